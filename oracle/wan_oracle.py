@@ -1,0 +1,336 @@
+"""CPU oracle for the Wan 2.1 DiT forward hot path.
+
+TEST INFRASTRUCTURE ONLY. This module is the plain, slow, obviously correct
+definition the CUDA library is checked against. Only the tests, the smoke check
+and the benchmark's CPU-baseline leg may import it; the library never calls it
+and shares no code with it.
+
+Every function works in float64 on one sample (no batch axis) and writes the
+definition out directly, with numpy matmul as the only library step. Sources are
+the pages on Wan 2.1:
+
+* [Wan-P2] "Wan: Open and Advanced Large-Scale Video Generative Models (Wan 2.1)",
+  zhao9797.github.io, sections "Diffusion Transformer", "I2V 架构扩展" (I2V
+  extension), "训练方法" (training method) and the config table.
+* [Wan-P1] "超越Sora！阿里正式完全开源 ... Wan2.1", 163.com, sections
+  "核心创新二" (DiT) and "核心创新四" (I2V).
+
+Where the pages are silent the plainest reading is taken; each such reading is
+named in the docstring ("reading: ...").
+
+Parity-pin status: every function here is pinned by a ``-m "not gpu"`` test
+against something other than itself (a library routine, a closed form, an
+invariant, or brute force). None is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+
+F64 = np.float64
+
+
+def _f(a) -> np.ndarray:
+    return np.asarray(a, dtype=F64)
+
+
+# --------------------------------------------------------------------------------------
+# Shapes
+# --------------------------------------------------------------------------------------
+
+def token_count(latent_frames: int, latent_h: int, latent_w: int) -> int:
+    """Sequence length after the (1,2,2) patchify [Wan-P2, "Diffusion Transformer"]:
+    L = (1+T/4) * H/16 * W/16 in pixel units; the latent grid is already H/8 x W/8
+    (Wan-VAE 4x8x8 compression, [Wan-P2, "Wan-VAE"]), so L = F * (h/2) * (w/2)."""
+    if latent_h % 2 or latent_w % 2:
+        raise ValueError("latent height and width must be even for (1,2,2) patches")
+    return latent_frames * (latent_h // 2) * (latent_w // 2)
+
+
+# --------------------------------------------------------------------------------------
+# Patchify / unpatchify  [Wan-P2, "Diffusion Transformer": patchify is a 3D convolution
+# with kernel (1,2,2); the sequence is unpatchified at the end]
+# --------------------------------------------------------------------------------------
+
+def patchify(latent, weight, bias) -> np.ndarray:
+    """3D convolution with kernel = stride = (1,2,2) over ``latent [C,F,H,W]`` with
+    ``weight [D,C,1,2,2]`` and ``bias [D]``, returning tokens ``[L,D]``.
+
+    Because the kernel equals the stride the patches do not overlap, so the
+    convolution is exactly: for every output position (f,i,j),
+    ``x[(f,i,j), d] = bias[d] + sum_{c,ph,pw} weight[d,c,0,ph,pw] * latent[c,f,2i+ph,2j+pw]``.
+    reading: tokens are ordered (f, i, j) row-major; the weight is flattened in
+    (c, ph, pw) order with pw fastest (the natural layout of the conv weight)."""
+    lat = _f(latent)
+    w = _f(weight)
+    C, F, H, W = lat.shape
+    D = w.shape[0]
+    assert w.shape == (D, C, 1, 2, 2)
+    patches = lat.reshape(C, F, H // 2, 2, W // 2, 2)          # c, f, i, ph, j, pw
+    patches = patches.transpose(1, 2, 4, 0, 3, 5)               # f, i, j, c, ph, pw
+    patches = patches.reshape(F * (H // 2) * (W // 2), C * 4)
+    return patches @ w.reshape(D, C * 4).T + _f(bias)[None, :]
+
+
+def unpatchify(tokens, out_ch: int, frames: int, height: int, width: int) -> np.ndarray:
+    """Inverse of the patch gather: ``tokens [L, out_ch*4]`` laid out (c, ph, pw) per
+    token, tokens ordered (f, i, j), back to ``[out_ch, F, H, W]``
+    [Wan-P2, "Diffusion Transformer": patchify -> blocks -> unpatchify]."""
+    y = _f(tokens)
+    hi, wi = height // 2, width // 2
+    y = y.reshape(frames, hi, wi, out_ch, 2, 2)                  # f, i, j, c, ph, pw
+    y = y.transpose(3, 0, 1, 4, 2, 5)                            # c, f, i, ph, j, pw
+    return y.reshape(out_ch, frames, height, width)
+
+
+# --------------------------------------------------------------------------------------
+# Timestep embedding and the shared AdaLN MLP
+# --------------------------------------------------------------------------------------
+
+def sinusoidal_embedding(t: float, dim: int = 256) -> np.ndarray:
+    """Sinusoidal timestep embedding; the frequency dimension is 256 [Wan-P2, note under
+    the config table]. reading: frequencies 10000^(-i/(dim/2)) for i < dim/2, cosines
+    first, then sines (the DiT lineage the page cites)."""
+    half = dim // 2
+    freqs = np.power(F64(10000.0), -np.arange(half, dtype=F64) / half)
+    args = F64(t) * freqs
+    return np.concatenate([np.cos(args), np.sin(args)])
+
+
+def silu(x) -> np.ndarray:
+    x = _f(x)
+    return x / (1.0 + np.exp(-x))
+
+
+def linear(x, weight, bias=None) -> np.ndarray:
+    """y = x W^T + b with ``weight [out, in]``."""
+    y = _f(x) @ _f(weight).T
+    if bias is not None:
+        y = y + _f(bias)
+    return y
+
+
+def time_mlp(t: float, w1, b1, w2, b2, freq_dim: int = 256) -> np.ndarray:
+    """Shared timestep MLP: one MLP of Linear + SiLU layers predicts the six
+    modulation vectors and is shared by all blocks [Wan-P2, "Diffusion Transformer";
+    Wan-P1, "核心创新二"]. reading: sinusoid(256) -> Linear(256,D) -> SiLU ->
+    Linear(D,6D), reshaped to ``[6, D]``."""
+    e = sinusoidal_embedding(t, freq_dim)
+    hdn = silu(linear(e, w1, b1))
+    out = linear(hdn, w2, b2)
+    return out.reshape(6, -1)
+
+
+def block_modulation(e, mod_bias) -> np.ndarray:
+    """Each block learns its own bias on top of the shared MLP output
+    [Wan-P2, "Diffusion Transformer"; Wan-P1, "核心创新二"]: ``mod = e + bias_b``.
+    reading: rows are (shift_msa, scale_msa, gate_msa, shift_ffn, scale_ffn, gate_ffn)."""
+    return _f(e) + _f(mod_bias)
+
+
+# --------------------------------------------------------------------------------------
+# Normalisation, activation, attention
+# --------------------------------------------------------------------------------------
+
+def layer_norm(x, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm over the last axis without affine parameters, biased variance
+    (divide by D), eps = 1e-6."""
+    x = _f(x)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def modulate(h, shift, scale) -> np.ndarray:
+    """AdaLN modulation. reading: ``h * (1 + scale) + shift`` (DiT convention)."""
+    return _f(h) * (1.0 + _f(scale)) + _f(shift)
+
+
+def gelu_tanh(x) -> np.ndarray:
+    """GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = _f(x)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def softmax(s, axis: int = -1) -> np.ndarray:
+    s = _f(s)
+    z = np.exp(s - s.max(axis=axis, keepdims=True))
+    return z / z.sum(axis=axis, keepdims=True)
+
+
+def attention(q, k, v, heads: int) -> np.ndarray:
+    """Multi-head scaled dot-product attention, non-causal, no dropout: per head,
+    ``softmax(q k^T / sqrt(d)) v`` with heads as contiguous d-wide slices of the model
+    width. Used for the full spatio-temporal self-attention [Wan-P2, "Diffusion
+    Transformer": full spatio-temporal attention] and the text cross-attention
+    [Wan-P1, "核心创新二": cross-attention in every block]. reading: no positional
+    encoding and no q/k normalisation (the pages mention neither)."""
+    q, k, v = _f(q), _f(k), _f(v)
+    Lq, D = q.shape
+    d = D // heads
+    out = np.empty((Lq, D), dtype=F64)
+    step = 512  # query rows are independent; this bound only limits memory
+    for hh in range(heads):
+        sl = slice(hh * d, (hh + 1) * d)
+        for r0 in range(0, Lq, step):
+            p = softmax(q[r0:r0 + step, sl] @ k[:, sl].T / math.sqrt(d), axis=-1)
+            out[r0:r0 + step, sl] = p @ v[:, sl]
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Block branches
+# --------------------------------------------------------------------------------------
+
+def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
+                          kv_source=None) -> np.ndarray:
+    """Self-attention sub-layer output before the gate: ``attn(h Wq, h Wk, h Wv) Wo^T + bo``.
+    The fused QKV weight ``w_qkv [3D, D]`` is stacked (q, k, v). ``kv_source`` (all rows
+    of h) lets the caller evaluate only some query rows; by default it is ``h``."""
+    h = _f(h)
+    D = h.shape[-1]
+    src = h if kv_source is None else _f(kv_source)
+    wqkv, bqkv = _f(w["w_qkv"]), _f(w["b_qkv"])
+    q = linear(h, wqkv[:D], bqkv[:D])
+    k = linear(src, wqkv[D:2 * D], bqkv[D:2 * D])
+    v = linear(src, wqkv[2 * D:], bqkv[2 * D:])
+    o = attention(q, k, v, heads)
+    return linear(o, w["w_o"], w["b_o"])
+
+
+def cross_attention_branch(h, ctx, w: Dict[str, np.ndarray], heads: int,
+                           img_ctx=None) -> np.ndarray:
+    """Cross-attention sub-layer: queries from the video tokens, keys and values from
+    the 512 umT5 text tokens [Wan-P2, "Diffusion Transformer" and "umT5"]. For I2V, a
+    decoupled second attention over image-context tokens with its own K/V projection
+    is added before the shared output projection [Wan-P2, "I2V 架构扩展"; Wan-P1,
+    "核心创新四"]. reading: ``o = attn(q,Kt,Vt) + attn(q,Ki,Vi)``, weight 1."""
+    D = _f(h).shape[-1]
+    q = linear(h, w["w_cq"], w["b_cq"])
+    kv = linear(ctx, w["w_ckv"], w["b_ckv"])
+    o = attention(q, kv[:, :D], kv[:, D:], heads)
+    if img_ctx is not None:
+        kvi = linear(img_ctx, w["w_ckv_img"], w["b_ckv_img"])
+        o = o + attention(q, kvi[:, :D], kvi[:, D:], heads)
+    return linear(o, w["w_co"], w["b_co"])
+
+
+def ffn_branch(h, w: Dict[str, np.ndarray]) -> np.ndarray:
+    """Feed-forward sub-layer: Linear(D,F) -> GELU-tanh -> Linear(F,D)
+    [Wan-P2 config table: FFN dimension 8960 / 13824]. reading: a plain two-matrix
+    FFN (a gated GLU would not match the 1.3B/14B parameter counts)."""
+    return linear(gelu_tanh(linear(h, w["w_1"], w["b_1"])), w["w_2"], w["b_2"])
+
+
+def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6,
+              img_ctx=None, rows: Optional[Sequence[int]] = None,
+              return_parts: bool = False):
+    """One DiT block [Wan-P2, "Diffusion Transformer"]:
+
+    1. ``x += gate_msa * SelfAttn(LN(x) (1 + scale_msa) + shift_msa)``
+    2. ``x += CrossAttn(LN(x), ctx[, img_ctx])``
+    3. ``x += gate_ffn * FFN(LN(x) (1 + scale_ffn) + shift_ffn)``
+
+    with ``mod = e + mod_bias`` (six vectors, see ``block_modulation``).
+    reading: self-attention, then cross-attention, then FFN; the cross-attention
+    input gets a plain LayerNorm and its residual has no gate (the pages give six
+    modulation vectors, i.e. two gated branches).
+
+    ``rows`` evaluates only those query rows; it is exact because every step but
+    self-attention is row-local, and self-attention still takes keys and values from
+    all rows. Returns ``x_out`` (of the selected rows), and with ``return_parts``
+    also a dict of intermediates for those rows.
+    """
+    x = _f(x)
+    mod = block_modulation(e, w["mod_bias"])
+    shift_msa, scale_msa, gate_msa, shift_ffn, scale_ffn, gate_ffn = mod
+    h_all = modulate(layer_norm(x, eps), shift_msa, scale_msa)
+    if rows is None:
+        xr, hr = x, h_all
+    else:
+        rows = np.asarray(rows)
+        xr, hr = x[rows], h_all[rows]
+    parts = {"h_msa": hr}
+    sa = self_attention_branch(hr, w, heads, kv_source=h_all)
+    parts["sa"] = sa
+    x1 = xr + gate_msa * sa
+    hc = layer_norm(x1, eps)
+    parts["h_cross"] = hc
+    ca = cross_attention_branch(hc, ctx, w, heads, img_ctx=img_ctx)
+    parts["ca"] = ca
+    x2 = x1 + ca
+    hf = modulate(layer_norm(x2, eps), shift_ffn, scale_ffn)
+    parts["h_ffn"] = hf
+    ff = ffn_branch(hf, w)
+    parts["ffn"] = ff
+    x3 = x2 + gate_ffn * ff
+    parts["x_after_sa"], parts["x_after_ca"] = x1, x2
+    return (x3, parts) if return_parts else x3
+
+
+# --------------------------------------------------------------------------------------
+# I2V input fusion and image context  [Wan-P2, "I2V 架构扩展"; Wan-P1, "核心创新四"]
+# --------------------------------------------------------------------------------------
+
+def i2v_mask(frame_keep, latent_frames: int, height: int, width: int,
+             temporal_stride: int = 4) -> np.ndarray:
+    """Binary mask (1 = keep, 0 = generate) over the pixel frames, reshaped to the VAE
+    temporal stride. reading: the first pixel frame's value is repeated ``stride``
+    times so the 1+T frames become ``latent_frames * stride`` values, which are
+    grouped as ``[latent_frames, stride]`` and put on the channel axis, giving
+    ``[stride, F, H, W]`` broadcast over the latent grid."""
+    m = np.asarray(frame_keep, dtype=F64).reshape(-1)
+    assert m.shape[0] == 1 + temporal_stride * (latent_frames - 1)
+    m = np.concatenate([np.repeat(m[:1], temporal_stride), m[1:]])
+    m = m.reshape(latent_frames, temporal_stride).T                  # [stride, F]
+    return np.broadcast_to(m[:, :, None, None], (temporal_stride, latent_frames, height, width)).copy()
+
+
+def i2v_input(noise, cond, mask) -> np.ndarray:
+    """Noise latent, condition latent and reshaped mask concatenated on channels."""
+    return np.concatenate([_f(noise), _f(cond), _f(mask)], axis=0)
+
+
+def image_context_mlp(feat, w1, b1, w2, b2, w3, b3) -> np.ndarray:
+    """Three-layer MLP projecting image-encoder features to the global image context.
+    reading: Linear(1280,D) -> GELU-tanh -> Linear(D,D) -> GELU-tanh -> Linear(D,D)."""
+    hdn = gelu_tanh(linear(feat, w1, b1))
+    hdn = gelu_tanh(linear(hdn, w2, b2))
+    return linear(hdn, w3, b3)
+
+
+# --------------------------------------------------------------------------------------
+# Head, stack and flow matching
+# --------------------------------------------------------------------------------------
+
+def head(x, w_head, b_head, eps: float = 1e-6) -> np.ndarray:
+    """Output head. reading: plain LayerNorm, then Linear(D, out_ch*4)."""
+    return linear(layer_norm(x, eps), w_head, b_head)
+
+
+def flow_matching_input(x1, x0, u: float) -> np.ndarray:
+    """Intermediate latent of rectified flow [Wan-P2, "训练方法"]: x_t = t x1 + (1-t) x0."""
+    return F64(u) * _f(x1) + (1.0 - F64(u)) * _f(x0)
+
+
+def flow_matching_target(x1, x0) -> np.ndarray:
+    """Ground-truth velocity v_t = x1 - x0 [Wan-P2, "训练方法"]."""
+    return _f(x1) - _f(x0)
+
+
+def dit_stack(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, heads: int,
+              eps: float = 1e-6, img_ctx=None, freq_dim: int = 256) -> np.ndarray:
+    """Whole DiT on one sample [Wan-P2, "Diffusion Transformer"]: patchify -> the time
+    MLP shared by all blocks -> N blocks (each with its own modulation bias) -> head ->
+    unpatchify. ``weights`` holds ``w_p, b_p, w_t1, b_t1, w_t2, b_t2, w_head, b_head``.
+    Returns the predicted velocity ``[out_ch, F, H, W]``."""
+    lat = _f(latent)
+    C, F, H, W = lat.shape
+    x = patchify(lat, weights["w_p"], weights["b_p"])
+    e = time_mlp(t, weights["w_t1"], weights["b_t1"], weights["w_t2"], weights["b_t2"], freq_dim)
+    for blk in blocks:
+        x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx)
+    y = head(x, weights["w_head"], weights["b_head"], eps)
+    return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)

@@ -1,0 +1,140 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and show the pins catch them:
+a dropped term, a wrong sign or index, a transposed operand, a wrong constant."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import wan_oracle as O
+import test_oracle_pins as P
+
+
+def _fails(check, *args):
+    with pytest.raises(AssertionError):
+        check(*args)
+
+
+def test_patchify_mutations_are_caught():
+    def swapped_ph_pw(latent, weight, bias):          # patch flattened (pw, ph) instead of (ph, pw)
+        w = np.asarray(weight).transpose(0, 1, 2, 4, 3)
+        return O.patchify(latent, w, bias)
+
+    def no_bias(latent, weight, bias):
+        return O.patchify(latent, weight, np.zeros_like(bias))
+    _fails(P.check_patchify, swapped_ph_pw)
+    _fails(P.check_patchify, no_bias)
+
+    def transposed_tokens(tokens, c, f, h, w):         # (j, i) token order in the inverse
+        y = np.asarray(tokens).reshape(f, h // 2, w // 2, -1).transpose(0, 2, 1, 3).reshape(len(tokens), -1)
+        return O.unpatchify(y, c, f, h, w)
+    _fails(P.check_patch_roundtrip, O.patchify, transposed_tokens)
+
+
+def test_embedding_mutations_are_caught():
+    def sin_first(t, dim=256):
+        e = O.sinusoidal_embedding(t, dim)
+        return np.concatenate([e[dim // 2:], e[:dim // 2]])
+
+    def wrong_base(t, dim=256):
+        half = dim // 2
+        a = t * np.power(1000.0, -np.arange(half) / half)
+        return np.concatenate([np.cos(a), np.sin(a)])
+    _fails(P.check_sinusoid, sin_first)
+    _fails(P.check_sinusoid, wrong_base)
+
+    def relu_mlp(t, w1, b1, w2, b2, freq_dim=256):
+        e = O.sinusoidal_embedding(t, freq_dim)
+        return O.linear(np.maximum(O.linear(e, w1, b1), 0), w2, b2).reshape(6, -1)
+    _fails(P.check_time_mlp, relu_mlp, O.block_modulation)
+    _fails(P.check_time_mlp, O.time_mlp, lambda e, b: np.asarray(e) + 0.5 * np.asarray(b))
+
+
+def test_norm_and_activation_mutations_are_caught():
+    def unbiased_ln(x, eps=1e-6):
+        x = np.asarray(x, np.float64)
+        return (x - x.mean(-1, keepdims=True)) / np.sqrt(x.var(-1, ddof=1, keepdims=True) + eps)
+
+    def eps_outside(x, eps=1e-6):
+        x = np.asarray(x, np.float64)
+        return (x - x.mean(-1, keepdims=True)) / (np.sqrt(x.var(-1, keepdims=True)) + eps)
+    _fails(P.check_layer_norm, unbiased_ln)
+    _fails(P.check_layer_norm, eps_outside)
+    _fails(P.check_modulate, lambda h, sh, sc: np.asarray(h) * np.asarray(sc) + sh, O.layer_norm)
+    _fails(P.check_modulate, lambda h, sh, sc: np.asarray(h) * (1 + np.asarray(sc)) - sh, O.layer_norm)
+
+    def erf_gelu(x):
+        x = np.asarray(x, np.float64)
+        return np.array([0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in x])
+    _fails(P.check_gelu, erf_gelu)
+    _fails(P.check_gelu, lambda x: 0.5 * x * (1 + np.tanh(math.sqrt(2 / math.pi) * (x + 0.0447 * x ** 3))))
+    _fails(P.check_softmax, lambda s, axis=-1: np.exp(s) / np.exp(s).sum(axis, keepdims=True) * 1.0000001)
+
+
+def test_attention_mutations_are_caught():
+    def unscaled(q, k, v, heads):
+        return O.attention(np.asarray(q) * math.sqrt(np.asarray(q).shape[1] // heads), k, v, heads)
+
+    def heads_interleaved(q, k, v, heads):            # head h takes columns h, h+H, ... instead of a slab
+        q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+        D = q.shape[1]
+        perm = np.arange(D).reshape(D // heads, heads).T.reshape(-1)
+        inv = np.argsort(perm)
+        return O.attention(q[:, perm], k[:, perm], v[:, perm], heads)[:, inv]
+
+    def softmax_over_queries(q, k, v, heads):
+        q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+        d = q.shape[1] // heads
+        out = np.empty((q.shape[0], q.shape[1]))
+        for hh in range(heads):
+            sl = slice(hh * d, (hh + 1) * d)
+            p = O.softmax(q[:, sl] @ k[:, sl].T / math.sqrt(d), axis=0)
+            out[:, sl] = p @ v[:, sl]
+        return out
+    _fails(P.check_attention, unscaled)
+    _fails(P.check_attention, heads_interleaved)
+    _fails(P.check_attention, softmax_over_queries)
+
+
+def test_block_mutations_are_caught(monkeypatch):
+    # gate applied to the cross-attention branch as well (wrong reading of the six vectors)
+    orig = O.cross_attention_branch
+
+    def gated_cross(h, ctx, w, heads, img_ctx=None):
+        return 0.5 * orig(h, ctx, w, heads, img_ctx=img_ctx)
+    monkeypatch.setattr(O, "cross_attention_branch", gated_cross)
+    _fails(P.check_block_vs_torch, O.dit_block)
+    monkeypatch.undo()
+
+    # shift and scale rows swapped in the modulation
+    orig_mod = O.block_modulation
+
+    def swapped(e, b):
+        m = orig_mod(e, b)
+        return m[[1, 0, 2, 4, 3, 5]]
+    monkeypatch.setattr(O, "block_modulation", swapped)
+    _fails(P.check_block_vs_torch, O.dit_block)
+    monkeypatch.undo()
+
+    # FFN with the activation dropped
+    monkeypatch.setattr(O, "gelu_tanh", lambda x: np.asarray(x, np.float64))
+    _fails(P.check_block_vs_torch, O.dit_block)
+    monkeypatch.undo()
+
+    # image-context attention subtracted instead of added (I2V)
+    orig_attn = O.attention
+    calls = {"n": 0}
+
+    def sign_flip_second(q, k, v, heads):
+        calls["n"] += 1
+        r = orig_attn(q, k, v, heads)
+        return -r if k.shape[0] == 5 else r           # the tiny I2V image context has 5 tokens
+    monkeypatch.setattr(O, "attention", sign_flip_second)
+    _fails(P.check_block_vs_torch, O.dit_block)
+    monkeypatch.undo()
+
+
+def test_i2v_mask_mutation_is_caught():
+    def no_repeat(keep, F, H, W, stride=4):
+        m = np.concatenate([np.asarray(keep, np.float64), np.zeros(3)]).reshape(F, stride).T
+        return np.broadcast_to(m[:, :, None, None], (stride, F, H, W)).copy()
+    _fails(P.check_i2v_mask, no_repeat)

@@ -1,0 +1,484 @@
+"""Pins of the CPU oracle to facts outside itself (library routines, closed forms,
+invariants, brute force, and the numbers the Wan 2.1 pages print).
+
+Each pin is written as a ``check_*`` function that takes the oracle function(s)
+under test, so ``test_oracle_mutations.py`` can plant plausible mistakes in the
+oracle and show that some pin fails.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as tF
+
+from oracle import wan_oracle as O
+from wan_inputs import WORKLOADS, make_inputs, round_bf16, bf16_bits, bits_to_f32, sample_rows
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = lambda s: np.random.Generator(np.random.PCG64(s))  # noqa: E731
+
+
+def t64(a):
+    return torch.as_tensor(np.asarray(a, dtype=np.float64))
+
+
+# ----------------------------------------------------------------------------------------
+# Golden: the pages' config table and shape formula
+# ----------------------------------------------------------------------------------------
+
+def test_token_count_matches_page_formula():
+    g = json.load(open(os.path.join(GOLDEN, "wan21_config_table.json")))
+    c = g["vae_compression"]
+    for vid in g["videos"]:
+        T = vid["T_plus_1"] - 1
+        L_page = (1 + T // 4) * (vid["H"] // 16) * (vid["W"] // 16)   # pixel-space formula
+        lat = (1 + T // c["t"], vid["H"] // c["h"], vid["W"] // c["w"])  # latent grid
+        assert O.token_count(*lat) == L_page
+    assert WORKLOADS["wan13b_480p_block"].tokens == 32760
+    assert WORKLOADS["wan14b_720p_block"].tokens == 75600
+    assert WORKLOADS["tiny_f32_block"].tokens == 32
+    with pytest.raises(ValueError):
+        O.token_count(2, 7, 8)
+
+
+def _block_param_count(D, F):
+    # self-attn qkv+o, cross-attn q+kv+o, FFN (weights and biases), per-block modulation bias
+    return (3 * D * D + 3 * D) + (D * D + D) + (D * D + D) + (2 * D * D + 2 * D) + (D * D + D) \
+        + (F * D + F) + (D * F + D) + 6 * D
+
+
+def test_parameter_count_matches_model_names():
+    """The block inventory (8 D^2 attention matrices, a plain 2-matrix FFN and a shared
+    AdaLN MLP) reproduces the 1.3B / 14B names of the config table; a GLU FFN or an
+    unshared AdaLN would not."""
+    g = json.load(open(os.path.join(GOLDEN, "wan21_config_table.json")))
+    for name, m in g["models"].items():
+        D, F, n = m["dim"], m["ffn"], m["layers"]
+        total = n * _block_param_count(D, F)
+        assert abs(total / m["nominal_params"] - 1) < 0.08, (name, total)
+        glu = n * (_block_param_count(D, F) + F * D)
+        assert glu / m["nominal_params"] > 1.18
+        unshared = n * 6 * D * D
+        frac = unshared / (total + unshared)
+        assert abs(frac - g["adaln_sharing_saves_fraction"]) < 0.07
+
+
+# ----------------------------------------------------------------------------------------
+# Patchify / unpatchify
+# ----------------------------------------------------------------------------------------
+
+def check_patchify(patchify):
+    rng = RNG(1)
+    for C, F, H, W, D in [(16, 2, 8, 8, 24), (36, 3, 6, 10, 7), (4, 1, 2, 2, 3)]:
+        lat = rng.standard_normal((C, F, H, W))
+        w = rng.standard_normal((D, C, 1, 2, 2))
+        b = rng.standard_normal(D)
+        ref = tF.conv3d(t64(lat)[None], t64(w), t64(b), stride=(1, 2, 2))[0]  # [D,F,H/2,W/2]
+        ref = ref.permute(1, 2, 3, 0).reshape(-1, D).numpy()
+        got = patchify(lat, w, b)
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_patchify_is_the_strided_conv3d():
+    check_patchify(O.patchify)
+
+
+def check_patch_roundtrip(patchify, unpatchify):
+    rng = RNG(2)
+    C, F, H, W = 16, 3, 6, 10
+    lat = rng.standard_normal((C, F, H, W))
+    onehot = np.zeros((C * 4, C, 1, 2, 2))
+    for c in range(C):
+        for ph in range(2):
+            for pw in range(2):
+                onehot[c * 4 + ph * 2 + pw, c, 0, ph, pw] = 1.0
+    tokens = patchify(lat, onehot, np.zeros(C * 4))
+    # brute-force gather of one token
+    f, i, j = 2, 1, 3
+    tok = tokens[(f * (H // 2) + i) * (W // 2) + j]
+    for c in range(C):
+        assert tok[c * 4 + 0] == lat[c, f, 2 * i, 2 * j]
+        assert tok[c * 4 + 3] == lat[c, f, 2 * i + 1, 2 * j + 1]
+    back = unpatchify(tokens, C, F, H, W)
+    assert np.array_equal(back, lat)           # exact permutation
+    y = rng.standard_normal((F * (H // 2) * (W // 2), C * 4))
+    assert np.array_equal(patchify(unpatchify(y, C, F, H, W), onehot, np.zeros(C * 4)), y)
+
+
+def test_patchify_unpatchify_roundtrip_exact():
+    check_patch_roundtrip(O.patchify, O.unpatchify)
+
+
+# ----------------------------------------------------------------------------------------
+# Timestep embedding, shared MLP, per-block bias
+# ----------------------------------------------------------------------------------------
+
+def check_sinusoid(emb_fn):
+    e0 = emb_fn(0.0, 256)
+    assert np.array_equal(e0, np.concatenate([np.ones(128), np.zeros(128)]))
+    e = emb_fn(math.pi / 2, 256)                 # first frequency is 1: cos(pi/2)=0, sin(pi/2)=1
+    assert abs(e[0]) < 1e-15 and abs(e[128] - 1) < 1e-15
+    for t in [0.3, 17.0, 999.9]:
+        e = emb_fn(t, 256)
+        np.testing.assert_allclose(e[:128] ** 2 + e[128:] ** 2, 1.0, atol=1e-14)
+        # independent route to the frequencies: exp(-ln(10000) i / 128)
+        f = torch.exp(-math.log(10000.0) * torch.arange(128, dtype=torch.float64) / 128)
+        ref = torch.cat([torch.cos(t * f), torch.sin(t * f)]).numpy()
+        np.testing.assert_allclose(e, ref, atol=1e-12)
+
+
+def test_sinusoid_closed_forms():
+    check_sinusoid(O.sinusoidal_embedding)
+
+
+def check_time_mlp(time_mlp, block_modulation):
+    rng = RNG(3)
+    D = 32
+    w1, b1 = rng.standard_normal((D, 256)) * 0.1, rng.standard_normal(D) * 0.1
+    w2, b2 = rng.standard_normal((6 * D, D)) * 0.1, rng.standard_normal(6 * D) * 0.1
+    t = 431.5
+    mlp = torch.nn.Sequential(torch.nn.Linear(256, D), torch.nn.SiLU(), torch.nn.Linear(D, 6 * D)).double()
+    with torch.no_grad():
+        mlp[0].weight.copy_(t64(w1)); mlp[0].bias.copy_(t64(b1))
+        mlp[2].weight.copy_(t64(w2)); mlp[2].bias.copy_(t64(b2))
+        ref = mlp(t64(O.sinusoidal_embedding(t, 256))).numpy().reshape(6, D)
+    e = time_mlp(t, w1, b1, w2, b2)
+    np.testing.assert_allclose(e, ref, rtol=1e-12, atol=1e-13)
+    bias = rng.standard_normal((6, D))
+    assert np.array_equal(block_modulation(e, bias), block_modulation(e, bias.copy()))  # equal biases
+    delta = rng.standard_normal((6, D))
+    np.testing.assert_allclose(block_modulation(e, bias + delta) - block_modulation(e, bias), delta,
+                               atol=1e-13)
+
+
+def test_shared_time_mlp_and_block_bias():
+    check_time_mlp(O.time_mlp, O.block_modulation)
+
+
+# ----------------------------------------------------------------------------------------
+# LayerNorm, modulation, GELU, softmax
+# ----------------------------------------------------------------------------------------
+
+def check_layer_norm(ln):
+    rng = RNG(4)
+    x = rng.standard_normal((7, 96)) * 3 + 1.5
+    ref = tF.layer_norm(t64(x), (96,), eps=1e-6).numpy()
+    np.testing.assert_allclose(ln(x, 1e-6), ref, rtol=1e-12, atol=1e-12)
+    y = ln(x, 1e-6)
+    var = x.var(axis=-1)
+    np.testing.assert_allclose(y.mean(axis=-1), 0.0, atol=1e-13)
+    np.testing.assert_allclose((y ** 2).mean(axis=-1), var / (var + 1e-6), rtol=1e-12)
+    c = np.full((2, 16), 3.25)                   # constant rows normalise to exactly 0
+    assert np.array_equal(ln(c, 1e-6), np.zeros_like(c))
+
+
+def test_layer_norm_pins():
+    check_layer_norm(O.layer_norm)
+
+
+def check_modulate(modulate, ln):
+    rng = RNG(5)
+    x = rng.standard_normal((5, 64))
+    h = ln(x, 1e-6)
+    z = np.zeros(64)
+    np.testing.assert_array_equal(modulate(h, z, z), h)            # scale = shift = 0: plain LN
+    sh = rng.standard_normal(64)
+    np.testing.assert_allclose(modulate(h, sh, -np.ones(64)), np.broadcast_to(sh, h.shape), atol=0)
+    sc = rng.standard_normal(64)
+    np.testing.assert_allclose(modulate(h, z, sc), h + h * sc, rtol=1e-15, atol=1e-15)
+
+
+def test_modulation_pins():
+    check_modulate(O.modulate, O.layer_norm)
+
+
+def check_gelu(gelu):
+    xs = np.linspace(-8, 8, 1001)
+    ref = np.array([0.5 * v * (1 + math.tanh(math.sqrt(2 / math.pi) * (v + 0.044715 * v ** 3))) for v in xs])
+    np.testing.assert_allclose(gelu(xs), ref, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(gelu(xs), tF.gelu(t64(xs), approximate="tanh").numpy(), rtol=1e-13, atol=1e-15)
+    assert gelu(np.array([0.0]))[0] == 0.0
+
+
+def test_gelu_tanh_pins():
+    check_gelu(O.gelu_tanh)
+
+
+def test_silu_pins():
+    xs = np.linspace(-20, 20, 401)
+    np.testing.assert_allclose(O.silu(xs), tF.silu(t64(xs)).numpy(), rtol=1e-14, atol=1e-300)
+
+
+def check_softmax(softmax):
+    rng = RNG(6)
+    s = rng.standard_normal((9, 33)) * 10
+    p = softmax(s, -1)
+    assert np.all(np.abs(p.sum(-1) - 1) < 1e-12)
+    np.testing.assert_allclose(p, torch.softmax(t64(s), -1).numpy(), rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(softmax(s + 1234.5, -1), p, rtol=1e-12, atol=1e-300)
+
+
+def test_softmax_pins():
+    check_softmax(O.softmax)
+
+
+# ----------------------------------------------------------------------------------------
+# Attention: brute force, library, special cases
+# ----------------------------------------------------------------------------------------
+
+def naive_attention_loops(q, k, v, heads):
+    """Independent triple-loop attention (pure Python) for tiny inputs."""
+    Lq, D = len(q), len(q[0])
+    Lk = len(k)
+    d = D // heads
+    out = [[0.0] * D for _ in range(Lq)]
+    for hh in range(heads):
+        for i in range(Lq):
+            scores = []
+            for j in range(Lk):
+                acc = 0.0
+                for c in range(hh * d, (hh + 1) * d):
+                    acc += q[i][c] * k[j][c]
+                scores.append(acc / math.sqrt(d))
+            mx = max(scores)
+            ex = [math.exp(sv - mx) for sv in scores]
+            den = sum(ex)
+            for c in range(hh * d, (hh + 1) * d):
+                out[i][c] = sum(ex[j] * v[j][c] for j in range(Lk)) / den
+    return np.array(out)
+
+
+def check_attention(attention):
+    rng = RNG(7)
+    for Lq, Lk, H, d in [(5, 7, 2, 4), (3, 1, 1, 8), (6, 13, 3, 2)]:
+        q = rng.standard_normal((Lq, H * d)) * 2
+        k = rng.standard_normal((Lk, H * d)) * 2
+        v = rng.standard_normal((Lk, H * d))
+        got = attention(q, k, v, H)
+        np.testing.assert_allclose(got, naive_attention_loops(q.tolist(), k.tolist(), v.tolist(), H),
+                                   rtol=1e-12, atol=1e-13)
+        qt = t64(q).reshape(Lq, H, d).transpose(0, 1)
+        kt = t64(k).reshape(Lk, H, d).transpose(0, 1)
+        vt = t64(v).reshape(Lk, H, d).transpose(0, 1)
+        ref = tF.scaled_dot_product_attention(qt, kt, vt).transpose(0, 1).reshape(Lq, H * d).numpy()
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+    # one key: output is that key's value
+    q = rng.standard_normal((4, 8)); k = rng.standard_normal((1, 8)); v = rng.standard_normal((1, 8))
+    np.testing.assert_allclose(attention(q, k, v, 2), np.repeat(v, 4, 0), rtol=1e-14)
+    # all keys equal: output is the mean of the values
+    k = np.repeat(rng.standard_normal((1, 8)), 6, 0); v = rng.standard_normal((6, 8))
+    np.testing.assert_allclose(attention(q, k, v, 2), np.repeat(v.mean(0, keepdims=True), 4, 0), rtol=1e-13)
+    # keys/values permuted together: same output
+    k = rng.standard_normal((9, 8)); v = rng.standard_normal((9, 8)); perm = rng.permutation(9)
+    np.testing.assert_allclose(attention(q, k[perm], v[perm], 2), attention(q, k, v, 2), rtol=1e-12)
+
+
+def test_attention_pins():
+    check_attention(O.attention)
+
+
+def test_attention_long_rows_chunking():
+    """Query-row chunking inside the oracle (memory bound only) changes nothing."""
+    rng = RNG(8)
+    q = rng.standard_normal((1100, 16)); k = rng.standard_normal((40, 16)); v = rng.standard_normal((40, 16))
+    full = O.attention(q, k, v, 2)
+    np.testing.assert_allclose(full[1000:], O.attention(q[1000:], k, v, 2), rtol=0, atol=0)
+
+
+# ----------------------------------------------------------------------------------------
+# Block: library re-expression, special cases, invariants, row sampling
+# ----------------------------------------------------------------------------------------
+
+def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None):
+    """The block re-expressed with torch library routines (layer_norm, linear,
+    scaled_dot_product_attention, gelu) in float64."""
+    X, E, C = t64(x), t64(e) + t64(w["mod_bias"]), t64(ctx)
+    D = X.shape[-1]
+    d = D // heads
+    W = {k: t64(v) for k, v in w.items()}
+
+    def mha(q, k, v):
+        Lq, Lk = q.shape[0], k.shape[0]
+        qh = q.reshape(Lq, heads, d).transpose(0, 1)
+        kh = k.reshape(Lk, heads, d).transpose(0, 1)
+        vh = v.reshape(Lk, heads, d).transpose(0, 1)
+        return tF.scaled_dot_product_attention(qh, kh, vh).transpose(0, 1).reshape(Lq, D)
+
+    ln = lambda t: tF.layer_norm(t, (D,), eps=eps)  # noqa: E731
+    h = ln(X) * (1 + E[1]) + E[0]
+    qkv = tF.linear(h, W["w_qkv"], W["b_qkv"])
+    X = X + E[2] * tF.linear(mha(qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]), W["w_o"], W["b_o"])
+    hc = ln(X)
+    q = tF.linear(hc, W["w_cq"], W["b_cq"])
+    kv = tF.linear(C, W["w_ckv"], W["b_ckv"])
+    o = mha(q, kv[:, :D], kv[:, D:])
+    if img_ctx is not None:
+        kvi = tF.linear(t64(img_ctx), W["w_ckv_img"], W["b_ckv_img"])
+        o = o + mha(q, kvi[:, :D], kvi[:, D:])
+    X = X + tF.linear(o, W["w_co"], W["b_co"])
+    hf = ln(X) * (1 + E[4]) + E[3]
+    ff = tF.linear(tF.gelu(tF.linear(hf, W["w_1"], W["b_1"]), approximate="tanh"), W["w_2"], W["b_2"])
+    return (X + E[5] * ff).numpy()
+
+
+def _tiny_block_inputs(i2v=False, seed=0):
+    w = WORKLOADS["wan13b_480p_i2v_block" if i2v else "tiny_f32_block"]
+    if i2v:
+        import dataclasses
+        w = dataclasses.replace(w, frames=2, height=4, width=8, dim=64, heads=2, ffn=96, text_len=9,
+                                img_len=5, img_feat=24, dtype="f32")
+    inp = make_inputs(w, seed=seed)
+    return w, inp
+
+
+def check_block_vs_torch(dit_block):
+    for i2v in (False, True):
+        w, inp = _tiny_block_inputs(i2v)
+        blk = inp["blocks"][0]
+        img = None
+        if i2v:
+            img = O.image_context_mlp(inp["img_feat"][0], inp["w_i1"], inp["b_i1"], inp["w_i2"],
+                                      inp["b_i2"], inp["w_i3"], inp["b_i3"])
+        got = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img)
+        ref = torch_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img)
+        np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(got - inp["x"][0], ref - inp["x"][0], rtol=1e-9, atol=1e-11)
+
+
+def test_block_matches_library_reexpression():
+    check_block_vs_torch(O.dit_block)
+
+
+def check_block_special_cases(dit_block):
+    w, inp = _tiny_block_inputs()
+    x, e, ctx = inp["x"][0].astype(np.float64), inp["e"][0].astype(np.float64), inp["ctx"][0]
+    blk = {k: np.asarray(v, dtype=np.float64) for k, v in inp["blocks"][0].items()}
+    e0 = e.copy()
+    e0[2] = -blk["mod_bias"][2]          # gate_msa = 0 exactly
+    e0[5] = -blk["mod_bias"][5]          # gate_ffn = 0 exactly
+    out = dit_block(x, e0, blk, ctx, w.heads)
+    ca = O.cross_attention_branch(O.layer_norm(x), ctx, blk, w.heads)
+    np.testing.assert_allclose(out, x + ca, rtol=1e-13, atol=1e-13)
+    blk0 = dict(blk, w_co=np.zeros_like(blk["w_co"]), b_co=np.zeros_like(blk["b_co"]))
+    assert np.array_equal(dit_block(x, e0, blk0, ctx, w.heads), x)      # identity block
+    perm = RNG(9).permutation(ctx.shape[0])                              # text order is irrelevant
+    np.testing.assert_allclose(dit_block(x, e, blk, ctx[perm], w.heads), dit_block(x, e, blk, ctx, w.heads),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_block_gates_identity_and_text_permutation():
+    check_block_special_cases(O.dit_block)
+
+
+def test_block_row_sampling_is_exact():
+    w, inp = _tiny_block_inputs()
+    x, e, ctx, blk = inp["x"][0], inp["e"][0], inp["ctx"][0], inp["blocks"][0]
+    full = O.dit_block(x, e, blk, ctx, w.heads)
+    rows = [0, 5, 17, 31]
+    np.testing.assert_allclose(O.dit_block(x, e, blk, ctx, w.heads, rows=rows), full[rows], rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------------------
+# I2V, image MLP, head, stack, flow matching
+# ----------------------------------------------------------------------------------------
+
+def check_i2v_mask(i2v_mask):
+    keep = np.zeros(81); keep[0] = 1
+    m = i2v_mask(keep, 21, 6, 4)
+    assert m.shape == (4, 21, 6, 4)
+    assert np.all(m[:, 0] == 1) and np.all(m[:, 1:] == 0)
+    keep = np.zeros(81); keep[80] = 1                  # last pixel frame -> channel 3 of the last latent frame
+    m = i2v_mask(keep, 21, 2, 2)
+    assert m[3, 20].min() == 1 and m.sum() == 4
+    keep = np.zeros(81); keep[1] = 1                   # second pixel frame -> channel 0 of latent frame 1
+    m = i2v_mask(keep, 21, 2, 2)
+    assert m[0, 1].min() == 1 and m.sum() == 4
+
+
+def test_i2v_mask_structure():
+    check_i2v_mask(O.i2v_mask)
+
+
+def test_i2v_zero_projection_equals_t2v():
+    rng = RNG(10)
+    D, F, H, W = 12, 2, 4, 6
+    noise, cond = rng.standard_normal((16, F, H, W)), rng.standard_normal((16, F, H, W))
+    keep = np.zeros(1 + 4 * (F - 1)); keep[0] = 1
+    x36 = O.i2v_input(noise, cond, O.i2v_mask(keep, F, H, W))
+    w16 = rng.standard_normal((D, 16, 1, 2, 2)); b = rng.standard_normal(D)
+    w36 = np.concatenate([w16, np.zeros((D, 20, 1, 2, 2))], axis=1)
+    assert np.array_equal(O.patchify(x36, w36, b), O.patchify(noise, w16, b))
+    w36[:, 16:] = rng.standard_normal((D, 20, 1, 2, 2))
+    assert not np.allclose(O.patchify(x36, w36, b), O.patchify(noise, w16, b))
+
+
+def test_image_context_mlp_vs_torch():
+    rng = RNG(11)
+    feat = rng.standard_normal((5, 24))
+    ws = [rng.standard_normal(s) * 0.2 for s in [(16, 24), (16,), (16, 16), (16,), (16, 16), (16,)]]
+    ref = t64(feat)
+    for i in range(3):
+        ref = tF.linear(ref, t64(ws[2 * i]), t64(ws[2 * i + 1]))
+        if i < 2:
+            ref = tF.gelu(ref, approximate="tanh")
+    np.testing.assert_allclose(O.image_context_mlp(feat, *ws), ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
+    w = WORKLOADS["tiny_f32_block"]
+    inp = make_inputs(w, seed=1, n_blocks=2)
+    lat, t, ctx = inp["noise"][0], float(inp["t"][0]), inp["ctx"][0]
+    zero = [{k: np.zeros_like(v) for k, v in b.items()} for b in inp["blocks"]]
+    v = O.dit_stack(lat, t, inp, zero, ctx, w.heads)
+    x = O.patchify(lat, inp["w_p"], inp["b_p"])
+    ref = O.unpatchify(tF.linear(tF.layer_norm(t64(x), (w.dim,), eps=1e-6), t64(inp["w_head"]),
+                                 t64(inp["b_head"])).numpy(), 16, w.frames, w.height, w.width)
+    np.testing.assert_allclose(v, ref, rtol=1e-12, atol=1e-12)
+    # two real blocks == the torch re-expression applied twice with the shared MLP output
+    v2 = O.dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads)
+    e = O.time_mlp(t, inp["w_t1"], inp["b_t1"], inp["w_t2"], inp["b_t2"])
+    xx = x
+    for b in inp["blocks"]:
+        xx = torch_block(xx, e, b, ctx, w.heads)
+    ref2 = O.unpatchify(O.head(xx, inp["w_head"], inp["b_head"]), 16, w.frames, w.height, w.width)
+    np.testing.assert_allclose(v2, ref2, rtol=1e-10, atol=1e-11)
+
+
+def test_flow_matching_endpoints():
+    rng = RNG(12)
+    x1, x0 = rng.standard_normal((3, 4)), rng.standard_normal((3, 4))
+    assert np.array_equal(O.flow_matching_input(x1, x0, 0.0), x0)
+    assert np.array_equal(O.flow_matching_input(x1, x0, 1.0), x1)
+    a, b = O.flow_matching_input(x1, x0, 0.25), O.flow_matching_input(x1, x0, 0.75)
+    np.testing.assert_allclose(b - a, 0.5 * O.flow_matching_target(x1, x0), rtol=1e-14, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------------------
+# Input generator (shared with the CUDA tests): bf16 rounding and row sampling
+# ----------------------------------------------------------------------------------------
+
+def test_bf16_rounding_matches_torch():
+    rng = RNG(13)
+    a = np.concatenate([rng.standard_normal(10000).astype(np.float32) * 100,
+                        np.array([0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.4e38, -1e-40], np.float32)])
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_bits(a), ref)
+    assert np.array_equal(round_bf16(a), torch.from_numpy(a).to(torch.bfloat16).float().numpy())
+    assert np.array_equal(bits_to_f32(bf16_bits(a)), round_bf16(a))
+
+
+def test_sample_rows_cover_ends_and_ragged_tail():
+    rows = sample_rows(32760)
+    assert len(rows) == 256 and rows[0] == 0 and rows[-1] == 32759
+    assert set(range(32640, 32760)).issubset(set(rows.tolist()))
+    assert np.array_equal(sample_rows(100), np.arange(100))
+
+
+def test_inputs_are_deterministic():
+    w = WORKLOADS["tiny_f32_block"]
+    a, b = make_inputs(w, seed=0), make_inputs(w, seed=0)
+    assert np.array_equal(a["x"], b["x"]) and np.array_equal(a["blocks"][0]["w_qkv"], b["blocks"][0]["w_qkv"])
+    assert not np.array_equal(a["x"], make_inputs(w, seed=1)["x"])
