@@ -1,0 +1,279 @@
+/*
+ * wan.h - C ABI of the B200 (sm_100a) library for the Wan 2.1 DiT forward hot path.
+ *
+ * The operations follow "Wan: Open and Advanced Large-Scale Video Generative Models
+ * (Wan 2.1)" (zhao9797.github.io), section "Diffusion Transformer" (patchify with a
+ * (1,2,2) 3D convolution, a shared Linear+SiLU timestep MLP predicting six modulation
+ * vectors with a learned bias per block, full spatio-temporal self-attention, text
+ * cross-attention, FFN, unpatchify), its config table (dim / FFN dim / heads / layers,
+ * frequency dim 256, latent dim 16), section "I2V 架构扩展" (I2V input fusion and
+ * decoupled image cross-attention) and section "训练方法" (rectified-flow
+ * interpolation and velocity target).
+ *
+ * Conventions for every call:
+ *  - Pointers to tensors are DEVICE pointers owned by the caller; the library never
+ *    allocates device memory. Calls that need scratch take a caller-provided device
+ *    workspace (size from wan_workspace_bytes). Struct pointers (config, weight
+ *    tables) are HOST pointers read during the call only.
+ *  - Tensors are dense, row-major, in the listed shapes. "act" means the activation /
+ *    weight dtype of the config (cfg->dtype: WAN_F32 or WAN_BF16). The residual
+ *    stream x, the modulation e and mod_bias, timesteps and outputs of patchify/head
+ *    are always fp32.
+ *  - Linear weights are [out_features, in_features] (y = x W^T + b), biases [out].
+ *  - Every device pointer must be 16-byte aligned.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). Arguments are validated on the host before any launch; on a
+ *    validation error nothing is launched and a negative wan_status is returned.
+ *    Launch failures return WAN_ERR_CUDA. Device-side waits are bounded: a wait that
+ *    runs out sets a device flag that wan_device_status() reports as WAN_ERR_TIMEOUT.
+ *  - Calls keep no state between them except the trace tables and the device error
+ *    flag; they are safe to call from several host threads on different streams.
+ *  - Shape limits: D = heads * head_dim; head_dim 128 (bf16) or <= 128 (fp32);
+ *    D, ffn_dim multiples of 64; latent H and W even; the fp32 path supports key
+ *    lengths up to 8192.
+ */
+#ifndef WAN_H
+#define WAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WAN_OK = 0,
+  WAN_ERR_NULL = -1,        /* a required pointer is NULL                          */
+  WAN_ERR_SHAPE = -2,       /* sizes inconsistent or outside the supported range   */
+  WAN_ERR_DTYPE = -3,       /* unknown dtype                                       */
+  WAN_ERR_ALIGN = -4,       /* a device pointer is not 16-byte aligned             */
+  WAN_ERR_WORKSPACE = -5,   /* workspace smaller than wan_workspace_bytes()        */
+  WAN_ERR_CUDA = -6,        /* a CUDA launch or runtime call failed                */
+  WAN_ERR_TIMEOUT = -7,     /* a bounded device-side wait ran out                  */
+  WAN_ERR_UNSUPPORTED = -8  /* valid request this build does not implement         */
+} wan_status;
+
+typedef enum { WAN_F32 = 0, WAN_BF16 = 1 } wan_dtype;
+
+/* Model hyper-parameters (config table of the Wan 2.1 page). */
+typedef struct {
+  int dim;          /* D: model width                       (1536 / 5120)   */
+  int heads;        /* attention heads                      (12 / 40)       */
+  int head_dim;     /* D / heads                            (128)           */
+  int ffn_dim;      /* F: FFN hidden width                  (8960 / 13824)  */
+  int in_ch;        /* DiT input channels: 16 (T2V) or 36 (I2V)             */
+  int out_ch;       /* output latent channels (16)                          */
+  int freq_dim;     /* sinusoidal timestep embedding width (256)            */
+  int img_feat_dim; /* image-encoder feature width for I2V (1280)           */
+  float eps;        /* LayerNorm epsilon (1e-6), no affine                  */
+  int dtype;        /* wan_dtype of weights and activations                 */
+} wan_dit_config;
+
+/* One DiT block's weights (act dtype unless noted). */
+typedef struct {
+  const float* mod_bias;            /* [6, D] fp32: per-block bias added to e  */
+  const void *w_qkv, *b_qkv;        /* [3D, D], [3D]: stacked q, k, v          */
+  const void *w_o, *b_o;            /* [D, D], [D]                             */
+  const void *w_cq, *b_cq;          /* [D, D], [D]: cross-attention query      */
+  const void *w_ckv, *b_ckv;        /* [2D, D], [2D]: text key, value          */
+  const void *w_co, *b_co;          /* [D, D], [D]: cross-attention output     */
+  const void *w_ckv_img, *b_ckv_img;/* [2D, D], [2D]: I2V image key, value; NULL for T2V */
+  const void *w_1, *b_1;            /* [F, D], [F]                             */
+  const void *w_2, *b_2;            /* [D, F], [D]                             */
+} wan_block_weights;
+
+/* Shared timestep MLP: sinusoid(freq_dim) -> Linear(freq_dim, D) -> SiLU -> Linear(D, 6D). */
+typedef struct {
+  const void *w_t1, *b_t1;          /* [D, freq_dim], [D]   */
+  const void *w_t2, *b_t2;          /* [6D, D], [6D]        */
+} wan_time_weights;
+
+/* I2V image-context MLP: Linear(img_feat, D) -> GELU -> Linear(D, D) -> GELU -> Linear(D, D). */
+typedef struct {
+  const void *w_1, *b_1;            /* [D, img_feat], [D] */
+  const void *w_2, *b_2;            /* [D, D], [D]        */
+  const void *w_3, *b_3;            /* [D, D], [D]        */
+} wan_image_mlp_weights;
+
+/* Non-block weights of the whole DiT. */
+typedef struct {
+  const void *w_p, *b_p;            /* patchify conv [D, in_ch, 1, 2, 2] (= [D, in_ch*4]), [D] */
+  wan_time_weights time;
+  const void *w_head, *b_head;      /* [out_ch*4, D], [out_ch*4]: head Linear, (c, ph, pw) order */
+} wan_stack_weights;
+
+/* Linear-layer epilogues of wan_linear_fwd (and of the block's GEMMs). */
+typedef enum {
+  WAN_EPI_STORE = 0,     /* out(act)  = A W^T + b                                  */
+  WAN_EPI_GELU = 1,      /* out(act)  = gelu_tanh(A W^T + b)                       */
+  WAN_EPI_RESIDUAL = 2,  /* out(fp32) += g * (A W^T + b), g = gate[b,n]+gate_bias[n] (1 if gate NULL) */
+  WAN_EPI_F32 = 3        /* out(fp32) = A W^T + b                                  */
+} wan_epilogue;
+
+/* Trace kinds (wan_trace_read). */
+typedef enum { WAN_KIND_NORM = 0, WAN_KIND_GEMM = 1, WAN_KIND_ATTN = 2, WAN_KIND_SMALL = 3,
+               WAN_KIND_COUNT = 4 } wan_kernel_kind;
+
+/* ---- library information ------------------------------------------------------- */
+
+/* Human-readable text of a wan_status. Never NULL; static storage. */
+const char* wan_status_string(int status);
+
+/* Device-memory workspace (bytes) that wan_dit_block_fwd / wan_dit_stack_fwd and the
+ * branch calls need for batch B, L video tokens, Lc text tokens and Li image tokens
+ * (Li = 0 for T2V). Returns 0 for an invalid config. */
+size_t wan_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int Li);
+
+/* Sync `stream`, then report and clear the device flag set by a bounded wait that ran
+ * out: WAN_OK, WAN_ERR_TIMEOUT, or WAN_ERR_CUDA if the sync itself failed. */
+int wan_device_status(void* stream);
+
+/* ---- the hot path -------------------------------------------------------------- */
+
+/* Patchify [Wan 2.1 page, "Diffusion Transformer": 3D conv, kernel = stride = (1,2,2)].
+ * latent [B, in_ch, F, H, W] act; x_out [B, L, D] fp32 with L = F*(H/2)*(W/2), tokens
+ * ordered (f, i, j). Workspace: B*L*in_ch*4 act elements (the gathered patches). */
+int wan_patchify(const wan_dit_config* cfg, const void* latent, int B, int F, int H, int W,
+                 const void* w_p, const void* b_p, float* x_out,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* Shared timestep MLP [Wan 2.1 page, "Diffusion Transformer"]: t [B] fp32 (0..1000
+ * scale) -> e_out [B, 6, D] fp32 = Linear(D,6D)(SiLU(Linear(256,D)(sinusoid(t)))).
+ * The sinusoid is [cos(t f_i) | sin(t f_i)], f_i = 10000^(-i/(freq_dim/2)). */
+int wan_time_mlp(const wan_dit_config* cfg, const float* t, int B, const wan_time_weights* w,
+                 float* e_out, void* stream);
+
+/* LayerNorm (eps, no affine) + AdaLN modulation [Wan 2.1 page, "Diffusion Transformer":
+ * six modulation vectors]. x [B, L, D] fp32 -> h_out [B, L, D] act with
+ * h = LN(x) * (1 + scale) + shift, where for chunk c in {0, 1}
+ * shift = e[b, 3c] + mod_bias[3c], scale = e[b, 3c+1] + mod_bias[3c+1]
+ * (chunk 0: self-attention input, chunk 1: FFN input). chunk = -1 gives plain LN and
+ * ignores e and mod_bias. mod_bias may be NULL (zero). */
+int wan_adaln_modulate(const wan_dit_config* cfg, const float* x, int B, int L,
+                       const float* e, const float* mod_bias, int chunk, void* h_out, void* stream);
+
+/* Self-attention branch with gated residual: x_inout[B, L, D] fp32 +=
+ * gate_msa * (Attn(h Wq, h Wk, h Wv) Wo^T + bo), gate_msa = e[b,2] + w->mod_bias[2].
+ * h [B, L, D] act is the modulated LN output. Attention is full (non-causal) over the
+ * L tokens of each sample, per head, scale 1/sqrt(head_dim). */
+int wan_self_attn_fwd(const wan_dit_config* cfg, const void* h, const wan_block_weights* w,
+                      const float* e, float* x_inout, int B, int L,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Cross-attention branch, plain residual [Wan 2.1 page, "Diffusion Transformer" and
+ * "I2V 架构扩展"]: x_inout += (Attn(q, Kt, Vt) [+ Attn(q, Ki, Vi)]) Wco^T + bco with
+ * q = h Wcq^T + bcq, [Kt|Vt] = ctx Wckv^T + bckv, [Ki|Vi] = img_ctx Wckv_img^T + b.
+ * h [B, L, D] act (plain LN of x); ctx [B, Lc, D] act; img_ctx [B, Li, D] act or NULL
+ * (Li = 0). */
+int wan_cross_attn_fwd(const wan_dit_config* cfg, const void* h, const void* ctx, int Lc,
+                       const void* img_ctx, int Li, const wan_block_weights* w,
+                       float* x_inout, int B, int L, void* workspace, size_t ws_bytes, void* stream);
+
+/* FFN branch with gated residual: x_inout += gate_ffn * (gelu_tanh(h W1^T + b1) W2^T + b2),
+ * gate_ffn = e[b,5] + w->mod_bias[5]. h [B, L, D] act. */
+int wan_ffn_fwd(const wan_dit_config* cfg, const void* h, const wan_block_weights* w,
+                const float* e, float* x_inout, int B, int L,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/* One DiT block, in place on the residual stream x_inout [B, L, D] fp32:
+ * self-attention (modulated LN, gated), cross-attention (plain LN, ungated), FFN
+ * (modulated LN, gated). e [B, 6, D] fp32 is the shared timestep-MLP output; the
+ * block adds w->mod_bias. ctx [B, Lc, D] act; img_ctx [B, Li, D] act or NULL. */
+int wan_dit_block_fwd(const wan_dit_config* cfg, float* x_inout, const float* e,
+                      const void* ctx, int Lc, const void* img_ctx, int Li,
+                      const wan_block_weights* w, int B, int L,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* The whole DiT: patchify -> shared timestep MLP -> n_blocks blocks (blocks is a HOST
+ * array of n_blocks weight tables) -> head (plain LN, Linear(D, out_ch*4)) ->
+ * unpatchify. latent [B, in_ch, F, H, W] act, t [B] fp32, ctx [B, Lc, D] act,
+ * img_ctx [B, Li, D] act or NULL; v_out [B, out_ch, F, H, W] fp32 (the predicted
+ * velocity). Workspace: wan_workspace_bytes(...) of this L. */
+int wan_dit_stack_fwd(const wan_dit_config* cfg, int n_blocks, const void* latent,
+                      int B, int F, int H, int W, const float* t,
+                      const wan_stack_weights* sw, const wan_block_weights* blocks,
+                      const void* ctx, int Lc, const void* img_ctx, int Li,
+                      float* v_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Head and unpatchify [Wan 2.1 page, "Diffusion Transformer"]: x [B, L, D] fp32 ->
+ * plain LN -> Linear(D, out_ch*4) -> v_out [B, out_ch, F, H, W] fp32, where output
+ * column c*4 + ph*2 + pw of token (f, i, j) lands at v_out[b, c, f, 2i+ph, 2j+pw].
+ * Workspace: B*L*D act elements. */
+int wan_head_fwd(const wan_dit_config* cfg, const float* x, int B, int F, int H, int W,
+                 const void* w_head, const void* b_head, float* v_out,
+                 void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- I2V and flow-matching pieces --------------------------------------------- */
+
+/* I2V input fusion [Wan 2.1 page, "I2V 架构扩展"]: out [B, 36, F, H, W] act =
+ * concat(noise [B,16,F,H,W], cond [B,16,F,H,W], mask [B,4,F,H,W]) where the mask is
+ * built from frame_keep [B, 1+4(F-1)] uint8 (1 = keep, 0 = generate): the first
+ * frame's value is repeated 4 times, the 4F values are grouped per latent frame and
+ * put on 4 channels, broadcast over H x W. */
+int wan_i2v_input(const wan_dit_config* cfg, const void* noise, const void* cond,
+                  const uint8_t* frame_keep, int B, int F, int H, int W, void* out, void* stream);
+
+/* I2V image-context MLP: feat [B, Li, img_feat] act -> img_ctx_out [B, Li, D] act.
+ * Workspace: 2 * B * Li * D act elements. */
+int wan_image_context_fwd(const wan_dit_config* cfg, const void* feat, int B, int Li,
+                          const wan_image_mlp_weights* w, void* img_ctx_out,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/* Rectified-flow interpolation [Wan 2.1 page, "训练方法"]: xt_out[b] = u[b] x1[b] +
+ * (1 - u[b]) x0[b] (act, n elements per sample), and t_out[b] = 1000 u[b] (fp32). */
+int wan_flow_matching_input(const wan_dit_config* cfg, const void* x1, const void* x0,
+                            const float* u, int B, int64_t n, void* xt_out, float* t_out,
+                            void* stream);
+
+/* Mean squared error per sample between the prediction v [B, n] fp32 and the
+ * velocity target x1 - x0 (act): loss_out [B] fp32. */
+int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void* x1,
+                           const void* x0, int B, int64_t n, float* loss_out, void* stream);
+
+/* ---- single-kernel entry points (used by the branch calls; exposed for tests) --- */
+
+/* Multi-head attention softmax(q k^T / sqrt(d)) v, non-causal. q [B, Lq, *], k and v
+ * [B, Lk, *], o [B, Lq, *] act; head h of each operand occupies columns
+ * [col0 + h*d, col0 + (h+1)*d) of rows with the given row strides (elements). */
+int wan_attention_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0,
+                      const void* k, int64_t k_row_stride, int k_col0,
+                      const void* v, int64_t v_row_stride, int v_col0,
+                      void* o, int64_t o_row_stride, int o_col0,
+                      int B, int heads, int Lq, int Lk, int head_dim, void* stream);
+
+/* y = A W^T + b with an epilogue. A [M, K] act (row stride K), W [N, K] act, bias [N]
+ * act or NULL. out: act [M, N] for STORE/GELU, fp32 [M, N] for F32/RESIDUAL. For
+ * RESIDUAL, gate (fp32) is indexed gate[(m / rows_per_batch) * gate_batch_stride + n]
+ * and gate_bias [N] fp32 is added (either may be NULL). */
+int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, const void* bias,
+                   void* out, int M, int N, int K, int epilogue,
+                   const float* gate, const float* gate_bias, int64_t gate_batch_stride,
+                   int rows_per_batch, void* stream);
+
+/* ---- tracing ------------------------------------------------------------------- */
+
+/* Total number of kernels this library has launched in this process. */
+int64_t wan_launch_count(void);
+
+/* Turn per-launch CUDA-event timing on (1) or off (0). While on, each launch is
+ * bracketed by events on its stream (a fixed pool of 16384 pairs per process). */
+int wan_trace_enable(int on);
+
+/* Drop all recorded launch timings. */
+int wan_trace_reset(void);
+
+/* Synchronise on the recorded events and return the total device time (ms) and the
+ * number of timed launches of one wan_kernel_kind since the last reset. */
+int wan_trace_read(int kind, double* total_ms, int64_t* launches);
+
+/* Per-launch records since the last reset, in launch order (host arrays of `cap`
+ * entries): kind, device time (ms) and algorithmic work - FLOPs (2 per multiply-add)
+ * for GEMM and attention launches, bytes read + written for the others. Returns the
+ * number of records written (<= cap) or a negative wan_status. */
+int wan_trace_launches(int cap, int* kinds, double* ms, double* work);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WAN_H */

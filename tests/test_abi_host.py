@@ -1,0 +1,113 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports every
+function include/wan.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wan.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(wan_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def wan():
+    from video_diffusion_transformer_wan_b200 import build
+    build.build()
+    import video_diffusion_transformer_wan_b200 as w
+    return w
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for required in ["wan_patchify", "wan_adaln_modulate", "wan_self_attn_fwd", "wan_cross_attn_fwd", "wan_ffn_fwd",
+                     "wan_dit_block_fwd", "wan_dit_stack_fwd", "wan_workspace_bytes", "wan_status_string"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(wan):
+    lib = ctypes.CDLL(wan.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(wan):
+    for code in range(0, -9, -1):
+        assert wan.status_string(code) and wan.status_string(code) != "unknown status"
+    assert wan.status_string(-100) == "unknown status"
+
+
+def _cfg(wan, **kw):
+    d = dict(dim=1536, heads=12, ffn=8960, dtype="bf16")
+    d.update(kw)
+    return wan.make_config(**d)
+
+
+def test_workspace_bytes_layout(wan):
+    cfg = _cfg(wan)
+    B, L, Lc = 1, 32760, 512
+    n = wan.workspace_bytes(cfg, B, L, Lc)
+    D, F = 1536, 8960
+    # h + max(5LD + 2LcD, LF) act elements + fp32 x + fp32 e, each region 256-aligned
+    lower = 2 * (B * L * D + max(5 * L * D + 2 * Lc * D, L * F)) + 4 * (B * L * D + 6 * D)
+    assert lower <= n <= lower + 4 * 256
+    assert wan.workspace_bytes(cfg, 2, L, Lc) > n
+    assert wan.workspace_bytes(_cfg(wan, heads=7), 1, 10, 10) == 0       # D != heads * head_dim
+
+
+def test_validation_rejects_before_launch(wan):
+    """Bad arguments return negative statuses without touching the GPU (pointers are
+    never dereferenced on the host, and no launch happens on a validation error)."""
+    L = wan.lib
+    launches = wan.launch_count()
+    cfg = _cfg(wan)
+    fake = 1 << 20                      # 16-byte aligned fake device address
+    bw = wan.BlockWeights(*([fake] * 17))
+    # NULL x
+    st = L.wan_dit_block_fwd(ctypes.byref(cfg), None, fake, fake, 512, None, 0, ctypes.byref(bw), 1, 32, fake,
+                             1 << 40, None)
+    assert st == -1
+    # misaligned x
+    st = L.wan_dit_block_fwd(ctypes.byref(cfg), fake + 4, fake, fake, 512, None, 0, ctypes.byref(bw), 1, 32, fake,
+                             1 << 40, None)
+    assert st == -4
+    # workspace too small
+    st = L.wan_dit_block_fwd(ctypes.byref(cfg), fake, fake, fake, 512, None, 0, ctypes.byref(bw), 1, 32, fake, 16, None)
+    assert st == -5
+    # empty text context
+    st = L.wan_dit_block_fwd(ctypes.byref(cfg), fake, fake, fake, 0, None, 0, ctypes.byref(bw), 1, 32, fake,
+                             1 << 40, None)
+    assert st == -2
+    # unknown dtype
+    bad = _cfg(wan)
+    bad.dtype = 7
+    assert L.wan_dit_block_fwd(ctypes.byref(bad), fake, fake, fake, 512, None, 0, ctypes.byref(bw), 1, 32, fake,
+                               1 << 40, None) == -3
+    # bf16 with head_dim 64 is not implemented by the tensor-core attention
+    c64 = _cfg(wan, dim=128, heads=2, ffn=256)
+    assert L.wan_dit_block_fwd(ctypes.byref(c64), fake, fake, fake, 16, None, 0, ctypes.byref(bw), 1, 32, fake,
+                               1 << 40, None) == -8
+    # odd latent width for patchify
+    assert L.wan_patchify(ctypes.byref(cfg), fake, 1, 2, 8, 7, fake, fake, fake, fake, 1 << 30, None) == -2
+    # I2V block without the image K/V weight
+    bw2 = wan.BlockWeights(*([fake] * 17))
+    bw2.w_ckv_img = None
+    assert L.wan_dit_block_fwd(ctypes.byref(cfg), fake, fake, fake, 512, fake, 257, ctypes.byref(bw2), 1, 32, fake,
+                               1 << 40, None) == -1
+    # attention: heads must match the config
+    assert L.wan_attention_fwd(ctypes.byref(cfg), fake, 4608, 0, fake, 4608, 1536, fake, 4608, 3072, fake, 1536, 0,
+                               1, 11, 32, 32, 128, None) == -2
+    # linear: N must be a multiple of 8
+    assert L.wan_linear_fwd(ctypes.byref(cfg), fake, fake, None, fake, 32, 12, 64, 0, None, None, 0, 1, None) == -2
+    assert wan.launch_count() == launches
+
+
+def test_trace_read_without_events(wan):
+    assert wan.trace_read(wan.KIND_ATTN) == (0.0, 0)

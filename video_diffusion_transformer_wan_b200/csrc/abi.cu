@@ -1,0 +1,690 @@
+// The C ABI (include/wan.h): argument validation, workspace layout, and the order of
+// kernel launches for the Wan 2.1 DiT block and stack ("Wan: Open and Advanced
+// Large-Scale Video Generative Models", section "Diffusion Transformer"). The host only
+// enqueues work on the caller's stream; nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace wan {
+
+// ------------------------------------------------------------------ device error flag
+__device__ int g_wan_error_flag;
+
+int* device_error_flag() {
+  static int* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wan_error_flag) == cudaSuccess) addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+// ------------------------------------------------------------------ trace
+namespace {
+constexpr int kTracePairs = 16384;
+struct Trace {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> start, stop;
+  std::vector<int> kind;
+  std::vector<double> work;
+  int used = 0;
+};
+Trace& trace() {
+  static Trace t;
+  return t;
+}
+std::atomic<int64_t> g_launches{0};
+thread_local int tl_slot = -1;
+}  // namespace
+
+void trace_launch_begin(int kind, cudaStream_t s, double work) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  Trace& t = trace();
+  tl_slot = -1;
+  std::lock_guard<std::mutex> lk(t.mu);
+  if (!t.on || t.used >= static_cast<int>(t.start.size())) return;
+  tl_slot = t.used++;
+  t.kind[tl_slot] = kind;
+  t.work[tl_slot] = work;
+  cudaEventRecord(t.start[tl_slot], s);
+}
+
+void trace_launch_end(int kind, cudaStream_t s) {
+  (void)kind;
+  if (tl_slot < 0) return;
+  Trace& t = trace();
+  std::lock_guard<std::mutex> lk(t.mu);
+  cudaEventRecord(t.stop[tl_slot], s);
+  tl_slot = -1;
+}
+
+// ------------------------------------------------------------------ tensor maps
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                    const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ validation helpers
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define WAN_REQUIRE(cond, code) \
+  do {                          \
+    if (!(cond)) return (code); \
+  } while (0)
+#define WAN_TRY(expr)               \
+  do {                              \
+    int _st = (expr);               \
+    if (_st != WAN_OK) return _st;  \
+  } while (0)
+
+int check_ptr(const void* p) {
+  if (!p) return WAN_ERR_NULL;
+  if (!aligned16(p)) return WAN_ERR_ALIGN;
+  return WAN_OK;
+}
+int check_opt_ptr(const void* p) { return p ? check_ptr(p) : WAN_OK; }
+
+// `attention`: the call runs attention, which fixes head_dim (128 on the bf16 tensor-core
+// path, <= 128 on the fp32 path).
+int check_cfg(const wan_dit_config* c, bool attention = false) {
+  WAN_REQUIRE(c, WAN_ERR_NULL);
+  WAN_REQUIRE(c->dtype == WAN_F32 || c->dtype == WAN_BF16, WAN_ERR_DTYPE);
+  WAN_REQUIRE(c->heads > 0 && c->head_dim > 0 && c->dim == c->heads * c->head_dim, WAN_ERR_SHAPE);
+  WAN_REQUIRE(c->dim % 64 == 0 && c->ffn_dim > 0 && c->ffn_dim % 64 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(c->in_ch > 0 && c->in_ch % 2 == 0 && c->out_ch > 0 && c->out_ch % 2 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(c->freq_dim > 0 && c->freq_dim % 2 == 0 && c->freq_dim <= 4096, WAN_ERR_SHAPE);
+  WAN_REQUIRE(c->eps > 0.f, WAN_ERR_SHAPE);
+  if (!attention) return WAN_OK;
+  if (c->dtype == WAN_BF16) {
+    WAN_REQUIRE(c->head_dim == 128, WAN_ERR_UNSUPPORTED);
+  } else {
+    WAN_REQUIRE(c->head_dim <= 128 && c->head_dim % 4 == 0, WAN_ERR_SHAPE);
+  }
+  return WAN_OK;
+}
+
+int check_block_w(const wan_dit_config* c, const wan_block_weights* w, bool need_img) {
+  WAN_REQUIRE(w, WAN_ERR_NULL);
+  WAN_TRY(check_opt_ptr(w->mod_bias));
+  const void* req[] = {w->w_qkv, w->w_o, w->w_cq, w->w_ckv, w->w_co, w->w_1, w->w_2};
+  for (const void* p : req) WAN_TRY(check_ptr(p));
+  const void* opt[] = {w->b_qkv, w->b_o, w->b_cq, w->b_ckv, w->b_co, w->b_1, w->b_2, w->b_ckv_img};
+  for (const void* p : opt) WAN_TRY(check_opt_ptr(p));
+  if (need_img) WAN_TRY(check_ptr(w->w_ckv_img));
+  (void)c;
+  return WAN_OK;
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t h;        // [B, L, D] act
+  size_t big;      // region R, see below
+  size_t x;        // [B, L, D] fp32 (stack)
+  size_t e;        // [B, 6, D] fp32 (stack)
+  size_t total;
+  size_t big_elems;
+};
+
+// Region R (act elements), reused by the three branches:
+//   self-attention: qkv [B*L, 3D] at 0, attention output [B*L, D] at 3*B*L*D
+//   cross-attention: q [B*L, D] at 0, attention output [B*L, D or 2D] at 3*B*L*D,
+//                    text K|V [B*Lc, 2D] at 5*B*L*D, image K|V [B*Li, 2D] after it
+//   FFN: hidden [B*L, F] at 0; patchify gather / image MLP scratch also start at 0.
+Layout layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
+  const size_t es = dtype_size(c->dtype);
+  const size_t D = c->dim, F = c->ffn_dim;
+  const size_t BL = static_cast<size_t>(B) * L;
+  size_t big = 5 * BL * D + 2 * static_cast<size_t>(B) * (Lc + Li) * D;
+  big = big > BL * F ? big : BL * F;
+  const size_t patch = BL * c->in_ch * 4;
+  big = big > patch ? big : patch;
+  const size_t img = 2 * static_cast<size_t>(B) * Li * D;
+  big = big > img ? big : img;
+  Layout l;
+  l.h = 0;
+  l.big = align_up(BL * D * es);
+  l.big_elems = big;
+  l.x = l.big + align_up(big * es);
+  l.e = l.x + align_up(BL * D * 4);
+  l.total = l.e + align_up(static_cast<size_t>(B) * 6 * D * 4);
+  return l;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+inline uint8_t* at(void* base, size_t off) { return static_cast<uint8_t*>(base) + off; }
+
+int gemm(const wan_dit_config* c, const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N,
+         int K, int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+  if (c->dtype == WAN_BF16) return launch_gemm_tc(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  return launch_gemm_simt(static_cast<const float*>(A), lda, static_cast<const float*>(W),
+                          static_cast<const float*>(bias), out, M, N, K, w_k_period, epi, s);
+}
+
+int attention(const wan_dit_config* c, AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t ors, int oc,
+              int B, int Lq, int Lk, cudaStream_t s) {
+  if (c->dtype == WAN_BF16) return launch_attn_tc(q, k, v, o, ors, oc, B, c->heads, Lq, Lk, s);
+  return launch_attn_simt(q, k, v, o, ors, oc, B, c->heads, Lq, Lk, c->head_dim, s);
+}
+
+GemmEpi epi_store(int64_t ldo, int kind = WAN_EPI_STORE) {
+  GemmEpi e{};
+  e.kind = kind;
+  e.ldo = ldo;
+  e.rows_per_batch = 1;
+  return e;
+}
+GemmEpi epi_residual(int64_t ldo, const float* gate, const float* gate_bias, int64_t bstride, int L) {
+  GemmEpi e{};
+  e.kind = WAN_EPI_RESIDUAL;
+  e.ldo = ldo;
+  e.gate = gate;
+  e.gate_bias = gate_bias;
+  e.gate_bstride = bstride;
+  e.rows_per_batch = L;
+  return e;
+}
+
+int self_attn_impl(const wan_dit_config* c, const void* h, const wan_block_weights* w, const float* e, float* x, int B,
+                   int L, void* ws, const Layout& ly, cudaStream_t s) {
+  const int D = c->dim;
+  const size_t es = dtype_size(c->dtype);
+  const int M = B * L;
+  uint8_t* R = at(ws, ly.big);
+  void* qkv = R;
+  void* o = R + static_cast<size_t>(3) * M * D * es;
+  WAN_TRY(gemm(c, h, D, w->w_qkv, w->b_qkv, qkv, M, 3 * D, D, 0, epi_store(3 * D), s));
+  WAN_TRY(attention(c, {qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, L, L, s));
+  const float* gb = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
+  return gemm(c, o, D, w->w_o, w->b_o, x, M, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, L), s);
+}
+
+int cross_attn_impl(const wan_dit_config* c, const void* h, const void* ctx, int Lc, const void* img, int Li,
+                    const wan_block_weights* w, float* x, int B, int L, void* ws, const Layout& ly, cudaStream_t s) {
+  const int D = c->dim;
+  const size_t es = dtype_size(c->dtype);
+  const int M = B * L;
+  uint8_t* R = at(ws, ly.big);
+  void* q = R;
+  void* ocat = R + static_cast<size_t>(3) * M * D * es;
+  void* kvt = R + static_cast<size_t>(5) * M * D * es;
+  void* kvi = static_cast<uint8_t*>(kvt) + static_cast<size_t>(2) * B * Lc * D * es;
+  const bool with_img = img && Li > 0;
+  const int ow = with_img ? 2 * D : D;
+  WAN_TRY(gemm(c, h, D, w->w_cq, w->b_cq, q, M, D, D, 0, epi_store(D), s));
+  WAN_TRY(gemm(c, ctx, D, w->w_ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
+  WAN_TRY(attention(c, {q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, L, Lc, s));
+  if (with_img) {
+    WAN_TRY(gemm(c, img, D, w->w_ckv_img, w->b_ckv_img, kvi, B * Li, 2 * D, D, 0, epi_store(2 * D), s));
+    WAN_TRY(attention(c, {q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, L, Li, s));
+    // (o_text + o_image) Wco^T as one reduction over [o_text | o_image] with Wco reused.
+    return gemm(c, ocat, ow, w->w_co, w->b_co, x, M, D, 2 * D, D, epi_residual(D, nullptr, nullptr, 0, L), s);
+  }
+  return gemm(c, ocat, D, w->w_co, w->b_co, x, M, D, D, 0, epi_residual(D, nullptr, nullptr, 0, L), s);
+}
+
+int ffn_impl(const wan_dit_config* c, const void* h, const wan_block_weights* w, const float* e, float* x, int B, int L,
+             void* ws, const Layout& ly, cudaStream_t s) {
+  const int D = c->dim, F = c->ffn_dim;
+  const int M = B * L;
+  void* hid = at(ws, ly.big);
+  WAN_TRY(gemm(c, h, D, w->w_1, w->b_1, hid, M, F, D, 0, epi_store(F, WAN_EPI_GELU), s));
+  const float* gb = w->mod_bias ? w->mod_bias + 5 * D : nullptr;
+  return gemm(c, hid, F, w->w_2, w->b_2, x, M, D, F, 0, epi_residual(D, e + 5 * D, gb, 6 * D, L), s);
+}
+
+int block_impl(const wan_dit_config* c, float* x, const float* e, const void* ctx, int Lc, const void* img, int Li,
+               const wan_block_weights* w, int B, int L, void* ws, const Layout& ly, cudaStream_t s) {
+  void* h = at(ws, ly.h);
+  const int64_t rows = static_cast<int64_t>(B) * L;
+  WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 0, h, c->dtype, c->eps, s));
+  WAN_TRY(self_attn_impl(c, h, w, e, x, B, L, ws, ly, s));
+  WAN_TRY(launch_layernorm(x, rows, c->dim, L, nullptr, nullptr, -1, h, c->dtype, c->eps, s));
+  WAN_TRY(cross_attn_impl(c, h, ctx, Lc, img, Li, w, x, B, L, ws, ly, s));
+  WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 1, h, c->dtype, c->eps, s));
+  return ffn_impl(c, h, w, e, x, B, L, ws, ly, s);
+}
+
+// Plain LN of the residual stream, then Linear(D, out_ch*4) whose epilogue scatters each
+// token's (c, ph, pw) outputs into the unpatchified latent.
+int head_impl(const wan_dit_config* c, const float* x, int B, int F, int H, int W, const void* w_head,
+              const void* b_head, float* v_out, void* h, cudaStream_t s) {
+  const int L = F * (H / 2) * (W / 2);
+  WAN_TRY(launch_layernorm(x, static_cast<int64_t>(B) * L, c->dim, L, nullptr, nullptr, -1, h, c->dtype, c->eps, s));
+  GemmEpi ep{};
+  ep.kind = kEpiHeadScatter;
+  ep.rows_per_batch = L;
+  ep.sc_C = c->out_ch;
+  ep.sc_F = F;
+  ep.sc_H = H;
+  ep.sc_W = W;
+  return gemm(c, h, c->dim, w_head, b_head, v_out, B * L, c->out_ch * 4, c->dim, 0, ep, s);
+}
+
+int check_tokens(const wan_dit_config* c, int B, int L, int Lc, int Li) {
+  WAN_REQUIRE(B >= 0 && L >= 0 && Lc >= 0 && Li >= 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(static_cast<int64_t>(B) * L < (int64_t(1) << 31), WAN_ERR_SHAPE);
+  if (c->dtype == WAN_F32) WAN_REQUIRE(L <= 8192 && Lc <= 8192 && Li <= 8192, WAN_ERR_SHAPE);
+  return WAN_OK;
+}
+
+int check_ws(const wan_dit_config* c, void* ws, size_t ws_bytes, int B, int L, int Lc, int Li) {
+  WAN_TRY(check_ptr(ws));
+  WAN_REQUIRE(ws_bytes >= layout(c, B, L, Lc, Li).total, WAN_ERR_WORKSPACE);
+  return WAN_OK;
+}
+
+}  // namespace
+}  // namespace wan
+
+using namespace wan;
+
+extern "C" {
+
+const char* wan_status_string(int status) {
+  switch (status) {
+    case WAN_OK: return "ok";
+    case WAN_ERR_NULL: return "a required pointer is NULL";
+    case WAN_ERR_SHAPE: return "sizes inconsistent or outside the supported range";
+    case WAN_ERR_DTYPE: return "unknown dtype";
+    case WAN_ERR_ALIGN: return "a device pointer or stride is not 16-byte aligned";
+    case WAN_ERR_WORKSPACE: return "workspace smaller than wan_workspace_bytes()";
+    case WAN_ERR_CUDA: return "a CUDA launch or runtime call failed";
+    case WAN_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case WAN_ERR_UNSUPPORTED: return "request not implemented by this build";
+    default: return "unknown status";
+  }
+}
+
+size_t wan_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int Li) {
+  if (check_cfg(cfg) != WAN_OK || B < 0 || L < 0 || Lc < 0 || Li < 0) return 0;
+  return layout(cfg, B, L, Lc, Li).total;
+}
+
+int wan_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return WAN_ERR_CUDA;
+  int* flag = device_error_flag();
+  if (!flag) return WAN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WAN_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return WAN_ERR_TIMEOUT;
+  }
+  return WAN_OK;
+}
+
+int wan_patchify(const wan_dit_config* cfg, const void* latent, int B, int F, int H, int W, const void* w_p,
+                 const void* b_p, float* x_out, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(latent));
+  WAN_TRY(check_ptr(w_p));
+  WAN_TRY(check_opt_ptr(b_p));
+  WAN_TRY(check_ptr(x_out));
+  WAN_TRY(check_ptr(workspace));
+  WAN_REQUIRE(B >= 0 && F >= 0 && H >= 0 && W >= 0 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
+  const int L = F * (H / 2) * (W / 2);
+  const int K = cfg->in_ch * 4;
+  WAN_REQUIRE(ws_bytes >= static_cast<size_t>(B) * L * K * dtype_size(cfg->dtype), WAN_ERR_WORKSPACE);
+  cudaStream_t s = as_stream(stream);
+  WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, workspace, cfg->dtype, s));
+  return gemm(cfg, workspace, K, w_p, b_p, x_out, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s);
+}
+
+int wan_time_mlp(const wan_dit_config* cfg, const float* t, int B, const wan_time_weights* w, float* e_out,
+                 void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_REQUIRE(w, WAN_ERR_NULL);
+  WAN_TRY(check_ptr(t));
+  WAN_TRY(check_ptr(w->w_t1));
+  WAN_TRY(check_ptr(w->w_t2));
+  WAN_TRY(check_ptr(w->b_t1));
+  WAN_TRY(check_ptr(w->b_t2));
+  WAN_TRY(check_ptr(e_out));
+  WAN_REQUIRE(B >= 0, WAN_ERR_SHAPE);
+  return launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, w->w_t1, w->b_t1, w->w_t2, w->b_t2, e_out, cfg->dtype,
+                         as_stream(stream));
+}
+
+int wan_adaln_modulate(const wan_dit_config* cfg, const float* x, int B, int L, const float* e, const float* mod_bias,
+                       int chunk, void* h_out, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(x));
+  WAN_TRY(check_ptr(h_out));
+  WAN_REQUIRE(chunk >= -1 && chunk <= 1 && B >= 0 && L >= 0, WAN_ERR_SHAPE);
+  if (chunk >= 0) WAN_TRY(check_ptr(e));
+  WAN_TRY(check_opt_ptr(mod_bias));
+  return launch_layernorm(x, static_cast<int64_t>(B) * L, cfg->dim, L, e, mod_bias, chunk, h_out, cfg->dtype,
+                          cfg->eps, as_stream(stream));
+}
+
+int wan_self_attn_fwd(const wan_dit_config* cfg, const void* h, const wan_block_weights* w, const float* e,
+                      float* x_inout, int B, int L, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  WAN_TRY(check_block_w(cfg, w, false));
+  WAN_TRY(check_ptr(h));
+  WAN_TRY(check_ptr(e));
+  WAN_TRY(check_ptr(x_inout));
+  WAN_TRY(check_tokens(cfg, B, L, 0, 0));
+  WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, 0, 0));
+  return self_attn_impl(cfg, h, w, e, x_inout, B, L, workspace, layout(cfg, B, L, 0, 0), as_stream(stream));
+}
+
+int wan_cross_attn_fwd(const wan_dit_config* cfg, const void* h, const void* ctx, int Lc, const void* img_ctx, int Li,
+                       const wan_block_weights* w, float* x_inout, int B, int L, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  const bool with_img = img_ctx && Li > 0;
+  WAN_TRY(check_block_w(cfg, w, with_img));
+  WAN_TRY(check_ptr(h));
+  WAN_TRY(check_ptr(ctx));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_TRY(check_ptr(x_inout));
+  WAN_REQUIRE(Lc > 0, WAN_ERR_SHAPE);
+  WAN_TRY(check_tokens(cfg, B, L, Lc, Li));
+  WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, Lc, with_img ? Li : 0));
+  return cross_attn_impl(cfg, h, ctx, Lc, img_ctx, with_img ? Li : 0, w, x_inout, B, L, workspace,
+                         layout(cfg, B, L, Lc, with_img ? Li : 0), as_stream(stream));
+}
+
+int wan_ffn_fwd(const wan_dit_config* cfg, const void* h, const wan_block_weights* w, const float* e, float* x_inout,
+                int B, int L, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_block_w(cfg, w, false));
+  WAN_TRY(check_ptr(h));
+  WAN_TRY(check_ptr(e));
+  WAN_TRY(check_ptr(x_inout));
+  WAN_TRY(check_tokens(cfg, B, L, 0, 0));
+  WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, 0, 0));
+  return ffn_impl(cfg, h, w, e, x_inout, B, L, workspace, layout(cfg, B, L, 0, 0), as_stream(stream));
+}
+
+int wan_dit_block_fwd(const wan_dit_config* cfg, float* x_inout, const float* e, const void* ctx, int Lc,
+                      const void* img_ctx, int Li, const wan_block_weights* w, int B, int L, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  const bool with_img = img_ctx && Li > 0;
+  WAN_TRY(check_block_w(cfg, w, with_img));
+  WAN_TRY(check_ptr(x_inout));
+  WAN_TRY(check_ptr(e));
+  WAN_TRY(check_ptr(ctx));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_REQUIRE(Lc > 0, WAN_ERR_SHAPE);
+  WAN_TRY(check_tokens(cfg, B, L, Lc, Li));
+  const int li = with_img ? Li : 0;
+  WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, Lc, li));
+  return block_impl(cfg, x_inout, e, ctx, Lc, img_ctx, li, w, B, L, workspace, layout(cfg, B, L, Lc, li),
+                    as_stream(stream));
+}
+
+int wan_dit_stack_fwd(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H, int W,
+                      const float* t, const wan_stack_weights* sw, const wan_block_weights* blocks, const void* ctx,
+                      int Lc, const void* img_ctx, int Li, float* v_out, void* workspace, size_t ws_bytes,
+                      void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  WAN_REQUIRE(sw && (blocks || n_blocks == 0), WAN_ERR_NULL);
+  WAN_REQUIRE(n_blocks >= 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(B >= 0 && F >= 0 && H % 2 == 0 && W % 2 == 0 && H >= 0 && W >= 0, WAN_ERR_SHAPE);
+  const bool with_img = img_ctx && Li > 0;
+  for (int i = 0; i < n_blocks; ++i) WAN_TRY(check_block_w(cfg, &blocks[i], with_img));
+  WAN_TRY(check_ptr(latent));
+  WAN_TRY(check_ptr(t));
+  WAN_TRY(check_ptr(ctx));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_TRY(check_ptr(v_out));
+  WAN_TRY(check_ptr(sw->w_p));
+  WAN_TRY(check_opt_ptr(sw->b_p));
+  WAN_TRY(check_ptr(sw->w_head));
+  WAN_TRY(check_opt_ptr(sw->b_head));
+  WAN_TRY(check_ptr(sw->time.w_t1));
+  WAN_TRY(check_ptr(sw->time.w_t2));
+  WAN_TRY(check_ptr(sw->time.b_t1));
+  WAN_TRY(check_ptr(sw->time.b_t2));
+  WAN_REQUIRE(Lc > 0, WAN_ERR_SHAPE);
+  const int L = F * (H / 2) * (W / 2);
+  const int li = with_img ? Li : 0;
+  WAN_TRY(check_tokens(cfg, B, L, Lc, li));
+  WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, Lc, li));
+  const Layout ly = layout(cfg, B, L, Lc, li);
+  cudaStream_t s = as_stream(stream);
+  float* x = reinterpret_cast<float*>(at(workspace, ly.x));
+  float* e = reinterpret_cast<float*>(at(workspace, ly.e));
+  void* patches = at(workspace, ly.big);
+  const int K = cfg->in_ch * 4;
+  WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, patches, cfg->dtype, s));
+  WAN_TRY(gemm(cfg, patches, K, sw->w_p, sw->b_p, x, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s));
+  WAN_TRY(launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, sw->time.w_t1, sw->time.b_t1, sw->time.w_t2, sw->time.b_t2,
+                          e, cfg->dtype, s));
+  for (int i = 0; i < n_blocks; ++i)
+    WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s));
+  return head_impl(cfg, x, B, F, H, W, sw->w_head, sw->b_head, v_out, at(workspace, ly.h), s);
+}
+
+int wan_head_fwd(const wan_dit_config* cfg, const float* x, int B, int F, int H, int W, const void* w_head,
+                 const void* b_head, float* v_out, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(x));
+  WAN_TRY(check_ptr(w_head));
+  WAN_TRY(check_opt_ptr(b_head));
+  WAN_TRY(check_ptr(v_out));
+  WAN_TRY(check_ptr(workspace));
+  WAN_REQUIRE(B >= 0 && F >= 0 && H >= 0 && W >= 0 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
+  const int L = F * (H / 2) * (W / 2);
+  WAN_REQUIRE(ws_bytes >= static_cast<size_t>(B) * L * cfg->dim * dtype_size(cfg->dtype), WAN_ERR_WORKSPACE);
+  return head_impl(cfg, x, B, F, H, W, w_head, b_head, v_out, workspace, as_stream(stream));
+}
+
+int wan_i2v_input(const wan_dit_config* cfg, const void* noise, const void* cond, const uint8_t* frame_keep, int B,
+                  int F, int H, int W, void* out, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(noise));
+  WAN_TRY(check_ptr(cond));
+  WAN_REQUIRE(frame_keep, WAN_ERR_NULL);
+  WAN_TRY(check_ptr(out));
+  WAN_REQUIRE(B >= 0 && F >= 1 && H >= 0 && W >= 0, WAN_ERR_SHAPE);
+  return launch_i2v_input(noise, cond, frame_keep, B, F, H, W, out, cfg->dtype, as_stream(stream));
+}
+
+int wan_image_context_fwd(const wan_dit_config* cfg, const void* feat, int B, int Li, const wan_image_mlp_weights* w,
+                          void* img_ctx_out, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_REQUIRE(w, WAN_ERR_NULL);
+  WAN_TRY(check_ptr(feat));
+  WAN_TRY(check_ptr(w->w_1));
+  WAN_TRY(check_ptr(w->w_2));
+  WAN_TRY(check_ptr(w->w_3));
+  WAN_TRY(check_opt_ptr(w->b_1));
+  WAN_TRY(check_opt_ptr(w->b_2));
+  WAN_TRY(check_opt_ptr(w->b_3));
+  WAN_TRY(check_ptr(img_ctx_out));
+  WAN_TRY(check_ptr(workspace));
+  WAN_REQUIRE(B >= 0 && Li >= 0 && cfg->img_feat_dim > 0 && cfg->img_feat_dim % 8 == 0, WAN_ERR_SHAPE);
+  const int D = cfg->dim;
+  const size_t es = dtype_size(cfg->dtype);
+  const size_t half = static_cast<size_t>(B) * Li * D * es;
+  WAN_REQUIRE(ws_bytes >= 2 * half, WAN_ERR_WORKSPACE);
+  cudaStream_t s = as_stream(stream);
+  void* t1 = workspace;
+  void* t2 = static_cast<uint8_t*>(workspace) + half;
+  const int M = B * Li;
+  WAN_TRY(gemm(cfg, feat, cfg->img_feat_dim, w->w_1, w->b_1, t1, M, D, cfg->img_feat_dim, 0,
+               epi_store(D, WAN_EPI_GELU), s));
+  WAN_TRY(gemm(cfg, t1, D, w->w_2, w->b_2, t2, M, D, D, 0, epi_store(D, WAN_EPI_GELU), s));
+  return gemm(cfg, t2, D, w->w_3, w->b_3, img_ctx_out, M, D, D, 0, epi_store(D), s);
+}
+
+int wan_flow_matching_input(const wan_dit_config* cfg, const void* x1, const void* x0, const float* u, int B, int64_t n,
+                            void* xt_out, float* t_out, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(x1));
+  WAN_TRY(check_ptr(x0));
+  WAN_TRY(check_ptr(u));
+  WAN_TRY(check_ptr(xt_out));
+  WAN_TRY(check_opt_ptr(t_out));
+  WAN_REQUIRE(B >= 0 && n >= 0, WAN_ERR_SHAPE);
+  return launch_flow_input(x1, x0, u, B, n, xt_out, t_out, cfg->dtype, as_stream(stream));
+}
+
+int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void* x1, const void* x0, int B, int64_t n,
+                           float* loss_out, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(v));
+  WAN_TRY(check_ptr(x1));
+  WAN_TRY(check_ptr(x0));
+  WAN_TRY(check_ptr(loss_out));
+  WAN_REQUIRE(B >= 0 && n > 0, WAN_ERR_SHAPE);
+  return launch_flow_loss(v, x1, x0, B, n, loss_out, cfg->dtype, as_stream(stream));
+}
+
+int wan_attention_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0, const void* k,
+                      int64_t k_row_stride, int k_col0, const void* v, int64_t v_row_stride, int v_col0, void* o,
+                      int64_t o_row_stride, int o_col0, int B, int heads, int Lq, int Lk, int head_dim,
+                      void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  WAN_TRY(check_ptr(q));
+  WAN_TRY(check_ptr(k));
+  WAN_TRY(check_ptr(v));
+  WAN_TRY(check_ptr(o));
+  WAN_REQUIRE(heads == cfg->heads && head_dim == cfg->head_dim, WAN_ERR_SHAPE);
+  WAN_REQUIRE(B >= 0 && Lq >= 0 && Lk > 0, WAN_ERR_SHAPE);
+  const int64_t need = static_cast<int64_t>(heads) * head_dim;
+  WAN_REQUIRE(q_col0 >= 0 && k_col0 >= 0 && v_col0 >= 0 && o_col0 >= 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(q_col0 + need <= q_row_stride && k_col0 + need <= k_row_stride && v_col0 + need <= v_row_stride &&
+                  o_col0 + need <= o_row_stride,
+              WAN_ERR_SHAPE);
+  if (cfg->dtype == WAN_F32) WAN_REQUIRE(Lk <= 8192, WAN_ERR_SHAPE);
+  return attention(cfg, {q, q_row_stride, q_col0}, {k, k_row_stride, k_col0}, {v, v_row_stride, v_col0}, o,
+                   o_row_stride, o_col0, B, Lq, Lk, as_stream(stream));
+}
+
+int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, const void* bias, void* out, int M, int N,
+                   int K, int epilogue, const float* gate, const float* gate_bias, int64_t gate_batch_stride,
+                   int rows_per_batch, void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(A));
+  WAN_TRY(check_ptr(W));
+  WAN_TRY(check_opt_ptr(bias));
+  WAN_TRY(check_ptr(out));
+  WAN_TRY(check_opt_ptr(gate));
+  WAN_TRY(check_opt_ptr(gate_bias));
+  WAN_REQUIRE(M >= 0 && N > 0 && K > 0 && N % 8 == 0 && K % 8 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(epilogue >= WAN_EPI_STORE && epilogue <= WAN_EPI_F32, WAN_ERR_SHAPE);
+  if (epilogue == WAN_EPI_RESIDUAL) {
+    WAN_REQUIRE(rows_per_batch > 0 && gate_batch_stride >= 0 && gate_batch_stride % 4 == 0, WAN_ERR_SHAPE);
+  }
+  GemmEpi ep = epilogue == WAN_EPI_RESIDUAL ? epi_residual(N, gate, gate_bias, gate_batch_stride, rows_per_batch)
+                                            : epi_store(N, epilogue);
+  return gemm(cfg, A, K, W, bias, out, M, N, K, 0, ep, as_stream(stream));
+}
+
+int64_t wan_launch_count(void) { return g_launches.load(); }
+
+int wan_trace_enable(int on) {
+  Trace& t = trace();
+  std::lock_guard<std::mutex> lk(t.mu);
+  if (on && t.start.empty()) {
+    t.start.resize(kTracePairs);
+    t.stop.resize(kTracePairs);
+    t.kind.assign(kTracePairs, -1);
+    t.work.assign(kTracePairs, 0.0);
+    for (int i = 0; i < kTracePairs; ++i) {
+      if (cudaEventCreate(&t.start[i]) != cudaSuccess || cudaEventCreate(&t.stop[i]) != cudaSuccess) {
+        t.start.resize(i);
+        t.stop.resize(i);
+        return WAN_ERR_CUDA;
+      }
+    }
+  }
+  t.on = on != 0;
+  return WAN_OK;
+}
+
+int wan_trace_reset(void) {
+  Trace& t = trace();
+  std::lock_guard<std::mutex> lk(t.mu);
+  t.used = 0;
+  return WAN_OK;
+}
+
+int wan_trace_read(int kind, double* total_ms, int64_t* launches) {
+  WAN_REQUIRE(total_ms && launches, WAN_ERR_NULL);
+  Trace& t = trace();
+  std::lock_guard<std::mutex> lk(t.mu);
+  double tot = 0.0;
+  int64_t n = 0;
+  for (int i = 0; i < t.used; ++i) {
+    if (t.kind[i] != kind) continue;
+    if (cudaEventSynchronize(t.stop[i]) != cudaSuccess) return WAN_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t.start[i], t.stop[i]) != cudaSuccess) return WAN_ERR_CUDA;
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
+  return WAN_OK;
+}
+
+int wan_trace_launches(int cap, int* kinds, double* ms, double* work) {
+  WAN_REQUIRE(cap >= 0 && (cap == 0 || (kinds && ms && work)), WAN_ERR_NULL);
+  Trace& t = trace();
+  std::lock_guard<std::mutex> lk(t.mu);
+  const int n = t.used < cap ? t.used : cap;
+  for (int i = 0; i < n; ++i) {
+    if (cudaEventSynchronize(t.stop[i]) != cudaSuccess) return WAN_ERR_CUDA;
+    float e = 0.f;
+    if (cudaEventElapsedTime(&e, t.start[i], t.stop[i]) != cudaSuccess) return WAN_ERR_CUDA;
+    kinds[i] = t.kind[i];
+    ms[i] = e;
+    work[i] = t.work[i];
+  }
+  return n;
+}
+
+}  // extern "C"

@@ -1,0 +1,362 @@
+// Kernel (c): persistent bf16 GEMM on the sm_100a tensor cores (tcgen05), computing
+// out = epilogue(A W^T + bias) for the DiT's Linear layers: the fused QKV projection,
+// the attention output projections with the gated residual, the FFN (GELU-tanh into
+// the hidden, gated residual out of it), the patchify projection (fp32 store) and the
+// head (scatter straight into the unpatchified latent).
+//
+// Tile 128 x BN x 64. One CTA per SM loops over output tiles:
+//   warp 0  : TMA producer, a ring of kStages (A, W) stages with 128-byte swizzle;
+//   warp 1  : one elected thread issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
+//             accumulator; two accumulators alternate so the epilogue of one tile
+//             overlaps the main loop of the next;
+//   warps 2-5: epilogue; warp w reads TMEM lanes 32*(w%4).. (rows of the tile) with
+//             tcgen05.ld, applies bias / activation / gate and writes global memory.
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace wan {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+};
+
+struct GemmParams {
+  int M, N, K;
+  int k_blocks;
+  int wk_period_blocks;  // > 0: W column block = k block mod this
+  int m_blocks, n_blocks;
+  const __nv_bfloat16* bias;
+  void* out;
+  GemmEpi epi;
+  int* err;
+};
+
+__device__ __forceinline__ float gelu_tanh_f(float v) {
+  const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
+  return 0.5f * v * (1.0f + tanh_approx(u));
+}
+
+// Apply the epilogue to 32 consecutive accumulator columns [n0, n0+32) of one row.
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int n0, const uint32_t (&r)[32]) {
+  if (row >= p.M || n0 >= p.N) return;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  const bool full = n0 + 32 <= p.N;
+  if (p.bias) {
+    if (full) {
+      const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint4 u = __ldg(bp + g);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float2 f = __bfloat1622float2(h[j]);
+          v[g * 8 + 2 * j] += f.x;
+          v[g * 8 + 2 * j + 1] += f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (n0 + i < p.N) v[i] += __bfloat162float(p.bias[n0 + i]);
+    }
+  }
+  const int kind = p.epi.kind;
+  if (kind == WAN_EPI_STORE || kind == WAN_EPI_GELU) {
+    if (kind == WAN_EPI_GELU) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_f(v[i]);
+    }
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (n0 + g * 8 < p.N) {
+        uint4 u;
+        u.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+        u.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+        u.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+        u.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+        reinterpret_cast<uint4*>(o)[g] = u;
+      }
+    }
+  } else if (kind == WAN_EPI_F32) {
+    float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      if (n0 + g * 4 < p.N)
+        reinterpret_cast<float4*>(o)[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+  } else if (kind == WAN_EPI_RESIDUAL) {
+    float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+    const float* gate = p.epi.gate ? p.epi.gate + static_cast<int64_t>(row / p.epi.rows_per_batch) * p.epi.gate_bstride + n0
+                                   : nullptr;
+    const float* gb = p.epi.gate_bias ? p.epi.gate_bias + n0 : nullptr;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (n0 + g * 4 < p.N) {
+        float4 x = reinterpret_cast<float4*>(o)[g];
+        float gg[4] = {1.f, 1.f, 1.f, 1.f};
+        if (gate) {
+          float4 t = __ldg(reinterpret_cast<const float4*>(gate) + g);
+          gg[0] = t.x; gg[1] = t.y; gg[2] = t.z; gg[3] = t.w;
+          if (gb) {
+            float4 u = __ldg(reinterpret_cast<const float4*>(gb) + g);
+            gg[0] += u.x; gg[1] += u.y; gg[2] += u.z; gg[3] += u.w;
+          }
+        }
+        x.x += gg[0] * v[4 * g];
+        x.y += gg[1] * v[4 * g + 1];
+        x.z += gg[2] * v[4 * g + 2];
+        x.w += gg[3] * v[4 * g + 3];
+        reinterpret_cast<float4*>(o)[g] = x;
+      }
+    }
+  } else {  // kEpiHeadScatter: n = c*4 + ph*2 + pw, row = b*L + (f*Hh + i)*Wh + j
+    const int L = p.epi.rows_per_batch;
+    const int b = row / L, l = row % L;
+    const int Hh = p.epi.sc_H / 2, Wh = p.epi.sc_W / 2;
+    const int f = l / (Hh * Wh), ii = (l / Wh) % Hh, jj = l % Wh;
+    float* o = static_cast<float*>(p.out);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int n = n0 + i;
+      if (n < p.N) {
+        const int c = n >> 2, ph = (n >> 1) & 1, pw = n & 1;
+        const int64_t idx = ((static_cast<int64_t>(b) * p.epi.sc_C + c) * p.epi.sc_F + f) * p.epi.sc_H * p.epi.sc_W +
+                            static_cast<int64_t>(2 * ii + ph) * p.epi.sc_W + (2 * jj + pw);
+        o[idx] = v[i];
+      }
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                        const GemmParams p) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::kStages * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::kStages * C::kBBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int num_tiles = p.m_blocks * p.n_blocks;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int m0 = (tile / p.n_blocks) * kBM;
+        const int n0 = (tile % p.n_blocks) * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          const int kbw = p.wk_period_blocks > 0 ? kb % p.wk_period_blocks : kb;
+          tma_load_2d(sA + stage * C::kABytes, &mapA, &full[stage], kb * kBK, m0);
+          tma_load_2d(sB + stage * C::kBBytes, &mapB, &full[stage], kbw * kBK, n0);
+          ++issued;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every issued tile load has landed before the CTA exits.
+      for (int s = 0; s < C::kStages; ++s) {
+        const int64_t n_s = issued / C::kStages + (s < issued % C::kStages ? 1 : 0);
+        if (n_s > 0) mbar_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1), p.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + k * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(&tfull[acc]);
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      tc_commit(drain);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    const int quarter = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, p.err)) break;
+      tc_fence_after();
+      const int m0 = (tile / p.n_blocks) * kBM;
+      const int n0 = (tile % p.n_blocks) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+        epilogue_chunk(p, row, n0 + c * 32, r);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    counts[dev] = n > 0 ? n : 148;
+  }
+  return counts[dev];
+}
+
+template <int BN>
+int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
+              int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  CUtensorMap mapA, mapB;
+  const uint64_t dimsA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * 2};
+  const uint32_t boxA[2] = {kBK, kBM};
+  const int kw = w_k_period > 0 ? w_k_period : K;
+  const uint64_t dimsB[2] = {static_cast<uint64_t>(kw), static_cast<uint64_t>(N)};
+  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * 2};
+  const uint32_t boxB[2] = {kBK, BN};
+  if (!make_tmap_bf16(&mapA, A, 2, dimsA, strA, boxA) || !make_tmap_bf16(&mapB, W, 2, dimsB, strB, boxB))
+    return WAN_ERR_CUDA;
+  GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.k_blocks = (K + kBK - 1) / kBK;
+  p.wk_period_blocks = w_k_period > 0 ? w_k_period / kBK : 0;
+  p.m_blocks = (M + kBM - 1) / kBM;
+  p.n_blocks = (N + BN - 1) / BN;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.out = out;
+  p.epi = epi;
+  p.err = device_error_flag();
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev & 63], [] {
+    cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(C::kSmemBytes));
+  });
+  const int tiles = p.m_blocks * p.n_blocks;
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  gemm_bf16_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
+                   int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+  if (M == 0 || N == 0) return WAN_OK;
+  if (K % 8 != 0 || lda % 8 != 0 || N % 8 != 0) return WAN_ERR_SHAPE;
+  if (w_k_period > 0 && (w_k_period % kBK != 0 || K % w_k_period != 0)) return WAN_ERR_SHAPE;
+  trace_launch_begin(WAN_KIND_GEMM, s, 2.0 * M * N * K);
+  int st;
+  if (N <= 64)
+    st = launch_bn<64>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  else if (N <= 128)
+    st = launch_bn<128>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  else
+    st = launch_bn<256>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  trace_launch_end(WAN_KIND_GEMM, s);
+  return st;
+}
+
+}  // namespace wan

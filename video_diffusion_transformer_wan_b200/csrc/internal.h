@@ -1,0 +1,85 @@
+// Host-side declarations shared by the library's translation units: kernel launchers,
+// tensor-map creation, the device error flag and the launch trace.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/wan.h"
+
+namespace wan {
+
+// ---------------------------------------------------------------- launch bookkeeping
+// Every kernel launch goes through trace_launch_begin/end: they count the launch and,
+// when tracing is on, bracket it with CUDA events on the launch stream.
+// `work`: algorithmic FLOPs (GEMM, attention) or bytes moved (other kernels).
+void trace_launch_begin(int kind, cudaStream_t s, double work = 0.0);
+void trace_launch_end(int kind, cudaStream_t s);
+int* device_error_flag();   // device address of the error flag of the current device
+
+// Returns WAN_ERR_CUDA if the last launch failed.
+inline int check_launch() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? WAN_OK : WAN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- tensor maps
+// 2D/3D bf16 tile maps with 128-byte swizzle. dims/strides innermost first; strides
+// in bytes for dims >= 1. Returns false if the driver rejects the map.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box);
+
+// ---------------------------------------------------------------- kernels
+// LayerNorm (+ modulation). rows = B*L; e/mod_bias may be NULL (chunk < 0: plain LN).
+int launch_layernorm(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias,
+                     int chunk, void* out, int dtype, float eps, cudaStream_t s);
+
+struct GemmEpi {
+  int kind;                 // wan_epilogue
+  const float* gate;        // RESIDUAL: gate[(m / rows_per_batch) * gate_bstride + n]
+  const float* gate_bias;   // RESIDUAL: + gate_bias[n]
+  int64_t gate_bstride;
+  int rows_per_batch;
+  int64_t ldo;              // output row stride (elements)
+  // head scatter (kind == kEpiHeadScatter): out[b, c, f, 2i+ph, 2j+pw]
+  int sc_F, sc_H, sc_W, sc_C;
+};
+enum : int { kEpiHeadScatter = 100 };
+
+// bf16 tcgen05 GEMM: out = epi(A[M,K] W[N,K]^T + bias). A's rows have stride lda
+// elements; W has K columns (row stride K). If w_k_period > 0, W has w_k_period
+// columns and the k-th reduction index reads W column (k mod w_k_period).
+int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
+                   int w_k_period, const GemmEpi& epi, cudaStream_t s);
+// fp32 SIMT GEMM with the same semantics (fp32 activations and weights).
+int launch_gemm_simt(const float* A, int64_t lda, const float* W, const float* bias, void* out, int M, int N,
+                     int K, int w_k_period, const GemmEpi& epi, cudaStream_t s);
+
+struct AttnOperand {
+  const void* ptr;
+  int64_t row_stride;  // elements
+  int col0;            // column of head 0
+};
+// bf16 tcgen05 flash attention, head_dim 128.
+int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
+                   int B, int H, int Lq, int Lk, cudaStream_t s);
+// fp32 SIMT attention, head_dim <= 128, Lk <= 8192.
+int launch_attn_simt(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
+                     int B, int H, int Lq, int Lk, int d, cudaStream_t s);
+
+// Small kernels.
+int launch_patch_gather(const void* latent, int B, int C, int F, int H, int W, void* patches, int dtype,
+                        cudaStream_t s);
+int launch_time_mlp(const float* t, int B, int D, int freq_dim, const void* w1, const void* b1, const void* w2,
+                    const void* b2, float* e_out, int dtype, cudaStream_t s);
+int launch_i2v_input(const void* noise, const void* cond, const uint8_t* keep, int B, int F, int H, int W,
+                     void* out, int dtype, cudaStream_t s);
+int launch_flow_input(const void* x1, const void* x0, const float* u, int B, int64_t n, void* xt, float* t_out,
+                      int dtype, cudaStream_t s);
+int launch_flow_loss(const float* v, const void* x1, const void* x0, int B, int64_t n, float* loss, int dtype,
+                     cudaStream_t s);
+
+inline size_t dtype_size(int dtype) { return dtype == WAN_BF16 ? 2 : 4; }
+
+}  // namespace wan

@@ -1,0 +1,263 @@
+// Small kernels of the Wan 2.1 DiT forward path ("Wan: Open and Advanced Large-Scale
+// Video Generative Models", sections "Diffusion Transformer", "I2V 架构扩展" and
+// "训练方法"): the (1,2,2) patch gather feeding the patchify GEMM, the shared timestep
+// MLP, I2V input fusion, and the rectified-flow interpolation and loss.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "internal.h"
+
+namespace wan {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ld(const T* p, int64_t i);
+template <>
+__device__ __forceinline__ float ld<float>(const float* p, int64_t i) {
+  return p[i];
+}
+template <>
+__device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+template <typename T>
+__device__ __forceinline__ T cvt(float v);
+template <>
+__device__ __forceinline__ float cvt<float>(float v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 cvt<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// patches[b*L + (f*Hh + i)*Wh + j, c*4 + ph*2 + pw] = latent[b, c, f, 2i+ph, 2j+pw]
+// One thread per (token, channel): two 2-element reads, one 4-element write.
+template <typename T>
+__global__ void patch_gather_kernel(const T* __restrict__ lat, int B, int C, int F, int H, int W,
+                                    T* __restrict__ out) {
+  const int Hh = H / 2, Wh = W / 2;
+  const int64_t L = static_cast<int64_t>(F) * Hh * Wh;
+  const int64_t total = static_cast<int64_t>(B) * L * C;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % C);
+    const int64_t tok = idx / C;
+    const int b = static_cast<int>(tok / L);
+    const int64_t l = tok % L;
+    const int f = static_cast<int>(l / (Hh * Wh));
+    const int i = static_cast<int>((l / Wh) % Hh);
+    const int j = static_cast<int>(l % Wh);
+    const T* src = lat + ((static_cast<int64_t>(b) * C + c) * F + f) * H * W + static_cast<int64_t>(2 * i) * W + 2 * j;
+    T* dst = out + tok * (C * 4) + c * 4;
+    dst[0] = src[0];
+    dst[1] = src[1];
+    dst[2] = src[W];
+    dst[3] = src[W + 1];
+  }
+}
+
+constexpr int kTimeThreads = 256;
+constexpr int kTimeOutPerBlock = 256;
+
+// e[b, m] = sum_n w2[m, n] silu(sum_k w1[n, k] emb_k(t_b) + b1[n]) + b2[m], m < 6D.
+// Each block recomputes the sinusoid (double-precision arguments) and the D hidden
+// units in shared memory, then produces 256 outputs, one warp per output row at a time.
+template <typename T>
+__global__ void __launch_bounds__(kTimeThreads) time_mlp_kernel(const float* __restrict__ t, int D, int freq_dim,
+                                                                 const T* __restrict__ w1, const T* __restrict__ b1,
+                                                                 const T* __restrict__ w2, const T* __restrict__ b2,
+                                                                 float* __restrict__ e) {
+  extern __shared__ float sm[];
+  float* emb = sm;              // [freq_dim]
+  float* hid = sm + freq_dim;   // [D]
+  const int b = blockIdx.y;
+  const int half = freq_dim / 2;
+  const double tb = static_cast<double>(t[b]);
+  for (int k = threadIdx.x; k < half; k += kTimeThreads) {
+    const double f = pow(10000.0, -static_cast<double>(k) / half);
+    emb[k] = static_cast<float>(cos(tb * f));
+    emb[half + k] = static_cast<float>(sin(tb * f));
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int n = warp; n < D; n += kTimeThreads / 32) {
+    float acc = 0.f;
+    for (int k = lane; k < freq_dim; k += 32) acc = fmaf(ld(w1, static_cast<int64_t>(n) * freq_dim + k), emb[k], acc);
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      const float z = acc + ld(b1, n);
+      hid[n] = z / (1.0f + expf(-z));
+    }
+  }
+  __syncthreads();
+  const int m_end = min(6 * D, (blockIdx.x + 1) * kTimeOutPerBlock);
+  for (int m = blockIdx.x * kTimeOutPerBlock + warp; m < m_end; m += kTimeThreads / 32) {
+    float acc = 0.f;
+    for (int n = lane; n < D; n += 32) acc = fmaf(ld(w2, static_cast<int64_t>(m) * D + n), hid[n], acc);
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) e[static_cast<int64_t>(b) * 6 * D + m] = acc + ld(b2, m);
+  }
+}
+
+// out[b, c, f, y, x]: c < 16 noise, c < 32 condition latent, c < 36 the frame mask,
+// where latent frame f, mask channel mc takes pixel frame 0 for f == 0 (the first frame
+// repeated 4 times) and pixel frame 4f + mc - 3 otherwise.
+template <typename T>
+__global__ void i2v_input_kernel(const T* __restrict__ noise, const T* __restrict__ cond,
+                                 const uint8_t* __restrict__ keep, int B, int F, int H, int W, T* __restrict__ out) {
+  const int64_t plane = static_cast<int64_t>(F) * H * W;
+  const int64_t total = static_cast<int64_t>(B) * 36 * plane;
+  const int nkeep = 1 + 4 * (F - 1);
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t within = idx % plane;
+    const int c = static_cast<int>((idx / plane) % 36);
+    const int b = static_cast<int>(idx / (36 * plane));
+    T v;
+    if (c < 16) {
+      v = noise[(static_cast<int64_t>(b) * 16 + c) * plane + within];
+    } else if (c < 32) {
+      v = cond[(static_cast<int64_t>(b) * 16 + (c - 16)) * plane + within];
+    } else {
+      const int f = static_cast<int>(within / (static_cast<int64_t>(H) * W));
+      const int mc = c - 32;
+      const int frame = f == 0 ? 0 : 4 * f + mc - 3;
+      v = cvt<T>(keep[static_cast<int64_t>(b) * nkeep + frame] ? 1.0f : 0.0f);
+    }
+    out[idx] = v;
+  }
+}
+
+template <typename T>
+__global__ void flow_input_kernel(const T* __restrict__ x1, const T* __restrict__ x0, const float* __restrict__ u,
+                                  int B, int64_t n, T* __restrict__ xt, float* __restrict__ t_out) {
+  const int64_t total = static_cast<int64_t>(B) * n;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float ub = u[idx / n];
+    xt[idx] = cvt<T>(ub * ld(x1, idx) + (1.0f - ub) * ld(x0, idx));
+    if (t_out && idx % n == 0) t_out[idx / n] = 1000.0f * ub;
+  }
+}
+
+// One block per sample: loss[b] = mean((v - (x1 - x0))^2), accumulated in double in a
+// fixed order (deterministic).
+template <typename T>
+__global__ void __launch_bounds__(256) flow_loss_kernel(const float* __restrict__ v, const T* __restrict__ x1,
+                                                        const T* __restrict__ x0, int64_t n, float* __restrict__ loss) {
+  __shared__ double red[8];
+  const int b = blockIdx.x;
+  const int64_t base = static_cast<int64_t>(b) * n;
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < n; i += 256) {
+    const double d = static_cast<double>(v[base + i]) - (static_cast<double>(ld(x1, base + i)) - ld(x0, base + i));
+    acc += d * d;
+  }
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 8; ++w) s += red[w];
+    loss[b] = static_cast<float>(s / static_cast<double>(n));
+  }
+}
+
+unsigned grid_for(int64_t total, int threads) {
+  int64_t g = (total + threads - 1) / threads;
+  if (g > 148 * 64) g = 148 * 64;
+  return static_cast<unsigned>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+int launch_patch_gather(const void* latent, int B, int C, int F, int H, int W, void* patches, int dtype,
+                        cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(B) * F * (H / 2) * (W / 2) * C;
+  if (total == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s);
+  if (dtype == WAN_BF16)
+    patch_gather_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(latent), B, C, F, H, W, static_cast<__nv_bfloat16*>(patches));
+  else
+    patch_gather_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(static_cast<const float*>(latent), B, C, F, H,
+                                                                    W, static_cast<float*>(patches));
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+int launch_time_mlp(const float* t, int B, int D, int freq_dim, const void* w1, const void* b1, const void* w2,
+                    const void* b2, float* e_out, int dtype, cudaStream_t s) {
+  if (B == 0) return WAN_OK;
+  dim3 grid((6 * D + kTimeOutPerBlock - 1) / kTimeOutPerBlock, B);
+  const size_t smem = static_cast<size_t>(freq_dim + D) * sizeof(float);
+  if (smem > 48 * 1024) return WAN_ERR_SHAPE;
+  trace_launch_begin(WAN_KIND_SMALL, s);
+  if (dtype == WAN_BF16)
+    time_mlp_kernel<__nv_bfloat16><<<grid, kTimeThreads, smem, s>>>(
+        t, D, freq_dim, static_cast<const __nv_bfloat16*>(w1), static_cast<const __nv_bfloat16*>(b1),
+        static_cast<const __nv_bfloat16*>(w2), static_cast<const __nv_bfloat16*>(b2), e_out);
+  else
+    time_mlp_kernel<float><<<grid, kTimeThreads, smem, s>>>(t, D, freq_dim, static_cast<const float*>(w1),
+                                                           static_cast<const float*>(b1),
+                                                           static_cast<const float*>(w2),
+                                                           static_cast<const float*>(b2), e_out);
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+int launch_i2v_input(const void* noise, const void* cond, const uint8_t* keep, int B, int F, int H, int W, void* out,
+                     int dtype, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(B) * 36 * F * H * W;
+  if (total == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s);
+  if (dtype == WAN_BF16)
+    i2v_input_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(noise), static_cast<const __nv_bfloat16*>(cond), keep, B, F, H, W,
+        static_cast<__nv_bfloat16*>(out));
+  else
+    i2v_input_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(static_cast<const float*>(noise),
+                                                                 static_cast<const float*>(cond), keep, B, F, H, W,
+                                                                 static_cast<float*>(out));
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+int launch_flow_input(const void* x1, const void* x0, const float* u, int B, int64_t n, void* xt, float* t_out,
+                      int dtype, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(B) * n;
+  if (total == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s);
+  if (dtype == WAN_BF16)
+    flow_input_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x1), static_cast<const __nv_bfloat16*>(x0), u, B, n,
+        static_cast<__nv_bfloat16*>(xt), t_out);
+  else
+    flow_input_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(static_cast<const float*>(x1),
+                                                                  static_cast<const float*>(x0), u, B, n,
+                                                                  static_cast<float*>(xt), t_out);
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+int launch_flow_loss(const float* v, const void* x1, const void* x0, int B, int64_t n, float* loss, int dtype,
+                     cudaStream_t s) {
+  if (B == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s);
+  if (dtype == WAN_BF16)
+    flow_loss_kernel<__nv_bfloat16><<<B, 256, 0, s>>>(v, static_cast<const __nv_bfloat16*>(x1),
+                                                      static_cast<const __nv_bfloat16*>(x0), n, loss);
+  else
+    flow_loss_kernel<float><<<B, 256, 0, s>>>(v, static_cast<const float*>(x1), static_cast<const float*>(x0), n,
+                                              loss);
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+}  // namespace wan
