@@ -29,8 +29,8 @@
  *  - Calls keep no state between them except the trace tables and the device error
  *    flag; they are safe to call from several host threads on different streams.
  *  - Shape limits: D = heads * head_dim; head_dim 128 (bf16) or <= 128 (fp32);
- *    D, ffn_dim multiples of 64; latent H and W even; the fp32 path supports key
- *    lengths up to 8192.
+ *    D, ffn_dim multiples of 64; freq_dim a multiple of 8; latent H and W even; the
+ *    fp32 path supports key lengths up to 8192.
  */
 #ifndef WAN_H
 #define WAN_H

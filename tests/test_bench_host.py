@@ -1,0 +1,62 @@
+"""Host-side checks of bench.py's accounting (no GPU): algorithmic FLOPs per block
+against the closed form, the workload shapes, and the clock-sample parser."""
+import importlib.util
+import os
+
+import pytest
+
+from wan_inputs import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+def test_block_flops_match_closed_form(bench):
+    w2 = WORKLOADS["wan13b_480p_block"]
+    w4 = WORKLOADS["wan14b_720p_block"]
+    # QKV 6LD^2, O 2LD^2, cross q 2LD^2, cross o 2LD^2, kv 4 Lc D^2: 12 L D^2 + 4 Lc D^2 in total
+    for w in (w2, w4):
+        L, D, F, Lc = w.tokens, w.dim, w.ffn, w.text_len
+        expect = 12 * L * D * D + 4 * Lc * D * D + 4 * L * L * D + 4 * L * Lc * D + 4 * L * D * F
+        assert bench.block_flops(w) == pytest.approx(expect, rel=1e-12)
+    assert bench.block_flops(w2) / 1e12 == pytest.approx(9.433, abs=0.002)
+    assert bench.block_flops(w4) / 1e12 == pytest.approx(163.08, abs=0.02)
+    wi = WORKLOADS["wan13b_480p_i2v_block"]
+    extra = 4 * wi.img_len * wi.dim ** 2 + 4 * wi.tokens * wi.img_len * wi.dim + 2 * wi.tokens * wi.dim ** 2
+    assert bench.block_flops(wi) - bench.block_flops(w2) == pytest.approx(extra, rel=1e-12)
+
+
+def test_attention_share_of_block(bench):
+    w = WORKLOADS["wan13b_480p_block"]
+    attn = 4 * w.tokens ** 2 * w.dim
+    assert 0.69 < attn / bench.block_flops(w) < 0.71
+
+
+def test_clock_sampler_parses_nvidia_smi_lines(bench):
+    class P:
+        def __init__(self, out):
+            self.out = out
+
+        def terminate(self):
+            pass
+
+        def communicate(self, timeout=None):
+            return self.out, ""
+    s = bench.ClockSampler(0)
+    s.proc = P("0, 1800, 1965, 900.1, 0x0, Not Active, Not Active, Not Active, Active\n"
+               "0, 1400, 1965, 1000.2, 0x4, Not Active, Not Active, Not Active, Active\n"
+               "0, 1500, 1965, 990.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    r = s.stop()
+    assert r["sm_mhz"] == 1500 and r["sm_max_mhz"] == 1965 and r["reasons"] == ["sw_power_cap"] and r["samples"] == 3
+
+
+def test_peaks_source(bench):
+    peaks, src = bench.load_peaks()
+    assert peaks["bf16_tflops_sustained"] > 0 and src in ("measured", "fallback")

@@ -21,7 +21,8 @@ __all__ = [
     "flow_matching_loss", "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwan_b200.so")
+LIB_PATH = os.environ.get("WAN_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                            "libwan_b200.so")
 WAN_F32, WAN_BF16 = 0, 1
 EPI_STORE, EPI_GELU, EPI_RESIDUAL, EPI_F32 = 0, 1, 2, 3
 KIND_NORM, KIND_GEMM, KIND_ATTN, KIND_SMALL = 0, 1, 2, 3

@@ -136,7 +136,7 @@ int check_cfg(const wan_dit_config* c, bool attention = false) {
   WAN_REQUIRE(c->heads > 0 && c->head_dim > 0 && c->dim == c->heads * c->head_dim, WAN_ERR_SHAPE);
   WAN_REQUIRE(c->dim % 64 == 0 && c->ffn_dim > 0 && c->ffn_dim % 64 == 0, WAN_ERR_SHAPE);
   WAN_REQUIRE(c->in_ch > 0 && c->in_ch % 2 == 0 && c->out_ch > 0 && c->out_ch % 2 == 0, WAN_ERR_SHAPE);
-  WAN_REQUIRE(c->freq_dim > 0 && c->freq_dim % 2 == 0 && c->freq_dim <= 4096, WAN_ERR_SHAPE);
+  WAN_REQUIRE(c->freq_dim > 0 && c->freq_dim % 8 == 0 && c->freq_dim <= 4096, WAN_ERR_SHAPE);
   WAN_REQUIRE(c->eps > 0.f, WAN_ERR_SHAPE);
   if (!attention) return WAN_OK;
   if (c->dtype == WAN_BF16) {

@@ -4,22 +4,24 @@
 // cross-attention over 512 umT5 tokens in every block). softmax(q k^T / sqrt(d)) v per
 // head, non-causal, bf16 inputs, fp32 accumulation and fp32 softmax, head_dim 128.
 //
-// One CTA = one 128-row query tile of one (sample, head); 192 threads:
-//   warp 0   : TMA producer - Q once, then K_0, V_0, K_1, V_1, ... through a 4-stage
-//              ring of 32 KB tiles (128 rows x 128 dims, two 64-dim halves with
-//              128-byte swizzle);
-//   warp 1   : one thread issues tcgen05.mma: S_j = Q K_j^T into one of two TMEM S
-//              buffers (so QK^T of tile j+1 runs while tile j is in softmax), then
-//              O += P_{j-1} V_{j-1} into the TMEM O accumulator (V is an MN-major
-//              operand, no transpose pass);
-//   warps 2-5: softmax, one thread per query row: tcgen05.ld of its S row, masking of
-//              the ragged last key tile, running max and sum in fp32, exponentials
-//              with ex2, P rounded to bf16 into swizzled shared memory for the PV MMA.
-//              The running max used as the exponent base is only moved when the new
-//              row max exceeds it by more than 2^8 in probability terms; O (in TMEM)
-//              and the sum are rescaled then. Softmax is invariant to the base, and
-//              p <= 256 stays well inside fp32 and bf16 range, so the result is the
-//              same softmax. At the end O is divided by the sum and stored as bf16.
+// One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 320 threads:
+//   warp 0    : TMA producer - both Q tiles once, then K_0, K_1, V_0, K_2, V_1, ...
+//               (the order the MMA warp consumes them) through a 3-stage ring of 32 KB
+//               tiles (128 rows x 128 dims as two 64-dim halves, 128-byte swizzle);
+//   warp 1    : one thread issues tcgen05.mma. For key tile j and each query tile t:
+//               O_t += P_t(j-1) V_{j-1}, then S_t = Q_t K_j^T, then a commit that
+//               signals S_t ready. MMAs of one thread complete in issue order, so that
+//               signal also means P_t's buffer is free and O_t holds every earlier PV;
+//   warps 2-5 : softmax of query tile 0, warps 6-9: of query tile 1; one thread per
+//               query row (warp % 4 selects the TMEM lane quarter). Two passes over
+//               the row's S in TMEM (max, then exponentials), so the row never has to
+//               sit in registers whole; fp32 max and sum, ex2, the ragged last key
+//               tile masked; P rounded to bf16 into 128-byte-swizzled shared memory.
+//               The exponent base moves only when the row max grows by more than 2^8
+//               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
+//               base and p <= 256 stays well inside fp32 and bf16 range.
+// While one tile's softmax runs, the tensor core works on the other tile's MMAs.
+// TMEM: S_0, S_1, O_0, O_1 = 4 x 128 of the 512 columns.
 #include <cuda_bf16.h>
 
 #include <math.h>
@@ -32,19 +34,26 @@
 namespace wan {
 namespace {
 
-constexpr int kAttnThreads = 192;
-constexpr int kTile = 128;            // query rows per CTA = key rows per tile
-constexpr int kHd = 128;              // head dim
-constexpr int kStages = 4;            // K/V ring depth
-constexpr int kTileBytes = kTile * kHd * 2;   // 32 KB
-constexpr int kHalfBytes = kTileBytes / 2;    // one 64-column half
-constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (1 + kStages + 2) + 256;
-constexpr float kRescaleLog2 = 8.0f;  // move the exponent base when the max grows by > 2^8
+constexpr int kAttnThreads = 320;
+constexpr int kTile = 128;                     // query rows per tile = key rows per tile
+constexpr int kHd = 128;                       // head dim
+constexpr int kQTiles = 2;                     // query tiles per CTA
+constexpr int kStages = 3;                     // K/V ring depth
+constexpr int kTileBytes = kTile * kHd * 2;    // 32 KB
+constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
+constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (2 * kQTiles + kStages) + 256;
+constexpr float kRescaleLog2 = 8.0f;
+// Of every 8 exponentials, how many run on the FMA pipes (exp2_poly) instead of the
+// MUFU unit (0..4): balances the two units.
+#ifndef WAN_ATTN_POLY_EXP
+#define WAN_ATTN_POLY_EXP 0
+#endif
+constexpr int kPolyExp = WAN_ATTN_POLY_EXP;
 
 struct AttnParams {
   int Lq, Lk, H;
   int q_col0, k_col0, v_col0;
-  float scale_log2;       // log2(e) / sqrt(d)
+  float scale_log2;  // log2(e) / sqrt(d)
   __nv_bfloat16* o;
   int64_t o_row_stride;
   int64_t o_batch_stride;
@@ -52,28 +61,31 @@ struct AttnParams {
   int* err;
 };
 
+// Ring position of K_j / V_j in the load order K_0, K_1, V_0, K_2, V_1, ..., V_{n-1}.
+__device__ __forceinline__ int pos_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__device__ __forceinline__ int pos_v(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 * j + 2; }
+
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sKV = sQ + kTileBytes;
-  uint8_t* sP = sKV + kStages * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kTileBytes);
+  uint8_t* sQ = smem;                                  // [2][32 KB]
+  uint8_t* sP = sQ + kQTiles * kTileBytes;             // [2][32 KB]
+  uint8_t* sKV = sP + kQTiles * kTileBytes;            // [kStages][32 KB]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * kTileBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 2;
+  uint64_t* s_full = kv_empty + kStages;   // [2]
+  uint64_t* p_full = s_full + kQTiles;     // [2]
+  uint64_t* o_final = p_full + kQTiles;    // [2]
+  uint64_t* drain = o_final + kQTiles;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kTile;
+  const int q0 = blockIdx.x * (kQTiles * kTile);
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int nkv = (p.Lk + kTile - 1) / kTile;
@@ -84,11 +96,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&o_done[i], 1);
+    for (int t = 0; t < kQTiles; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_final[t], 1);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -106,22 +117,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t tmem_o = tmem_base + 256;
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kTileBytes);
+      mbar_arrive_expect_tx(q_full, kQTiles * kTileBytes);
       const int qc = p.q_col0 + h * kHd;
-      tma_load_3d(sQ, &mapQ, q_full, qc, q0, b);
-      tma_load_3d(sQ + kHalfBytes, &mapQ, q_full, qc + 64, q0, b);
+      for (int t = 0; t < kQTiles; ++t) {
+        tma_load_3d(sQ + t * kTileBytes, &mapQ, q_full, qc, q0 + t * kTile, b);
+        tma_load_3d(sQ + t * kTileBytes + kHalfBytes, &mapQ, q_full, qc + 64, q0 + t * kTile, b);
+      }
       const int n_loads = 2 * nkv;
       int issued = 0;
       for (int ld = 0; ld < n_loads; ++ld) {
         const int stage = ld % kStages;
         const uint32_t phase = static_cast<uint32_t>((ld / kStages) & 1);
         if (!mbar_wait(&kv_empty[stage], phase ^ 1u, p.err)) break;
-        const bool is_v = ld & 1;
-        const int j = ld >> 1;
+        bool is_v;
+        int j;
+        if (ld == 0) {
+          is_v = false, j = 0;
+        } else if (ld == n_loads - 1) {
+          is_v = true, j = nkv - 1;
+        } else if (ld & 1) {
+          is_v = false, j = (ld + 1) >> 1;
+        } else {
+          is_v = true, j = (ld >> 1) - 1;
+        }
         const CUtensorMap* map = is_v ? &mapV : &mapK;
         const int col = (is_v ? p.v_col0 : p.k_col0) + h * kHd;
         uint8_t* dst = sKV + stage * kTileBytes;
@@ -143,159 +164,202 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t kv_addr = smem_u32(sKV);
       const uint32_t p_addr = smem_u32(sP);
-      bool ok = mbar_wait(q_full, 0, p.err);
-      auto issue_pv = [&](int i) -> bool {
-        const int ld = 2 * i + 1;
-        const int stage = ld % kStages;
-        if (!mbar_wait(&p_full[i & 1], static_cast<uint32_t>((i >> 1) & 1), p.err)) return false;
-        if (!mbar_wait(&kv_full[stage], static_cast<uint32_t>((ld / kStages) & 1), p.err)) return false;
-        tc_fence_after();
-        const uint32_t pa = p_addr + (i & 1) * kTileBytes;
-        const uint32_t va = kv_addr + stage * kTileBytes;
+      auto wait_pos = [&](int pos) {
+        return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
+      };
+      auto pv = [&](int t, int i, int vstage) {
+        const uint32_t pa = p_addr + t * kTileBytes;
+        const uint32_t va = kv_addr + vstage * kTileBytes;
+        const uint32_t o_tmem = tmem_base + 256 + t * kTile;
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
           const uint64_t ad = sdesc_sw128(pa + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(va + k * 16 * 128, kHalfBytes, 1024);
-          tc_mma_bf16(tmem_o, ad, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+          tc_mma_bf16(o_tmem, ad, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
         }
-        tc_commit(&kv_empty[stage]);
-        tc_commit(&o_done[i & 1]);
-        return true;
       };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int ld = 2 * j;
-        const int stage = ld % kStages;
-        if (!mbar_wait(&kv_full[stage], static_cast<uint32_t>((ld / kStages) & 1), p.err)) break;
-        if (!mbar_wait(&s_free[j & 1], static_cast<uint32_t>(((j >> 1) & 1) ^ 1), p.err)) break;
-        tc_fence_after();
-        const uint32_t s_tmem = tmem_base + (j & 1) * kTile;
-        const uint32_t ka = kv_addr + stage * kTileBytes;
+      auto qk = [&](int t, int kstage) {
+        const uint32_t qa = q_addr + t * kTileBytes;
+        const uint32_t ka = kv_addr + kstage * kTileBytes;
+        const uint32_t s_tmem = tmem_base + t * kTile;
 #pragma unroll
         for (int k = 0; k < kHd / 16; ++k) {
           const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-          tc_mma_bf16(s_tmem, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk,
+          tc_mma_bf16(s_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk,
                       k > 0 ? 1u : 0u);
         }
-        tc_commit(&kv_empty[stage]);
-        tc_commit(&s_full[j & 1]);
-        if (j > 0) ok = issue_pv(j - 1);
+      };
+      bool ok = mbar_wait(q_full, 0, p.err);
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int pk = pos_k(j);
+        if (!wait_pos(pk)) break;
+        int pvpos = -1;
+        if (j > 0) {
+          pvpos = pos_v(j - 1, nkv);
+          if (!wait_pos(pvpos)) break;
+        }
+        for (int t = 0; ok && t < kQTiles; ++t) {
+          if (j > 0) {
+            if (!mbar_wait(&p_full[t], static_cast<uint32_t>((j - 1) & 1), p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            pv(t, j - 1, pvpos % kStages);
+          }
+          qk(t, pk % kStages);
+          tc_commit(&s_full[t]);
+        }
+        if (!ok) break;
+        tc_commit(&kv_empty[pk % kStages]);
+        if (j > 0) tc_commit(&kv_empty[pvpos % kStages]);
       }
-      if (ok && nkv > 0) issue_pv(nkv - 1);
+      if (ok && nkv > 0) {
+        const int last = nkv - 1;
+        const int pvpos = pos_v(last, nkv);
+        ok = wait_pos(pvpos);
+        for (int t = 0; ok && t < kQTiles; ++t) {
+          if (!mbar_wait(&p_full[t], static_cast<uint32_t>(last & 1), p.err)) break;
+          tc_fence_after();
+          pv(t, last, pvpos % kStages);
+          tc_commit(&o_final[t]);
+        }
+        tc_commit(&kv_empty[pvpos % kStages]);
+      }
       tc_commit(drain);
       mbar_wait(drain, 0, p.err);
     }
   } else {
-    // Softmax warps: TMEM lane quarter (warp % 4) holds query rows 32*quarter + lane.
+    // Softmax: query tile t, TMEM lane quarter (warp % 4), row 32 * quarter + lane.
+    const int t = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_row = tmem_base + lane_off + t * kTile;
+    const uint32_t o_row = tmem_base + lane_off + 256 + t * kTile;
+    uint8_t* prow = sP + t * kTileBytes + row * 128;
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; ok && j < nkv; ++j) {
-      if (!mbar_wait(&s_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), p.err)) {
+      if (!mbar_wait_warp(&s_full[t], static_cast<uint32_t>(j & 1), p.err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[kTile];
-      {
-        const uint32_t sa = tmem_base + lane_off + (j & 1) * kTile;
+      const int valid = p.Lk - j * kTile;  // keys of this tile that exist (mask the rest)
+      // Pass 1: row max over the two 64-column halves.
+      float mx8[8];
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(sa + c * 32, r);
-          tmem_ld_wait();
+      for (int a = 0; a < 8; ++a) mx8[a] = -INFINITY;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(s_row + hf * 64, r0);
+        tmem_ld32(s_row + hf * 64 + 32, r1);
+        tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          const float v0 = (hf * 64 + i < valid) ? __uint_as_float(r0[i]) : -INFINITY;
+          const float v1 = (hf * 64 + 32 + i < valid) ? __uint_as_float(r1[i]) : -INFINITY;
+          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(v0, v1));
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[j & 1]);
-      const int valid = p.Lk - j * kTile;
-      if (valid < kTile) {
-#pragma unroll
-        for (int i = 0; i < kTile; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int i = 1; i < kTile; ++i) mx = fmaxf(mx, s[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // The TMEM loads and stores of a rescale are warp-collective, so the decision is
+      // taken per warp: if any row of the warp needs it, every row moves its base to
+      // max(old base, tile max) (alpha = 1 for rows whose max did not grow).
+      const bool grow = (mx - m_run) * sl2 > kRescaleLog2;
       if (j == 0) {
         m_run = mx;
-      } else if ((mx - m_run) * sl2 > kRescaleLog2) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled.
-        if (!mbar_wait(&o_done[(j - 1) & 1], static_cast<uint32_t>(((j - 1) >> 1) & 1), p.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float alpha = ex2_approx((m_run - mx) * sl2);
+      } else if (__any_sync(0xffffffffu, grow)) {
+        // S_t(j) ready implies PV_t(j-1) completed: O_t is current and may be rescaled.
+        const float m_new = fmaxf(m_run, mx);
+        const float alpha = ex2_approx((m_run - m_new) * sl2);
 #pragma unroll
-        for (int c = 0; c < kHd / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, r);
+        for (int c = 0; c < kHd / 64; ++c) {
+          uint32_t r[32], r2[32];
+          tmem_ld32(o_row + c * 64, r);
+          tmem_ld32(o_row + c * 64 + 32, r2);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tmem_o + lane_off + c * 32, r);
+          for (int i = 0; i < 32; ++i) {
+            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            r2[i] = __float_as_uint(__uint_as_float(r2[i]) * alpha);
+          }
+          tmem_st32(o_row + c * 64, r);
+          tmem_st32(o_row + c * 64 + 32, r2);
         }
         tmem_st_wait();
         l_run *= alpha;
-        m_run = mx;
+        m_run = m_new;
       }
+      // Pass 2: exponentials, row sum, P (bf16) into swizzled shared memory.
       const float nb = -m_run * sl2;
-      float rs = 0.f;
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(s_row + hf * 64, r0);
+        tmem_ld32(s_row + hf * 64 + 32, r1);
+        tmem_ld_wait();
+        // exponentials in place (the registers now hold p as fp32 bits)
 #pragma unroll
-      for (int i = 0; i < kTile; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], sl2, nb));
-        rs += s[i];
-      }
-      l_run += rs;
-      // The P buffer of this parity was last read by PV_{j-2}.
-      if (j >= 2 && !mbar_wait(&o_done[j & 1], static_cast<uint32_t>(((j - 2) >> 1) & 1), p.err)) {
-        ok = false;
-        break;
-      }
-      uint8_t* prow = sP + (j & 1) * kTileBytes + row * 128;
+        for (int i = 0; i < 32; ++i) {
+          const float v0 = (hf * 64 + i < valid) ? __uint_as_float(r0[i]) : -INFINITY;
+          const float v1 = (hf * 64 + 32 + i < valid) ? __uint_as_float(r1[i]) : -INFINITY;
+          const float e0 = ex2_approx(fmaf(v0, sl2, nb));
+          const float x1 = fmaf(v1, sl2, nb);
+          const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
+          rs8[i & 7] += e0 + e1;
+          r0[i] = __float_as_uint(e0);
+          r1[i] = __float_as_uint(e1);
+        }
 #pragma unroll
-      for (int c16 = 0; c16 < kTile / 8; ++c16) {
-        const int half = c16 >> 3, ch = c16 & 7;
-        uint4 u;
-        u.x = pack_bf16x2(s[c16 * 8 + 0], s[c16 * 8 + 1]);
-        u.y = pack_bf16x2(s[c16 * 8 + 2], s[c16 * 8 + 3]);
-        u.z = pack_bf16x2(s[c16 * 8 + 4], s[c16 * 8 + 5]);
-        u.w = pack_bf16x2(s[c16 * 8 + 6], s[c16 * 8 + 7]);
-        *reinterpret_cast<uint4*>(prow + half * kHalfBytes + ((ch ^ (row & 7)) << 4)) = u;
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t* src = ch < 4 ? r0 + ch * 8 : r1 + (ch - 4) * 8;
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
+          u.y = pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3]));
+          u.z = pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5]));
+          u.w = pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7]));
+          *reinterpret_cast<uint4*>(prow + hf * kHalfBytes + ((ch ^ (row & 7)) << 4)) = u;
+        }
       }
+      l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[t]);
     }
-    if (ok && nkv > 0) {
-      const int last = nkv - 1;
-      if (mbar_wait(&o_done[last & 1], static_cast<uint32_t>((last >> 1) & 1), p.err)) {
-        tc_fence_after();
-        const float inv = 1.0f / l_run;
-        const int grow = q0 + row;
-        __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride +
-                              static_cast<int64_t>(grow) * p.o_row_stride + p.o_col0 + h * kHd;
+    if (ok && nkv > 0 && mbar_wait_warp(&o_final[t], 0, p.err)) {
+      tc_fence_after();
+      const float inv = 1.0f / l_run;
+      const int grow = q0 + t * kTile + row;
+      __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride +
+                            static_cast<int64_t>(grow) * p.o_row_stride + p.o_col0 + h * kHd;
 #pragma unroll
-        for (int c = 0; c < kHd / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, r);
-          tmem_ld_wait();
-          if (grow < p.Lq) {
+      for (int c = 0; c < kHd / 64; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(o_row + c * 64, r0);
+        tmem_ld32(o_row + c * 64 + 32, r1);
+        tmem_ld_wait();
+        if (grow < p.Lq) {
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(r[g * 8 + 0]) * inv, __uint_as_float(r[g * 8 + 1]) * inv);
-              u.y = pack_bf16x2(__uint_as_float(r[g * 8 + 2]) * inv, __uint_as_float(r[g * 8 + 3]) * inv);
-              u.z = pack_bf16x2(__uint_as_float(r[g * 8 + 4]) * inv, __uint_as_float(r[g * 8 + 5]) * inv);
-              u.w = pack_bf16x2(__uint_as_float(r[g * 8 + 6]) * inv, __uint_as_float(r[g * 8 + 7]) * inv);
-              reinterpret_cast<uint4*>(orow + c * 32)[g] = u;
-            }
+          for (int g = 0; g < 4; ++g) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(r0[g * 8 + 0]) * inv, __uint_as_float(r0[g * 8 + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(r0[g * 8 + 2]) * inv, __uint_as_float(r0[g * 8 + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(r0[g * 8 + 4]) * inv, __uint_as_float(r0[g * 8 + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(r0[g * 8 + 6]) * inv, __uint_as_float(r0[g * 8 + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 64)[g] = u;
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(r1[g * 8 + 0]) * inv, __uint_as_float(r1[g * 8 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(r1[g * 8 + 2]) * inv, __uint_as_float(r1[g * 8 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(r1[g * 8 + 4]) * inv, __uint_as_float(r1[g * 8 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(r1[g * 8 + 6]) * inv, __uint_as_float(r1[g * 8 + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 64 + 32)[g] = w;
           }
         }
       }
@@ -349,7 +413,7 @@ int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t
     cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kAttnSmem));
   });
-  dim3 grid((Lq + kTile - 1) / kTile, H, B);
+  dim3 grid((Lq + kQTiles * kTile - 1) / (kQTiles * kTile), H, B);
   trace_launch_begin(WAN_KIND_ATTN, s, 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd);
   attn_fwd_tc_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(mq, mk, mv, p);
   int st = check_launch();

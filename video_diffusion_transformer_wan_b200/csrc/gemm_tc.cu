@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
-      if (!mbar_wait(&tfull[acc], (it >> 1) & 1, p.err)) break;
+      if (!mbar_wait_warp(&tfull[acc], (it >> 1) & 1, p.err)) break;
       tc_fence_after();
       const int m0 = (tile / p.n_blocks) * kBM;
       const int n0 = (tile % p.n_blocks) * BN;

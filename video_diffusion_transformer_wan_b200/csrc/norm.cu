@@ -3,12 +3,18 @@
 // Large-Scale Video Generative Models", section "Diffusion Transformer": a shared MLP
 // predicts six modulation vectors, each block adds its own bias).
 //
-// HBM-bound: per row it reads D fp32 and writes D outputs. TPR threads own a row; each
-// thread holds NU units of 8 consecutive floats in registers (two 128-bit loads per
-// unit, one 128-bit bf16 store), so the row is read from HBM exactly once. Mean and
-// variance are two passes over the registers (warp shuffles, then shared memory when
-// a row spans several warps).
+// HBM-bound: per row it reads D fp32 and writes D outputs, i.e. 6 bytes per element
+// for a bf16 output. A row group of TPR threads owns one row at a time; each thread
+// holds NU units of 8 consecutive floats (two 128-bit loads, one 128-bit bf16 store).
+// The kernel is persistent: a row group walks rows with a grid-wide stride, keeps its
+// slice of shift and (1 + scale) in registers for as long as the sample does not
+// change (so modulation costs no memory traffic per row), and loads the next row
+// while it normalises the current one (two rows in flight per group). Mean and
+// variance are two passes over the registers: warp shuffles within a row group of
+// <= 32 threads, shared memory across the warps of a larger group.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "internal.h"
 
@@ -39,105 +45,120 @@ __device__ __forceinline__ void store8<float>(float* dst, const float (&v)[8]) {
   reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// Threads per block: several row groups of <= 32 threads, or one larger group.
 template <int TPR>
-__device__ __forceinline__ float row_sum(float v, float* red, int row_in_block, int t) {
+constexpr int norm_block() {
+  return TPR <= 32 ? kNormThreads : TPR;
+}
+
+template <int TPR>
+__device__ __forceinline__ float group_sum(float v, float* red, int t) {
   constexpr int W = TPR < 32 ? TPR : 32;
 #pragma unroll
   for (int o = W / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, W);
   if constexpr (TPR > 32) {
     constexpr int NW = TPR / 32;
-    float* r = red + row_in_block * NW;
-    __syncthreads();
-    if ((t & 31) == 0) r[t >> 5] = v;
+    if ((t & 31) == 0) red[t >> 5] = v;
     __syncthreads();
     v = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) v += r[w];
+    for (int w = 0; w < NW; ++w) v += red[w];
+    __syncthreads();
   }
   return v;
 }
 
-template <int TPR, int NU, typename OutT>
-__global__ void __launch_bounds__(kNormThreads) layernorm_mod_kernel(
+template <int TPR, int NU, bool MOD, typename OutT>
+__global__ void __launch_bounds__(norm_block<TPR>()) layernorm_mod_kernel(
     const float* __restrict__ x, int64_t rows, int D, int L, const float* __restrict__ e,
     const float* __restrict__ mod_bias, int chunk, OutT* __restrict__ out, float eps) {
-  constexpr int RPB = kNormThreads / TPR;
-  __shared__ float red[(TPR > 32) ? RPB * (TPR / 32) : 1];
-  const int row_in_block = threadIdx.x / TPR;
+  constexpr int G = norm_block<TPR>() / TPR;  // row groups per block
+  __shared__ float red[TPR > 32 ? TPR / 32 : 1];
+  const int group = threadIdx.x / TPR;
   const int t = threadIdx.x % TPR;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * RPB + row_in_block;
-  const bool active = row < rows;
-  const float* xr = x + (active ? row : 0) * D;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * G;
+  const float inv_d = 1.0f / static_cast<float>(D);
 
-  float v[NU][8];
-#pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const int col = (u * TPR + t) * 8;
-    const float4 a = __ldcs(reinterpret_cast<const float4*>(xr + col));
-    const float4 b = __ldcs(reinterpret_cast<const float4*>(xr + col + 4));
-    v[u][0] = a.x; v[u][1] = a.y; v[u][2] = a.z; v[u][3] = a.w;
-    v[u][4] = b.x; v[u][5] = b.y; v[u][6] = b.z; v[u][7] = b.w;
-  }
-  float s = 0.f;
-#pragma unroll
-  for (int u = 0; u < NU; ++u)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s += v[u][i];
-  const float mean = row_sum<TPR>(s, red, row_in_block, t) / static_cast<float>(D);
-  float q = 0.f;
-#pragma unroll
-  for (int u = 0; u < NU; ++u)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float c = v[u][i] - mean;
-      q += c * c;
-    }
-  const float var = row_sum<TPR>(q, red, row_in_block, t) / static_cast<float>(D);
-  const float rstd = 1.0f / sqrtf(var + eps);
-  if (!active) return;
+  float shv[MOD ? NU : 1][8];
+  float scv[MOD ? NU : 1][8];
+  int64_t cur_b = -1;
+  float va[NU][8], vb[NU][8];
 
-  const float* shift = nullptr;
-  const float* scale = nullptr;
-  const float* bshift = nullptr;
-  const float* bscale = nullptr;
-  if (chunk >= 0) {
-    const int64_t b = row / L;
-    shift = e + (b * 6 + 3 * chunk) * D;
-    scale = shift + D;
-    if (mod_bias) {
-      bshift = mod_bias + (3 * chunk) * D;
-      bscale = bshift + D;
+  auto load = [&](float (&v)[NU][8], int64_t r) {
+    const float* xr = x + (r < rows ? r : rows - 1) * D;
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+      const int col = (u * TPR + t) * 8;
+      const float4 a = __ldcs(reinterpret_cast<const float4*>(xr + col));
+      const float4 b = __ldcs(reinterpret_cast<const float4*>(xr + col + 4));
+      v[u][0] = a.x; v[u][1] = a.y; v[u][2] = a.z; v[u][3] = a.w;
+      v[u][4] = b.x; v[u][5] = b.y; v[u][6] = b.z; v[u][7] = b.w;
     }
-  }
-  OutT* orow = out + row * D;
+  };
+  auto process = [&](float (&v)[NU][8], int64_t r) {
+    float s = 0.f;
 #pragma unroll
-  for (int u = 0; u < NU; ++u) {
-    const int col = (u * TPR + t) * 8;
-    float o[8];
+    for (int u = 0; u < NU; ++u)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) o[i] = (v[u][i] - mean) * rstd;
-    if (chunk >= 0) {
-      float sh[8], sc[8];
-      *reinterpret_cast<float4*>(sh) = *reinterpret_cast<const float4*>(shift + col);
-      *reinterpret_cast<float4*>(sh + 4) = *reinterpret_cast<const float4*>(shift + col + 4);
-      *reinterpret_cast<float4*>(sc) = *reinterpret_cast<const float4*>(scale + col);
-      *reinterpret_cast<float4*>(sc + 4) = *reinterpret_cast<const float4*>(scale + col + 4);
-      if (bshift) {
-        float bs[8], bc[8];
-        *reinterpret_cast<float4*>(bs) = *reinterpret_cast<const float4*>(bshift + col);
-        *reinterpret_cast<float4*>(bs + 4) = *reinterpret_cast<const float4*>(bshift + col + 4);
-        *reinterpret_cast<float4*>(bc) = *reinterpret_cast<const float4*>(bscale + col);
-        *reinterpret_cast<float4*>(bc + 4) = *reinterpret_cast<const float4*>(bscale + col + 4);
+      for (int i = 0; i < 8; ++i) s += v[u][i];
+    const float mean = group_sum<TPR>(s, red, t) * inv_d;
+    float q = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          sh[i] += bs[i];
-          sc[i] += bc[i];
+    for (int u = 0; u < NU; ++u)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float c = v[u][i] - mean;
+        q += c * c;
+      }
+    const float rstd = 1.0f / sqrtf(group_sum<TPR>(q, red, t) * inv_d + eps);
+    if (r >= rows) return;
+    if constexpr (MOD) {
+      const int64_t b = r / L;
+      if (b != cur_b) {
+        cur_b = b;
+        const float* sh = e + (b * 6 + 3 * chunk) * D;
+        const float* sc = sh + D;
+        const float* bsh = mod_bias ? mod_bias + (3 * chunk) * D : nullptr;
+#pragma unroll
+        for (int u = 0; u < NU; ++u) {
+          const int col = (u * TPR + t) * 8;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            shv[u][i] = sh[col + i] + (bsh ? bsh[col + i] : 0.f);
+            scv[u][i] = 1.0f + sc[col + i] + (bsh ? bsh[D + col + i] : 0.f);
+          }
         }
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = o[i] * (1.0f + sc[i]) + sh[i];
     }
-    store8<OutT>(orow + col, o);
+    OutT* orow = out + r * D;
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+      float o[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        o[i] = (v[u][i] - mean) * rstd;
+        if constexpr (MOD) o[i] = fmaf(o[i], scv[u][i], shv[u][i]);
+      }
+      store8<OutT>(orow + (u * TPR + t) * 8, o);
+    }
+  };
+
+  // The block's rows advance together (base is uniform across the block), so shuffles
+  // and barriers never diverge; groups past the end load a valid row and skip stores.
+  int64_t base = static_cast<int64_t>(blockIdx.x) * G;
+  if (base >= rows) return;
+  load(va, base + group);
+  while (true) {
+    const int64_t nb = base + stride;
+    if (nb < rows) load(vb, nb + group);
+    process(va, base + group);
+    base = nb;
+    if (base >= rows) break;
+    const int64_t nb2 = base + stride;
+    if (nb2 < rows) load(va, nb2 + group);
+    process(vb, base + group);
+    base = nb2;
+    if (base >= rows) break;
   }
 }
 
@@ -185,44 +206,72 @@ __global__ void __launch_bounds__(kNormThreads) layernorm_mod_generic(
   }
 }
 
-template <typename OutT, int TPR, int NU>
+int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+template <typename OutT, int TPR, int NU, bool MOD>
 int launch_fixed(const float* x, int64_t rows, int D, int L, const float* e, const float* mb, int chunk,
                  OutT* out, float eps, cudaStream_t s) {
-  constexpr int RPB = kNormThreads / TPR;
-  const int64_t blocks = (rows + RPB - 1) / RPB;
-  layernorm_mod_kernel<TPR, NU, OutT><<<static_cast<unsigned>(blocks), kNormThreads, 0, s>>>(
-      x, rows, D, L, e, mb, chunk, out, eps);
+  constexpr int BT = norm_block<TPR>();
+  constexpr int G = BT / TPR;
+  auto kern = layernorm_mod_kernel<TPR, NU, MOD, OutT>;
+  static int per_sm[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (per_sm[dev & 63] == 0) {
+    int v = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kern, BT, 0);
+    per_sm[dev & 63] = v > 0 ? v : 1;
+  }
+  int64_t blocks = (rows + G - 1) / G;
+  const int64_t cap = static_cast<int64_t>(per_sm[dev & 63]) * num_sms();
+  if (blocks > cap) blocks = cap;
+  kern<<<static_cast<unsigned>(blocks), BT, 0, s>>>(x, rows, D, L, e, mb, chunk, out, eps);
+  return check_launch();
+}
+
+template <typename OutT, bool MOD>
+int launch_mod(const float* x, int64_t rows, int D, int L, const float* e, const float* mb, int chunk, OutT* out,
+               float eps, cudaStream_t s) {
+  const int units = D / 8;
+#define WAN_LN_CASE(TPR, NU) \
+  if (units == (TPR) * (NU)) return launch_fixed<OutT, TPR, NU, MOD>(x, rows, D, L, e, mb, chunk, out, eps, s);
+  WAN_LN_CASE(8, 1)
+  WAN_LN_CASE(16, 1)
+  WAN_LN_CASE(32, 1)
+  WAN_LN_CASE(32, 2)
+  WAN_LN_CASE(64, 2)     // D = 1024
+  WAN_LN_CASE(64, 3)     // D = 1536
+  WAN_LN_CASE(64, 4)     // D = 2048
+  WAN_LN_CASE(128, 3)    // D = 3072
+  WAN_LN_CASE(128, 4)    // D = 4096
+  WAN_LN_CASE(128, 5)    // D = 5120
+#undef WAN_LN_CASE
+  layernorm_mod_generic<OutT><<<static_cast<unsigned>(rows), kNormThreads, 0, s>>>(x, rows, D, L, e, mb, chunk,
+                                                                                     out, eps);
   return check_launch();
 }
 
 template <typename OutT>
 int launch_typed(const float* x, int64_t rows, int D, int L, const float* e, const float* mb, int chunk, OutT* out,
                  float eps, cudaStream_t s) {
-  const int units = D / 8;
-  if (D % 8 == 0) {
-#define WAN_LN_CASE(TPR, NU) \
-  if (units == (TPR) * (NU)) return launch_fixed<OutT, TPR, NU>(x, rows, D, L, e, mb, chunk, out, eps, s);
-    WAN_LN_CASE(8, 1)
-    WAN_LN_CASE(16, 1)
-    WAN_LN_CASE(32, 1)
-    WAN_LN_CASE(32, 2)
-    WAN_LN_CASE(32, 3)
-    WAN_LN_CASE(32, 4)
-    WAN_LN_CASE(32, 5)
-    WAN_LN_CASE(32, 6)
-    WAN_LN_CASE(32, 7)
-    WAN_LN_CASE(32, 8)
-    WAN_LN_CASE(128, 3)
-    WAN_LN_CASE(128, 4)
-    WAN_LN_CASE(128, 5)
-    WAN_LN_CASE(128, 6)
-    WAN_LN_CASE(128, 7)
-    WAN_LN_CASE(128, 8)
-#undef WAN_LN_CASE
+  if (D % 8 != 0) {
+    layernorm_mod_generic<OutT><<<static_cast<unsigned>(rows), kNormThreads, 0, s>>>(x, rows, D, L, e, mb, chunk,
+                                                                                       out, eps);
+    return check_launch();
   }
-  layernorm_mod_generic<OutT><<<static_cast<unsigned>(rows), kNormThreads, 0, s>>>(x, rows, D, L, e, mb, chunk,
-                                                                                     out, eps);
-  return check_launch();
+  return chunk >= 0 ? launch_mod<OutT, true>(x, rows, D, L, e, mb, chunk, out, eps, s)
+                    : launch_mod<OutT, false>(x, rows, D, L, e, mb, chunk, out, eps, s);
 }
 
 }  // namespace

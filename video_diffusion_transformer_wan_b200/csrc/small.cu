@@ -57,12 +57,71 @@ __global__ void patch_gather_kernel(const T* __restrict__ lat, int B, int C, int
   }
 }
 
-constexpr int kTimeThreads = 256;
+constexpr int kTimeThreads = 512;
 constexpr int kTimeOutPerBlock = 256;
+constexpr int kTimeRows = 4;  // weight rows a warp reduces at once (independent loads in flight)
+
+// 16-byte vector loads of weight rows, widened to fp32.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __bfloat1622float2(h[i]);
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float (&f)[4]) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  }
+};
+
+// acc[r] = sum_k w[(row0 + r) * n + k] * v[k] for kTimeRows rows (rows >= nrows are
+// computed on a valid row and ignored by the caller); the result is in every lane.
+template <typename T>
+__device__ __forceinline__ void warp_dot_rows(const T* __restrict__ w, int row0, int nrows, int n,
+                                              const float* __restrict__ v, int lane, float (&acc)[kTimeRows]) {
+  constexpr int V = Vec16<T>::N;
+  const T* rp[kTimeRows];
+#pragma unroll
+  for (int r = 0; r < kTimeRows; ++r) {
+    acc[r] = 0.f;
+    rp[r] = w + static_cast<int64_t>(min(row0 + r, nrows - 1)) * n;
+  }
+  const int nv = (n / V) * V;
+  for (int k = lane * V; k < nv; k += 32 * V) {
+    float f[kTimeRows][V];
+#pragma unroll
+    for (int r = 0; r < kTimeRows; ++r) Vec16<T>::load(rp[r] + k, f[r]);
+#pragma unroll
+    for (int r = 0; r < kTimeRows; ++r)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[r] = fmaf(f[r][i], v[k + i], acc[r]);
+  }
+  for (int k = nv + lane; k < n; k += 32)
+#pragma unroll
+    for (int r = 0; r < kTimeRows; ++r) acc[r] = fmaf(ld(rp[r], k), v[k], acc[r]);
+#pragma unroll
+  for (int r = 0; r < kTimeRows; ++r)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], off);
+}
 
 // e[b, m] = sum_n w2[m, n] silu(sum_k w1[n, k] emb_k(t_b) + b1[n]) + b2[m], m < 6D.
 // Each block recomputes the sinusoid (double-precision arguments) and the D hidden
-// units in shared memory, then produces 256 outputs, one warp per output row at a time.
+// units in shared memory (W1 is small and L2-resident), then produces 256 outputs;
+// a warp reduces kTimeRows weight rows at a time with 16-byte loads.
 template <typename T>
 __global__ void __launch_bounds__(kTimeThreads) time_mlp_kernel(const float* __restrict__ t, int D, int freq_dim,
                                                                  const T* __restrict__ w1, const T* __restrict__ b1,
@@ -80,23 +139,33 @@ __global__ void __launch_bounds__(kTimeThreads) time_mlp_kernel(const float* __r
     emb[half + k] = static_cast<float>(sin(tb * f));
   }
   __syncthreads();
+  constexpr int kWarps = kTimeThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int n = warp; n < D; n += kTimeThreads / 32) {
-    float acc = 0.f;
-    for (int k = lane; k < freq_dim; k += 32) acc = fmaf(ld(w1, static_cast<int64_t>(n) * freq_dim + k), emb[k], acc);
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      const float z = acc + ld(b1, n);
-      hid[n] = z / (1.0f + expf(-z));
+  for (int n0 = warp * kTimeRows; n0 < D; n0 += kWarps * kTimeRows) {
+    float acc[kTimeRows];
+    warp_dot_rows(w1, n0, D, freq_dim, emb, lane, acc);
+    if (lane < kTimeRows && n0 + lane < D) {
+      float a = acc[0];
+#pragma unroll
+      for (int r = 1; r < kTimeRows; ++r)
+        if (lane == r) a = acc[r];
+      const float z = a + ld(b1, n0 + lane);
+      hid[n0 + lane] = z / (1.0f + expf(-z));
     }
   }
   __syncthreads();
-  const int m_end = min(6 * D, (blockIdx.x + 1) * kTimeOutPerBlock);
-  for (int m = blockIdx.x * kTimeOutPerBlock + warp; m < m_end; m += kTimeThreads / 32) {
-    float acc = 0.f;
-    for (int n = lane; n < D; n += 32) acc = fmaf(ld(w2, static_cast<int64_t>(m) * D + n), hid[n], acc);
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) e[static_cast<int64_t>(b) * 6 * D + m] = acc + ld(b2, m);
+  const int m_beg = blockIdx.x * kTimeOutPerBlock;
+  const int m_end = min(6 * D, m_beg + kTimeOutPerBlock);
+  for (int m0 = m_beg + warp * kTimeRows; m0 < m_end; m0 += kWarps * kTimeRows) {
+    float acc[kTimeRows];
+    warp_dot_rows(w2, m0, 6 * D, D, hid, lane, acc);
+    if (lane < kTimeRows && m0 + lane < m_end) {
+      float a = acc[0];
+#pragma unroll
+      for (int r = 1; r < kTimeRows; ++r)
+        if (lane == r) a = acc[r];
+      e[static_cast<int64_t>(b) * 6 * D + m0 + lane] = a + ld(b2, m0 + lane);
+    }
   }
 }
 
