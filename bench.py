@@ -68,17 +68,21 @@ def load_peaks():
 
 
 def attn_traffic_per_launch():
-    """DRAM bytes per self-attention launch from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken."""
-    p = os.path.join(PROFILES, "attn_traffic.json")
+    """DRAM bytes (read + write) per self-attention launch from the committed ncu
+    summary, or None when the kernel source changed since the counters were taken."""
+    p = os.path.join(PROFILES, "attn_fwd_tc_kernel__self_L32760_H12.md")
     src = os.path.join(ROOT, "video_diffusion_transformer_wan_b200", "csrc", "attn_tc.cu")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if d.get("attn_tc_sha256") != h:
+    sha = byts = None
+    for line in open(p):
+        if line.startswith("- attn_tc.cu sha256:"):
+            sha = line.split(":", 1)[1].strip()
+        elif line.startswith("- dram bytes per launch (read+write):"):
+            byts = float(line.split(":", 1)[1])
+    if sha != hashlib.sha256(open(src, "rb").read()).hexdigest():
         return None
-    return d.get("bytes_per_launch")
+    return byts
 
 
 class ClockSampler:

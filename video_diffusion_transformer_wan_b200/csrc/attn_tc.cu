@@ -27,6 +27,7 @@
 #include <math.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -249,25 +250,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_after();
       const int valid = p.Lk - j * kTile;  // keys of this tile that exist (mask the rest)
-      // Pass 1: row max over the two 64-column halves.
-      float mx8[8];
+      // Only the last key tile can be ragged: the mask is compiled into that case alone
+      // (the branch is uniform across the CTA).
+      auto row_max = [&](auto masked) -> float {
+        constexpr bool kMask = decltype(masked)::value;
+        float mx8[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx8[a] = -INFINITY;
+        for (int a = 0; a < 8; ++a) mx8[a] = -INFINITY;
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(s_row + hf * 64, r0);
-        tmem_ld32(s_row + hf * 64 + 32, r1);
-        tmem_ld_wait();
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(s_row + hf * 64, r0);
+          tmem_ld32(s_row + hf * 64 + 32, r1);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float v0 = (hf * 64 + i < valid) ? __uint_as_float(r0[i]) : -INFINITY;
-          const float v1 = (hf * 64 + 32 + i < valid) ? __uint_as_float(r1[i]) : -INFINITY;
-          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(v0, v1));
+          for (int i = 0; i < 32; ++i) {
+            float v0 = __uint_as_float(r0[i]);
+            float v1 = __uint_as_float(r1[i]);
+            if constexpr (kMask) {
+              v0 = (hf * 64 + i < valid) ? v0 : -INFINITY;
+              v1 = (hf * 64 + 32 + i < valid) ? v1 : -INFINITY;
+            }
+            mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(v0, v1));
+          }
         }
-      }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      };
+      const float mx = valid >= kTile ? row_max(std::false_type{}) : row_max(std::true_type{});
       // The TMEM loads and stores of a rescale are warp-collective, so the decision is
       // taken per warp: if any row of the warp needs it, every row moves its base to
       // max(old base, tile max) (alpha = 1 for rows whose max did not grow).
@@ -299,35 +309,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Pass 2: exponentials, row sum, P (bf16) into swizzled shared memory.
       const float nb = -m_run * sl2;
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      auto exps = [&](auto masked) {
+        constexpr bool kMask = decltype(masked)::value;
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(s_row + hf * 64, r0);
-        tmem_ld32(s_row + hf * 64 + 32, r1);
-        tmem_ld_wait();
-        // exponentials in place (the registers now hold p as fp32 bits)
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(s_row + hf * 64, r0);
+          tmem_ld32(s_row + hf * 64 + 32, r1);
+          tmem_ld_wait();
+          // exponentials in place (the registers now hold p as fp32 bits)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float v0 = (hf * 64 + i < valid) ? __uint_as_float(r0[i]) : -INFINITY;
-          const float v1 = (hf * 64 + 32 + i < valid) ? __uint_as_float(r1[i]) : -INFINITY;
-          const float e0 = ex2_approx(fmaf(v0, sl2, nb));
-          const float x1 = fmaf(v1, sl2, nb);
-          const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
-          rs8[i & 7] += e0 + e1;
-          r0[i] = __float_as_uint(e0);
-          r1[i] = __float_as_uint(e1);
-        }
+          for (int i = 0; i < 32; ++i) {
+            float v0 = __uint_as_float(r0[i]);
+            float v1 = __uint_as_float(r1[i]);
+            if constexpr (kMask) {
+              v0 = (hf * 64 + i < valid) ? v0 : -INFINITY;
+              v1 = (hf * 64 + 32 + i < valid) ? v1 : -INFINITY;
+            }
+            const float e0 = ex2_approx(fmaf(v0, sl2, nb));
+            const float x1 = fmaf(v1, sl2, nb);
+            const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
+            rs8[i & 7] += e0 + e1;
+            r0[i] = __float_as_uint(e0);
+            r1[i] = __float_as_uint(e1);
+          }
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t* src = ch < 4 ? r0 + ch * 8 : r1 + (ch - 4) * 8;
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
-          u.y = pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3]));
-          u.z = pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5]));
-          u.w = pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7]));
-          *reinterpret_cast<uint4*>(prow + hf * kHalfBytes + ((ch ^ (row & 7)) << 4)) = u;
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t* src = ch < 4 ? r0 + ch * 8 : r1 + (ch - 4) * 8;
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
+            u.y = pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3]));
+            u.z = pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5]));
+            u.w = pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7]));
+            *reinterpret_cast<uint4*>(prow + hf * kHalfBytes + ((ch ^ (row & 7)) << 4)) = u;
+          }
         }
-      }
+      };
+      if (valid >= kTile)
+        exps(std::false_type{});
+      else
+        exps(std::true_type{});
       l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       fence_async_smem();
       tc_fence_before();

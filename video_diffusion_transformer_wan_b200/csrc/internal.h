@@ -6,7 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/wan.h"
+#include "wan.h"
 
 namespace wan {
 
