@@ -204,6 +204,30 @@ int wan_head_fwd(const wan_dit_config* cfg, const float* x, int B, int F, int H,
                  const void* w_head, const void* b_head, float* v_out,
                  void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- patchify without a workspace --------------------------------------------- */
+
+/* Bytes of the fixed device scratch array that wan_patchify_noalloc uses. */
+#define WAN_PATCHIFY_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* wan_patchify for callers that cannot allocate device memory: code that must not call
+ * the CUDA allocator (a host callback, an allocation-free real-time loop), a plug-in
+ * that its host framework hands only input and output pointers, or a process whose
+ * device-memory budget is fixed at start-up. The Wan 2.1 pages have no counterpart of
+ * this call; it exists for such callers of this library.
+ * Same arguments, layout and result as wan_patchify minus the workspace: the gathered
+ * patches go to a fixed array of WAN_PATCHIFY_NOALLOC_SCRATCH_BYTES (16 MiB) inside the
+ * library, which every GPU that loads the library holds until the process exits. A
+ * request whose patches (B*L*in_ch*4 act elements) exceed it returns WAN_ERR_SHAPE
+ * before any launch. The call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).
+ * The first call on a device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture. All calls
+ * share the one array and each leaves its contents behind: calls whose work overlaps
+ * on the GPU (other streams, other host threads) race on it, so the caller must order
+ * them. No part of the array needs to start at zero. */
+int wan_patchify_noalloc(const wan_dit_config* cfg, const void* latent, int B, int F, int H, int W,
+                         const void* w_p, const void* b_p, float* x_out, void* stream);
+
 /* ---- I2V and flow-matching pieces --------------------------------------------- */
 
 /* I2V input fusion [Wan 2.1 page, "I2V 架构扩展"]: out [B, 36, F, H, W] act =

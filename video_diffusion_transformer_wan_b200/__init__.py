@@ -15,7 +15,7 @@ from typing import Dict, Optional, Sequence
 __all__ = [
     "LIB_PATH", "lib", "WanError", "WAN_F32", "WAN_BF16", "EPI_STORE", "EPI_GELU", "EPI_RESIDUAL", "EPI_F32",
     "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights",
-    "ImageMlpWeights", "StackWeights", "make_config", "workspace_bytes", "device_status", "patchify", "time_mlp",
+    "ImageMlpWeights", "StackWeights", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
     "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
     "flow_matching_loss", "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "wan_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i]),
         "wan_device_status": (_i, [_vp]),
         "wan_patchify": (_i, [P(Config), _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+        "wan_patchify_noalloc": (_i, [P(Config), _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
         "wan_time_mlp": (_i, [P(Config), _vp, _i, P(TimeWeights), _vp, _vp]),
         "wan_adaln_modulate": (_i, [P(Config), _vp, _i, _i, _vp, _vp, _i, _vp, _vp]),
         "wan_self_attn_fwd": (_i, [P(Config), _vp, P(BlockWeights), _vp, _vp, _i, _i, _vp, _sz, _vp]),
@@ -164,6 +165,13 @@ def patchify(cfg, latent, w_p, b_p, x_out, ws, stream=None):
     B, C, F, H, W = latent.shape
     _check(_lib().wan_patchify(ctypes.byref(cfg), _p(latent), B, F, H, W, _p(w_p), _p(b_p), _p(x_out), _p(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "wan_patchify")
+
+
+def patchify_noalloc(cfg, latent, w_p, b_p, x_out, stream=None):
+    """wan_patchify without a workspace (fixed scratch inside the library)."""
+    B, C, F, H, W = latent.shape
+    _check(_lib().wan_patchify_noalloc(ctypes.byref(cfg), _p(latent), B, F, H, W, _p(w_p), _p(b_p), _p(x_out),
+                                       _stream(stream)), "wan_patchify_noalloc")
 
 
 def time_mlp(cfg, t, tw: TimeWeights, e_out, stream=None):
