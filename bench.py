@@ -135,6 +135,22 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the slowest replica sets the time)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_step: float, ms_per_step: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas timed by the slowest one."""
+    return world * tokens_per_step / (ms_per_step / 1e3)
+
+
 def _oracle_prefix(inp):
     from oracle import wan_oracle as O
     x = O.patchify(inp["noise"][0], inp["w_p"], inp["b_p"])
@@ -237,13 +253,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # Independent replicas: every rank draws its own sample (seed = rank).
     inp = make_inputs(w, seed=rank, block_input=False)
     cfg = config_for(w)
@@ -306,12 +315,12 @@ def main():
     clocks = sampler.stop()
     barrier()
     launches = wan.launch_count() - launches0
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     recs = wan.trace_launches()
     wan.trace_enable(False)
     ms_step = ms_total / args.steps
     tokens_step = B * L
-    value = world * tokens_step / (ms_step / 1e3)
+    value = replica_throughput(world, tokens_step, ms_step)
     flops = step_flops(w)
 
     # dominant kernel: the self-attention launch (largest attention work per step)
@@ -356,8 +365,8 @@ def main():
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e2.elapsed_time(e3)) / args.steps
-    e2e_value = world * tokens_step / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2.elapsed_time(e3), world, "cuda") / args.steps
+    e2e_value = replica_throughput(world, tokens_step, e2e_ms)
     status = wan.device_status()
     if status != 0:
         raise RuntimeError(f"device status {wan.status_string(status)} after timing")

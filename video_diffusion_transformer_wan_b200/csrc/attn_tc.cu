@@ -6,22 +6,25 @@
 //
 // One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 320 threads:
 //   warp 0    : TMA producer - both Q tiles once, then K_0, K_1, V_0, K_2, V_1, ...
-//               (the order the MMA warp consumes them) through a 3-stage ring of 32 KB
+//               (the order the MMA warp consumes them) through a 5-stage ring of 32 KB
 //               tiles (128 rows x 128 dims as two 64-dim halves, 128-byte swizzle);
 //   warp 1    : one thread issues tcgen05.mma. For key tile j and each query tile t:
-//               O_t += P_t(j-1) V_{j-1}, then S_t = Q_t K_j^T, then a commit that
-//               signals S_t ready. MMAs of one thread complete in issue order, so that
-//               signal also means P_t's buffer is free and O_t holds every earlier PV;
+//               O_t += P_t(j-1) V_{j-1} (P read from tensor memory, V an MN-major
+//               operand in shared memory), then S_t = Q_t K_j^T, then a commit that
+//               signals S_t ready. MMAs of one thread execute in issue order, so that
+//               signal also means P_t has been consumed and O_t holds every earlier PV;
 //   warps 2-5 : softmax of query tile 0, warps 6-9: of query tile 1; one thread per
 //               query row (warp % 4 selects the TMEM lane quarter). Two passes over
-//               the row's S in TMEM (max, then exponentials), so the row never has to
-//               sit in registers whole; fp32 max and sum, ex2, the ragged last key
-//               tile masked; P rounded to bf16 into 128-byte-swizzled shared memory.
+//               the row's S in TMEM (max, then exponentials); fp32 max and sum, ex2,
+//               the ragged last key tile masked in a separate compiled path. P is
+//               rounded to bf16 and written back into tensor memory over the S columns
+//               already consumed (two bf16 per 32-bit column, the layout of a K-major
+//               MMA operand), so P never touches shared memory.
 //               The exponent base moves only when the row max grows by more than 2^8
 //               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
 //               base and p <= 256 stays well inside fp32 and bf16 range.
 // While one tile's softmax runs, the tensor core works on the other tile's MMAs.
-// TMEM: S_0, S_1, O_0, O_1 = 4 x 128 of the 512 columns.
+// TMEM: S_0 (later P_0), S_1 (P_1), O_0, O_1 = 4 x 128 of the 512 columns.
 #include <cuda_bf16.h>
 
 #include <math.h>
@@ -39,10 +42,10 @@ constexpr int kAttnThreads = 320;
 constexpr int kTile = 128;                     // query rows per tile = key rows per tile
 constexpr int kHd = 128;                       // head dim
 constexpr int kQTiles = 2;                     // query tiles per CTA
-constexpr int kStages = 3;                     // K/V ring depth
+constexpr int kStages = 5;                     // K/V ring depth
 constexpr int kTileBytes = kTile * kHd * 2;    // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
-constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (2 * kQTiles + kStages) + 256;
+constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
 constexpr float kRescaleLog2 = 8.0f;
 // Of every 8 exponentials, how many run on the FMA pipes (exp2_poly) instead of the
 // MUFU unit (0..4): balances the two units.
@@ -72,8 +75,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                  // [2][32 KB]
-  uint8_t* sP = sQ + kQTiles * kTileBytes;             // [2][32 KB]
-  uint8_t* sKV = sP + kQTiles * kTileBytes;            // [kStages][32 KB]
+  uint8_t* sKV = sQ + kQTiles * kTileBytes;            // [kStages][32 KB]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * kTileBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
@@ -164,19 +166,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(kTile, kHd, 0, 1);
       const uint32_t q_addr = smem_u32(sQ);
       const uint32_t kv_addr = smem_u32(sKV);
-      const uint32_t p_addr = smem_u32(sP);
       auto wait_pos = [&](int pos) {
         return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
       };
       auto pv = [&](int t, int i, int vstage) {
-        const uint32_t pa = p_addr + t * kTileBytes;
+        // A = P_t in TMEM: bf16 pairs packed in the first 64 columns of S_t's region.
+        const uint32_t p_tmem = tmem_base + t * kTile;
         const uint32_t va = kv_addr + vstage * kTileBytes;
         const uint32_t o_tmem = tmem_base + 256 + t * kTile;
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(pa + (k >> 2) * kHalfBytes + (k & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(va + k * 16 * 128, kHalfBytes, 1024);
-          tc_mma_bf16(o_tmem, ad, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
         }
       };
       auto qk = [&](int t, int kstage) {
@@ -238,7 +239,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_row = tmem_base + lane_off + t * kTile;
     const uint32_t o_row = tmem_base + lane_off + 256 + t * kTile;
-    uint8_t* prow = sP + t * kTileBytes + row * 128;
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY;
     float l_run = 0.f;
@@ -333,16 +333,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             r0[i] = __float_as_uint(e0);
             r1[i] = __float_as_uint(e1);
           }
+          // P (bf16 pairs) over the S columns already consumed: half hf of the row goes to
+          // packed columns [32 hf, 32 hf + 32) of S_t's region.
+          uint32_t pk[32];
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t* src = ch < 4 ? r0 + ch * 8 : r1 + (ch - 4) * 8;
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
-            u.y = pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3]));
-            u.z = pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5]));
-            u.w = pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7]));
-            *reinterpret_cast<uint4*>(prow + hf * kHalfBytes + ((ch ^ (row & 7)) << 4)) = u;
+          for (int i = 0; i < 16; ++i) {
+            pk[i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+            pk[16 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
           }
+          tmem_st32(s_row + hf * 32, pk);
         }
       };
       if (valid >= kTile)
@@ -350,7 +349,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       else
         exps(std::true_type{});
       l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      fence_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }

@@ -9,8 +9,12 @@
 //   warp 1  : one elected thread issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
 //             accumulator; two accumulators alternate so the epilogue of one tile
 //             overlaps the main loop of the next;
-//   warps 2-5: epilogue; warp w reads TMEM lanes 32*(w%4).. (rows of the tile) with
-//             tcgen05.ld, applies bias / activation / gate and writes global memory.
+//   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).. (rows of the tile) and one
+//             half of the tile's columns with tcgen05.ld, applies bias / activation /
+//             gate and writes global memory. Two warps per lane quarter and column
+//             chunks taken in pairs (the fp32 residual of both chunks is loaded before
+//             either is updated) keep enough bytes in flight that the epilogue of one
+//             tile hides under the main loop of the next even when K is short.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -23,7 +27,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
 template <int BN>
 struct GemmCfg {
@@ -146,6 +151,50 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   }
 }
 
+// Two adjacent 32-column chunks [n0, n0+64) of one row. For the residual epilogue the
+// fp32 residual of both chunks is loaded before either is updated (16 loads in flight
+// per thread); other epilogues go chunk by chunk.
+__device__ __forceinline__ void epilogue_pair(const GemmParams& p, int row, int n0, const uint32_t (&r0)[32],
+                                              const uint32_t (&r1)[32]) {
+  if (p.epi.kind != WAN_EPI_RESIDUAL || row >= p.M || n0 + 64 > p.N) {
+    epilogue_chunk(p, row, n0, r0);
+    epilogue_chunk(p, row, n0 + 32, r1);
+    return;
+  }
+  float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+  float4 x[16];
+#pragma unroll
+  for (int g = 0; g < 16; ++g) x[g] = reinterpret_cast<const float4*>(o)[g];
+  const float* gate = p.epi.gate ? p.epi.gate + static_cast<int64_t>(row / p.epi.rows_per_batch) * p.epi.gate_bstride + n0
+                                 : nullptr;
+  const float* gb = p.epi.gate_bias ? p.epi.gate_bias + n0 : nullptr;
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {
+    const uint32_t* rr = g < 8 ? r0 + 4 * g : r1 + 4 * (g - 8);
+    float v0 = __uint_as_float(rr[0]), v1 = __uint_as_float(rr[1]);
+    float v2 = __uint_as_float(rr[2]), v3 = __uint_as_float(rr[3]);
+    if (p.bias) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.bias + n0) + g);
+      const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+      const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+      v0 += b01.x; v1 += b01.y; v2 += b23.x; v3 += b23.y;
+    }
+    if (gate) {
+      float4 t = __ldg(reinterpret_cast<const float4*>(gate) + g);
+      if (gb) {
+        const float4 u = __ldg(reinterpret_cast<const float4*>(gb) + g);
+        t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+      }
+      v0 *= t.x; v1 *= t.y; v2 *= t.z; v3 *= t.w;
+    }
+    x[g].x += v0;
+    x[g].y += v1;
+    x[g].z += v2;
+    x[g].w += v3;
+    reinterpret_cast<float4*>(o)[g] = x[g];
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
@@ -171,7 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * kEpiWarps);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -260,22 +309,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_wait(drain, 0, p.err);
     }
   } else {
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;           // TMEM lanes 32*quarter .. (rows of the tile)
+    const int colhalf = (warp - 2) >> 2;    // which half of the tile's columns
+    constexpr int kMine = BN / 64;          // 32-column chunks per warp
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       if (!mbar_wait_warp(&tfull[acc], (it >> 1) & 1, p.err)) break;
       tc_fence_after();
       const int m0 = (tile / p.n_blocks) * kBM;
-      const int n0 = (tile % p.n_blocks) * BN;
+      const int n0 = (tile % p.n_blocks) * BN + colhalf * (BN / 2);
       const int row = m0 + quarter * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN + colhalf * (BN / 2));
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        tmem_ld_wait();
-        epilogue_chunk(p, row, n0 + c * 32, r);
+      for (int c = 0; c < kMine; c += 2) {
+        if (c + 1 < kMine) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_row + c * 32, r0);
+          tmem_ld32(t_row + (c + 1) * 32, r1);
+          tmem_ld_wait();
+          epilogue_pair(p, row, n0 + c * 32, r0, r1);
+        } else {
+          uint32_t r0[32];
+          tmem_ld32(t_row + c * 32, r0);
+          tmem_ld_wait();
+          epilogue_chunk(p, row, n0 + c * 32, r0);
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
