@@ -14,12 +14,14 @@
 //               signals S_t ready. MMAs of one thread execute in issue order, so that
 //               signal also means P_t has been consumed and O_t holds every earlier PV;
 //   warps 2-5 : softmax of query tile 0, warps 6-9: of query tile 1; one thread per
-//               query row (warp % 4 selects the TMEM lane quarter). Two passes over
-//               the row's S in TMEM (max, then exponentials); fp32 max and sum, ex2,
-//               the ragged last key tile masked in a separate compiled path. P is
-//               rounded to bf16 and written back into tensor memory over the S columns
-//               already consumed (two bf16 per 32-bit column, the layout of a K-major
-//               MMA operand), so P never touches shared memory.
+//               query row (warp % 4 selects the TMEM lane quarter). The row's 128 S
+//               values are read from TMEM with a single wait (the wait covers every
+//               outstanding TMEM load, so reading in pieces would expose its latency
+//               once per piece); fp32 max and sum, ex2, the ragged last key tile
+//               masked only on that tile. P is rounded to bf16, packed in place and
+//               written back into tensor memory over the S columns already read (two
+//               bf16 per 32-bit column, the layout of a K-major MMA operand), so P
+//               never touches shared memory.
 //               The exponent base moves only when the row max grows by more than 2^8
 //               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
 //               base and p <= 256 stays well inside fp32 and bf16 range.
@@ -30,7 +32,6 @@
 #include <math.h>
 
 #include <mutex>
-#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -48,7 +49,7 @@ constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
 constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
 constexpr float kRescaleLog2 = 8.0f;
 // Of every 8 exponentials, how many run on the FMA pipes (exp2_poly) instead of the
-// MUFU unit (0..4): balances the two units.
+// MUFU unit (0..4). Measured best at 0 for this kernel (1 and 2 were slower).
 #ifndef WAN_ATTN_POLY_EXP
 #define WAN_ATTN_POLY_EXP 0
 #endif
@@ -250,104 +251,65 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_after();
       const int valid = p.Lk - j * kTile;  // keys of this tile that exist (mask the rest)
-      // Only the last key tile can be ragged: the mask is compiled into that case alone
-      // (the branch is uniform across the CTA).
-      auto row_max = [&](auto masked) -> float {
-        constexpr bool kMask = decltype(masked)::value;
-        float mx8[8];
+      // The whole S row (128 fp32) is read with one wait; P is then packed in place into
+      // the first 64 registers (pair i of the row lands in register i <= 2i, so the pass
+      // never overwrites a value it still has to read) and stored over S in TMEM.
+      uint32_t r[kTile];
+      tmem_ld32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+      tmem_ld32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      tmem_ld32(s_row + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+      tmem_ld32(s_row + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+      tmem_ld_wait();
+      if (valid < kTile) {
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = -INFINITY;
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(s_row + hf * 64, r0);
-          tmem_ld32(s_row + hf * 64 + 32, r1);
-          tmem_ld_wait();
+        for (int i = 0; i < kTile; ++i)
+          if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+      }
+      float mx8[8];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float v0 = __uint_as_float(r0[i]);
-            float v1 = __uint_as_float(r1[i]);
-            if constexpr (kMask) {
-              v0 = (hf * 64 + i < valid) ? v0 : -INFINITY;
-              v1 = (hf * 64 + 32 + i < valid) ? v1 : -INFINITY;
-            }
-            mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(v0, v1));
-          }
-        }
-        return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      };
-      const float mx = valid >= kTile ? row_max(std::false_type{}) : row_max(std::true_type{});
-      // The TMEM loads and stores of a rescale are warp-collective, so the decision is
-      // taken per warp: if any row of the warp needs it, every row moves its base to
-      // max(old base, tile max) (alpha = 1 for rows whose max did not grow).
+      for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(r[a]);
+#pragma unroll
+      for (int i = 8; i < kTile; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[i]));
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const bool grow = (mx - m_run) * sl2 > kRescaleLog2;
+      float alpha = 1.0f;
+      bool rescale = false;
       if (j == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, grow)) {
-        // S_t(j) ready implies PV_t(j-1) completed: O_t is current and may be rescaled.
         const float m_new = fmaxf(m_run, mx);
-        const float alpha = ex2_approx((m_run - m_new) * sl2);
-#pragma unroll
-        for (int c = 0; c < kHd / 64; ++c) {
-          uint32_t r[32], r2[32];
-          tmem_ld32(o_row + c * 64, r);
-          tmem_ld32(o_row + c * 64 + 32, r2);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            r2[i] = __float_as_uint(__uint_as_float(r2[i]) * alpha);
-          }
-          tmem_st32(o_row + c * 64, r);
-          tmem_st32(o_row + c * 64 + 32, r2);
-        }
-        tmem_st_wait();
-        l_run *= alpha;
+        alpha = ex2_approx((m_run - m_new) * sl2);
         m_run = m_new;
+        rescale = true;
       }
-      // Pass 2: exponentials, row sum, P (bf16) into swizzled shared memory.
       const float nb = -m_run * sl2;
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      auto exps = [&](auto masked) {
-        constexpr bool kMask = decltype(masked)::value;
+#pragma unroll
+      for (int i = 0; i < kTile / 2; ++i) {
+        const float x0 = fmaf(__uint_as_float(r[2 * i]), sl2, nb);
+        const float x1 = fmaf(__uint_as_float(r[2 * i + 1]), sl2, nb);
+        const float e0 = ex2_approx(x0);
+        const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
+        rs8[i & 7] += e0 + e1;
+        r[i] = pack_bf16x2(e0, e1);
+      }
+      tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+      tmem_st32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+      if (rescale) {
+        // S_t(j) ready implies PV_t(j-1) completed, and PV_t(j) waits for this thread's
+        // arrival below: O_t is current and idle while it is rescaled here.
 #pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(s_row + hf * 64, r0);
-          tmem_ld32(s_row + hf * 64 + 32, r1);
+        for (int c = 0; c < kHd / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_row + c * 32, o);
           tmem_ld_wait();
-          // exponentials in place (the registers now hold p as fp32 bits)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float v0 = __uint_as_float(r0[i]);
-            float v1 = __uint_as_float(r1[i]);
-            if constexpr (kMask) {
-              v0 = (hf * 64 + i < valid) ? v0 : -INFINITY;
-              v1 = (hf * 64 + 32 + i < valid) ? v1 : -INFINITY;
-            }
-            const float e0 = ex2_approx(fmaf(v0, sl2, nb));
-            const float x1 = fmaf(v1, sl2, nb);
-            const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
-            rs8[i & 7] += e0 + e1;
-            r0[i] = __float_as_uint(e0);
-            r1[i] = __float_as_uint(e1);
-          }
-          // P (bf16 pairs) over the S columns already consumed: half hf of the row goes to
-          // packed columns [32 hf, 32 hf + 32) of S_t's region.
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            pk[i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-            pk[16 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
-          }
-          tmem_st32(s_row + hf * 32, pk);
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st32(o_row + c * 32, o);
         }
-      };
-      if (valid >= kTile)
-        exps(std::false_type{});
-      else
-        exps(std::true_type{});
+        l_run *= alpha;
+      }
       l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_st_wait();
       tc_fence_before();
