@@ -334,3 +334,44 @@ def dit_stack(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, head
         x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx)
     y = head(x, weights["w_head"], weights["b_head"], eps)
     return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)
+
+
+# --------------------------------------------------------------------------------------
+# Sampling: rectified-flow Euler integration with classifier-free guidance
+# [Wan-P2, "Infra": about 50 sampling steps; "训练方法": the model predicts the velocity
+# x1 - x0 along x_t = t x1 + (1 - t) x0, noise at t = 0]
+# --------------------------------------------------------------------------------------
+
+def euler_cfg(x0, n_steps: int, guidance: float, velocity_cond, velocity_uncond) -> np.ndarray:
+    """Integrate dx/dt = v(x, t) from t = 0 (noise) to t = 1 with ``n_steps`` Euler
+    steps on the uniform grid t_k = k / n_steps, where the velocity is the guided
+    combination ``v_u + guidance * (v_c - v_u)`` of the conditional and unconditional
+    predictions ``velocity_*(x, t_k)``. reading: uniform grid in t, explicit Euler,
+    guidance applied to the velocity (the pages give only the step count and a
+    guidance scale)."""
+    x = _f(x0).copy()
+    dt = 1.0 / n_steps
+    for k in range(n_steps):
+        t = k * dt
+        vc = _f(velocity_cond(x, t))
+        vu = _f(velocity_uncond(x, t))
+        x = x + dt * (vu + guidance * (vc - vu))
+    return x
+
+
+def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks: Sequence[Dict], ctx_cond,
+                     ctx_uncond, heads: int, eps: float = 1e-6, img_ctx=None, cond_channels=None,
+                     freq_dim: int = 256) -> np.ndarray:
+    """Generate a latent with the DiT as the velocity model: ``euler_cfg`` with
+    ``v(x, t) = dit_stack(input(x), 1000 t, ...)`` under the text context (conditional)
+    and the unconditional context. ``noise [16, F, H, W]`` is x at t = 0. For I2V,
+    ``cond_channels [20, F, H, W]`` (condition latent and mask) are appended to x on the
+    channel axis at every step and stay fixed. reading: the image context is used by
+    both branches; only the text context differs."""
+    def make_input(x):
+        return x if cond_channels is None else np.concatenate([x, _f(cond_channels)], axis=0)
+
+    def vel(ctx):
+        return lambda x, t: dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps,
+                                      img_ctx=img_ctx, freq_dim=freq_dim)
+    return euler_cfg(noise, n_steps, guidance, vel(ctx_cond), vel(ctx_uncond))

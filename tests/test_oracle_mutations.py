@@ -138,3 +138,17 @@ def test_i2v_mask_mutation_is_caught():
         m = np.concatenate([np.asarray(keep, np.float64), np.zeros(3)]).reshape(F, stride).T
         return np.broadcast_to(m[:, :, None, None], (stride, F, H, W)).copy()
     _fails(P.check_i2v_mask, no_repeat)
+
+
+def test_euler_cfg_mutations_are_caught():
+    def guidance_on_wrong_branch(x0, n, g, vc, vu):
+        return O.euler_cfg(x0, n, g, vu, vc)
+
+    def right_endpoint_grid(x0, n, g, vc, vu):
+        x = np.asarray(x0, np.float64).copy()
+        for k in range(n):
+            t = (k + 1) / n
+            x = x + (vu(x, t) + g * (vc(x, t) - vu(x, t))) / n
+        return x
+    _fails(P.check_euler_cfg, guidance_on_wrong_branch)
+    _fails(P.check_euler_cfg, right_endpoint_grid)
