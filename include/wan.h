@@ -255,6 +255,41 @@ int wan_flow_matching_input(const wan_dit_config* cfg, const void* x1, const voi
 int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void* x1,
                            const void* x0, int B, int64_t n, float* loss_out, void* stream);
 
+/* ---- sampling ----------------------------------------------------------------- */
+
+/* Device workspace (bytes) of wan_sample_euler_cfg for these sizes (0 on a bad cfg). */
+size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W,
+                                  int Lc, int Li);
+
+/* Generation loop with the DiT as the velocity model [Wan 2.1 page, "训练方法" (the
+ * rectified-flow velocity) and "Infra" (a fixed number of sampling steps, about 50); the
+ * Baidu cloud article on Wan 2.1 names the step count and the guidance scale as the
+ * user's knobs]. The pages fix neither the time grid nor the solver nor the guidance
+ * formula; this call takes the plainest reading that the velocity definition supports:
+ * x(0) is the noise, x(1) the sample, n_steps explicit Euler steps on the uniform grid
+ * t_k = k / n_steps, x += (1/n_steps) (v_u + guidance (v_c - v_u)), where
+ * v_c = DiT(input(x), 1000 t_k, ctx_cond) and v_u = DiT(input(x), 1000 t_k, ctx_uncond)
+ * are evaluated as ONE stack pass over a batch of 2B samples.
+ *   input [B, in_ch, F, H, W] act (device): the noise in channels [0, out_ch) and, for
+ *     I2V (in_ch > out_ch), the condition channels [out_ch, in_ch) that are appended to
+ *     x unchanged at every step. out_ch <= in_ch.
+ *   ctx_cond, ctx_uncond [B, Lc, D] act; img_ctx [B, Li, D] act or NULL (Li = 0): the
+ *     image context is shared by both branches.
+ *   latent_out [B, out_ch, F, H, W] fp32: the state x, written with the noise at the
+ *     start and holding x(1) on return. The DiT input is x rounded to act each step.
+ *   blocks: HOST array of n_blocks weight tables; sw: stack weights.
+ *   Cross-attention K|V of both contexts are projected once per call and kept for all
+ *   steps. workspace >= wan_sample_workspace_bytes(...) device bytes.
+ * Errors (before any launch): WAN_ERR_NULL, WAN_ERR_SHAPE (n_steps < 1, a guidance that
+ * is not finite, out_ch > in_ch, Lc = 0, odd H or W), WAN_ERR_WORKSPACE, WAN_ERR_ALIGN.
+ * B = 0 returns WAN_OK without work. Enqueued on `stream`; returns before the GPU work
+ * ends. */
+int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* input, int B, int F, int H,
+                         int W, int n_steps, float guidance, const wan_stack_weights* sw,
+                         const wan_block_weights* blocks, const void* ctx_cond, const void* ctx_uncond,
+                         int Lc, const void* img_ctx, int Li, float* latent_out, void* workspace,
+                         size_t ws_bytes, void* stream);
+
 /* ---- single-kernel entry points (used by the branch calls; exposed for tests) --- */
 
 /* Multi-head attention softmax(q k^T / sqrt(d)) v, non-causal. q [B, Lq, *], k and v

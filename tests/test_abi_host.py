@@ -109,5 +109,35 @@ def test_validation_rejects_before_launch(wan):
     assert wan.launch_count() == launches
 
 
+def test_sampler_validation_and_workspace(wan):
+    """The sampling call checks its arguments before any launch; its workspace covers
+    the 2B-sample stack pass plus the per-block K|V caches."""
+    L = wan.lib
+    launches = wan.launch_count()
+    cfg = _cfg(wan)
+    fake = 1 << 20
+    bws = (wan.BlockWeights * 2)(*[wan.BlockWeights(*([fake] * 17)) for _ in range(2)])
+    sw = wan.StackWeights(fake, fake, wan.TimeWeights(fake, fake, fake, fake), fake, fake)
+    B, F, H, W, Lc = 1, 21, 60, 104, 512
+    need = wan.sample_workspace_bytes(cfg, 2, B, F, H, W, Lc)
+    Lt = F * (H // 2) * (W // 2)
+    assert need > wan.workspace_bytes(cfg, 2 * B, Lt, Lc) + 2 * 2 * (2 * B * Lc * 2 * 1536)
+    assert wan.sample_workspace_bytes(_cfg(wan, heads=7), 2, B, F, H, W, Lc) == 0
+
+    def call(n_steps=4, g=5.0, c=cfg, ctx_u=fake, ws=1 << 40, b=B, h=H):
+        return L.wan_sample_euler_cfg(ctypes.byref(c), 2, fake, b, F, h, W, n_steps, g, ctypes.byref(sw), bws, fake,
+                                      ctx_u, Lc, None, 0, fake, fake, ws, None)
+    assert call(n_steps=0) == -2
+    assert call(g=float("nan")) == -2
+    assert call(g=float("inf")) == -2
+    assert call(ctx_u=None) == -1
+    assert call(ws=need - 1) == -5
+    assert call(h=59) == -2
+    c2 = _cfg(wan, in_ch=16, out_ch=20)
+    assert call(c=c2) == -2
+    assert call(b=0) == 0
+    assert wan.launch_count() == launches
+
+
 def test_trace_read_without_events(wan):
     assert wan.trace_read(wan.KIND_ATTN) == (0.0, 0)

@@ -32,10 +32,10 @@ def small_bf16(i2v=False, **kw):
 class Run:
     """Inputs on the device and the ABI tables for one workload."""
 
-    def __init__(self, wan, w, seed=0, n_blocks=None, zero_wx=True):
+    def __init__(self, wan, w, seed=0, n_blocks=None, zero_wx=True, uncond=False):
         from video_diffusion_transformer_wan_b200.model import DitModel, config_for, to_device
         self.w = w
-        self.inp = make_inputs(w, seed=seed, n_blocks=n_blocks, zero_wx=zero_wx)
+        self.inp = make_inputs(w, seed=seed, n_blocks=n_blocks, zero_wx=zero_wx, uncond=uncond)
         self.cfg = config_for(w)
         self.model = DitModel(self.cfg, self.inp)
         act = self.model.act
@@ -43,6 +43,7 @@ class Run:
         self.x = to_device(self.inp["x"], torch.float32)
         self.e = to_device(self.inp["e"], torch.float32)
         self.ctx = to_device(self.inp["ctx"], act)
+        self.ctx_uncond = to_device(self.inp["ctx_uncond"], act) if uncond else None
         self.img_ctx = None
         self.img_np = None
         Li = 0

@@ -18,7 +18,7 @@ __all__ = [
     "ImageMlpWeights", "StackWeights", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
     "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
-    "flow_matching_loss", "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
+    "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
 LIB_PATH = os.environ.get("WAN_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
@@ -88,6 +88,9 @@ def _load() -> ctypes.CDLL:
         "wan_attention_fwd": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _i,
                                    _i, _i, _i, _vp]),
         "wan_linear_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i, _vp]),
+        "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i]),
+        "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
+                                      P(BlockWeights), _vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
         "wan_launch_count": (_i64, []),
         "wan_trace_enable": (_i, [_i]),
         "wan_trace_reset": (_i, []),
@@ -224,6 +227,23 @@ def dit_stack_fwd(cfg, latent, t, sw: StackWeights, blocks: Sequence[BlockWeight
     _check(_lib().wan_dit_stack_fwd(ctypes.byref(cfg), len(blocks), _p(latent), B, F, H, W, _p(t), ctypes.byref(sw),
                                  arr, _p(ctx), ctx.shape[1], _p(img_ctx), Li, _p(v_out), *_ws(ws), _stream(stream)),
            "wan_dit_stack_fwd")
+
+
+def sample_workspace_bytes(cfg: Config, n_blocks: int, B: int, F: int, H: int, W: int, Lc: int, Li: int = 0) -> int:
+    return int(_lib().wan_sample_workspace_bytes(ctypes.byref(cfg), n_blocks, B, F, H, W, Lc, Li))
+
+
+def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, blocks: Sequence[BlockWeights],
+                     ctx_cond, ctx_uncond, img_ctx, latent_out, ws, stream=None):
+    """inp [B, in_ch, F, H, W]: the noise in its first out_ch channels (and, for I2V, the
+    fixed condition channels after them); latent_out [B, out_ch, F, H, W] fp32."""
+    B, C, F, H, W = inp.shape
+    arr = (BlockWeights * max(1, len(blocks)))(*blocks)
+    Li = 0 if img_ctx is None else img_ctx.shape[1]
+    _check(_lib().wan_sample_euler_cfg(ctypes.byref(cfg), len(blocks), _p(inp), B, F, H, W, n_steps, guidance,
+                                    ctypes.byref(sw), arr, _p(ctx_cond), _p(ctx_uncond), ctx_cond.shape[1],
+                                    _p(img_ctx), Li, _p(latent_out), *_ws(ws), _stream(stream)),
+           "wan_sample_euler_cfg")
 
 
 def attention_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0, o_col0=0, stream=None):

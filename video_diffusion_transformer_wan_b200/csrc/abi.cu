@@ -244,8 +244,11 @@ int self_attn_impl(const wan_dit_config* c, const void* h, const wan_block_weigh
   return gemm(c, o, D, w->w_o, w->b_o, x, M, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, L), s);
 }
 
+// kvt_cached / kvi_cached: text / image K|V already projected ([B*Lc, 2D], [B*Li, 2D]
+// act), e.g. kept across sampling steps; the projections are skipped when given.
 int cross_attn_impl(const wan_dit_config* c, const void* h, const void* ctx, int Lc, const void* img, int Li,
-                    const wan_block_weights* w, float* x, int B, int L, void* ws, const Layout& ly, cudaStream_t s) {
+                    const wan_block_weights* w, float* x, int B, int L, void* ws, const Layout& ly, cudaStream_t s,
+                    const void* kvt_cached = nullptr, const void* kvi_cached = nullptr) {
   const int D = c->dim;
   const size_t es = dtype_size(c->dtype);
   const int M = B * L;
@@ -257,10 +260,16 @@ int cross_attn_impl(const wan_dit_config* c, const void* h, const void* ctx, int
   const bool with_img = img && Li > 0;
   const int ow = with_img ? 2 * D : D;
   WAN_TRY(gemm(c, h, D, w->w_cq, w->b_cq, q, M, D, D, 0, epi_store(D), s));
-  WAN_TRY(gemm(c, ctx, D, w->w_ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
+  if (kvt_cached)
+    kvt = const_cast<void*>(kvt_cached);
+  else
+    WAN_TRY(gemm(c, ctx, D, w->w_ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
   WAN_TRY(attention(c, {q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, L, Lc, s));
   if (with_img) {
-    WAN_TRY(gemm(c, img, D, w->w_ckv_img, w->b_ckv_img, kvi, B * Li, 2 * D, D, 0, epi_store(2 * D), s));
+    if (kvi_cached)
+      kvi = const_cast<void*>(kvi_cached);
+    else
+      WAN_TRY(gemm(c, img, D, w->w_ckv_img, w->b_ckv_img, kvi, B * Li, 2 * D, D, 0, epi_store(2 * D), s));
     WAN_TRY(attention(c, {q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, L, Li, s));
     // (o_text + o_image) Wco^T as one reduction over [o_text | o_image] with Wco reused.
     return gemm(c, ocat, ow, w->w_co, w->b_co, x, M, D, 2 * D, D, epi_residual(D, nullptr, nullptr, 0, L), s);
@@ -279,13 +288,14 @@ int ffn_impl(const wan_dit_config* c, const void* h, const wan_block_weights* w,
 }
 
 int block_impl(const wan_dit_config* c, float* x, const float* e, const void* ctx, int Lc, const void* img, int Li,
-               const wan_block_weights* w, int B, int L, void* ws, const Layout& ly, cudaStream_t s) {
+               const wan_block_weights* w, int B, int L, void* ws, const Layout& ly, cudaStream_t s,
+               const void* kvt_cached = nullptr, const void* kvi_cached = nullptr) {
   void* h = at(ws, ly.h);
   const int64_t rows = static_cast<int64_t>(B) * L;
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 0, h, c->dtype, c->eps, s));
   WAN_TRY(self_attn_impl(c, h, w, e, x, B, L, ws, ly, s));
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, nullptr, nullptr, -1, h, c->dtype, c->eps, s));
-  WAN_TRY(cross_attn_impl(c, h, ctx, Lc, img, Li, w, x, B, L, ws, ly, s));
+  WAN_TRY(cross_attn_impl(c, h, ctx, Lc, img, Li, w, x, B, L, ws, ly, s, kvt_cached, kvi_cached));
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 1, h, c->dtype, c->eps, s));
   return ffn_impl(c, h, w, e, x, B, L, ws, ly, s);
 }
@@ -304,6 +314,50 @@ int head_impl(const wan_dit_config* c, const float* x, int B, int F, int H, int 
   ep.sc_H = H;
   ep.sc_W = W;
   return gemm(c, h, c->dim, w_head, b_head, v_out, B * L, c->out_ch * 4, c->dim, 0, ep, s);
+}
+
+// patchify -> timestep MLP -> blocks -> head. kvt/kvi: per-block cached cross-attention
+// K|V (arrays of n_blocks pointers) or NULL.
+int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H, int W,
+               const float* t, const wan_stack_weights* sw, const wan_block_weights* blocks, const void* ctx, int Lc,
+               const void* img_ctx, int li, float* v_out, void* workspace, const Layout& ly, cudaStream_t s,
+               const void* const* kvt, const void* const* kvi) {
+  const int L = F * (H / 2) * (W / 2);
+  float* x = reinterpret_cast<float*>(at(workspace, ly.x));
+  float* e = reinterpret_cast<float*>(at(workspace, ly.e));
+  void* patches = at(workspace, ly.big);
+  const int K = cfg->in_ch * 4;
+  WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, patches, cfg->dtype, s));
+  WAN_TRY(gemm(cfg, patches, K, sw->w_p, sw->b_p, x, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s));
+  WAN_TRY(launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, sw->time.w_t1, sw->time.b_t1, sw->time.w_t2, sw->time.b_t2,
+                          e, cfg->dtype, s));
+  for (int i = 0; i < n_blocks; ++i)
+    WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s, kvt ? kvt[i] : nullptr,
+                       kvi ? kvi[i] : nullptr));
+  return head_impl(cfg, x, B, F, H, W, sw->w_head, sw->b_head, v_out, at(workspace, ly.h), s);
+}
+
+// Sampler workspace: the stack's workspace for 2B samples, the 2B-sample DiT input, the
+// 2B velocities (fp32), the 2B timesteps, and per block the cached text and image K|V
+// of both contexts.
+struct SampleLayout {
+  size_t in2, v, t, kvt, kvi, total;
+  size_t kvt_block, kvi_block;  // bytes per block
+};
+SampleLayout sample_layout(const wan_dit_config* c, int n_blocks, int B, int F, int H, int W, int Lc, int Li) {
+  const size_t es = dtype_size(c->dtype);
+  const int L = F * (H / 2) * (W / 2);
+  const size_t fhw = static_cast<size_t>(F) * H * W;
+  SampleLayout l;
+  l.in2 = align_up(layout(c, 2 * B, L, Lc, Li).total);
+  l.v = l.in2 + align_up(2 * static_cast<size_t>(B) * c->in_ch * fhw * es);
+  l.t = l.v + align_up(2 * static_cast<size_t>(B) * c->out_ch * fhw * 4);
+  l.kvt = l.t + align_up(2 * static_cast<size_t>(B) * 4);
+  l.kvt_block = align_up(2 * static_cast<size_t>(B) * Lc * 2 * c->dim * es);
+  l.kvi_block = align_up(2 * static_cast<size_t>(B) * Li * 2 * c->dim * es);
+  l.kvi = l.kvt + static_cast<size_t>(n_blocks) * l.kvt_block;
+  l.total = l.kvi + static_cast<size_t>(n_blocks) * l.kvi_block;
+  return l;
 }
 
 int check_tokens(const wan_dit_config* c, int B, int L, int Lc, int Li) {
@@ -491,19 +545,84 @@ int wan_dit_stack_fwd(const wan_dit_config* cfg, int n_blocks, const void* laten
   const int li = with_img ? Li : 0;
   WAN_TRY(check_tokens(cfg, B, L, Lc, li));
   WAN_TRY(check_ws(cfg, workspace, ws_bytes, B, L, Lc, li));
-  const Layout ly = layout(cfg, B, L, Lc, li);
+  return stack_impl(cfg, n_blocks, latent, B, F, H, W, t, sw, blocks, ctx, Lc, img_ctx, li, v_out, workspace,
+                    layout(cfg, B, L, Lc, li), as_stream(stream), nullptr, nullptr);
+}
+
+size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W, int Lc,
+                                  int Li) {
+  if (check_cfg(cfg) != WAN_OK || n_blocks < 0 || B < 0 || F < 0 || H < 0 || W < 0 || Lc < 0 || Li < 0) return 0;
+  return sample_layout(cfg, n_blocks, B, F, H, W, Lc, Li).total;
+}
+
+int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* input, int B, int F, int H, int W,
+                         int n_steps, float guidance, const wan_stack_weights* sw, const wan_block_weights* blocks,
+                         const void* ctx_cond, const void* ctx_uncond, int Lc, const void* img_ctx, int Li,
+                         float* latent_out, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  WAN_REQUIRE(sw && (blocks || n_blocks == 0), WAN_ERR_NULL);
+  WAN_REQUIRE(n_blocks >= 0 && n_steps >= 1 && guidance == guidance && guidance - guidance == 0.0f, WAN_ERR_SHAPE);
+  WAN_REQUIRE(B >= 0 && F >= 1 && H >= 2 && W >= 2 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(cfg->out_ch <= cfg->in_ch && Lc > 0, WAN_ERR_SHAPE);
+  const bool with_img = img_ctx && Li > 0;
+  for (int i = 0; i < n_blocks; ++i) WAN_TRY(check_block_w(cfg, &blocks[i], with_img));
+  WAN_TRY(check_ptr(input));
+  WAN_TRY(check_ptr(ctx_cond));
+  WAN_TRY(check_ptr(ctx_uncond));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_TRY(check_ptr(latent_out));
+  WAN_TRY(check_ptr(sw->w_p));
+  WAN_TRY(check_opt_ptr(sw->b_p));
+  WAN_TRY(check_ptr(sw->w_head));
+  WAN_TRY(check_opt_ptr(sw->b_head));
+  WAN_TRY(check_ptr(sw->time.w_t1));
+  WAN_TRY(check_ptr(sw->time.w_t2));
+  WAN_TRY(check_ptr(sw->time.b_t1));
+  WAN_TRY(check_ptr(sw->time.b_t2));
+  WAN_TRY(check_ptr(workspace));
+  const int L = F * (H / 2) * (W / 2);
+  const int li = with_img ? Li : 0;
+  WAN_TRY(check_tokens(cfg, 2 * B, L, Lc, li));
+  const SampleLayout sl = sample_layout(cfg, n_blocks, B, F, H, W, Lc, li);
+  WAN_REQUIRE(ws_bytes >= sl.total, WAN_ERR_WORKSPACE);
+  if (B == 0) return WAN_OK;
   cudaStream_t s = as_stream(stream);
-  float* x = reinterpret_cast<float*>(at(workspace, ly.x));
-  float* e = reinterpret_cast<float*>(at(workspace, ly.e));
-  void* patches = at(workspace, ly.big);
-  const int K = cfg->in_ch * 4;
-  WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, patches, cfg->dtype, s));
-  WAN_TRY(gemm(cfg, patches, K, sw->w_p, sw->b_p, x, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s));
-  WAN_TRY(launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, sw->time.w_t1, sw->time.b_t1, sw->time.w_t2, sw->time.b_t2,
-                          e, cfg->dtype, s));
-  for (int i = 0; i < n_blocks; ++i)
-    WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s));
-  return head_impl(cfg, x, B, F, H, W, sw->w_head, sw->b_head, v_out, at(workspace, ly.h), s);
+  const int D = cfg->dim;
+  const size_t es = dtype_size(cfg->dtype);
+  const int64_t fhw = static_cast<int64_t>(F) * H * W;
+  const int64_t n = cfg->out_ch * fhw, in_stride = cfg->in_ch * fhw;
+  void* in2 = at(workspace, sl.in2);
+  float* v = reinterpret_cast<float*>(at(workspace, sl.v));
+  float* t = reinterpret_cast<float*>(at(workspace, sl.t));
+  WAN_TRY(launch_sampler_init(input, B, n, in_stride, latent_out, in2, t, cfg->dtype, s));
+  // Cross-attention K|V of both contexts, once per block for all steps.
+  std::vector<const void*> kvt(n_blocks), kvi(n_blocks, nullptr);
+  for (int i = 0; i < n_blocks; ++i) {
+    uint8_t* ct = at(workspace, sl.kvt + i * sl.kvt_block);
+    const size_t half_t = static_cast<size_t>(B) * Lc * 2 * D * es;
+    WAN_TRY(gemm(cfg, ctx_cond, D, blocks[i].w_ckv, blocks[i].b_ckv, ct, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
+    WAN_TRY(gemm(cfg, ctx_uncond, D, blocks[i].w_ckv, blocks[i].b_ckv, ct + half_t, B * Lc, 2 * D, D, 0,
+                 epi_store(2 * D), s));
+    kvt[i] = ct;
+    if (with_img) {
+      uint8_t* ci = at(workspace, sl.kvi + i * sl.kvi_block);
+      const size_t half_i = static_cast<size_t>(B) * li * 2 * D * es;
+      for (int h = 0; h < 2; ++h)
+        WAN_TRY(gemm(cfg, img_ctx, D, blocks[i].w_ckv_img, blocks[i].b_ckv_img, ci + h * half_i, B * li, 2 * D, D,
+                     0, epi_store(2 * D), s));
+      kvi[i] = ci;
+    }
+  }
+  const Layout ly = layout(cfg, 2 * B, L, Lc, li);
+  const float dt = 1.0f / static_cast<float>(n_steps);
+  for (int k = 0; k < n_steps; ++k) {
+    WAN_TRY(stack_impl(cfg, n_blocks, in2, 2 * B, F, H, W, t, sw, blocks, ctx_cond, Lc,
+                       with_img ? img_ctx : nullptr, li, v, workspace, ly, s,
+                       n_blocks ? kvt.data() : nullptr, with_img && n_blocks ? kvi.data() : nullptr));
+    const float t_next = static_cast<float>(1000.0 * (k + 1) / n_steps);
+    WAN_TRY(launch_euler_cfg(v, B, n, in_stride, dt, guidance, latent_out, in2, t, t_next, cfg->dtype, s));
+  }
+  return WAN_OK;
 }
 
 int wan_head_fwd(const wan_dit_config* cfg, const float* x, int B, int F, int H, int W, const void* w_head,

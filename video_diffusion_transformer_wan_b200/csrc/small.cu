@@ -233,6 +233,46 @@ __global__ void __launch_bounds__(256) flow_loss_kernel(const float* __restrict_
   }
 }
 
+// Sampler set-up: the 2B-sample DiT input (both halves = the caller's input, which
+// holds the noise in its first n elements per sample and, for I2V, fixed condition
+// channels after them), the fp32 state x = noise, and the timestep of step 0.
+template <typename T>
+__global__ void sampler_init_kernel(const T* __restrict__ input, int B, int64_t n, int64_t in_stride,
+                                    float* __restrict__ x, T* __restrict__ in2, float* __restrict__ t) {
+  const int64_t total = static_cast<int64_t>(B) * in_stride;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = idx / in_stride, i = idx % in_stride;
+    const T v = input[idx];
+    in2[idx] = v;
+    in2[static_cast<int64_t>(B) * in_stride + idx] = v;
+    if (i < n) x[b * n + i] = ld(input, idx);
+    if (idx < 2 * B) t[idx] = 0.0f;
+  }
+}
+
+// One guided Euler step: x += dt * (v_u + g (v_c - v_u)) with v = [v_c (B samples) |
+// v_u (B samples)]; the new x (rounded to the activation type) goes into the first n
+// elements of both halves of the next DiT input, and the timestep becomes t_next.
+template <typename T>
+__global__ void euler_cfg_kernel(const float* __restrict__ v, int B, int64_t n, int64_t in_stride, float dt,
+                                 float g, float* __restrict__ x, T* __restrict__ in2, float* __restrict__ t,
+                                 float t_next) {
+  const int64_t total = static_cast<int64_t>(B) * n;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t b = idx / n, i = idx % n;
+    const float vc = v[idx];
+    const float vu = v[total + idx];
+    const float xv = x[idx] + dt * (vu + g * (vc - vu));
+    x[idx] = xv;
+    const T xt = cvt<T>(xv);
+    in2[b * in_stride + i] = xt;
+    in2[(b + B) * in_stride + i] = xt;
+    if (idx < 2 * B) t[idx] = t_next;
+  }
+}
+
 unsigned grid_for(int64_t total, int threads) {
   int64_t g = (total + threads - 1) / threads;
   if (g > 148 * 64) g = 148 * 64;
@@ -240,6 +280,38 @@ unsigned grid_for(int64_t total, int threads) {
 }
 
 }  // namespace
+
+int launch_sampler_init(const void* input, int B, int64_t n, int64_t in_stride, float* x, void* in2, float* t,
+                        int dtype, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(B) * in_stride;
+  if (total == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s, static_cast<double>(total) * dtype_size(dtype) * 3.0);
+  if (dtype == WAN_BF16)
+    sampler_init_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(input), B, n, in_stride, x, static_cast<__nv_bfloat16*>(in2), t);
+  else
+    sampler_init_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(static_cast<const float*>(input), B, n,
+                                                                    in_stride, x, static_cast<float*>(in2), t);
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
+
+int launch_euler_cfg(const float* v, int B, int64_t n, int64_t in_stride, float dt, float g, float* x, void* in2,
+                     float* t, float t_next, int dtype, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(B) * n;
+  if (total == 0) return WAN_OK;
+  trace_launch_begin(WAN_KIND_SMALL, s, static_cast<double>(total) * (16.0 + 2.0 * dtype_size(dtype)));
+  if (dtype == WAN_BF16)
+    euler_cfg_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
+        v, B, n, in_stride, dt, g, x, static_cast<__nv_bfloat16*>(in2), t, t_next);
+  else
+    euler_cfg_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(v, B, n, in_stride, dt, g, x,
+                                                                 static_cast<float*>(in2), t, t_next);
+  int st = check_launch();
+  trace_launch_end(WAN_KIND_SMALL, s);
+  return st;
+}
 
 int launch_patch_gather(const void* latent, int B, int C, int F, int H, int W, void* patches, int dtype,
                         cudaStream_t s) {

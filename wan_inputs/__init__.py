@@ -131,7 +131,7 @@ def _normal(rng: np.random.Generator, shape, std: float) -> np.ndarray:
 
 
 def make_inputs(w: Workload, seed: int = 0, *, n_blocks: Optional[int] = None,
-                zero_wx: bool = True, block_input: bool = True) -> Dict[str, object]:
+                zero_wx: bool = True, block_input: bool = True, uncond: bool = False) -> Dict[str, object]:
     """Draw every tensor of a workload, in this fixed order:
 
     1. latent noise ``[B,16,F,H,W]`` ~ N(0,1)
@@ -149,6 +149,9 @@ def make_inputs(w: Workload, seed: int = 0, *, n_blocks: Optional[int] = None,
     10. head: ``w_head [64,D]``, ``b_head [64]``
     11. (block_input) a residual-stream block input ``x [B,L,D]`` ~ N(0,1) fp32 and a
         shared-MLP output ``e [B,6,D]`` ~ N(0,0.2) fp32, for the block-level sub-calls.
+    12. (uncond) a second text context ``ctx_uncond [B,Lc,D]`` ~ N(0,1), the
+        unconditional branch of guided sampling (drawn last so that it leaves every
+        other tensor of the seed unchanged).
 
     Weights and biases (except ``mod_bias``), latents, context and image features are
     rounded to bf16 for bf16 workloads; everything stays fp32 for f32 workloads.
@@ -207,6 +210,8 @@ def make_inputs(w: Workload, seed: int = 0, *, n_blocks: Optional[int] = None,
     if block_input:
         out["x"] = _normal(rng, (B, L, D), 1.0)
         out["e"] = _normal(rng, (B, 6, D), 0.2)
+    if uncond:
+        out["ctx_uncond"] = rb(_normal(rng, (B, w.text_len, D), 1.0))
     return out
 
 
