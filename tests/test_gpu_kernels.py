@@ -184,6 +184,36 @@ def test_attention_planted_peak_and_strided_layout(wan):
     assert rel_err(got[0, rows, D:], ref[rows]) <= BF16_TOL
 
 
+def test_attention_running_max_jumps(wan):
+    """Rows whose score maximum jumps up in later key tiles, by less and by more than the
+    kernel's lazy-rescale threshold (2^8 in exp2 units, 62.7 in raw logits at d = 128),
+    so the running base moves (O and the sum rescaled) once or several times per row."""
+    r = rng(13)
+    B, Lq, H, d = 1, 256, 1, 128
+    Lk = 4 * 128 + 50
+    q = r.standard_normal((B, Lq, d))
+    k = r.standard_normal((B, Lk, d))
+    v = r.standard_normal((B, Lk, d))
+    plan = {3: [(150, 60.0)], 40: [(130, 80.0), (300, 200.0)], 130: [(260, 70.0), (400, 150.0), (555, 300.0)],
+            255: [(520, 90.0), (521, 90.0)]}
+    for i, keys in plan.items():
+        qi = q[0, i]
+        for j, logit in keys:
+            k[0, j] = logit * qi * math.sqrt(d) / qi.dot(qi)
+    q, k, v = (round_bf16(a) for a in (q, k, v))
+    cfg = _cfg(wan, "bf16", D=d, heads=H)
+    o = torch.empty(B, Lq, d, dtype=torch.bfloat16, device="cuda")
+    wan.attention_fwd(cfg, dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), o, H, d)
+    torch.cuda.synchronize()
+    got = host(o)
+    ref = O.attention(q[0], k[0], v[0], H)
+    assert rel_err(got[0], ref) <= BF16_TOL
+    rows = sorted(plan)
+    assert rel_err(got[0, rows], ref[rows]) <= BF16_TOL
+    # row 255's two equal planted keys dominate: its output is their mean value
+    np.testing.assert_allclose(got[0, 255], 0.5 * (v[0, 520] + v[0, 521]), atol=2e-2)
+
+
 def test_attention_long_sequence_sampled_rows(wan):
     r = rng(12)
     B, L, H, d = 1, 4100, 1, 128

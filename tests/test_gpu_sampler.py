@@ -68,10 +68,9 @@ def test_sampler_matches_oracle(wan, i2v):
         e_x, e_d = rel_err(got[b], ref), rel_err(got[b] - x0, ref - x0)
         print(f"sampler i2v={i2v} b={b}: latent {e_x:.2e} displacement {e_d:.2e}")
         assert e_x <= BF16_TOL
-        # The step is x += dt (v_u + g (v_c - v_u)): an error of eps max|v| in each branch
-        # reaches the guided velocity as (|1 - g| + |g|) eps max|v| at most, which is
-        # about |g| times the bf16 bar when measured against the guided displacement.
-        assert e_d <= BF16_TOL * (abs(1 - g) + abs(g)) / 2
+        # The displacement sum_k dt (v_u + g (v_c - v_u)) is held to the same bf16 bar
+        # (guidance amplifies the branch difference, not the rounding of the stack).
+        assert e_d <= BF16_TOL
 
 
 @pytest.mark.parametrize("g", [1.0, 0.0])

@@ -15,6 +15,11 @@
 //             chunks taken in pairs (the fp32 residual of both chunks is loaded before
 //             either is updated) keep enough bytes in flight that the epilogue of one
 //             tile hides under the main loop of the next even when K is short.
+//
+// Tile order: the row blocks are cut into groups of group_m; within a group the row
+// block varies fastest, so the 148 tiles in flight share a slab of at most
+// group_m row blocks of A (sized to stay in L2) and a few column blocks of W, and each
+// operand comes from DRAM about once per group instead of once per wave.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -29,6 +34,9 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+#ifndef WAN_GEMM_SLAB_MB
+#define WAN_GEMM_SLAB_MB 32  // bytes of A (MiB) one tile group keeps resident in L2
+#endif
 
 template <int BN>
 struct GemmCfg {
@@ -45,6 +53,7 @@ struct GemmParams {
   int k_blocks;
   int wk_period_blocks;  // > 0: W column block = k block mod this
   int m_blocks, n_blocks;
+  int group_m;           // row blocks per tile group
   const __nv_bfloat16* bias;
   void* out;
   GemmEpi epi;
@@ -54,6 +63,17 @@ struct GemmParams {
 __device__ __forceinline__ float gelu_tanh_f(float v) {
   const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);
   return 0.5f * v * (1.0f + tanh_approx(u));
+}
+
+// Output tile -> (row block, column block), row block fastest within a group.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& mb, int& nb) {
+  const int per_group = p.group_m * p.n_blocks;
+  const int g = tile / per_group;
+  const int r = tile - g * per_group;
+  const int m_first = g * p.group_m;
+  const int gm = min(p.group_m, p.m_blocks - m_first);
+  mb = m_first + r % gm;
+  nb = r / gm;
 }
 
 // Apply the epilogue to 32 consecutive accumulator columns [n0, n0+32) of one row.
@@ -246,8 +266,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int m0 = (tile / p.n_blocks) * kBM;
-        const int n0 = (tile % p.n_blocks) * BN;
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
+        const int m0 = mb * kBM;
+        const int n0 = nb * BN;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
             ok = false;
@@ -317,8 +339,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int acc = it & 1;
       if (!mbar_wait_warp(&tfull[acc], (it >> 1) & 1, p.err)) break;
       tc_fence_after();
-      const int m0 = (tile / p.n_blocks) * kBM;
-      const int n0 = (tile % p.n_blocks) * BN + colhalf * (BN / 2);
+      int mb, nb;
+      tile_coords(p, tile, mb, nb);
+      const int m0 = mb * kBM;
+      const int n0 = nb * BN + colhalf * (BN / 2);
       const int row = m0 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + colhalf * (BN / 2));
@@ -383,6 +407,10 @@ int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void*
   p.wk_period_blocks = w_k_period > 0 ? w_k_period / kBK : 0;
   p.m_blocks = (M + kBM - 1) / kBM;
   p.n_blocks = (N + BN - 1) / BN;
+  {
+    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * 2 * kBM);
+    p.group_m = static_cast<int>(slab_rows < 1 ? 1 : (slab_rows > p.m_blocks ? p.m_blocks : slab_rows));
+  }
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.out = out;
   p.epi = epi;
