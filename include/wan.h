@@ -255,6 +255,43 @@ int wan_flow_matching_input(const wan_dit_config* cfg, const void* x1, const voi
 int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void* x1,
                            const void* x0, int B, int64_t n, float* loss_out, void* stream);
 
+/* ---- sequence parallelism (Ulysses) ------------------------------------------ */
+
+/* Self-attention of one block split over P = sp_size ranks along the token axis, the
+ * intra-machine layer of the pages' context parallelism [163.com article on Wan2.1,
+ * "核心创新三" (inference: context parallelism; inside a machine, Ulysses); Wan 2.1 page,
+ * "Infra" (2D CP = outer Ring Attention x inner Ulysses)]. Rank r owns tokens
+ * [r L/P, (r+1) L/P) of every sample, and heads [r H/P, (r+1) H/P) while attending.
+ * Everything except attention is row-local and uses the ordinary calls on L/P rows.
+ * The exchange is fused into the producing kernels: each call stores its results
+ * straight into the buffers of the ranks that consume them (pointers that may be peer
+ * GPUs' memory, e.g. CUDA IPC mappings over NVLink; on one GPU, local buffers). The
+ * caller orders the phases across ranks (all ranks finish phase 1 before any starts
+ * phase 2, and so on), e.g. with a one-element all-reduce on the stream.
+ * Requirements: bf16 config (WAN_ERR_UNSUPPORTED otherwise), 1 <= P <= 8, H % P == 0,
+ * L % P == 0, 0 <= sp_rank < P; pointer arrays are HOST arrays of P device pointers,
+ * each 16-byte aligned. Errors are returned before any launch. */
+
+/* Phase 1 - QKV projection and scatter: h [B, L/P, D] act (this rank's rows of the
+ * modulated LN output). Computes h Wqkv^T + b and stores, for every rank s, the q, k and
+ * v columns of s's heads into qkv_dst[s] [B, L, 3D/P] act (q | k | v slabs of D/P
+ * columns) at this rank's rows. */
+int wan_sp_qkv_fwd(const wan_dit_config* cfg, int sp_size, int sp_rank, const void* h, int B, int L,
+                   const wan_block_weights* w, void* const* qkv_dst, void* stream);
+
+/* Phase 2 - attention and gather: qkv [B, L, 3D/P] act (this rank's heads, all rows, as
+ * phase 1 left it). Attends over all L tokens and stores each row's output of this
+ * rank's heads into o_dst[owner] [B, L/P, D] act, columns [sp_rank D/P, (sp_rank+1) D/P),
+ * where owner = row / (L/P). */
+int wan_sp_attn_fwd(const wan_dit_config* cfg, int sp_size, int sp_rank, const void* qkv, int B, int L,
+                    void* const* o_dst, void* stream);
+
+/* Phase 3 - output projection with the gated residual on this rank's rows:
+ * x_inout [B, L/P, D] fp32 += gate_msa * (o Wo^T + bo), o [B, L/P, D] act from phase 2,
+ * gate_msa = e[b, 2] + w->mod_bias[2] (e [B, 6, D] fp32). */
+int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const wan_block_weights* w,
+                   const float* e, float* x_inout, int B, int L, void* stream);
+
 /* ---- sampling ----------------------------------------------------------------- */
 
 /* Device workspace (bytes) of wan_sample_euler_cfg for these sizes (0 on a bad cfg). */

@@ -18,7 +18,8 @@ __all__ = [
     "ImageMlpWeights", "StackWeights", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
     "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
-    "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
+    "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd",
+    "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
 LIB_PATH = os.environ.get("WAN_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
@@ -91,6 +92,9 @@ def _load() -> ctypes.CDLL:
         "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i]),
         "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
                                       P(BlockWeights), _vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+        "wan_sp_qkv_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(BlockWeights), P(_vp), _vp]),
+        "wan_sp_attn_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(_vp), _vp]),
+        "wan_sp_out_fwd": (_i, [P(Config), _i, _vp, P(BlockWeights), _vp, _vp, _i, _i, _vp]),
         "wan_launch_count": (_i64, []),
         "wan_trace_enable": (_i, [_i]),
         "wan_trace_reset": (_i, []),
@@ -244,6 +248,28 @@ def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, 
                                     ctypes.byref(sw), arr, _p(ctx_cond), _p(ctx_uncond), ctx_cond.shape[1],
                                     _p(img_ctx), Li, _p(latent_out), *_ws(ws), _stream(stream)),
            "wan_sample_euler_cfg")
+
+
+def _ptr_table(bufs):
+    return (_vp * len(bufs))(*[_p(b) for b in bufs])
+
+
+def sp_qkv_fwd(cfg, sp_size: int, sp_rank: int, h, L: int, bw: BlockWeights, qkv_dst, stream=None):
+    """h [B, L/P, D] (this rank's rows); qkv_dst: P buffers [B, L, 3D/P]."""
+    _check(_lib().wan_sp_qkv_fwd(ctypes.byref(cfg), sp_size, sp_rank, _p(h), h.shape[0], L, ctypes.byref(bw),
+                              _ptr_table(qkv_dst), _stream(stream)), "wan_sp_qkv_fwd")
+
+
+def sp_attn_fwd(cfg, sp_size: int, sp_rank: int, qkv, L: int, o_dst, stream=None):
+    """qkv [B, L, 3D/P] (this rank's heads); o_dst: P buffers [B, L/P, D]."""
+    _check(_lib().wan_sp_attn_fwd(ctypes.byref(cfg), sp_size, sp_rank, _p(qkv), qkv.shape[0], L,
+                               _ptr_table(o_dst), _stream(stream)), "wan_sp_attn_fwd")
+
+
+def sp_out_fwd(cfg, sp_size: int, o, bw: BlockWeights, e, x_inout, L: int, stream=None):
+    """o [B, L/P, D] act, x_inout [B, L/P, D] fp32, e [B, 6, D] fp32."""
+    _check(_lib().wan_sp_out_fwd(ctypes.byref(cfg), sp_size, _p(o), ctypes.byref(bw), _p(e), _p(x_inout),
+                              o.shape[0], L, _stream(stream)), "wan_sp_out_fwd")
 
 
 def attention_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0, o_col0=0, stream=None):

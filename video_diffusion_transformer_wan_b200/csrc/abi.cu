@@ -549,6 +549,71 @@ int wan_dit_stack_fwd(const wan_dit_config* cfg, int n_blocks, const void* laten
                     layout(cfg, B, L, Lc, li), as_stream(stream), nullptr, nullptr);
 }
 
+namespace {
+int check_sp(const wan_dit_config* cfg, int P, int r, int B, int L, void* const* ptrs) {
+  WAN_TRY(check_cfg(cfg, true));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  WAN_REQUIRE(P >= 1 && P <= kMaxSeqRanks && r >= 0 && r < P, WAN_ERR_SHAPE);
+  WAN_REQUIRE(cfg->heads % P == 0 && B >= 0 && L >= 0 && L % P == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(ptrs, WAN_ERR_NULL);
+  for (int s = 0; s < P; ++s) WAN_TRY(check_ptr(ptrs[s]));
+  return check_tokens(cfg, B, L, 0, 0);
+}
+}  // namespace
+
+int wan_sp_qkv_fwd(const wan_dit_config* cfg, int sp_size, int sp_rank, const void* h, int B, int L,
+                   const wan_block_weights* w, void* const* qkv_dst, void* stream) {
+  WAN_TRY(check_sp(cfg, sp_size, sp_rank, B, L, qkv_dst));
+  WAN_REQUIRE(w, WAN_ERR_NULL);
+  WAN_TRY(check_ptr(w->w_qkv));
+  WAN_TRY(check_opt_ptr(w->b_qkv));
+  WAN_TRY(check_ptr(h));
+  const int D = cfg->dim, Ll = L / sp_size;
+  if (B == 0 || L == 0) return WAN_OK;
+  GemmEpi ep = epi_store(3 * D / sp_size);
+  ep.kind = kEpiSeqScatter;
+  for (int s = 0; s < sp_size; ++s) ep.sp_dst[s] = qkv_dst[s];
+  ep.sp_rows_local = Ll;
+  ep.sp_rows_total = L;
+  ep.sp_row_off = sp_rank * Ll;
+  ep.sp_part_cols = D;
+  ep.sp_rank_cols = D / sp_size;
+  return gemm(cfg, h, D, w->w_qkv, w->b_qkv, nullptr, B * Ll, 3 * D, D, 0, ep, as_stream(stream));
+}
+
+int wan_sp_attn_fwd(const wan_dit_config* cfg, int sp_size, int sp_rank, const void* qkv, int B, int L,
+                    void* const* o_dst, void* stream) {
+  WAN_TRY(check_sp(cfg, sp_size, sp_rank, B, L, o_dst));
+  WAN_TRY(check_ptr(qkv));
+  const int D = cfg->dim, Dl = D / sp_size;
+  if (B == 0 || L == 0) return WAN_OK;
+  SeqScatter sc{};
+  sc.ranks = sp_size;
+  sc.rows_local = L / sp_size;
+  for (int s = 0; s < sp_size; ++s) sc.dst[s] = o_dst[s];
+  return launch_attn_tc({qkv, 3 * Dl, 0}, {qkv, 3 * Dl, Dl}, {qkv, 3 * Dl, 2 * Dl}, nullptr, D, sp_rank * Dl, B,
+                        cfg->heads / sp_size, L, L, as_stream(stream), &sc);
+}
+
+int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const wan_block_weights* w,
+                   const float* e, float* x_inout, int B, int L, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  WAN_REQUIRE(sp_size >= 1 && sp_size <= kMaxSeqRanks && L % sp_size == 0 && B >= 0 && L >= 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(w, WAN_ERR_NULL);
+  WAN_TRY(check_ptr(w->w_o));
+  WAN_TRY(check_opt_ptr(w->b_o));
+  WAN_TRY(check_opt_ptr(w->mod_bias));
+  WAN_TRY(check_ptr(o));
+  WAN_TRY(check_ptr(e));
+  WAN_TRY(check_ptr(x_inout));
+  const int D = cfg->dim, Ll = L / sp_size;
+  if (B == 0 || L == 0) return WAN_OK;
+  const float* gb = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
+  return gemm(cfg, o, D, w->w_o, w->b_o, x_inout, B * Ll, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, Ll),
+              as_stream(stream));
+}
+
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W, int Lc,
                                   int Li) {
   if (check_cfg(cfg) != WAN_OK || n_blocks < 0 || B < 0 || F < 0 || H < 0 || W < 0 || Lc < 0 || Li < 0) return 0;

@@ -63,6 +63,7 @@ struct AttnParams {
   int64_t o_row_stride;
   int64_t o_batch_stride;
   int o_col0;
+  SeqScatter sc;  // sc.ranks > 0: rows go to their owners' buffers
   int* err;
 };
 
@@ -319,8 +320,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const int grow = q0 + t * kTile + row;
-      __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride +
-                            static_cast<int64_t>(grow) * p.o_row_stride + p.o_col0 + h * kHd;
+      __nv_bfloat16* orow;
+      if (p.sc.ranks > 0) {
+        const int owner = min(grow / p.sc.rows_local, p.sc.ranks - 1);
+        const int64_t lrow = static_cast<int64_t>(b) * p.sc.rows_local + (grow - owner * p.sc.rows_local);
+        orow = static_cast<__nv_bfloat16*>(p.sc.dst[owner]) + lrow * p.o_row_stride + p.o_col0 + h * kHd;
+      } else {
+        orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride + static_cast<int64_t>(grow) * p.o_row_stride +
+               p.o_col0 + h * kHd;
+      }
 #pragma unroll
       for (int c = 0; c < kHd / 64; ++c) {
         uint32_t r0[32], r1[32];
@@ -367,7 +375,7 @@ bool make_operand_map(CUtensorMap* map, const AttnOperand& op, int B, int L) {
 }  // namespace
 
 int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0, int B,
-                   int H, int Lq, int Lk, cudaStream_t s) {
+                   int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc) {
   if (B == 0 || Lq == 0) return WAN_OK;
   if (Lk <= 0) return WAN_ERR_SHAPE;
   if (q.row_stride % 8 || k.row_stride % 8 || v.row_stride % 8 || o_row_stride % 8) return WAN_ERR_ALIGN;
@@ -387,6 +395,10 @@ int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t
   p.o_row_stride = o_row_stride;
   p.o_batch_stride = o_row_stride * Lq;
   p.o_col0 = o_col0;
+  p.sc = sc ? *sc : SeqScatter{};
+  if (sc && (sc->ranks < 1 || sc->ranks > kMaxSeqRanks || sc->rows_local < 1 ||
+             static_cast<int64_t>(sc->rows_local) * sc->ranks < Lq))
+    return WAN_ERR_SHAPE;
   p.err = device_error_flag();
   static std::once_flag once[64];
   int dev = 0;

@@ -104,12 +104,23 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
     }
   }
   const int kind = p.epi.kind;
-  if (kind == WAN_EPI_STORE || kind == WAN_EPI_GELU) {
+  if (kind == WAN_EPI_STORE || kind == WAN_EPI_GELU || kind == kEpiSeqScatter) {
     if (kind == WAN_EPI_GELU) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_f(v[i]);
     }
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+    __nv_bfloat16* o;
+    if (kind == kEpiSeqScatter) {
+      // The 32 columns lie inside one head, hence inside one destination rank's slab.
+      const int b = row / p.epi.sp_rows_local, i = row - b * p.epi.sp_rows_local;
+      const int part = n0 / p.epi.sp_part_cols, c = n0 - part * p.epi.sp_part_cols;
+      const int s = c / p.epi.sp_rank_cols;
+      const int64_t drow = static_cast<int64_t>(b) * p.epi.sp_rows_total + p.epi.sp_row_off + i;
+      o = static_cast<__nv_bfloat16*>(p.epi.sp_dst[s]) + drow * p.epi.ldo + part * p.epi.sp_rank_cols +
+          (c - s * p.epi.sp_rank_cols);
+    } else {
+      o = static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
+    }
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       if (n0 + g * 8 < p.N) {

@@ -35,6 +35,8 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
 int launch_layernorm(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias,
                      int chunk, void* out, int dtype, float eps, cudaStream_t s);
 
+constexpr int kMaxSeqRanks = 8;  // sequence-parallel group size limit
+
 struct GemmEpi {
   int kind;                 // wan_epilogue
   const float* gate;        // RESIDUAL: gate[(m / rows_per_batch) * gate_bstride + n]
@@ -44,8 +46,14 @@ struct GemmEpi {
   int64_t ldo;              // output row stride (elements)
   // head scatter (kind == kEpiHeadScatter): out[b, c, f, 2i+ph, 2j+pw]
   int sc_F, sc_H, sc_W, sc_C;
+  // sequence-parallel scatter (kind == kEpiSeqScatter, a bf16 store): local row
+  // m = b*sp_rows_local + i goes to row b*sp_rows_total + sp_row_off + i of rank s's
+  // buffer sp_dst[s]; column n = part*sp_part_cols + s*sp_rank_cols + c goes to column
+  // part*sp_rank_cols + c there (row stride ldo = parts * sp_rank_cols).
+  void* sp_dst[kMaxSeqRanks];
+  int sp_rows_local, sp_rows_total, sp_row_off, sp_part_cols, sp_rank_cols;
 };
-enum : int { kEpiHeadScatter = 100 };
+enum : int { kEpiHeadScatter = 100, kEpiSeqScatter = 101 };
 
 // bf16 tcgen05 GEMM: out = epi(A[M,K] W[N,K]^T + bias). A's rows have stride lda
 // elements; W has K columns (row stride K). If w_k_period > 0, W has w_k_period
@@ -61,9 +69,17 @@ struct AttnOperand {
   int64_t row_stride;  // elements
   int col0;            // column of head 0
 };
-// bf16 tcgen05 flash attention, head_dim 128.
+// Sequence-parallel output scatter: query row l of sample b goes to rank
+// r = l / rows_local, row b*rows_local + (l - r*rows_local) of dst[r].
+struct SeqScatter {
+  int ranks;
+  int rows_local;
+  void* dst[kMaxSeqRanks];
+};
+// bf16 tcgen05 flash attention, head_dim 128. With sc, o is ignored and each output row
+// is written to its owner's buffer (row stride o_row_stride, columns from o_col0).
 int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
-                   int B, int H, int Lq, int Lk, cudaStream_t s);
+                   int B, int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc = nullptr);
 // fp32 SIMT attention, head_dim <= 128, Lk <= 8192.
 int launch_attn_simt(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
                      int B, int H, int Lq, int Lk, int d, cudaStream_t s);

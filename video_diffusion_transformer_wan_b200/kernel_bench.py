@@ -4,8 +4,12 @@ command the committed ncu summaries were captured with.
   python -m video_diffusion_transformer_wan_b200.kernel_bench attention --L 32760 --heads 12
   python -m video_diffusion_transformer_wan_b200.kernel_bench gemm --M 32760 --N 4608 --K 1536 --epi store
   python -m video_diffusion_transformer_wan_b200.kernel_bench layernorm --L 32760 --dim 1536
+  python -m video_diffusion_transformer_wan_b200.kernel_bench sample --blocks 30 --steps 2
 
-Inputs are random device tensors (the kernels' timing does not depend on values).
+Inputs are random device tensors (the kernels' timing does not depend on values); the
+``sample`` mode draws the 1.3B 480P workload's seeded weights and times the guided
+Euler loop (one call of ``steps`` steps, conditional and unconditional branches as one
+batch of two).
 Prints one JSON line with the per-launch time and the achieved rate.
 """
 from __future__ import annotations
@@ -31,9 +35,38 @@ def _time(fn, iters: int, warmup: int) -> float:
     return a.elapsed_time(b) / max(iters, 1)
 
 
+def _sample(a) -> dict:
+    import dataclasses
+
+    from wan_inputs import WORKLOADS, make_inputs
+
+    from .model import DitModel, config_for, to_device
+    w = dataclasses.replace(WORKLOADS["wan13b_480p_block"], n_blocks=a.blocks)
+    inp = make_inputs(w, seed=0, block_input=False, uncond=True)
+    cfg = config_for(w)
+    model = DitModel(cfg, inp)
+    B, F, H, W, L, D = w.batch, w.frames, w.height, w.width, w.tokens, w.dim
+    noise = to_device(inp["noise"], model.act)
+    ctx, ctx_u = to_device(inp["ctx"], model.act), to_device(inp["ctx_uncond"], model.act)
+    out = torch.empty(B, w.out_ch, F, H, W, dtype=torch.float32, device="cuda")
+    ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len), dtype=torch.uint8,
+                     device="cuda")
+    ms = _time(lambda: wan.sample_euler_cfg(cfg, noise, a.steps, a.guidance, model.stack_table,
+                                            model.block_tables, ctx, ctx_u, None, out, ws), a.iters, a.warmup)
+    Lc, Fd = w.text_len, w.ffn
+    # per step; the text K|V projections are made once per call and not counted
+    block = 2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * L * Lc * D + 4 * L * D * Fd
+    flops_step = 2 * B * (a.blocks * block + 2 * L * D * 64 * 2)
+    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, ms_per_call=ms, ms_per_euler_step=ms / a.steps,
+                latent_tokens_per_s=B * L * a.steps / (ms / 1e3), tflops=flops_step * a.steps / ms / 1e9)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm"])
+    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample"])
+    ap.add_argument("--blocks", type=int, default=30, help="sample: DiT blocks")
+    ap.add_argument("--steps", type=int, default=2, help="sample: Euler steps per call")
+    ap.add_argument("--guidance", type=float, default=5.0)
     ap.add_argument("--L", type=int, default=32760)
     ap.add_argument("--Lk", type=int, default=0, help="key length (default: L, self-attention)")
     ap.add_argument("--heads", type=int, default=12)
@@ -76,6 +109,8 @@ def main(argv=None):
         ms = _time(lambda: wan.linear_fwd(cfg, A, W, bias, C, epi, rows_per_batch=a.M), a.iters, a.warmup)
         flops = 2.0 * a.M * a.N * a.K
         out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, ms=ms, tflops=flops / ms / 1e9)
+    elif a.kernel == "sample":
+        out.update(_sample(a))
     else:
         cfg = wan.make_config(a.dim, a.dim // 64, a.dim)
         x = torch.randn(1, a.L, a.dim, device="cuda", generator=g)
