@@ -184,9 +184,8 @@ def attention(q, k, v, heads: int) -> np.ndarray:
 # Block branches
 # --------------------------------------------------------------------------------------
 
-def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
-                          kv_source=None) -> np.ndarray:
-    """Self-attention sub-layer output before the gate: ``attn(h Wq, h Wk, h Wv) Wo^T + bo``.
+def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None) -> np.ndarray:
+    """The attention output ``attn(h Wq, h Wk, h Wv)`` before the output projection.
     The fused QKV weight ``w_qkv [3D, D]`` is stacked (q, k, v). ``kv_source`` (all rows
     of h) lets the caller evaluate only some query rows; by default it is ``h``."""
     h = _f(h)
@@ -196,7 +195,16 @@ def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
     q = linear(h, wqkv[:D], bqkv[:D])
     k = linear(src, wqkv[D:2 * D], bqkv[D:2 * D])
     v = linear(src, wqkv[2 * D:], bqkv[2 * D:])
-    o = attention(q, k, v, heads)
+    return attention(q, k, v, heads)
+
+
+def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
+                          kv_source=None, o=None) -> np.ndarray:
+    """Self-attention sub-layer output before the gate: ``attn(h Wq, h Wk, h Wv) Wo^T + bo``.
+    ``o`` replaces the attention output when given (an output kept from an earlier
+    sampling step, see ``dit_block``'s ``attn_cache``)."""
+    if o is None:
+        o = self_attention_core(h, w, heads, kv_source)
     return linear(o, w["w_o"], w["b_o"])
 
 
@@ -226,7 +234,7 @@ def ffn_branch(h, w: Dict[str, np.ndarray]) -> np.ndarray:
 
 def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6,
               img_ctx=None, rows: Optional[Sequence[int]] = None,
-              return_parts: bool = False):
+              return_parts: bool = False, attn_cache: Optional[Dict] = None):
     """One DiT block [Wan-P2, "Diffusion Transformer"]:
 
     1. ``x += gate_msa * SelfAttn(LN(x) (1 + scale_msa) + shift_msa)``
@@ -242,6 +250,12 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
     self-attention is row-local, and self-attention still takes keys and values from
     all rows. Returns ``x_out`` (of the selected rows), and with ``return_parts``
     also a dict of intermediates for those rows.
+
+    ``attn_cache`` (the attention cache of a sampling loop, see
+    ``sample_euler_cfg_cached``): a dict whose ``"o"`` holds this block's last computed
+    attention output. With ``attn_cache["reuse"]`` true that output replaces the
+    attention (q, k and v are not formed); otherwise the attention is computed and
+    stored in ``attn_cache["o"]``.
     """
     x = _f(x)
     mod = block_modulation(e, w["mod_bias"])
@@ -253,7 +267,13 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
         rows = np.asarray(rows)
         xr, hr = x[rows], h_all[rows]
     parts = {"h_msa": hr}
-    sa = self_attention_branch(hr, w, heads, kv_source=h_all)
+    if attn_cache is not None and attn_cache.get("reuse"):
+        sa = self_attention_branch(hr, w, heads, o=attn_cache["o"])
+    else:
+        o = self_attention_core(hr, w, heads, kv_source=h_all)
+        if attn_cache is not None:
+            attn_cache["o"] = o
+        sa = self_attention_branch(hr, w, heads, o=o)
     parts["sa"] = sa
     x1 = xr + gate_msa * sa
     hc = layer_norm(x1, eps)
@@ -321,17 +341,20 @@ def flow_matching_target(x1, x0) -> np.ndarray:
 
 
 def dit_stack(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, heads: int,
-              eps: float = 1e-6, img_ctx=None, freq_dim: int = 256) -> np.ndarray:
+              eps: float = 1e-6, img_ctx=None, freq_dim: int = 256,
+              attn_caches: Optional[Sequence[Dict]] = None) -> np.ndarray:
     """Whole DiT on one sample [Wan-P2, "Diffusion Transformer"]: patchify -> the time
     MLP shared by all blocks -> N blocks (each with its own modulation bias) -> head ->
     unpatchify. ``weights`` holds ``w_p, b_p, w_t1, b_t1, w_t2, b_t2, w_head, b_head``.
+    ``attn_caches`` gives each block its attention cache (see ``dit_block``).
     Returns the predicted velocity ``[out_ch, F, H, W]``."""
     lat = _f(latent)
     C, F, H, W = lat.shape
     x = patchify(lat, weights["w_p"], weights["b_p"])
     e = time_mlp(t, weights["w_t1"], weights["b_t1"], weights["w_t2"], weights["b_t2"], freq_dim)
-    for blk in blocks:
-        x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx)
+    for i, blk in enumerate(blocks):
+        x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx,
+                      attn_cache=None if attn_caches is None else attn_caches[i])
     y = head(x, weights["w_head"], weights["b_head"], eps)
     return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)
 
@@ -375,3 +398,72 @@ def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks
         return lambda x, t: dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps,
                                       img_ctx=img_ctx, freq_dim=freq_dim)
     return euler_cfg(noise, n_steps, guidance, vel(ctx_cond), vel(ctx_uncond))
+
+
+# --------------------------------------------------------------------------------------
+# Diffusion cache  [Wan-P2, "Infra", inference optimisation: (1) a block's attention
+# output changes little from one sampling step to the next, so it is computed every few
+# steps and reused in between; (2) late in sampling the conditional and unconditional
+# predictions are close, so the unconditional pass is skipped and replaced by the
+# conditional one corrected by a kept residual]
+# --------------------------------------------------------------------------------------
+
+def diffusion_cache_schedule(n_steps: int, attn_start: int, attn_interval: int, cfg_start: int,
+                             cfg_interval: int):
+    """Per sampling step k, ``(reuse_attention, skip_unconditional)``. reading: before
+    ``attn_start`` every step computes attention; from it on, steps
+    ``attn_start + m * attn_interval`` compute it and the others reuse each block's
+    last output (``attn_interval = 1``: never reuse). The unconditional pass follows
+    the same rule with ``cfg_start`` and ``cfg_interval``. Step 0 always computes
+    both (``*_start >= 1`` or a computing step at 0)."""
+    out = []
+    for k in range(n_steps):
+        ra = k >= attn_start and (k - attn_start) % attn_interval != 0
+        su = k >= cfg_start and (k - cfg_start) % cfg_interval != 0
+        out.append((ra, su))
+    return out
+
+
+def euler_cfg_cached(x0, n_steps: int, guidance: float, velocity_cond, velocity_uncond, schedule) -> np.ndarray:
+    """``euler_cfg`` with the diffusion cache. ``velocity_*(x, t, reuse_attention)``.
+    On a step that skips the unconditional pass, the guided velocity is
+    ``v_c + (guidance - 1) * delta`` with ``delta = v_c - v_u`` kept from the last step
+    that ran both passes. reading: the residual compensation is that kept difference
+    (the unconditional prediction is taken as ``v_c - delta``)."""
+    x = _f(x0).copy()
+    dt = 1.0 / n_steps
+    delta = None
+    for k in range(n_steps):
+        t = k * dt
+        reuse, skip = schedule[k]
+        vc = _f(velocity_cond(x, t, reuse))
+        if skip:
+            v = vc + (guidance - 1.0) * delta
+        else:
+            vu = _f(velocity_uncond(x, t, reuse))
+            delta = vc - vu
+            v = vu + guidance * delta
+        x = x + dt * v
+    return x
+
+
+def sample_euler_cfg_cached(noise, n_steps: int, guidance: float, weights: Dict, blocks: Sequence[Dict], ctx_cond,
+                            ctx_uncond, heads: int, schedule, eps: float = 1e-6, img_ctx=None, cond_channels=None,
+                            freq_dim: int = 256) -> np.ndarray:
+    """``sample_euler_cfg`` with the diffusion cache of ``schedule``
+    (``diffusion_cache_schedule``). Each branch keeps its own per-block attention
+    outputs: a branch that reuses attention takes the outputs of the last step on which
+    that branch computed it."""
+    caches = {"c": [{} for _ in blocks], "u": [{} for _ in blocks]}
+
+    def make_input(x):
+        return x if cond_channels is None else np.concatenate([x, _f(cond_channels)], axis=0)
+
+    def vel(ctx, key):
+        def f(x, t, reuse):
+            for c in caches[key]:
+                c["reuse"] = reuse
+            return dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps, img_ctx=img_ctx,
+                             freq_dim=freq_dim, attn_caches=caches[key])
+        return f
+    return euler_cfg_cached(noise, n_steps, guidance, vel(ctx_cond, "c"), vel(ctx_uncond, "u"), schedule)

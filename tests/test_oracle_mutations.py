@@ -152,3 +152,50 @@ def test_euler_cfg_mutations_are_caught():
         return x
     _fails(P.check_euler_cfg, guidance_on_wrong_branch)
     _fails(P.check_euler_cfg, right_endpoint_grid)
+
+
+def test_diffusion_cache_mutations_are_caught(monkeypatch):
+    def unshifted(n, a0, ai, c0, ci):                 # period counted from step 0, not from the start
+        return [(k >= a0 and k % ai != 0, k >= c0 and k % ci != 0) for k in range(n)]
+    _fails(P.check_cache_schedule, unshifted)
+
+    def flipped_residual(x0, n, g, vc, vu, sched):    # v_c - (g - 1) delta
+        x = np.asarray(x0, np.float64).copy()
+        delta = None
+        for k in range(n):
+            reuse, skip = sched[k]
+            c = vc(x, k / n, reuse)
+            if skip:
+                v = c - (g - 1) * delta
+            else:
+                u = vu(x, k / n, reuse)
+                delta = c - u
+                v = u + g * delta
+            x = x + v / n
+        return x
+
+    def stale_residual(x0, n, g, vc, vu, sched):      # delta from the first step only
+        x = np.asarray(x0, np.float64).copy()
+        delta = None
+        for k in range(n):
+            reuse, skip = sched[k]
+            c = vc(x, k / n, reuse)
+            if skip:
+                v = c + (g - 1) * delta
+            else:
+                u = vu(x, k / n, reuse)
+                delta = c - u if delta is None else delta
+                v = u + g * (c - u)
+            x = x + v / n
+        return x
+    _fails(P.check_euler_cfg_cached, flipped_residual)
+    _fails(P.check_euler_cfg_cached, stale_residual)
+
+    orig = O.dit_block
+
+    def ignores_cache(x, e, w, ctx, heads, eps=1e-6, img_ctx=None, rows=None, return_parts=False, attn_cache=None):
+        if attn_cache is not None and not attn_cache.get("reuse"):
+            attn_cache["o"] = O.self_attention_core(O.modulate(O.layer_norm(x, eps), *O.block_modulation(
+                e, w["mod_bias"])[:2]), w, heads)
+        return orig(x, e, w, ctx, heads, eps, img_ctx, rows, return_parts)
+    _fails(P.check_block_attention_cache, ignores_cache)

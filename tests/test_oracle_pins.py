@@ -526,3 +526,94 @@ def test_sampler_uses_stack_velocity():
     np.testing.assert_allclose(got1, x0 + v_c, rtol=1e-12, atol=1e-12)
     got0 = O.sample_euler_cfg(x0, 1, 0.0, inp, inp["blocks"], ctx_c, ctx_u, w.heads)
     np.testing.assert_allclose(got0, x0 + v_u, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ diffusion cache
+def check_cache_schedule(schedule_fn):
+    s = schedule_fn(10, 2, 3, 5, 2)
+    assert [k for k, (ra, _) in enumerate(s) if ra] == [3, 4, 6, 7, 9]
+    assert [k for k, (_, su) in enumerate(s) if su] == [6, 8]
+    assert not any(ra or su for ra, su in schedule_fn(6, 0, 1, 0, 1))       # interval 1: never reuse
+    assert not any(ra or su for ra, su in schedule_fn(4, 4, 2, 9, 2))       # starts past the end
+    assert schedule_fn(3, 0, 2, 1, 5) == [(False, False), (True, False), (False, True)]
+
+
+def test_cache_schedule_closed_forms():
+    check_cache_schedule(O.diffusion_cache_schedule)
+
+
+def check_euler_cfg_cached(euler_cfg_cached):
+    rng = RNG(16)
+    x0 = rng.standard_normal((3, 4))
+    c, u = rng.standard_normal((3, 4)), rng.standard_normal((3, 4))
+    never = [(False, False)] * 5
+    # no caching: the uncached loop, bitwise
+    fc = lambda x, t, r: 0.3 * x + t * c                                     # noqa: E731
+    fu = lambda x, t, r: -0.2 * x + u                                        # noqa: E731
+    ref = O.euler_cfg(x0, 5, 4.0, lambda x, t: fc(x, t, False), lambda x, t: fu(x, t, False))
+    assert np.array_equal(euler_cfg_cached(x0, 5, 4.0, fc, fu, never), ref)
+    # constant velocities: the kept difference is exact, any schedule gives x0 + u + g (c - u)
+    sched = [(False, False), (True, True), (True, False), (False, True), (True, True)]
+    got = euler_cfg_cached(x0, 5, 5.0, lambda x, t, r: c, lambda x, t, r: u, sched)
+    np.testing.assert_allclose(got, x0 + u + 5.0 * (c - u), rtol=1e-12, atol=1e-12)
+    # linear velocities a x, b x, two steps, the second skips the unconditional pass:
+    # x1 = x0 + (b + g (a - b)) x0 / 2, x2 = x1 + (a x1 + (g - 1)(a - b) x0) / 2
+    a, b, g = 0.7, -0.4, 3.0
+    got = euler_cfg_cached(x0, 2, g, lambda x, t, r: a * x, lambda x, t, r: b * x, [(False, False), (False, True)])
+    x1 = x0 + 0.5 * (b + g * (a - b)) * x0
+    np.testing.assert_allclose(got, x1 + 0.5 * (a * x1 + (g - 1) * (a - b) * x0), rtol=1e-12)
+    # the reuse flag of each step reaches both velocity calls; skipped steps call v_u not at all
+    seen = []
+    euler_cfg_cached(x0, 3, 2.0, lambda x, t, r: seen.append(("c", t, r)) or c,
+                     lambda x, t, r: seen.append(("u", t, r)) or u, [(False, False), (True, True), (True, False)])
+    assert seen == [("c", 0.0, False), ("u", 0.0, False), ("c", 1 / 3, True), ("c", 2 / 3, True), ("u", 2 / 3, True)]
+
+
+def test_euler_cfg_cached_closed_forms():
+    check_euler_cfg_cached(O.euler_cfg_cached)
+
+
+def check_block_attention_cache(dit_block):
+    w, inp = _tiny_block_inputs(seed=3)
+    x, e, blk, ctx = inp["x"][0], inp["e"][0], inp["blocks"][0], inp["ctx"][0]
+    cache = {}
+    y0 = dit_block(x, e, blk, ctx, w.heads, attn_cache=cache)
+    o0 = cache["o"].copy()
+    # same input, reuse: identical output, cache untouched
+    cache["reuse"] = True
+    assert np.array_equal(dit_block(x, e, blk, ctx, w.heads, attn_cache=cache), y0)
+    assert np.array_equal(cache["o"], o0)
+    # a new input with reuse keeps the old attention output o0 (then the output
+    # projection, gate, cross-attention and FFN of the new input)
+    x2 = x + 0.3 * RNG(17).standard_normal(x.shape)
+    got = dit_block(x2, e, blk, ctx, w.heads, attn_cache=cache)
+    mod = O.block_modulation(e, blk["mod_bias"])
+    x1 = x2 + mod[2] * (o0 @ blk["w_o"].astype(np.float64).T + blk["b_o"])
+    x2b = x1 + O.cross_attention_branch(O.layer_norm(x1), ctx, blk, w.heads)
+    want = x2b + mod[5] * O.ffn_branch(O.modulate(O.layer_norm(x2b), mod[3], mod[4]), blk)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(got, dit_block(x2, e, blk, ctx, w.heads))           # reuse did change the result
+    # recomputing on the new input refreshes the cache and equals the plain block
+    cache["reuse"] = False
+    np.testing.assert_allclose(dit_block(x2, e, blk, ctx, w.heads, attn_cache=cache),
+                               dit_block(x2, e, blk, ctx, w.heads), rtol=1e-12, atol=1e-12)
+    assert not np.allclose(cache["o"], o0)
+
+
+def test_block_attention_cache():
+    check_block_attention_cache(O.dit_block)
+
+
+def test_cached_sampler_without_reuse_is_the_sampler():
+    w = WORKLOADS["tiny_f32_block"]
+    inp = make_inputs(w, seed=4, n_blocks=2)
+    x0 = inp["noise"][0]
+    ctx_c, ctx_u = inp["ctx"][0], RNG(18).standard_normal(inp["ctx"][0].shape)
+    sched = O.diffusion_cache_schedule(3, 0, 1, 0, 1)
+    got = O.sample_euler_cfg_cached(x0, 3, 4.0, inp, inp["blocks"], ctx_c, ctx_u, w.heads, sched)
+    assert np.array_equal(got, O.sample_euler_cfg(x0, 3, 4.0, inp, inp["blocks"], ctx_c, ctx_u, w.heads))
+    # with reuse the result moves, but stays close (the cache is an approximation)
+    sched = O.diffusion_cache_schedule(3, 1, 2, 2, 2)
+    assert sched == [(False, False), (False, False), (True, False)]
+    got2 = O.sample_euler_cfg_cached(x0, 3, 4.0, inp, inp["blocks"], ctx_c, ctx_u, w.heads, sched)
+    assert not np.array_equal(got2, got)
