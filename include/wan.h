@@ -294,9 +294,26 @@ int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const 
 
 /* ---- sampling ----------------------------------------------------------------- */
 
-/* Device workspace (bytes) of wan_sample_euler_cfg for these sizes (0 on a bad cfg). */
+/* Diffusion cache of the sampling loop [Wan 2.1 page, "Infra", inference optimisation:
+ * a block's attention output changes little between steps and is computed every few
+ * steps; late steps skip the unconditional pass and correct the conditional prediction
+ * by a kept residual]. Step k reuses every block's attention output when
+ * k >= attn_start and (k - attn_start) % attn_interval != 0, and skips the
+ * unconditional pass when k >= cfg_start and (k - cfg_start) % cfg_interval != 0.
+ * Intervals >= 1 (1 = never); starts >= 0; step 0 always runs both passes in full. On a
+ * skipped step the guided velocity is v_c + (guidance - 1) delta, delta = v_c - v_u
+ * from the last step that ran both passes. Each pass keeps its own attention outputs
+ * (those of the last step on which that pass computed attention). */
+typedef struct {
+  int attn_start, attn_interval;
+  int cfg_start, cfg_interval;
+} wan_diffusion_cache;
+
+/* Device workspace (bytes) of wan_sample_euler_cfg for these sizes and cache (NULL =
+ * no cache); 0 on a bad cfg. The cache adds n_blocks x 2B x L x D act elements of kept
+ * attention outputs and B x out_ch x F x H x W fp32 of kept residual. */
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W,
-                                  int Lc, int Li);
+                                  int Lc, int Li, const wan_diffusion_cache* cache);
 
 /* Generation loop with the DiT as the velocity model [Wan 2.1 page, "训练方法" (the
  * rectified-flow velocity) and "Infra" (a fixed number of sampling steps, about 50); the
@@ -316,16 +333,18 @@ size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B
  *     start and holding x(1) on return. The DiT input is x rounded to act each step.
  *   blocks: HOST array of n_blocks weight tables; sw: stack weights.
  *   Cross-attention K|V of both contexts are projected once per call and kept for all
- *   steps. workspace >= wan_sample_workspace_bytes(...) device bytes.
+ *   steps. cache: NULL (every step runs both passes in full) or the diffusion cache
+ *   above. workspace >= wan_sample_workspace_bytes(...) device bytes (same cache).
  * Errors (before any launch): WAN_ERR_NULL, WAN_ERR_SHAPE (n_steps < 1, a guidance that
- * is not finite, out_ch > in_ch, Lc = 0, odd H or W), WAN_ERR_WORKSPACE, WAN_ERR_ALIGN.
+ * is not finite, out_ch > in_ch, Lc = 0, odd H or W, a cache interval < 1 or start < 0),
+ * WAN_ERR_WORKSPACE, WAN_ERR_ALIGN.
  * B = 0 returns WAN_OK without work. Enqueued on `stream`; returns before the GPU work
  * ends. */
 int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* input, int B, int F, int H,
                          int W, int n_steps, float guidance, const wan_stack_weights* sw,
                          const wan_block_weights* blocks, const void* ctx_cond, const void* ctx_uncond,
-                         int Lc, const void* img_ctx, int Li, float* latent_out, void* workspace,
-                         size_t ws_bytes, void* stream);
+                         int Lc, const void* img_ctx, int Li, const wan_diffusion_cache* cache,
+                         float* latent_out, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---- single-kernel entry points (used by the branch calls; exposed for tests) --- */
 

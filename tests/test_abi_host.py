@@ -124,9 +124,10 @@ def test_sampler_validation_and_workspace(wan):
     assert need > wan.workspace_bytes(cfg, 2 * B, Lt, Lc) + 2 * 2 * (2 * B * Lc * 2 * 1536)
     assert wan.sample_workspace_bytes(_cfg(wan, heads=7), 2, B, F, H, W, Lc) == 0
 
-    def call(n_steps=4, g=5.0, c=cfg, ctx_u=fake, ws=1 << 40, b=B, h=H):
+    def call(n_steps=4, g=5.0, c=cfg, ctx_u=fake, ws=1 << 40, b=B, h=H, cache=None):
         return L.wan_sample_euler_cfg(ctypes.byref(c), 2, fake, b, F, h, W, n_steps, g, ctypes.byref(sw), bws, fake,
-                                      ctx_u, Lc, None, 0, fake, fake, ws, None)
+                                      ctx_u, Lc, None, 0, None if cache is None else ctypes.byref(cache), fake, fake,
+                                      ws, None)
     assert call(n_steps=0) == -2
     assert call(g=float("nan")) == -2
     assert call(g=float("inf")) == -2
@@ -136,6 +137,11 @@ def test_sampler_validation_and_workspace(wan):
     c2 = _cfg(wan, in_ch=16, out_ch=20)
     assert call(c=c2) == -2
     assert call(b=0) == 0
+    assert call(cache=wan.DiffusionCache(1, 0, 2, 2)) == -2          # interval 0
+    assert call(cache=wan.DiffusionCache(-1, 2, 2, 2)) == -2         # negative start
+    kept = wan.sample_workspace_bytes(cfg, 2, B, F, H, W, Lc, cache=wan.DiffusionCache(1, 2, 3, 2))
+    assert kept - need >= 2 * 2 * B * Lt * 1536 * 2 + B * 16 * F * H * W * 4      # attention outputs + residual
+    assert call(cache=wan.DiffusionCache(1, 2, 3, 2), ws=kept - 1) == -5
     assert wan.launch_count() == launches
 
 

@@ -37,16 +37,16 @@ def _input(wan, r, i2v):
     return inp, cc
 
 
-def _sample(wan, r, inp, n_steps, g, ctx=None, ctx_uncond=None):
+def _sample(wan, r, inp, n_steps, g, ctx=None, ctx_uncond=None, cache=None):
     B, _, F, H, W = inp.shape
     ctx = r.ctx if ctx is None else ctx
     ctx_uncond = r.ctx_uncond if ctx_uncond is None else ctx_uncond
     Li = 0 if r.img_ctx is None else r.img_ctx.shape[1]
-    ws = torch.empty(wan.sample_workspace_bytes(r.cfg, len(r.model.block_tables), B, F, H, W, r.w.text_len, Li),
-                     dtype=torch.uint8, device="cuda")
+    ws = torch.empty(wan.sample_workspace_bytes(r.cfg, len(r.model.block_tables), B, F, H, W, r.w.text_len, Li,
+                                                cache), dtype=torch.uint8, device="cuda")
     out = torch.full((B, 16, F, H, W), float("nan"), dtype=torch.float32, device="cuda")
     wan.sample_euler_cfg(r.cfg, inp, n_steps, g, r.model.stack_table, r.model.block_tables, ctx, ctx_uncond,
-                         r.img_ctx, out, ws)
+                         r.img_ctx, out, ws, cache=cache)
     torch.cuda.synchronize()
     assert wan.device_status() == 0
     return out
@@ -103,3 +103,36 @@ def test_sampler_deterministic_and_batch_independent(wan):
     assert torch.equal(a, b)
     one = _sample(wan, r, inp[1:].contiguous(), 3, 4.0, r.ctx[1:].contiguous(), r.ctx_uncond[1:].contiguous())
     assert torch.equal(one[0], a[1])
+
+
+@pytest.mark.parametrize("i2v", [False, True])
+def test_cached_sampler_matches_oracle(wan, i2v):
+    """Six steps with the diffusion cache (attention reused on steps 2, 4; unconditional
+    pass skipped on steps 4, 5): against the oracle's cached loop, same schedule."""
+    w = small_bf16(i2v=i2v, n_blocks=2, batch=2)
+    r = Run(wan, w, zero_wx=False, uncond=True)
+    inp, cc = _input(wan, r, i2v)
+    n_steps, g = 6, 5.0
+    pol = (1, 2, 3, 3)    # attn_start, attn_interval, cfg_start, cfg_interval
+    sched = O.diffusion_cache_schedule(n_steps, *pol)
+    assert [k for k, (a, _) in enumerate(sched) if a] == [2, 4] and [k for k, (_, c) in enumerate(sched) if c] == [4, 5]
+    got = host(_sample(wan, r, inp, n_steps, g, cache=wan.DiffusionCache(*pol)))
+    for b in range(w.batch):
+        x0 = r.inp["noise"][b]
+        ref = O.sample_euler_cfg_cached(x0, n_steps, g, r.inp, r.inp["blocks"], r.inp["ctx"][b],
+                                        r.inp["ctx_uncond"][b], w.heads, sched,
+                                        img_ctx=None if r.img_np is None else r.img_np[b], cond_channels=cc[b])
+        e_x, e_d = rel_err(got[b], ref), rel_err(got[b] - x0, ref - x0)
+        print(f"cached sampler i2v={i2v} b={b}: latent {e_x:.2e} displacement {e_d:.2e}")
+        assert e_x <= BF16_TOL
+        assert e_d <= BF16_TOL
+
+
+def test_cache_without_reuse_is_the_plain_loop(wan):
+    """Intervals of 1 never reuse: bitwise the loop without a cache."""
+    w = small_bf16(n_blocks=2, batch=2)
+    r = Run(wan, w, zero_wx=False, uncond=True)
+    inp, _ = _input(wan, r, False)
+    a = _sample(wan, r, inp, 3, 4.0)
+    b = _sample(wan, r, inp, 3, 4.0, cache=wan.DiffusionCache(0, 1, 0, 1))
+    assert torch.equal(a, b)

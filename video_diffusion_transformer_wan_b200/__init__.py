@@ -15,7 +15,7 @@ from typing import Dict, Optional, Sequence
 __all__ = [
     "LIB_PATH", "lib", "WanError", "WAN_F32", "WAN_BF16", "EPI_STORE", "EPI_GELU", "EPI_RESIDUAL", "EPI_F32",
     "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights",
-    "ImageMlpWeights", "StackWeights", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
+    "ImageMlpWeights", "StackWeights", "DiffusionCache", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
     "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
     "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd",
@@ -56,6 +56,12 @@ class StackWeights(ctypes.Structure):
     _fields_ = [("w_p", _vp), ("b_p", _vp), ("time", TimeWeights), ("w_head", _vp), ("b_head", _vp)]
 
 
+class DiffusionCache(ctypes.Structure):
+    """Attention reuse and unconditional-pass skipping of the sampling loop (see
+    ``wan_diffusion_cache`` in include/wan.h)."""
+    _fields_ = [("attn_start", _i), ("attn_interval", _i), ("cfg_start", _i), ("cfg_interval", _i)]
+
+
 class WanError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -89,9 +95,10 @@ def _load() -> ctypes.CDLL:
         "wan_attention_fwd": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _i,
                                    _i, _i, _i, _vp]),
         "wan_linear_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i, _vp]),
-        "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i]),
+        "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i, P(DiffusionCache)]),
         "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
-                                      P(BlockWeights), _vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+                                      P(BlockWeights), _vp, _vp, _i, _vp, _i, P(DiffusionCache), _vp, _vp, _sz,
+                                      _vp]),
         "wan_sp_qkv_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(BlockWeights), P(_vp), _vp]),
         "wan_sp_attn_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(_vp), _vp]),
         "wan_sp_out_fwd": (_i, [P(Config), _i, _vp, P(BlockWeights), _vp, _vp, _i, _i, _vp]),
@@ -233,12 +240,18 @@ def dit_stack_fwd(cfg, latent, t, sw: StackWeights, blocks: Sequence[BlockWeight
            "wan_dit_stack_fwd")
 
 
-def sample_workspace_bytes(cfg: Config, n_blocks: int, B: int, F: int, H: int, W: int, Lc: int, Li: int = 0) -> int:
-    return int(_lib().wan_sample_workspace_bytes(ctypes.byref(cfg), n_blocks, B, F, H, W, Lc, Li))
+def _cache_ref(cache: Optional[DiffusionCache]):
+    return None if cache is None else ctypes.byref(cache)
+
+
+def sample_workspace_bytes(cfg: Config, n_blocks: int, B: int, F: int, H: int, W: int, Lc: int, Li: int = 0,
+                           cache: Optional[DiffusionCache] = None) -> int:
+    return int(_lib().wan_sample_workspace_bytes(ctypes.byref(cfg), n_blocks, B, F, H, W, Lc, Li, _cache_ref(cache)))
 
 
 def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, blocks: Sequence[BlockWeights],
-                     ctx_cond, ctx_uncond, img_ctx, latent_out, ws, stream=None):
+                     ctx_cond, ctx_uncond, img_ctx, latent_out, ws, stream=None,
+                     cache: Optional[DiffusionCache] = None):
     """inp [B, in_ch, F, H, W]: the noise in its first out_ch channels (and, for I2V, the
     fixed condition channels after them); latent_out [B, out_ch, F, H, W] fp32."""
     B, C, F, H, W = inp.shape
@@ -246,7 +259,8 @@ def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, 
     Li = 0 if img_ctx is None else img_ctx.shape[1]
     _check(_lib().wan_sample_euler_cfg(ctypes.byref(cfg), len(blocks), _p(inp), B, F, H, W, n_steps, guidance,
                                     ctypes.byref(sw), arr, _p(ctx_cond), _p(ctx_uncond), ctx_cond.shape[1],
-                                    _p(img_ctx), Li, _p(latent_out), *_ws(ws), _stream(stream)),
+                                    _p(img_ctx), Li, _cache_ref(cache), _p(latent_out), *_ws(ws),
+                                    _stream(stream)),
            "wan_sample_euler_cfg")
 
 

@@ -230,16 +230,22 @@ GemmEpi epi_residual(int64_t ldo, const float* gate, const float* gate_bias, int
   return e;
 }
 
+// attn_kept: where the attention output goes (and stays, e.g. across sampling steps), or
+// NULL for the workspace; with attn_reuse the kept output is used as it is and neither
+// the QKV projection nor the attention runs.
 int self_attn_impl(const wan_dit_config* c, const void* h, const wan_block_weights* w, const float* e, float* x, int B,
-                   int L, void* ws, const Layout& ly, cudaStream_t s) {
+                   int L, void* ws, const Layout& ly, cudaStream_t s, void* attn_kept = nullptr,
+                   bool attn_reuse = false) {
   const int D = c->dim;
   const size_t es = dtype_size(c->dtype);
   const int M = B * L;
   uint8_t* R = at(ws, ly.big);
   void* qkv = R;
-  void* o = R + static_cast<size_t>(3) * M * D * es;
-  WAN_TRY(gemm(c, h, D, w->w_qkv, w->b_qkv, qkv, M, 3 * D, D, 0, epi_store(3 * D), s));
-  WAN_TRY(attention(c, {qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, L, L, s));
+  void* o = attn_kept ? attn_kept : R + static_cast<size_t>(3) * M * D * es;
+  if (!(attn_kept && attn_reuse)) {
+    WAN_TRY(gemm(c, h, D, w->w_qkv, w->b_qkv, qkv, M, 3 * D, D, 0, epi_store(3 * D), s));
+    WAN_TRY(attention(c, {qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, L, L, s));
+  }
   const float* gb = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
   return gemm(c, o, D, w->w_o, w->b_o, x, M, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, L), s);
 }
@@ -289,11 +295,12 @@ int ffn_impl(const wan_dit_config* c, const void* h, const wan_block_weights* w,
 
 int block_impl(const wan_dit_config* c, float* x, const float* e, const void* ctx, int Lc, const void* img, int Li,
                const wan_block_weights* w, int B, int L, void* ws, const Layout& ly, cudaStream_t s,
-               const void* kvt_cached = nullptr, const void* kvi_cached = nullptr) {
+               const void* kvt_cached = nullptr, const void* kvi_cached = nullptr, void* attn_kept = nullptr,
+               bool attn_reuse = false) {
   void* h = at(ws, ly.h);
   const int64_t rows = static_cast<int64_t>(B) * L;
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 0, h, c->dtype, c->eps, s));
-  WAN_TRY(self_attn_impl(c, h, w, e, x, B, L, ws, ly, s));
+  WAN_TRY(self_attn_impl(c, h, w, e, x, B, L, ws, ly, s, attn_kept, attn_reuse));
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, nullptr, nullptr, -1, h, c->dtype, c->eps, s));
   WAN_TRY(cross_attn_impl(c, h, ctx, Lc, img, Li, w, x, B, L, ws, ly, s, kvt_cached, kvi_cached));
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 1, h, c->dtype, c->eps, s));
@@ -321,7 +328,8 @@ int head_impl(const wan_dit_config* c, const float* x, int B, int F, int H, int 
 int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H, int W,
                const float* t, const wan_stack_weights* sw, const wan_block_weights* blocks, const void* ctx, int Lc,
                const void* img_ctx, int li, float* v_out, void* workspace, const Layout& ly, cudaStream_t s,
-               const void* const* kvt, const void* const* kvi) {
+               const void* const* kvt, const void* const* kvi, void* const* attn_kept = nullptr,
+               bool attn_reuse = false) {
   const int L = F * (H / 2) * (W / 2);
   float* x = reinterpret_cast<float*>(at(workspace, ly.x));
   float* e = reinterpret_cast<float*>(at(workspace, ly.e));
@@ -333,7 +341,7 @@ int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int 
                           e, cfg->dtype, s));
   for (int i = 0; i < n_blocks; ++i)
     WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s, kvt ? kvt[i] : nullptr,
-                       kvi ? kvi[i] : nullptr));
+                       kvi ? kvi[i] : nullptr, attn_kept ? attn_kept[i] : nullptr, attn_reuse));
   return head_impl(cfg, x, B, F, H, W, sw->w_head, sw->b_head, v_out, at(workspace, ly.h), s);
 }
 
@@ -341,10 +349,11 @@ int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int 
 // 2B velocities (fp32), the 2B timesteps, and per block the cached text and image K|V
 // of both contexts.
 struct SampleLayout {
-  size_t in2, v, t, kvt, kvi, total;
-  size_t kvt_block, kvi_block;  // bytes per block
+  size_t in2, v, t, kvt, kvi, attn, delta, total;
+  size_t kvt_block, kvi_block, attn_block;  // bytes per block
 };
-SampleLayout sample_layout(const wan_dit_config* c, int n_blocks, int B, int F, int H, int W, int Lc, int Li) {
+SampleLayout sample_layout(const wan_dit_config* c, int n_blocks, int B, int F, int H, int W, int Lc, int Li,
+                           bool cache) {
   const size_t es = dtype_size(c->dtype);
   const int L = F * (H / 2) * (W / 2);
   const size_t fhw = static_cast<size_t>(F) * H * W;
@@ -356,7 +365,10 @@ SampleLayout sample_layout(const wan_dit_config* c, int n_blocks, int B, int F, 
   l.kvt_block = align_up(2 * static_cast<size_t>(B) * Lc * 2 * c->dim * es);
   l.kvi_block = align_up(2 * static_cast<size_t>(B) * Li * 2 * c->dim * es);
   l.kvi = l.kvt + static_cast<size_t>(n_blocks) * l.kvt_block;
-  l.total = l.kvi + static_cast<size_t>(n_blocks) * l.kvi_block;
+  l.attn = l.kvi + static_cast<size_t>(n_blocks) * l.kvi_block;
+  l.attn_block = cache ? align_up(2 * static_cast<size_t>(B) * L * c->dim * es) : 0;
+  l.delta = l.attn + static_cast<size_t>(n_blocks) * l.attn_block;
+  l.total = l.delta + (cache ? align_up(static_cast<size_t>(B) * c->out_ch * fhw * 4) : 0);
   return l;
 }
 
@@ -615,17 +627,22 @@ int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const 
 }
 
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W, int Lc,
-                                  int Li) {
+                                  int Li, const wan_diffusion_cache* cache) {
   if (check_cfg(cfg) != WAN_OK || n_blocks < 0 || B < 0 || F < 0 || H < 0 || W < 0 || Lc < 0 || Li < 0) return 0;
-  return sample_layout(cfg, n_blocks, B, F, H, W, Lc, Li).total;
+  return sample_layout(cfg, n_blocks, B, F, H, W, Lc, Li, cache != nullptr).total;
 }
 
 int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* input, int B, int F, int H, int W,
                          int n_steps, float guidance, const wan_stack_weights* sw, const wan_block_weights* blocks,
                          const void* ctx_cond, const void* ctx_uncond, int Lc, const void* img_ctx, int Li,
-                         float* latent_out, void* workspace, size_t ws_bytes, void* stream) {
+                         const wan_diffusion_cache* cache, float* latent_out, void* workspace, size_t ws_bytes,
+                         void* stream) {
   WAN_TRY(check_cfg(cfg, true));
   WAN_REQUIRE(sw && (blocks || n_blocks == 0), WAN_ERR_NULL);
+  if (cache)
+    WAN_REQUIRE(cache->attn_start >= 0 && cache->attn_interval >= 1 && cache->cfg_start >= 0 &&
+                    cache->cfg_interval >= 1,
+                WAN_ERR_SHAPE);
   WAN_REQUIRE(n_blocks >= 0 && n_steps >= 1 && guidance == guidance && guidance - guidance == 0.0f, WAN_ERR_SHAPE);
   WAN_REQUIRE(B >= 0 && F >= 1 && H >= 2 && W >= 2 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
   WAN_REQUIRE(cfg->out_ch <= cfg->in_ch && Lc > 0, WAN_ERR_SHAPE);
@@ -648,7 +665,7 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
   const int L = F * (H / 2) * (W / 2);
   const int li = with_img ? Li : 0;
   WAN_TRY(check_tokens(cfg, 2 * B, L, Lc, li));
-  const SampleLayout sl = sample_layout(cfg, n_blocks, B, F, H, W, Lc, li);
+  const SampleLayout sl = sample_layout(cfg, n_blocks, B, F, H, W, Lc, li, cache != nullptr);
   WAN_REQUIRE(ws_bytes >= sl.total, WAN_ERR_WORKSPACE);
   if (B == 0) return WAN_OK;
   cudaStream_t s = as_stream(stream);
@@ -678,14 +695,30 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
       kvi[i] = ci;
     }
   }
+  // Kept attention outputs [2B, L, D] per block (conditional samples first, so a
+  // conditional-only pass over B samples uses the first half) and the kept residual.
+  std::vector<void*> kept;
+  float* delta = nullptr;
+  if (cache) {
+    for (int i = 0; i < n_blocks; ++i) kept.push_back(at(workspace, sl.attn + i * sl.attn_block));
+    delta = reinterpret_cast<float*>(at(workspace, sl.delta));
+  }
   const Layout ly = layout(cfg, 2 * B, L, Lc, li);
   const float dt = 1.0f / static_cast<float>(n_steps);
   for (int k = 0; k < n_steps; ++k) {
-    WAN_TRY(stack_impl(cfg, n_blocks, in2, 2 * B, F, H, W, t, sw, blocks, ctx_cond, Lc,
+    bool reuse = false, skip = false;
+    if (cache) {
+      reuse = k >= cache->attn_start && (k - cache->attn_start) % cache->attn_interval != 0;
+      skip = k >= cache->cfg_start && (k - cache->cfg_start) % cache->cfg_interval != 0;
+    }
+    const int Bp = skip ? B : 2 * B;  // samples in this step's pass
+    WAN_TRY(stack_impl(cfg, n_blocks, in2, Bp, F, H, W, t, sw, blocks, ctx_cond, Lc,
                        with_img ? img_ctx : nullptr, li, v, workspace, ly, s,
-                       n_blocks ? kvt.data() : nullptr, with_img && n_blocks ? kvi.data() : nullptr));
+                       n_blocks ? kvt.data() : nullptr, with_img && n_blocks ? kvi.data() : nullptr,
+                       cache && n_blocks ? kept.data() : nullptr, reuse));
     const float t_next = static_cast<float>(1000.0 * (k + 1) / n_steps);
-    WAN_TRY(launch_euler_cfg(v, B, n, in_stride, dt, guidance, latent_out, in2, t, t_next, cfg->dtype, s));
+    WAN_TRY(launch_euler_cfg(v, B, n, in_stride, dt, guidance, latent_out, in2, t, t_next, cfg->dtype, s, delta,
+                             skip));
   }
   return WAN_OK;
 }

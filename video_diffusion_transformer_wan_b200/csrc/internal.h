@@ -96,7 +96,7 @@ int launch_flow_input(const void* x1, const void* x0, const float* u, int B, int
 int launch_sampler_init(const void* input, int B, int64_t n, int64_t in_stride, float* x, void* in2, float* t,
                         int dtype, cudaStream_t s);
 int launch_euler_cfg(const float* v, int B, int64_t n, int64_t in_stride, float dt, float g, float* x, void* in2,
-                     float* t, float t_next, int dtype, cudaStream_t s);
+                     float* t, float t_next, int dtype, cudaStream_t s, float* delta = nullptr, bool skip = false);
 int launch_flow_loss(const float* v, const void* x1, const void* x0, int B, int64_t n, float* loss, int dtype,
                      cudaStream_t s);
 

@@ -251,20 +251,31 @@ __global__ void sampler_init_kernel(const T* __restrict__ input, int B, int64_t 
   }
 }
 
-// One guided Euler step: x += dt * (v_u + g (v_c - v_u)) with v = [v_c (B samples) |
-// v_u (B samples)]; the new x (rounded to the activation type) goes into the first n
-// elements of both halves of the next DiT input, and the timestep becomes t_next.
+// One guided Euler step. Both passes ran (skip = 0): v = [v_c (B samples) | v_u (B
+// samples)], delta = v_c - v_u (kept in `delta` when it is not null) and
+// x += dt * (v_u + g delta). The unconditional pass was skipped (skip = 1): v = v_c
+// (B samples) and x += dt * (v_c + (g - 1) delta) with the kept delta. The new x
+// (rounded to the activation type) goes into the first n elements of both halves of
+// the next DiT input, and the timestep becomes t_next.
 template <typename T>
 __global__ void euler_cfg_kernel(const float* __restrict__ v, int B, int64_t n, int64_t in_stride, float dt,
                                  float g, float* __restrict__ x, T* __restrict__ in2, float* __restrict__ t,
-                                 float t_next) {
+                                 float t_next, float* __restrict__ delta, int skip) {
   const int64_t total = static_cast<int64_t>(B) * n;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t b = idx / n, i = idx % n;
     const float vc = v[idx];
-    const float vu = v[total + idx];
-    const float xv = x[idx] + dt * (vu + g * (vc - vu));
+    float vel;
+    if (skip) {
+      vel = vc + (g - 1.0f) * delta[idx];
+    } else {
+      const float vu = v[total + idx];
+      const float d = vc - vu;
+      if (delta) delta[idx] = d;
+      vel = vu + g * d;
+    }
+    const float xv = x[idx] + dt * vel;
     x[idx] = xv;
     const T xt = cvt<T>(xv);
     in2[b * in_stride + i] = xt;
@@ -298,16 +309,16 @@ int launch_sampler_init(const void* input, int B, int64_t n, int64_t in_stride, 
 }
 
 int launch_euler_cfg(const float* v, int B, int64_t n, int64_t in_stride, float dt, float g, float* x, void* in2,
-                     float* t, float t_next, int dtype, cudaStream_t s) {
+                     float* t, float t_next, int dtype, cudaStream_t s, float* delta, bool skip) {
   const int64_t total = static_cast<int64_t>(B) * n;
   if (total == 0) return WAN_OK;
   trace_launch_begin(WAN_KIND_SMALL, s, static_cast<double>(total) * (16.0 + 2.0 * dtype_size(dtype)));
   if (dtype == WAN_BF16)
     euler_cfg_kernel<__nv_bfloat16><<<grid_for(total, 256), 256, 0, s>>>(
-        v, B, n, in_stride, dt, g, x, static_cast<__nv_bfloat16*>(in2), t, t_next);
+        v, B, n, in_stride, dt, g, x, static_cast<__nv_bfloat16*>(in2), t, t_next, delta, skip ? 1 : 0);
   else
-    euler_cfg_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(v, B, n, in_stride, dt, g, x,
-                                                                 static_cast<float*>(in2), t, t_next);
+    euler_cfg_kernel<float><<<grid_for(total, 256), 256, 0, s>>>(
+        v, B, n, in_stride, dt, g, x, static_cast<float*>(in2), t, t_next, delta, skip ? 1 : 0);
   int st = check_launch();
   trace_launch_end(WAN_KIND_SMALL, s);
   return st;

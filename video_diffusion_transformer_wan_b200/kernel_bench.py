@@ -49,16 +49,20 @@ def _sample(a) -> dict:
     noise = to_device(inp["noise"], model.act)
     ctx, ctx_u = to_device(inp["ctx"], model.act), to_device(inp["ctx_uncond"], model.act)
     out = torch.empty(B, w.out_ch, F, H, W, dtype=torch.float32, device="cuda")
-    ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len), dtype=torch.uint8,
+    cache = wan.DiffusionCache(*[int(v) for v in a.cache.split(",")]) if a.cache else None
+    ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len, 0, cache), dtype=torch.uint8,
                      device="cuda")
     ms = _time(lambda: wan.sample_euler_cfg(cfg, noise, a.steps, a.guidance, model.stack_table,
-                                            model.block_tables, ctx, ctx_u, None, out, ws), a.iters, a.warmup)
+                                            model.block_tables, ctx, ctx_u, None, out, ws, cache=cache),
+               a.iters, a.warmup)
     Lc, Fd = w.text_len, w.ffn
     # per step; the text K|V projections are made once per call and not counted
     block = 2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * L * Lc * D + 4 * L * D * Fd
     flops_step = 2 * B * (a.blocks * block + 2 * L * D * 64 * 2)
-    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, ms_per_call=ms, ms_per_euler_step=ms / a.steps,
-                latent_tokens_per_s=B * L * a.steps / (ms / 1e3), tflops=flops_step * a.steps / ms / 1e9)
+    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, cache=a.cache or None, ms_per_call=ms,
+                ms_per_euler_step=ms / a.steps,
+                latent_tokens_per_s=B * L * a.steps / (ms / 1e3),
+                tflops_uncached_equivalent=flops_step * a.steps / ms / 1e9)
 
 
 def main(argv=None):
@@ -67,6 +71,7 @@ def main(argv=None):
     ap.add_argument("--blocks", type=int, default=30, help="sample: DiT blocks")
     ap.add_argument("--steps", type=int, default=2, help="sample: Euler steps per call")
     ap.add_argument("--guidance", type=float, default=5.0)
+    ap.add_argument("--cache", default="", help="sample: diffusion cache attn_start,attn_interval,cfg_start,cfg_interval")
     ap.add_argument("--L", type=int, default=32760)
     ap.add_argument("--Lk", type=int, default=0, help="key length (default: L, self-attention)")
     ap.add_argument("--heads", type=int, default=12)
