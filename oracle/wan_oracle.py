@@ -184,14 +184,19 @@ def attention(q, k, v, heads: int) -> np.ndarray:
 # Block branches
 # --------------------------------------------------------------------------------------
 
-def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None) -> np.ndarray:
+def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None, fp8: bool = False) -> np.ndarray:
     """The attention output ``attn(h Wq, h Wk, h Wv)`` before the output projection.
     The fused QKV weight ``w_qkv [3D, D]`` is stacked (q, k, v). ``kv_source`` (all rows
-    of h) lets the caller evaluate only some query rows; by default it is ``h``."""
+    of h) lets the caller evaluate only some query rows; by default it is ``h``. With
+    ``fp8`` the projection is ``linear_fp8`` of the fused weight (one weight scale)."""
     h = _f(h)
     D = h.shape[-1]
     src = h if kv_source is None else _f(kv_source)
     wqkv, bqkv = _f(w["w_qkv"]), _f(w["b_qkv"])
+    if fp8:
+        q = linear_fp8(h, wqkv, bqkv)[:, :D]
+        kv = linear_fp8(src, wqkv, bqkv)
+        return attention(q, kv[:, D:2 * D], kv[:, 2 * D:], heads)
     q = linear(h, wqkv[:D], bqkv[:D])
     k = linear(src, wqkv[D:2 * D], bqkv[D:2 * D])
     v = linear(src, wqkv[2 * D:], bqkv[2 * D:])
@@ -199,42 +204,44 @@ def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None)
 
 
 def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
-                          kv_source=None, o=None) -> np.ndarray:
+                          kv_source=None, o=None, fp8: bool = False) -> np.ndarray:
     """Self-attention sub-layer output before the gate: ``attn(h Wq, h Wk, h Wv) Wo^T + bo``.
     ``o`` replaces the attention output when given (an output kept from an earlier
     sampling step, see ``dit_block``'s ``attn_cache``)."""
     if o is None:
-        o = self_attention_core(h, w, heads, kv_source)
-    return linear(o, w["w_o"], w["b_o"])
+        o = self_attention_core(h, w, heads, kv_source, fp8)
+    return (linear_fp8 if fp8 else linear)(o, w["w_o"], w["b_o"])
 
 
 def cross_attention_branch(h, ctx, w: Dict[str, np.ndarray], heads: int,
-                           img_ctx=None) -> np.ndarray:
+                           img_ctx=None, fp8: bool = False) -> np.ndarray:
     """Cross-attention sub-layer: queries from the video tokens, keys and values from
     the 512 umT5 text tokens [Wan-P2, "Diffusion Transformer" and "umT5"]. For I2V, a
     decoupled second attention over image-context tokens with its own K/V projection
     is added before the shared output projection [Wan-P2, "I2V 架构扩展"; Wan-P1,
     "核心创新四"]. reading: ``o = attn(q,Kt,Vt) + attn(q,Ki,Vi)``, weight 1."""
+    lin = linear_fp8 if fp8 else linear
     D = _f(h).shape[-1]
-    q = linear(h, w["w_cq"], w["b_cq"])
-    kv = linear(ctx, w["w_ckv"], w["b_ckv"])
+    q = lin(h, w["w_cq"], w["b_cq"])
+    kv = lin(ctx, w["w_ckv"], w["b_ckv"])
     o = attention(q, kv[:, :D], kv[:, D:], heads)
     if img_ctx is not None:
-        kvi = linear(img_ctx, w["w_ckv_img"], w["b_ckv_img"])
+        kvi = lin(img_ctx, w["w_ckv_img"], w["b_ckv_img"])
         o = o + attention(q, kvi[:, :D], kvi[:, D:], heads)
-    return linear(o, w["w_co"], w["b_co"])
+    return lin(o, w["w_co"], w["b_co"])
 
 
-def ffn_branch(h, w: Dict[str, np.ndarray]) -> np.ndarray:
+def ffn_branch(h, w: Dict[str, np.ndarray], fp8: bool = False) -> np.ndarray:
     """Feed-forward sub-layer: Linear(D,F) -> GELU-tanh -> Linear(F,D)
     [Wan-P2 config table: FFN dimension 8960 / 13824]. reading: a plain two-matrix
     FFN (a gated GLU would not match the 1.3B/14B parameter counts)."""
-    return linear(gelu_tanh(linear(h, w["w_1"], w["b_1"])), w["w_2"], w["b_2"])
+    lin = linear_fp8 if fp8 else linear
+    return lin(gelu_tanh(lin(h, w["w_1"], w["b_1"])), w["w_2"], w["b_2"])
 
 
 def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6,
               img_ctx=None, rows: Optional[Sequence[int]] = None,
-              return_parts: bool = False, attn_cache: Optional[Dict] = None):
+              return_parts: bool = False, attn_cache: Optional[Dict] = None, fp8: bool = False):
     """One DiT block [Wan-P2, "Diffusion Transformer"]:
 
     1. ``x += gate_msa * SelfAttn(LN(x) (1 + scale_msa) + shift_msa)``
@@ -256,6 +263,10 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
     attention output. With ``attn_cache["reuse"]`` true that output replaces the
     attention (q, k and v are not formed); otherwise the attention is computed and
     stored in ``attn_cache["o"]``.
+
+    ``fp8`` runs every linear layer of the block as ``linear_fp8`` (per-token input
+    codes, per-tensor weight codes; the sum of the text and image attention outputs is
+    quantised as one input).
     """
     x = _f(x)
     mod = block_modulation(e, w["mod_bias"])
@@ -268,22 +279,22 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
         xr, hr = x[rows], h_all[rows]
     parts = {"h_msa": hr}
     if attn_cache is not None and attn_cache.get("reuse"):
-        sa = self_attention_branch(hr, w, heads, o=attn_cache["o"])
+        sa = self_attention_branch(hr, w, heads, o=attn_cache["o"], fp8=fp8)
     else:
-        o = self_attention_core(hr, w, heads, kv_source=h_all)
+        o = self_attention_core(hr, w, heads, kv_source=h_all, fp8=fp8)
         if attn_cache is not None:
             attn_cache["o"] = o
-        sa = self_attention_branch(hr, w, heads, o=o)
+        sa = self_attention_branch(hr, w, heads, o=o, fp8=fp8)
     parts["sa"] = sa
     x1 = xr + gate_msa * sa
     hc = layer_norm(x1, eps)
     parts["h_cross"] = hc
-    ca = cross_attention_branch(hc, ctx, w, heads, img_ctx=img_ctx)
+    ca = cross_attention_branch(hc, ctx, w, heads, img_ctx=img_ctx, fp8=fp8)
     parts["ca"] = ca
     x2 = x1 + ca
     hf = modulate(layer_norm(x2, eps), shift_ffn, scale_ffn)
     parts["h_ffn"] = hf
-    ff = ffn_branch(hf, w)
+    ff = ffn_branch(hf, w, fp8=fp8)
     parts["ffn"] = ff
     x3 = x2 + gate_ffn * ff
     parts["x_after_sa"], parts["x_after_ca"] = x1, x2
@@ -467,3 +478,62 @@ def sample_euler_cfg_cached(noise, n_steps: int, guidance: float, weights: Dict,
                              freq_dim=freq_dim, attn_caches=caches[key])
         return f
     return euler_cfg_cached(noise, n_steps, guidance, vel(ctx_cond, "c"), vel(ctx_uncond, "u"), schedule)
+
+
+# --------------------------------------------------------------------------------------
+# FP8 (E4M3) linear layers  [Wan-P2, "Infra", inference optimisation: FP8 GEMM with a
+# per-tensor scale for the weights and a per-token scale for the activations]
+# --------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an 8-bit E4M3 code: sign bit, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent field 0 holds the subnormals m/8 * 2^-6; there are no infinities and
+    S.1111.111 is NaN."""
+    s = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 0xF, code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return s * (m / 8.0) * 2.0 ** -6
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def round_e4m3(x) -> np.ndarray:
+    """Nearest E4M3 value (ties to the even code), saturated to +-448. Normal numbers
+    (|x| >= 2^-6) have a spacing of 2^(e-3) in [2^e, 2^(e+1)); below 2^-6 the spacing is
+    2^-9 (subnormals)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)
+    q = np.exp2(e - 3)
+    r = np.rint(a / q) * q                      # np.rint: round half to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.sign(x) * r
+
+
+def quantize_e4m3(x, axis=None):
+    """Scale and codes for ``x ~ scale * q``: ``scale = amax / 448`` over the whole
+    tensor (``axis=None``, weights) or per row (``axis=-1``, activations: one scale per
+    token), ``q = round_e4m3(x / scale)``. reading: the scale maps the largest magnitude
+    onto the largest code; an all-zero row or tensor gets scale 1. The scale and the
+    division are float32 operations, the precision the kernels decide the code in.
+    Returns ``(q, scale)`` with q as float64 values on the E4M3 grid."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=axis, keepdims=axis is not None).astype(np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = round_e4m3((x32 / scale).astype(np.float32))
+    return q, (scale if axis is not None else np.float32(scale))
+
+
+def linear_fp8(x, weight, bias=None) -> np.ndarray:
+    """``y = (q_x q_w^T) * s_x[row] * s_w + b`` with per-token codes of the input and
+    per-tensor codes of the weight (``quantize_e4m3``); the product of the codes is
+    exact in float64."""
+    qx, sx = quantize_e4m3(x, axis=-1)
+    qw, sw = quantize_e4m3(weight)
+    y = (qx @ qw.T) * sx.astype(np.float64) * np.float64(sw)
+    return y if bias is None else y + _f(bias)

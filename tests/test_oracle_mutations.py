@@ -99,8 +99,8 @@ def test_block_mutations_are_caught(monkeypatch):
     # gate applied to the cross-attention branch as well (wrong reading of the six vectors)
     orig = O.cross_attention_branch
 
-    def gated_cross(h, ctx, w, heads, img_ctx=None):
-        return 0.5 * orig(h, ctx, w, heads, img_ctx=img_ctx)
+    def gated_cross(h, ctx, w, heads, img_ctx=None, fp8=False):
+        return 0.5 * orig(h, ctx, w, heads, img_ctx=img_ctx, fp8=fp8)
     monkeypatch.setattr(O, "cross_attention_branch", gated_cross)
     _fails(P.check_block_vs_torch, O.dit_block)
     monkeypatch.undo()
@@ -199,3 +199,28 @@ def test_diffusion_cache_mutations_are_caught(monkeypatch):
                 e, w["mod_bias"])[:2]), w, heads)
         return orig(x, e, w, ctx, heads, eps, img_ctx, rows, return_parts)
     _fails(P.check_block_attention_cache, ignores_cache)
+
+
+def test_fp8_mutations_are_caught(monkeypatch):
+    def ties_away(x):                                  # round half away from zero instead of to even
+        x = np.asarray(x, np.float64)
+        a = np.abs(x)
+        e = np.clip(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6, 8)
+        q = np.exp2(e - 3)
+        return np.sign(x) * np.minimum(np.floor(a / q + 0.5) * q, 448.0)
+
+    def no_subnormals(x):                              # flush below 2^-6
+        r = O.round_e4m3(x)
+        return np.where(np.abs(np.asarray(x)) < 2.0 ** -6, 0.0, r)
+    _fails(P.check_round_e4m3, ties_away)
+    _fails(P.check_round_e4m3, no_subnormals)
+    _fails(P.check_e4m3_decode, lambda c: O.e4m3_decode(c) * (2.0 if (c >> 3) & 0xF == 0 else 1.0))
+
+    orig = O.quantize_e4m3
+
+    def tensor_scales(x, axis=None):                   # one scale for all tokens instead of one per token
+        q, s = orig(x)
+        return (q, np.full((np.asarray(x).shape[0], 1), s, np.float32)) if axis == -1 else (q, s)
+    monkeypatch.setattr(O, "quantize_e4m3", tensor_scales)
+    _fails(P.check_block_fp8_vs_torch, O.dit_block)
+    monkeypatch.undo()

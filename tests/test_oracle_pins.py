@@ -292,10 +292,25 @@ def test_attention_long_rows_chunking():
 # Block: library re-expression, special cases, invariants, row sampling
 # ----------------------------------------------------------------------------------------
 
-def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None):
+def torch_fp8_linear(t, W, b):
+    """linear with E4M3 codes made by torch's float8_e4m3fn conversion: per-row scales of
+    the input, one scale for the weight (scale = amax / 448 in float32)."""
+    def codes(a, dim):
+        a32 = a.to(torch.float32)
+        amax = a32.abs().amax(dim=dim, keepdim=True) if dim is not None else a32.abs().amax()
+        sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        return (a32 / sc).to(torch.float8_e4m3fn).to(torch.float64), sc.to(torch.float64)
+    qx, sx = codes(t, -1)
+    qw, sw = codes(W, None)
+    return (qx @ qw.T) * sx * sw + b
+
+
+def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None, fp8=False):
     """The block re-expressed with torch library routines (layer_norm, linear,
-    scaled_dot_product_attention, gelu) in float64."""
+    scaled_dot_product_attention, gelu) in float64; with ``fp8`` every linear layer
+    uses torch's E4M3 conversion (``torch_fp8_linear``)."""
     X, E, C = t64(x), t64(e) + t64(w["mod_bias"]), t64(ctx)
+    lin = torch_fp8_linear if fp8 else tF.linear
     D = X.shape[-1]
     d = D // heads
     W = {k: t64(v) for k, v in w.items()}
@@ -309,18 +324,18 @@ def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None):
 
     ln = lambda t: tF.layer_norm(t, (D,), eps=eps)  # noqa: E731
     h = ln(X) * (1 + E[1]) + E[0]
-    qkv = tF.linear(h, W["w_qkv"], W["b_qkv"])
-    X = X + E[2] * tF.linear(mha(qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]), W["w_o"], W["b_o"])
+    qkv = lin(h, W["w_qkv"], W["b_qkv"])
+    X = X + E[2] * lin(mha(qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]), W["w_o"], W["b_o"])
     hc = ln(X)
-    q = tF.linear(hc, W["w_cq"], W["b_cq"])
-    kv = tF.linear(C, W["w_ckv"], W["b_ckv"])
+    q = lin(hc, W["w_cq"], W["b_cq"])
+    kv = lin(C, W["w_ckv"], W["b_ckv"])
     o = mha(q, kv[:, :D], kv[:, D:])
     if img_ctx is not None:
-        kvi = tF.linear(t64(img_ctx), W["w_ckv_img"], W["b_ckv_img"])
+        kvi = lin(t64(img_ctx), W["w_ckv_img"], W["b_ckv_img"])
         o = o + mha(q, kvi[:, :D], kvi[:, D:])
-    X = X + tF.linear(o, W["w_co"], W["b_co"])
+    X = X + lin(o, W["w_co"], W["b_co"])
     hf = ln(X) * (1 + E[4]) + E[3]
-    ff = tF.linear(tF.gelu(tF.linear(hf, W["w_1"], W["b_1"]), approximate="tanh"), W["w_2"], W["b_2"])
+    ff = lin(tF.gelu(lin(hf, W["w_1"], W["b_1"]), approximate="tanh"), W["w_2"], W["b_2"])
     return (X + E[5] * ff).numpy()
 
 
@@ -617,3 +632,78 @@ def test_cached_sampler_without_reuse_is_the_sampler():
     assert sched == [(False, False), (False, False), (True, False)]
     got2 = O.sample_euler_cfg_cached(x0, 3, 4.0, inp, inp["blocks"], ctx_c, ctx_u, w.heads, sched)
     assert not np.array_equal(got2, got)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3)
+def check_e4m3_decode(decode):
+    assert decode(0x7E) == 448.0 and decode(0x38) == 1.0 and decode(0x08) == 2.0 ** -6
+    assert decode(0x01) == 2.0 ** -9 and decode(0x00) == 0.0 and decode(0x3C) == 1.5
+    assert math.isnan(decode(0x7F)) and math.isnan(decode(0xFF))
+    vals = [decode(c) for c in range(0x7F)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))                     # monotone in code order
+    assert all(decode(c | 0x80) == -decode(c) for c in range(0x7F))
+
+
+def test_e4m3_decode_closed_forms():
+    check_e4m3_decode(O.e4m3_decode)
+
+
+def check_round_e4m3(round_fn):
+    vals = np.array([O.e4m3_decode(c) for c in range(0x7F)])
+    assert np.array_equal(round_fn(vals), vals) and np.array_equal(round_fn(-vals), -vals)   # fixed points
+    mids = (vals[:-1] + vals[1:]) / 2                                        # ties go to the even code
+    got = round_fn(mids)
+    even = np.where(np.arange(len(mids)) % 2 == 0, vals[:-1], vals[1:])
+    assert np.array_equal(got, even)
+    x = RNG(19).uniform(-448, 448, 20000) * np.exp2(RNG(20).integers(-14, 1, 20000))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(round_fn(x), ref)                                  # library conversion, in range
+    assert np.array_equal(round_fn(np.array([449.0, 1e6, -500.0])), np.array([448.0, 448.0, -448.0]))
+
+
+def test_round_e4m3_grid_ties_and_library():
+    check_round_e4m3(O.round_e4m3)
+
+
+def test_quantize_e4m3_scales():
+    a = RNG(21).standard_normal((7, 33)) * np.exp2(RNG(22).integers(-8, 8, (7, 1)))
+    a[3] = 0.0
+    q, s = O.quantize_e4m3(a, axis=-1)
+    assert s.shape == (7, 1) and s[3, 0] == 1.0 and not q[3].any()
+    rows = [r for r in range(7) if r != 3]
+    assert np.all(np.abs(q[rows]).max(axis=1) == 448.0)                     # the row max maps to 448
+    err = np.abs(q * s.astype(np.float64) - a)
+    assert np.all(err <= 2.0 ** -4 * np.abs(a) + s.astype(np.float64) * 2.0 ** -10 + 1e-30)
+    qt, st = O.quantize_e4m3(a)
+    assert np.ndim(st) == 0 and np.abs(qt).max() == 448.0
+
+
+def test_linear_fp8_is_the_dequantised_product():
+    r = RNG(23)
+    x, w, b = r.standard_normal((9, 40)), 0.02 * r.standard_normal((24, 40)), r.standard_normal(24)
+    qx, sx = O.quantize_e4m3(x, axis=-1)
+    qw, sw = O.quantize_e4m3(w)
+    ref = O.linear(qx * sx.astype(np.float64), qw * np.float64(sw), b)
+    np.testing.assert_allclose(O.linear_fp8(x, w, b), ref, rtol=1e-12, atol=1e-12)
+    exact = O.linear(x, w, b) - b
+    assert np.abs(O.linear_fp8(x, w, b) - b - exact).max() < 0.1 * np.abs(exact).max()   # an approximation of it
+
+
+def check_block_fp8_vs_torch(dit_block):
+    for i2v in (False, True):
+        w, inp = _tiny_block_inputs(i2v, seed=6)
+        blk = inp["blocks"][0]
+        img = None
+        if i2v:
+            img = O.image_context_mlp(inp["img_feat"][0], inp["w_i1"], inp["b_i1"], inp["w_i2"],
+                                      inp["b_i2"], inp["w_i3"], inp["b_i3"])
+        got = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True)
+        ref = torch_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True)
+        np.testing.assert_allclose(got - inp["x"][0], ref - inp["x"][0], rtol=1e-9, atol=1e-10)
+        plain = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img)
+        d, dp = got - inp["x"][0], plain - inp["x"][0]
+        assert 0 < np.abs(d - dp).max() < 0.2 * np.abs(dp).max()             # close to, not equal to, bf16
+
+
+def test_block_fp8_matches_library_reexpression():
+    check_block_fp8_vs_torch(O.dit_block)
