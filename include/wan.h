@@ -255,6 +255,52 @@ int wan_flow_matching_input(const wan_dit_config* cfg, const void* x1, const voi
 int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void* x1,
                            const void* x0, int B, int64_t n, float* loss_out, void* stream);
 
+/* ---- FP8 (E4M3) linear layers ------------------------------------------------- */
+
+/* FP8 GEMMs as the pages describe for inference [Wan 2.1 page, "Infra", inference
+ * optimisation: FP8 GEMM with a per-tensor scale for the weights and a per-token scale
+ * for the activations]. Codes are E4M3 (OCP FP8: bias 7, subnormals, no infinities),
+ * q = round-to-nearest-even-satfinite(x / s), s = amax / 448 (1 for an all-zero row or
+ * tensor), computed in IEEE float32. Requires a bf16 config; E4M3 arrays are bytes. */
+
+/* Per-tensor scales (device fp32 scalars) of a block's E4M3 weights. ckv_img may be
+ * NULL for T2V. */
+typedef struct {
+  const float *qkv, *o, *cq, *ckv, *co, *ckv_img, *ffn1, *ffn2;
+} wan_fp8_scales;
+
+/* Codes of x [M, K] act, one scale per row: q [M, K] E4M3, scale [M] fp32 (device).
+ * K % 16 == 0. */
+int wan_fp8_quantize_rows(const wan_dit_config* cfg, const void* x, int M, int K, void* q, float* scale,
+                          void* stream);
+
+/* Codes of a whole tensor x [n] act with one scale: q [n] E4M3, scale[0] fp32 (device;
+ * it is used as scratch while the work runs). n % 16 == 0. For weights, once. */
+int wan_fp8_quantize_tensor(const wan_dit_config* cfg, const void* x, int64_t n, void* q, float* scale,
+                            void* stream);
+
+/* y = a_scale[m] * w_scale[0] * (A W^T) + bias, then the epilogue of wan_linear_fwd.
+ * A [M, K] E4M3 (row stride K), a_scale [M] fp32, W [N, K] E4M3, w_scale [1] fp32,
+ * bias [N] act or NULL. K % 16 == 0, N % 8 == 0. tcgen05 kind::f8f6f4. */
+int wan_linear_fp8_fwd(const wan_dit_config* cfg, const void* A, const float* a_scale, const void* W,
+                       const float* w_scale, const void* bias, void* out, int M, int N, int K, int epilogue,
+                       const float* gate, const float* gate_bias, int64_t gate_batch_stride,
+                       int rows_per_batch, void* stream);
+
+/* Workspace (bytes) of wan_dit_block_fp8_fwd. */
+size_t wan_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int Li);
+
+/* wan_dit_block_fwd with every linear layer in FP8: w holds E4M3 codes for the eight
+ * weight matrices (biases and mod_bias as in the bf16 call) and sc their scales. The
+ * LayerNorm kernels write E4M3 codes with per-row scales directly; the attention
+ * outputs, the context, the image context and the FFN hidden are quantised per row by
+ * a separate pass (the I2V text and image attention outputs are summed first).
+ * Attention itself stays bf16 with fp32 accumulation. D % 16 == 0, F % 16 == 0, and
+ * D in {512, 1536, 5120} (WAN_ERR_UNSUPPORTED else). */
+int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x_inout, const float* e, const void* ctx, int Lc,
+                          const void* img_ctx, int Li, const wan_block_weights* w, const wan_fp8_scales* sc,
+                          int B, int L, void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- sequence parallelism (Ulysses) ------------------------------------------ */
 
 /* Self-attention of one block split over P = sp_size ranks along the token axis, the

@@ -3,6 +3,16 @@ import numpy as np
 
 BF16_TOL = 2e-2   # max|gpu - oracle| / max|oracle| for bf16 paths
 F32_TOL = 1e-4    # same, fp32 path
+# FP8 (E4M3) block against the oracle's FP8 block. E4M3 codes are 2^-3 apart (relative),
+# so an input that moves by one bf16 rounding step (2^-9) changes its code with
+# probability ~1/64 and then by a whole code. The GPU's quantiser inputs (attention
+# output, FFN hidden) are bf16 tensors whose values differ from the oracle's float64
+# ones at that level. Perturbing exactly those tensors by +-2^-9 in the oracle moves its
+# FP8 block by at most 3.3 % (max-norm) and 1.6 % (RMS) over 16 seeded trials (T2V and
+# I2V), so the bars are 1.5x those: 5e-2 and 2.5e-2. The RMS bar also separates the FP8
+# block from the bf16 one, which is 5 % RMS away.
+FP8_TOL_MAX = 5e-2
+FP8_TOL_RMS = 2.5e-2
 
 
 def rel_err(got, ref) -> float:
@@ -23,3 +33,10 @@ def host(t):
 
 def rng(seed):
     return np.random.Generator(np.random.PCG64(seed))
+
+
+def rms_err(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.sqrt(np.mean(ref ** 2))
+    return float(np.sqrt(np.mean((got - ref) ** 2)) / (den if den > 0 else 1.0))

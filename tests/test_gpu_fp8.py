@@ -1,0 +1,144 @@
+"""FP8 (E4M3) path through the C ABI against the oracle: quantisation codes and scales
+bit-exact (same float32 input, same float32 decision), the kind::f8f6f4 GEMM against
+the product of the codes, and the FP8 block against the oracle's FP8 block (T2V, I2V,
+and the 1.3B 480P block on sampled rows)."""
+import numpy as np
+import pytest
+
+from oracle import wan_oracle as O
+from wan_inputs import WORKLOADS, make_inputs, round_bf16, sample_rows
+from gpu_util import FP8_TOL_MAX, FP8_TOL_RMS, dev, host, rel_err, rms_err, rng
+from test_gpu_block import Run, small_bf16
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+E4M3 = np.array([O.e4m3_decode(c) for c in range(256)])
+
+
+@pytest.fixture(scope="module")
+def wan():
+    import video_diffusion_transformer_wan_b200 as w
+    return w
+
+
+def _cfg(wan, dtype="bf16"):
+    return wan.make_config(128, 1, 128, dtype=dtype)
+
+
+def _rows_input(seed, M, K):
+    r = rng(seed)
+    a = r.standard_normal((M, K)) * np.exp2(r.integers(-12, 10, (M, 1)))
+    a[1] = 0.0                                   # all-zero row: scale 1
+    a[2, :7] = [448.0, -1e-8, 3e-5, 2 ** -9, 1.5 * 2 ** -9, 17.0, -19.0]
+    return a
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("M,K", [(37, 1536), (5, 8960), (300, 64)])
+def test_quantize_rows_bit_exact(wan, dtype, M, K):
+    a = _rows_input(M + K, M, K)
+    a = round_bf16(a) if dtype == "bf16" else a.astype(np.float32)
+    act = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    s = torch.empty(M, dtype=torch.float32, device="cuda")
+    wan.fp8_quantize_rows(_cfg(wan, dtype), dev(a, act), q, s)
+    torch.cuda.synchronize()
+    ref_q, ref_s = O.quantize_e4m3(np.asarray(a, np.float32), axis=-1)
+    assert np.array_equal(s.cpu().numpy(), ref_s[:, 0])
+    assert np.array_equal(E4M3[q.cpu().numpy()], ref_q)
+
+
+def test_quantize_tensor_bit_exact(wan):
+    w = round_bf16(0.02 * rng(3).standard_normal((384, 1536)))
+    q = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    wan.fp8_quantize_tensor(_cfg(wan), dev(w, torch.bfloat16), q, s)
+    torch.cuda.synchronize()
+    ref_q, ref_s = O.quantize_e4m3(np.asarray(w, np.float32))
+    assert s.item() == float(ref_s)
+    assert np.array_equal(E4M3[q.cpu().numpy()], ref_q)
+
+
+@pytest.mark.parametrize("M,N,K,epi", [(333, 1536, 1536, "store"), (300, 256, 8960, "f32"), (129, 64, 512, "f32"),
+                                       (200, 128, 1536, "store"), (257, 1536, 1536, "residual"),
+                                       (130, 4608, 1536, "gelu")])
+def test_linear_fp8(wan, M, N, K, epi):
+    r = rng(M * 7 + N + K)
+    x = round_bf16(r.standard_normal((M, K)))
+    w = round_bf16(0.02 * r.standard_normal((N, K)))
+    b = round_bf16(0.1 * r.standard_normal(N))
+    cfg = _cfg(wan)
+    xq = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    wq = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(1, dtype=torch.float32, device="cuda")
+    wan.fp8_quantize_rows(cfg, dev(x, torch.bfloat16), xq, xs)
+    wan.fp8_quantize_tensor(cfg, dev(w, torch.bfloat16), wq, ws)
+    ref = O.linear_fp8(x, w, b)
+    kind = {"store": wan.EPI_STORE, "gelu": wan.EPI_GELU, "f32": wan.EPI_F32, "residual": wan.EPI_RESIDUAL}[epi]
+    gate = gate_b = None
+    if epi in ("store", "gelu"):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    elif epi == "f32":
+        out = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    else:
+        x0 = r.standard_normal((M, N)).astype(np.float32)
+        g = r.standard_normal(N).astype(np.float32)
+        out = torch.from_numpy(x0).cuda()
+        gate = torch.from_numpy(g).cuda()
+        ref = x0 + g * ref
+    wan.linear_fp8_fwd(cfg, xq, xs, wq, ws, dev(b, torch.bfloat16), out, kind, gate=gate,
+                       rows_per_batch=M)
+    torch.cuda.synchronize()
+    if epi == "gelu":
+        ref = O.gelu_tanh(ref)
+    tol = 1e-4 if epi in ("f32", "residual") else 8e-3          # fp32 accumulation; bf16 output rounding
+    assert rel_err(host(out), ref) <= tol
+
+
+@pytest.mark.parametrize("i2v", [False, True])
+def test_block_fp8_matches_oracle(wan, i2v):
+    from video_diffusion_transformer_wan_b200.model import Fp8Block
+    w = small_bf16(i2v=i2v, dim=512, heads=4, ffn=1024)
+    r = Run(wan, w, zero_wx=False)
+    fb = Fp8Block(r.cfg, r.model.blocks[0])
+    ws = torch.empty(wan.fp8_workspace_bytes(r.cfg, w.batch, w.tokens, w.text_len, w.img_len if i2v else 0),
+                     dtype=torch.uint8, device="cuda")
+    x = r.x.clone()
+    wan.dit_block_fp8_fwd(r.cfg, x, r.e, r.ctx, r.img_ctx, fb.table, fb.scale_table, ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(x)
+    for b in range(w.batch):
+        img = None if r.img_np is None else r.img_np[b]
+        ref = O.dit_block(r.inp["x"][b], r.inp["e"][b], r.inp["blocks"][0], r.inp["ctx"][b], w.heads, img_ctx=img,
+                          fp8=True)
+        d_got, d_ref = got[b] - r.inp["x"][b], ref - r.inp["x"][b]
+        print(f"fp8 block i2v={i2v} b={b}: max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
+        assert rel_err(d_got, d_ref) <= FP8_TOL_MAX
+        assert rms_err(d_got, d_ref) <= FP8_TOL_RMS
+
+
+def test_block_fp8_full_size_sampled_rows(wan):
+    """The 1.3B 480P block (L = 32760) in FP8, 256 sampled rows against the oracle."""
+    from video_diffusion_transformer_wan_b200.model import DitModel, Fp8Block, config_for, to_device
+    w = WORKLOADS["wan13b_480p_block"]
+    inp = make_inputs(w, seed=0)
+    cfg = config_for(w)
+    model = DitModel(cfg, inp)
+    fb = Fp8Block(cfg, model.blocks[0])
+    x = to_device(inp["x"], torch.float32)
+    e = to_device(inp["e"], torch.float32)
+    ctx = to_device(inp["ctx"], torch.bfloat16)
+    ws = torch.empty(wan.fp8_workspace_bytes(cfg, 1, w.tokens, w.text_len), dtype=torch.uint8, device="cuda")
+    wan.dit_block_fp8_fwd(cfg, x, e, ctx, None, fb.table, fb.scale_table, ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    rows = sample_rows(w.tokens)
+    got = x[0].cpu().numpy().astype(np.float64)[rows]
+    ref = O.dit_block(inp["x"][0], inp["e"][0], inp["blocks"][0], inp["ctx"][0], w.heads, rows=rows, fp8=True)
+    d_got, d_ref = got - inp["x"][0][rows], ref - inp["x"][0][rows]
+    print(f"fp8 block 1.3B sampled rows: max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
+    assert rel_err(d_got, d_ref) <= FP8_TOL_MAX
+    assert rms_err(d_got, d_ref) <= FP8_TOL_RMS

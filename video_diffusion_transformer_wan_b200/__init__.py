@@ -15,10 +15,11 @@ from typing import Dict, Optional, Sequence
 __all__ = [
     "LIB_PATH", "lib", "WanError", "WAN_F32", "WAN_BF16", "EPI_STORE", "EPI_GELU", "EPI_RESIDUAL", "EPI_F32",
     "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights",
-    "ImageMlpWeights", "StackWeights", "DiffusionCache", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
+    "ImageMlpWeights", "StackWeights", "DiffusionCache", "Fp8Scales", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
     "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
     "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd",
+    "fp8_quantize_rows", "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd",
     "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
@@ -62,6 +63,11 @@ class DiffusionCache(ctypes.Structure):
     _fields_ = [("attn_start", _i), ("attn_interval", _i), ("cfg_start", _i), ("cfg_interval", _i)]
 
 
+class Fp8Scales(ctypes.Structure):
+    """Device pointers of the per-tensor scales of a block's E4M3 weights."""
+    _fields_ = [(n, _vp) for n in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]]
+
+
 class WanError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -102,6 +108,13 @@ def _load() -> ctypes.CDLL:
         "wan_sp_qkv_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(BlockWeights), P(_vp), _vp]),
         "wan_sp_attn_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(_vp), _vp]),
         "wan_sp_out_fwd": (_i, [P(Config), _i, _vp, P(BlockWeights), _vp, _vp, _i, _i, _vp]),
+        "wan_fp8_quantize_rows": (_i, [P(Config), _vp, _i, _i, _vp, _vp, _vp]),
+        "wan_fp8_quantize_tensor": (_i, [P(Config), _vp, _i64, _vp, _vp, _vp]),
+        "wan_linear_fp8_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i,
+                                    _vp]),
+        "wan_fp8_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i]),
+        "wan_dit_block_fp8_fwd": (_i, [P(Config), _vp, _vp, _vp, _i, _vp, _i, P(BlockWeights), P(Fp8Scales), _i,
+                                       _i, _vp, _sz, _vp]),
         "wan_launch_count": (_i64, []),
         "wan_trace_enable": (_i, [_i]),
         "wan_trace_reset": (_i, []),
@@ -262,6 +275,41 @@ def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, 
                                     _p(img_ctx), Li, _cache_ref(cache), _p(latent_out), *_ws(ws),
                                     _stream(stream)),
            "wan_sample_euler_cfg")
+
+
+def fp8_quantize_rows(cfg, x, q, scale, stream=None):
+    """x [..., K] act -> q [..., K] uint8 (E4M3 codes), scale [rows] fp32."""
+    K = x.shape[-1]
+    _check(_lib().wan_fp8_quantize_rows(ctypes.byref(cfg), _p(x), x.numel() // K, K, _p(q), _p(scale),
+                                     _stream(stream)), "wan_fp8_quantize_rows")
+
+
+def fp8_quantize_tensor(cfg, x, q, scale, stream=None):
+    """x act (any shape) -> q uint8 codes, scale [1] fp32 (one scale for the tensor)."""
+    _check(_lib().wan_fp8_quantize_tensor(ctypes.byref(cfg), _p(x), x.numel(), _p(q), _p(scale),
+                                       _stream(stream)), "wan_fp8_quantize_tensor")
+
+
+def linear_fp8_fwd(cfg, A, a_scale, W, w_scale, bias, out, epilogue, gate=None, gate_bias=None,
+                   gate_batch_stride=0, rows_per_batch=1, stream=None):
+    K = A.shape[-1]
+    M = A.numel() // K
+    N = W.shape[0]
+    _check(_lib().wan_linear_fp8_fwd(ctypes.byref(cfg), _p(A), _p(a_scale), _p(W), _p(w_scale), _p(bias), _p(out),
+                                  M, N, K, epilogue, _p(gate), _p(gate_bias), gate_batch_stride, rows_per_batch,
+                                  _stream(stream)), "wan_linear_fp8_fwd")
+
+
+def fp8_workspace_bytes(cfg: Config, B: int, L: int, Lc: int, Li: int = 0) -> int:
+    return int(_lib().wan_fp8_workspace_bytes(ctypes.byref(cfg), B, L, Lc, Li))
+
+
+def dit_block_fp8_fwd(cfg, x_inout, e, ctx, img_ctx, bw: BlockWeights, sc: Fp8Scales, ws, stream=None):
+    B, L, _ = x_inout.shape
+    Li = 0 if img_ctx is None else img_ctx.shape[1]
+    _check(_lib().wan_dit_block_fp8_fwd(ctypes.byref(cfg), _p(x_inout), _p(e), _p(ctx), ctx.shape[1], _p(img_ctx),
+                                     Li, ctypes.byref(bw), ctypes.byref(sc), B, L, *_ws(ws), _stream(stream)),
+           "wan_dit_block_fp8_fwd")
 
 
 def _ptr_table(bufs):

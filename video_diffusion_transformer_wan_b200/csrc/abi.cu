@@ -89,8 +89,21 @@ EncodeTiledFn encode_fn() {
 }
 }  // namespace
 
+static bool make_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box);
+
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                     const uint32_t* box) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+bool make_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                  const uint32_t* box) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes, box);
+}
+
+static bool make_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t d[5], st[4];
@@ -101,7 +114,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
     es[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx,
+  return fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, st, bx,
             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -127,6 +140,11 @@ int check_ptr(const void* p) {
   return WAN_OK;
 }
 int check_opt_ptr(const void* p) { return p ? check_ptr(p) : WAN_OK; }
+// Non-null and 4-byte aligned (fp32 scalars and scale vectors).
+int check_ptr_any(const void* p) {
+  if (!p) return WAN_ERR_NULL;
+  return (reinterpret_cast<uintptr_t>(p) & 3u) == 0 ? WAN_OK : WAN_ERR_ALIGN;
+}
 
 // `attention`: the call runs attention, which fixes head_dim (128 on the bf16 tensor-core
 // path, <= 128 on the fp32 path).
@@ -624,6 +642,164 @@ int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const 
   const float* gb = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
   return gemm(cfg, o, D, w->w_o, w->b_o, x_inout, B * Ll, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, Ll),
               as_stream(stream));
+}
+
+// ------------------------------------------------------------------ FP8 (E4M3)
+namespace {
+// FP8 block workspace: the bf16 block's layout (its h region unused), then E4M3 codes
+// of the block inputs ([B*L, max(D, F)], reused by each linear layer in turn), codes of
+// the text / image context ([B*max(Lc, Li), D]) and the per-row scales of both.
+struct Fp8Layout {
+  Layout base;
+  size_t codes, ctx_codes, scales, ctx_scales, total;
+};
+Fp8Layout fp8_layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
+  Fp8Layout l;
+  l.base = layout(c, B, L, Lc, Li);
+  const size_t BL = static_cast<size_t>(B) * L;
+  const size_t Lx = static_cast<size_t>(B) * (Lc > Li ? Lc : Li);
+  const size_t wmax = c->ffn_dim > c->dim ? c->ffn_dim : c->dim;
+  l.codes = l.base.total;
+  l.ctx_codes = l.codes + align_up(BL * wmax);
+  l.scales = l.ctx_codes + align_up(Lx * c->dim);
+  l.ctx_scales = l.scales + align_up(BL * 4);
+  l.total = l.ctx_scales + align_up(Lx * 4);
+  return l;
+}
+
+int check_scales(const wan_fp8_scales* sc, bool with_img) {
+  WAN_REQUIRE(sc, WAN_ERR_NULL);
+  WAN_TRY(check_ptr_any(sc->qkv));
+  WAN_TRY(check_ptr_any(sc->o));
+  WAN_TRY(check_ptr_any(sc->cq));
+  WAN_TRY(check_ptr_any(sc->ckv));
+  WAN_TRY(check_ptr_any(sc->co));
+  WAN_TRY(check_ptr_any(sc->ffn1));
+  WAN_TRY(check_ptr_any(sc->ffn2));
+  if (with_img) WAN_TRY(check_ptr_any(sc->ckv_img));
+  return WAN_OK;
+}
+
+int e4m3_gemm(const void* A, const float* as, const void* W, const float* wsc, const void* bias, void* out, int M,
+              int N, int K, const GemmEpi& ep, cudaStream_t s) {
+  return launch_gemm_e4m3(A, K, as, W, wsc, bias, out, M, N, K, ep, s);
+}
+}  // namespace
+
+int wan_fp8_quantize_rows(const wan_dit_config* cfg, const void* x, int M, int K, void* q, float* scale,
+                          void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(x));
+  WAN_TRY(check_ptr(q));
+  WAN_TRY(check_ptr_any(scale));
+  WAN_REQUIRE(M >= 0 && K > 0 && K % 16 == 0, WAN_ERR_SHAPE);
+  return launch_quantize_rows(x, K, M, K, false, q, scale, cfg->dtype, as_stream(stream));
+}
+
+int wan_fp8_quantize_tensor(const wan_dit_config* cfg, const void* x, int64_t n, void* q, float* scale,
+                            void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  WAN_TRY(check_ptr(x));
+  WAN_TRY(check_ptr(q));
+  WAN_TRY(check_ptr_any(scale));
+  WAN_REQUIRE(n > 0 && n % 16 == 0, WAN_ERR_SHAPE);
+  return launch_quantize_tensor(x, n, q, scale, cfg->dtype, as_stream(stream));
+}
+
+int wan_linear_fp8_fwd(const wan_dit_config* cfg, const void* A, const float* a_scale, const void* W,
+                       const float* w_scale, const void* bias, void* out, int M, int N, int K, int epilogue,
+                       const float* gate, const float* gate_bias, int64_t gate_batch_stride, int rows_per_batch,
+                       void* stream) {
+  WAN_TRY(check_cfg(cfg));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  WAN_TRY(check_ptr(A));
+  WAN_TRY(check_ptr(W));
+  WAN_TRY(check_ptr_any(a_scale));
+  WAN_TRY(check_ptr_any(w_scale));
+  WAN_TRY(check_opt_ptr(bias));
+  WAN_TRY(check_ptr(out));
+  WAN_TRY(check_opt_ptr(gate));
+  WAN_TRY(check_opt_ptr(gate_bias));
+  WAN_REQUIRE(M >= 0 && N > 0 && K > 0 && N % 8 == 0 && K % 16 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(epilogue >= WAN_EPI_STORE && epilogue <= WAN_EPI_F32, WAN_ERR_SHAPE);
+  if (epilogue == WAN_EPI_RESIDUAL)
+    WAN_REQUIRE(rows_per_batch > 0 && gate_batch_stride >= 0 && gate_batch_stride % 4 == 0, WAN_ERR_SHAPE);
+  GemmEpi ep = epilogue == WAN_EPI_RESIDUAL ? epi_residual(N, gate, gate_bias, gate_batch_stride, rows_per_batch)
+                                            : epi_store(N, epilogue);
+  return e4m3_gemm(A, a_scale, W, w_scale, bias, out, M, N, K, ep, as_stream(stream));
+}
+
+size_t wan_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int Li) {
+  if (check_cfg(cfg) != WAN_OK || B < 0 || L < 0 || Lc < 0 || Li < 0) return 0;
+  return fp8_layout(cfg, B, L, Lc, Li).total;
+}
+
+int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x, const float* e, const void* ctx, int Lc,
+                          const void* img_ctx, int Li, const wan_block_weights* w, const wan_fp8_scales* sc, int B,
+                          int L, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  const bool with_img = img_ctx && Li > 0;
+  WAN_TRY(check_block_w(cfg, w, with_img));
+  WAN_TRY(check_scales(sc, with_img));
+  WAN_TRY(check_ptr(x));
+  WAN_TRY(check_ptr(e));
+  WAN_TRY(check_ptr(ctx));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_REQUIRE(Lc > 0 && cfg->dim % 16 == 0 && cfg->ffn_dim % 16 == 0, WAN_ERR_SHAPE);
+  const int li = with_img ? Li : 0;
+  WAN_TRY(check_tokens(cfg, B, L, Lc, li));
+  WAN_TRY(check_ptr(workspace));
+  const Fp8Layout fl = fp8_layout(cfg, B, L, Lc, li);
+  WAN_REQUIRE(ws_bytes >= fl.total, WAN_ERR_WORKSPACE);
+  if (B == 0 || L == 0) return WAN_OK;
+  cudaStream_t s = as_stream(stream);
+  const int D = cfg->dim, Fd = cfg->ffn_dim;
+  const int M = B * L;
+  const int64_t rows = M;
+  uint8_t* R = at(workspace, fl.base.big);
+  void* codes = at(workspace, fl.codes);
+  void* ctx_codes = at(workspace, fl.ctx_codes);
+  float* scales = reinterpret_cast<float*>(at(workspace, fl.scales));
+  float* ctx_scales = reinterpret_cast<float*>(at(workspace, fl.ctx_scales));
+  const size_t MD = static_cast<size_t>(M) * D * 2;  // bytes of one [M, D] bf16 slab
+  // self-attention
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 0, codes, scales, cfg->eps, s));
+  void* qkv = R;
+  void* o = R + 3 * MD;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_qkv, sc->qkv, w->b_qkv, qkv, M, 3 * D, D, epi_store(3 * D), s));
+  WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s));
+  WAN_TRY(launch_quantize_rows(o, D, M, D, false, codes, scales, WAN_BF16, s));
+  const float* gb_msa = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_o, sc->o, w->b_o, x, M, D, D, epi_residual(D, e + 2 * D, gb_msa, 6 * D, L), s));
+  // cross-attention
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, nullptr, nullptr, -1, codes, scales, cfg->eps, s));
+  void* q = R;
+  void* ocat = R + 3 * MD;
+  void* kvt = R + 5 * MD;
+  void* kvi = static_cast<uint8_t*>(kvt) + static_cast<size_t>(B) * Lc * 2 * D * 2;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_cq, sc->cq, w->b_cq, q, M, D, D, epi_store(D), s));
+  WAN_TRY(launch_quantize_rows(ctx, D, B * Lc, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
+  WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv, sc->ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, epi_store(2 * D), s));
+  const int ow = with_img ? 2 * D : D;
+  WAN_TRY(launch_attn_tc({q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, cfg->heads, L, Lc, s));
+  if (with_img) {
+    WAN_TRY(launch_quantize_rows(img_ctx, D, B * li, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
+    WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv_img, sc->ckv_img, w->b_ckv_img, kvi, B * li, 2 * D, D,
+                      epi_store(2 * D), s));
+    WAN_TRY(launch_attn_tc({q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, cfg->heads, L, li, s));
+  }
+  // the text and image outputs are summed while quantised
+  WAN_TRY(launch_quantize_rows(ocat, ow, M, D, with_img, codes, scales, WAN_BF16, s));
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_co, sc->co, w->b_co, x, M, D, D, epi_residual(D, nullptr, nullptr, 0, L), s));
+  // FFN
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 1, codes, scales, cfg->eps, s));
+  void* hid = R;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_1, sc->ffn1, w->b_1, hid, M, Fd, D, epi_store(Fd, WAN_EPI_GELU), s));
+  WAN_TRY(launch_quantize_rows(hid, Fd, M, Fd, false, codes, scales, WAN_BF16, s));
+  const float* gb_ffn = w->mod_bias ? w->mod_bias + 5 * D : nullptr;
+  return e4m3_gemm(codes, scales, w->w_2, sc->ffn2, w->b_2, x, M, D, Fd,
+                   epi_residual(D, e + 5 * D, gb_ffn, 6 * D, L), s);
 }
 
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W, int Lc,

@@ -41,8 +41,8 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 template <int BN>
 struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int kABytes = kBM * kBK * 2;
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kABytes = kBM * 128;  // 128-byte rows: 64 bf16 or 128 E4M3 elements
+  static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
@@ -54,6 +54,9 @@ struct GemmParams {
   int wk_period_blocks;  // > 0: W column block = k block mod this
   int m_blocks, n_blocks;
   int group_m;           // row blocks per tile group
+  int bk;                // elements of K per stage (64 bf16, 128 E4M3)
+  const float* a_scale;  // E4M3: per-row scale of A (acc * a_scale[m] * w_scale[0]), else NULL
+  const float* w_scale;
   const __nv_bfloat16* bias;
   void* out;
   GemmEpi epi;
@@ -82,6 +85,11 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.a_scale) {
+    const float sc = __ldg(p.a_scale + row) * __ldg(p.w_scale);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= sc;
+  }
   const bool full = n0 + 32 <= p.N;
   if (p.bias) {
     if (full) {
@@ -199,11 +207,12 @@ __device__ __forceinline__ void epilogue_pair(const GemmParams& p, int row, int 
   const float* gate = p.epi.gate ? p.epi.gate + static_cast<int64_t>(row / p.epi.rows_per_batch) * p.epi.gate_bstride + n0
                                  : nullptr;
   const float* gb = p.epi.gate_bias ? p.epi.gate_bias + n0 : nullptr;
+  const float sc = p.a_scale ? __ldg(p.a_scale + row) * __ldg(p.w_scale) : 1.0f;
 #pragma unroll
   for (int g = 0; g < 16; ++g) {
     const uint32_t* rr = g < 8 ? r0 + 4 * g : r1 + 4 * (g - 8);
-    float v0 = __uint_as_float(rr[0]), v1 = __uint_as_float(rr[1]);
-    float v2 = __uint_as_float(rr[2]), v3 = __uint_as_float(rr[3]);
+    float v0 = __uint_as_float(rr[0]) * sc, v1 = __uint_as_float(rr[1]) * sc;
+    float v2 = __uint_as_float(rr[2]) * sc, v3 = __uint_as_float(rr[3]) * sc;
     if (p.bias) {
       const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.bias + n0) + g);
       const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
@@ -226,10 +235,8 @@ __device__ __forceinline__ void epilogue_pair(const GemmParams& p, int row, int 
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                        const GemmParams p) {
+template <int BN, bool kF8>
+__device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -288,8 +295,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           const int kbw = p.wk_period_blocks > 0 ? kb % p.wk_period_blocks : kb;
-          tma_load_2d(sA + stage * C::kABytes, &mapA, &full[stage], kb * kBK, m0);
-          tma_load_2d(sB + stage * C::kBBytes, &mapB, &full[stage], kbw * kBK, n0);
+          tma_load_2d(sA + stage * C::kABytes, &mapA, &full[stage], kb * p.bk, m0);
+          tma_load_2d(sB + stage * C::kBBytes, &mapB, &full[stage], kbw * p.bk, n0);
           ++issued;
           if (++stage == C::kStages) {
             stage = 0;
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, 0);
+      const uint32_t idesc = kF8 ? idesc_e4m3_f32(kBM, BN) : idesc_bf16_f32(kBM, BN, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -324,10 +331,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_addr = smem_u32(sA + stage * C::kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per MMA: 16 bf16 or 32 E4M3
             const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + k * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            if (kF8)
+              tc_mma_e4m3(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == C::kStages) {
@@ -383,6 +393,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                        const GemmParams p) {
+  gemm_body<BN, false>(mapA, mapB, p);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_e4m3_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                        const GemmParams p) {
+  gemm_body<BN, true>(mapA, mapB, p);
+}
+
 int sm_count() {
   static int counts[64] = {0};
   int dev = 0;
@@ -396,32 +420,40 @@ int sm_count() {
   return counts[dev];
 }
 
-template <int BN>
+template <int BN, bool kF8>
 int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
-              int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+              int w_k_period, const GemmEpi& epi, cudaStream_t s, const float* a_scale = nullptr,
+              const float* w_scale = nullptr) {
   using C = GemmCfg<BN>;
+  constexpr int bk = kF8 ? 128 : 64;  // elements per 128-byte row
+  constexpr int es = kF8 ? 1 : 2;
   CUtensorMap mapA, mapB;
   const uint64_t dimsA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * 2};
-  const uint32_t boxA[2] = {kBK, kBM};
+  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * es};
+  const uint32_t boxA[2] = {bk, kBM};
   const int kw = w_k_period > 0 ? w_k_period : K;
   const uint64_t dimsB[2] = {static_cast<uint64_t>(kw), static_cast<uint64_t>(N)};
-  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * 2};
-  const uint32_t boxB[2] = {kBK, BN};
-  if (!make_tmap_bf16(&mapA, A, 2, dimsA, strA, boxA) || !make_tmap_bf16(&mapB, W, 2, dimsB, strB, boxB))
-    return WAN_ERR_CUDA;
+  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * es};
+  const uint32_t boxB[2] = {bk, BN};
+  const bool maps_ok = kF8 ? make_tmap_u8(&mapA, A, 2, dimsA, strA, boxA) && make_tmap_u8(&mapB, W, 2, dimsB, strB, boxB)
+                           : make_tmap_bf16(&mapA, A, 2, dimsA, strA, boxA) &&
+                                 make_tmap_bf16(&mapB, W, 2, dimsB, strB, boxB);
+  if (!maps_ok) return WAN_ERR_CUDA;
   GemmParams p;
   p.M = M;
   p.N = N;
   p.K = K;
-  p.k_blocks = (K + kBK - 1) / kBK;
-  p.wk_period_blocks = w_k_period > 0 ? w_k_period / kBK : 0;
+  p.bk = bk;
+  p.k_blocks = (K + bk - 1) / bk;
+  p.wk_period_blocks = w_k_period > 0 ? w_k_period / bk : 0;
   p.m_blocks = (M + kBM - 1) / kBM;
   p.n_blocks = (N + BN - 1) / BN;
   {
-    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * 2 * kBM);
+    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * es * kBM);
     p.group_m = static_cast<int>(slab_rows < 1 ? 1 : (slab_rows > p.m_blocks ? p.m_blocks : slab_rows));
   }
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.out = out;
   p.epi = epi;
@@ -430,12 +462,19 @@ int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void*
   int dev = 0;
   cudaGetDevice(&dev);
   std::call_once(once[dev & 63], [] {
-    cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(C::kSmemBytes));
+    if (kF8)
+      cudaFuncSetAttribute(gemm_e4m3_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(C::kSmemBytes));
+    else
+      cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(C::kSmemBytes));
   });
   const int tiles = p.m_blocks * p.n_blocks;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  gemm_bf16_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
+  if (kF8)
+    gemm_e4m3_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
+  else
+    gemm_bf16_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
   return check_launch();
 }
 
@@ -449,11 +488,27 @@ int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, 
   trace_launch_begin(WAN_KIND_GEMM, s, 2.0 * M * N * K);
   int st;
   if (N <= 64)
-    st = launch_bn<64>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+    st = launch_bn<64, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   else if (N <= 128)
-    st = launch_bn<128>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+    st = launch_bn<128, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   else
-    st = launch_bn<256>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+    st = launch_bn<256, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  trace_launch_end(WAN_KIND_GEMM, s);
+  return st;
+}
+
+int launch_gemm_e4m3(const void* A, int64_t lda, const float* a_scale, const void* W, const float* w_scale,
+                     const void* bias, void* out, int M, int N, int K, const GemmEpi& epi, cudaStream_t s) {
+  if (M == 0 || N == 0) return WAN_OK;
+  if (K % 16 != 0 || lda % 16 != 0 || N % 8 != 0) return WAN_ERR_SHAPE;
+  trace_launch_begin(WAN_KIND_GEMM, s, 2.0 * M * N * K);
+  int st;
+  if (N <= 64)
+    st = launch_bn<64, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
+  else if (N <= 128)
+    st = launch_bn<128, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
+  else
+    st = launch_bn<256, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
   trace_launch_end(WAN_KIND_GEMM, s);
   return st;
 }

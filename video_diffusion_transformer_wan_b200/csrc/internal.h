@@ -29,11 +29,18 @@ inline int check_launch() {
 // in bytes for dims >= 1. Returns false if the driver rejects the map.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
+// The same for 8-bit elements (E4M3 codes).
+bool make_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box);
 
 // ---------------------------------------------------------------- kernels
 // LayerNorm (+ modulation). rows = B*L; e/mod_bias may be NULL (chunk < 0: plain LN).
 int launch_layernorm(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias,
                      int chunk, void* out, int dtype, float eps, cudaStream_t s);
+// The same LN (+ modulation) writing E4M3 codes [rows, D] and one fp32 scale per row
+// (amax / 448, 1 for an all-zero row). D in {512, 1536, 5120}; WAN_ERR_UNSUPPORTED else.
+int launch_layernorm_e4m3(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias,
+                          int chunk, void* out, float* row_scale, float eps, cudaStream_t s);
 
 constexpr int kMaxSeqRanks = 8;  // sequence-parallel group size limit
 
@@ -60,6 +67,18 @@ enum : int { kEpiHeadScatter = 100, kEpiSeqScatter = 101 };
 // columns and the k-th reduction index reads W column (k mod w_k_period).
 int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
                    int w_k_period, const GemmEpi& epi, cudaStream_t s);
+// E4M3 codes of x [M, K] (act dtype, row stride x_stride elements; with sum_halves the
+// row is x[:, :K] + x[:, K:2K]) with one scale per row. K, x_stride multiples of 8.
+int launch_quantize_rows(const void* x, int64_t x_stride, int M, int K, bool sum_halves, void* q, float* scale,
+                         int dtype, cudaStream_t s);
+// E4M3 codes of a whole tensor (n elements, multiple of 8) with one scale; scale[0] is
+// used as the amax accumulator and holds the scale when the work completes.
+int launch_quantize_tensor(const void* x, int64_t n, void* q, float* scale, int dtype, cudaStream_t s);
+// E4M3 tcgen05 GEMM (kind::f8f6f4): out = epi(a_scale[m] * w_scale[0] * (A[M,K] W[N,K]^T)
+// + bias) with A and W E4M3 codes (row stride lda and K bytes), a_scale [M] and w_scale
+// [1] fp32 in device memory. K and lda multiples of 16.
+int launch_gemm_e4m3(const void* A, int64_t lda, const float* a_scale, const void* W, const float* w_scale,
+                     const void* bias, void* out, int M, int N, int K, const GemmEpi& epi, cudaStream_t s);
 // fp32 SIMT GEMM with the same semantics (fp32 activations and weights).
 int launch_gemm_simt(const float* A, int64_t lda, const float* W, const float* bias, void* out, int M, int N,
                      int K, int w_k_period, const GemmEpi& epi, cudaStream_t s);

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace wan {
 namespace {
@@ -68,10 +69,30 @@ __device__ __forceinline__ float group_sum(float v, float* red, int t) {
   return v;
 }
 
+template <int TPR>
+__device__ __forceinline__ float group_max(float v, float* red, int t) {
+  constexpr int W = TPR < 32 ? TPR : 32;
+#pragma unroll
+  for (int o = W / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o, W));
+  if constexpr (TPR > 32) {
+    constexpr int NW = TPR / 32;
+    if ((t & 31) == 0) red[t >> 5] = v;
+    __syncthreads();
+    v = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) v = fmaxf(v, red[w]);
+    __syncthreads();
+  }
+  return v;
+}
+
+// OutT = uint8_t writes E4M3 codes of h / s with one scale per row, s = amax(|h|) / 448
+// (1 for an all-zero row), into out and row_scale.
 template <int TPR, int NU, bool MOD, typename OutT>
 __global__ void __launch_bounds__(norm_block<TPR>()) layernorm_mod_kernel(
     const float* __restrict__ x, int64_t rows, int D, int L, const float* __restrict__ e,
-    const float* __restrict__ mod_bias, int chunk, OutT* __restrict__ out, float eps) {
+    const float* __restrict__ mod_bias, int chunk, OutT* __restrict__ out, float eps,
+    float* __restrict__ row_scale) {
   constexpr int G = norm_block<TPR>() / TPR;  // row groups per block
   __shared__ float red[TPR > 32 ? TPR / 32 : 1];
   const int group = threadIdx.x / TPR;
@@ -79,8 +100,8 @@ __global__ void __launch_bounds__(norm_block<TPR>()) layernorm_mod_kernel(
   const int64_t stride = static_cast<int64_t>(gridDim.x) * G;
   const float inv_d = 1.0f / static_cast<float>(D);
 
-  float shv[MOD ? NU : 1][8];
-  float scv[MOD ? NU : 1][8];
+  float shv[MOD ? NU : 1][8] = {};
+  float scv[MOD ? NU : 1][8] = {};
   int64_t cur_b = -1;
   float va[NU][8], vb[NU][8];
 
@@ -111,35 +132,81 @@ __global__ void __launch_bounds__(norm_block<TPR>()) layernorm_mod_kernel(
         q += c * c;
       }
     const float rstd = 1.0f / sqrtf(group_sum<TPR>(q, red, t) * inv_d + eps);
-    if (r >= rows) return;
-    if constexpr (MOD) {
-      const int64_t b = r / L;
-      if (b != cur_b) {
-        cur_b = b;
-        const float* sh = e + (b * 6 + 3 * chunk) * D;
-        const float* sc = sh + D;
-        const float* bsh = mod_bias ? mod_bias + (3 * chunk) * D : nullptr;
+    if constexpr (sizeof(OutT) == 1) {
+      // E4M3: the row's amax is a group reduction, taken by every group (also those past
+      // the last row, which store nothing) so that the block's barriers stay uniform.
+      if (MOD && r < rows) {
+        const int64_t b = r / L;
+        if (b != cur_b) {
+          cur_b = b;
+          const float* sh = e + (b * 6 + 3 * chunk) * D;
+          const float* sc = sh + D;
+          const float* bsh = mod_bias ? mod_bias + (3 * chunk) * D : nullptr;
 #pragma unroll
-        for (int u = 0; u < NU; ++u) {
-          const int col = (u * TPR + t) * 8;
+          for (int u = 0; u < NU; ++u) {
+            const int col = (u * TPR + t) * 8;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            shv[u][i] = sh[col + i] + (bsh ? bsh[col + i] : 0.f);
-            scv[u][i] = 1.0f + sc[col + i] + (bsh ? bsh[D + col + i] : 0.f);
+            for (int i = 0; i < 8; ++i) {
+              shv[u][i] = sh[col + i] + (bsh ? bsh[col + i] : 0.f);
+              scv[u][i] = 1.0f + sc[col + i] + (bsh ? bsh[D + col + i] : 0.f);
+            }
           }
         }
       }
-    }
-    OutT* orow = out + r * D;
+      float am = 0.f;
 #pragma unroll
-    for (int u = 0; u < NU; ++u) {
-      float o[8];
+      for (int u = 0; u < NU; ++u)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        o[i] = (v[u][i] - mean) * rstd;
-        if constexpr (MOD) o[i] = fmaf(o[i], scv[u][i], shv[u][i]);
+        for (int i = 0; i < 8; ++i) {
+          v[u][i] = (v[u][i] - mean) * rstd;
+          if constexpr (MOD) v[u][i] = fmaf(v[u][i], scv[u][i], shv[u][i]);
+          am = fmaxf(am, fabsf(v[u][i]));
+        }
+      am = group_max<TPR>(am, red, t);
+      if (r >= rows) return;
+      const float sc = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      if (t == 0) row_scale[r] = sc;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(out) + r * D;
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        uint2 c;
+        c.x = pack_e4m3x4(__fdiv_rn(v[u][0], sc), __fdiv_rn(v[u][1], sc), __fdiv_rn(v[u][2], sc),
+                          __fdiv_rn(v[u][3], sc));
+        c.y = pack_e4m3x4(__fdiv_rn(v[u][4], sc), __fdiv_rn(v[u][5], sc), __fdiv_rn(v[u][6], sc),
+                          __fdiv_rn(v[u][7], sc));
+        *reinterpret_cast<uint2*>(orow + (u * TPR + t) * 8) = c;
       }
-      store8<OutT>(orow + (u * TPR + t) * 8, o);
+    } else {
+      if (r >= rows) return;
+      if constexpr (MOD) {
+        const int64_t b = r / L;
+        if (b != cur_b) {
+          cur_b = b;
+          const float* sh = e + (b * 6 + 3 * chunk) * D;
+          const float* sc = sh + D;
+          const float* bsh = mod_bias ? mod_bias + (3 * chunk) * D : nullptr;
+#pragma unroll
+          for (int u = 0; u < NU; ++u) {
+            const int col = (u * TPR + t) * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              shv[u][i] = sh[col + i] + (bsh ? bsh[col + i] : 0.f);
+              scv[u][i] = 1.0f + sc[col + i] + (bsh ? bsh[D + col + i] : 0.f);
+            }
+          }
+        }
+      }
+      OutT* orow = out + r * D;
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          o[i] = (v[u][i] - mean) * rstd;
+          if constexpr (MOD) o[i] = fmaf(o[i], scv[u][i], shv[u][i]);
+        }
+        store8<OutT>(orow + (u * TPR + t) * 8, o);
+      }
     }
   };
 
@@ -221,7 +288,7 @@ int num_sms() {
 
 template <typename OutT, int TPR, int NU, bool MOD>
 int launch_fixed(const float* x, int64_t rows, int D, int L, const float* e, const float* mb, int chunk,
-                 OutT* out, float eps, cudaStream_t s) {
+                 OutT* out, float eps, cudaStream_t s, float* row_scale = nullptr) {
   constexpr int BT = norm_block<TPR>();
   constexpr int G = BT / TPR;
   auto kern = layernorm_mod_kernel<TPR, NU, MOD, OutT>;
@@ -236,7 +303,7 @@ int launch_fixed(const float* x, int64_t rows, int D, int L, const float* e, con
   int64_t blocks = (rows + G - 1) / G;
   const int64_t cap = static_cast<int64_t>(per_sm[dev & 63]) * num_sms();
   if (blocks > cap) blocks = cap;
-  kern<<<static_cast<unsigned>(blocks), BT, 0, s>>>(x, rows, D, L, e, mb, chunk, out, eps);
+  kern<<<static_cast<unsigned>(blocks), BT, 0, s>>>(x, rows, D, L, e, mb, chunk, out, eps, row_scale);
   return check_launch();
 }
 
@@ -274,7 +341,34 @@ int launch_typed(const float* x, int64_t rows, int D, int L, const float* e, con
                     : launch_mod<OutT, false>(x, rows, D, L, e, mb, chunk, out, eps, s);
 }
 
+template <bool MOD>
+int launch_e4m3(const float* x, int64_t rows, int D, int L, const float* e, const float* mb, int chunk, uint8_t* out,
+                float* row_scale, float eps, cudaStream_t s) {
+  const int units = D / 8;
+#define WAN_LN_CASE(TPR, NU)                                                                             \
+  if (units == (TPR) * (NU))                                                                             \
+    return launch_fixed<uint8_t, TPR, NU, MOD>(x, rows, D, L, e, mb, chunk, out, eps, s, row_scale);
+  WAN_LN_CASE(32, 2)     // D = 512
+  WAN_LN_CASE(64, 3)     // D = 1536
+  WAN_LN_CASE(128, 5)    // D = 5120
+#undef WAN_LN_CASE
+  return WAN_ERR_UNSUPPORTED;
+}
+
 }  // namespace
+
+int launch_layernorm_e4m3(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias,
+                          int chunk, void* out, float* row_scale, float eps, cudaStream_t s) {
+  if (rows == 0) return WAN_OK;
+  if (D % 8 != 0) return WAN_ERR_UNSUPPORTED;
+  trace_launch_begin(WAN_KIND_NORM, s, static_cast<double>(rows) * (D * 5.0 + 4.0));
+  const int st = chunk >= 0 ? launch_e4m3<true>(x, rows, D, L, e, mod_bias, chunk, static_cast<uint8_t*>(out),
+                                                row_scale, eps, s)
+                            : launch_e4m3<false>(x, rows, D, L, e, mod_bias, chunk, static_cast<uint8_t*>(out),
+                                                 row_scale, eps, s);
+  trace_launch_end(WAN_KIND_NORM, s);
+  return st;
+}
 
 int launch_layernorm(const float* x, int64_t rows, int D, int L, const float* e, const float* mod_bias, int chunk,
                      void* out, int dtype, float eps, cudaStream_t s) {

@@ -65,9 +65,39 @@ def _sample(a) -> dict:
                 tflops_uncached_equivalent=flops_step * a.steps / ms / 1e9)
 
 
+def _block(a) -> dict:
+    """One DiT block call (bf16 or FP8 linear layers) on a workload's shapes."""
+    from wan_inputs import WORKLOADS, make_inputs
+
+    from .model import DitModel, Fp8Block, config_for, to_device
+    w = WORKLOADS[a.workload]
+    inp = make_inputs(w, seed=0, n_blocks=1)
+    cfg = config_for(w)
+    model = DitModel(cfg, inp)
+    x0 = to_device(inp["x"], torch.float32)
+    e = to_device(inp["e"], torch.float32)
+    ctx = to_device(inp["ctx"], model.act)
+    x = x0.clone()
+    B, L = w.batch, w.tokens
+    if a.fp8:
+        fb = Fp8Block(cfg, model.blocks[0])
+        ws = torch.empty(wan.fp8_workspace_bytes(cfg, B, L, w.text_len), dtype=torch.uint8, device="cuda")
+        ms = _time(lambda: wan.dit_block_fp8_fwd(cfg, x, e, ctx, None, fb.table, fb.scale_table, ws), a.iters,
+                   a.warmup)
+    else:
+        ws = torch.empty(wan.workspace_bytes(cfg, B, L, w.text_len), dtype=torch.uint8, device="cuda")
+        ms = _time(lambda: wan.dit_block_fwd(cfg, x, e, ctx, None, model.block_tables[0], ws), a.iters, a.warmup)
+    D, F, Lc = w.dim, w.ffn, w.text_len
+    flops = B * (2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * Lc * D * D + 4 * L * Lc * D
+                 + 4 * L * D * F)
+    return dict(workload=w.name, fp8=a.fp8, ms=ms, tokens_per_s=B * L / (ms / 1e3), tflops=flops / ms / 1e9)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample"])
+    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block"])
+    ap.add_argument("--fp8", action="store_true", help="gemm / block: E4M3 operands (kind::f8f6f4)")
+    ap.add_argument("--workload", default="wan13b_480p_block", help="block: workload name")
     ap.add_argument("--blocks", type=int, default=30, help="sample: DiT blocks")
     ap.add_argument("--steps", type=int, default=2, help="sample: Euler steps per call")
     ap.add_argument("--guidance", type=float, default=5.0)
@@ -111,9 +141,22 @@ def main(argv=None):
         else:
             C = torch.zeros(a.M, a.N, dtype=torch.float32, device="cuda")
         epi = {"store": wan.EPI_STORE, "gelu": wan.EPI_GELU, "residual": wan.EPI_RESIDUAL, "f32": wan.EPI_F32}[a.epi]
-        ms = _time(lambda: wan.linear_fwd(cfg, A, W, bias, C, epi, rows_per_batch=a.M), a.iters, a.warmup)
+        if a.fp8:
+            Aq = torch.empty(a.M, a.K, dtype=torch.uint8, device="cuda")
+            As = torch.empty(a.M, dtype=torch.float32, device="cuda")
+            Wq = torch.empty(a.N, a.K, dtype=torch.uint8, device="cuda")
+            Ws = torch.empty(1, dtype=torch.float32, device="cuda")
+            wan.fp8_quantize_rows(cfg, A, Aq, As)
+            wan.fp8_quantize_tensor(cfg, W, Wq, Ws)
+            del A, W
+            ms = _time(lambda: wan.linear_fp8_fwd(cfg, Aq, As, Wq, Ws, bias, C, epi, rows_per_batch=a.M), a.iters,
+                       a.warmup)
+        else:
+            ms = _time(lambda: wan.linear_fwd(cfg, A, W, bias, C, epi, rows_per_batch=a.M), a.iters, a.warmup)
         flops = 2.0 * a.M * a.N * a.K
-        out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, ms=ms, tflops=flops / ms / 1e9)
+        out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, fp8=a.fp8, ms=ms, tflops=flops / ms / 1e9)
+    elif a.kernel == "block":
+        out.update(_block(a))
     elif a.kernel == "sample":
         out.update(_sample(a))
     else:

@@ -14,7 +14,8 @@ from typing import Dict, List, Optional
 import numpy as np
 import torch
 
-from . import (BlockWeights, Config, ImageMlpWeights, StackWeights, TimeWeights, block_weights, make_config)
+from . import (BlockWeights, Config, Fp8Scales, ImageMlpWeights, StackWeights, TimeWeights, block_weights,
+               fp8_quantize_tensor, make_config)
 
 
 def to_device(a, dtype: torch.dtype, device="cuda") -> torch.Tensor:
@@ -59,3 +60,30 @@ def config_for(workload) -> Config:
     return make_config(workload.dim, workload.heads, workload.ffn, in_ch=workload.in_ch, out_ch=workload.out_ch,
                        freq_dim=workload.freq_dim, img_feat=workload.img_feat, eps=workload.eps,
                        dtype=workload.dtype)
+
+
+FP8_WEIGHTS = {"w_qkv": "qkv", "w_o": "o", "w_cq": "cq", "w_ckv": "ckv", "w_co": "co", "w_ckv_img": "ckv_img",
+               "w_1": "ffn1", "w_2": "ffn2"}
+
+
+class Fp8Block:
+    """A block's weights as E4M3 codes with per-tensor scales, quantised on the GPU by
+    ``wan_fp8_quantize_tensor`` from the bf16 device weights; biases and ``mod_bias``
+    are shared with the bf16 block."""
+
+    def __init__(self, cfg: Config, block: Dict[str, torch.Tensor]):
+        self.codes: Dict[str, torch.Tensor] = {}
+        self.scales: Dict[str, torch.Tensor] = {}
+        for name, key in FP8_WEIGHTS.items():
+            if name not in block:
+                continue
+            w = block[name]
+            q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+            sc = torch.empty(1, dtype=torch.float32, device=w.device)
+            fp8_quantize_tensor(cfg, w, q, sc)
+            self.codes[name], self.scales[key] = q, sc
+        tables = dict(block)
+        tables.update(self.codes)
+        self.table = block_weights(tables)
+        self.scale_table = Fp8Scales(*(self.scales[k].data_ptr() if k in self.scales else None
+                                       for k in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]))
