@@ -338,6 +338,10 @@ def main():
     norm = [(ms, wk) for k, ms, wk in recs if k == wan.KIND_NORM]
 
     # ---------------- end to end through the C ABI with host buffers
+    # Every step copies its inputs from pinned host memory and its velocity back. Two
+    # sets of device buffers and a copy stream let step k+1's inputs and step k-1's
+    # result cross PCIe while step k computes; the timed interval covers the first
+    # upload to the last download.
     lat_h = torch.empty(lat.shape, dtype=act, pin_memory=True)
     lat_h.copy_(lat.cpu())
     t_h = torch.from_numpy(t_host).pin_memory()
@@ -346,22 +350,39 @@ def main():
     v_h = torch.empty(v.shape, dtype=torch.float32, pin_memory=True)
     h2d = lat_h.numel() * lat_h.element_size() + t_h.numel() * 4 + ctx_h.numel() * ctx_h.element_size()
     d2h = v_h.numel() * 4
+    bufs = [(lat, t, ctx, v), (torch.empty_like(lat), torch.empty_like(t), torch.empty_like(ctx), torch.empty_like(v))]
+    copy = torch.cuda.Stream()
+    ready = [torch.cuda.Event() for _ in range(2)]      # inputs of the buffer set uploaded
+    done = [torch.cuda.Event() for _ in range(2)]       # step on the buffer set finished
+    drained = [torch.cuda.Event() for _ in range(2)]    # its velocity downloaded
 
-    def e2e_step():
-        lat.copy_(lat_h, non_blocking=True)
-        t.copy_(t_h, non_blocking=True)
-        ctx.copy_(ctx_h, non_blocking=True)
-        step()
-        v_h.copy_(v, non_blocking=True)
+    def e2e_run(n):
+        for k in range(n):
+            i = k % 2
+            lat_i, t_i, ctx_i, v_i = bufs[i]
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(drained[i])
+                lat_i.copy_(lat_h, non_blocking=True)
+                t_i.copy_(t_h, non_blocking=True)
+                ctx_i.copy_(ctx_h, non_blocking=True)
+                ready[i].record(copy)
+            stream.wait_event(ready[i])
+            wan.dit_stack_fwd(cfg, lat_i, t_i, model.stack_table, model.block_tables, ctx_i, img_ctx, v_i, ws)
+            done[i].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(done[i])
+                v_h.copy_(v_i, non_blocking=True)
+                drained[i].record(copy)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(2)
     barrier()
     torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    copy.wait_event(e2)
+    e2e_run(args.steps)
+    stream.wait_stream(copy)
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -396,12 +396,19 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
 
 /* Multi-head attention softmax(q k^T / sqrt(d)) v, non-causal. q [B, Lq, *], k and v
  * [B, Lk, *], o [B, Lq, *] act; head h of each operand occupies columns
- * [col0 + h*d, col0 + (h+1)*d) of rows with the given row strides (elements). */
+ * [col0 + h*d, col0 + (h+1)*d) of rows with the given row strides (elements).
+ * workspace (optional, device, NULL with ws_bytes 0): with at least
+ * wan_attention_workspace_bytes(...) bytes, a last wave of work units that would fill
+ * at most half of the SMs is split over the key tiles and merged (bf16 path). */
 int wan_attention_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0,
                       const void* k, int64_t k_row_stride, int k_col0,
                       const void* v, int64_t v_row_stride, int v_col0,
                       void* o, int64_t o_row_stride, int o_col0,
-                      int B, int heads, int Lq, int Lk, int head_dim, void* stream);
+                      int B, int heads, int Lq, int Lk, int head_dim, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/* Bytes of the optional wan_attention_fwd workspace for B samples of Lq queries. */
+size_t wan_attention_workspace_bytes(const wan_dit_config* cfg, int B, int Lq);
 
 /* y = A W^T + b with an epilogue. A [M, K] act (row stride K), W [N, K] act, bias [N]
  * act or NULL. out: act [M, N] for STORE/GELU, fp32 [M, N] for F32/RESIDUAL. For

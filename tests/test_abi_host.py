@@ -55,9 +55,11 @@ def test_workspace_bytes_layout(wan):
     B, L, Lc = 1, 32760, 512
     n = wan.workspace_bytes(cfg, B, L, Lc)
     D, F = 1536, 8960
-    # h + max(5LD + 2LcD, LF) act elements + fp32 x + fp32 e, each region 256-aligned
-    lower = 2 * (B * L * D + max(5 * L * D + 2 * Lc * D, L * F)) + 4 * (B * L * D + 6 * D)
-    assert lower <= n <= lower + 4 * 256
+    # h + max(5LD + 2LcD, LF) act elements + fp32 x + fp32 e, each region 256-aligned,
+    # + partial outputs for at most 74 key-split attention units (2 x 2 x 128 rows x 520 B)
+    split = min(B * 12 * ((L + 255) // 256), 74) * 2 * 2 * 128 * 520
+    lower = 2 * (B * L * D + max(5 * L * D + 2 * Lc * D, L * F)) + 4 * (B * L * D + 6 * D) + split
+    assert lower <= n <= lower + 5 * 256
     assert wan.workspace_bytes(cfg, 2, L, Lc) > n
     assert wan.workspace_bytes(_cfg(wan, heads=7), 1, 10, 10) == 0       # D != heads * head_dim
 
@@ -103,7 +105,9 @@ def test_validation_rejects_before_launch(wan):
                                1 << 40, None) == -1
     # attention: heads must match the config
     assert L.wan_attention_fwd(ctypes.byref(cfg), fake, 4608, 0, fake, 4608, 1536, fake, 4608, 3072, fake, 1536, 0,
-                               1, 11, 32, 32, 128, None) == -2
+                               1, 11, 32, 32, 128, None, 0, None) == -2
+    assert wan.attention_workspace_bytes(cfg, 1, 32760) == 74 * 2 * 2 * 128 * 520   # 1536 units: capped at 74
+    assert wan.attention_workspace_bytes(cfg, 1, 256) == 12 * 2 * 2 * 128 * 520     # 12 units
     # linear: N must be a multiple of 8
     assert L.wan_linear_fwd(ctypes.byref(cfg), fake, fake, None, fake, 32, 12, 64, 0, None, None, 0, 1, None) == -2
     assert wan.launch_count() == launches

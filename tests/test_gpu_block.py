@@ -247,3 +247,20 @@ def test_flow_matching_velocity_and_loss(wan):
         assert rel_err(host(v)[b], ref) <= BF16_TOL
         ref_loss = np.mean((ref - O.flow_matching_target(r.inp["x1"][b], r.inp["noise"][b])) ** 2)
         assert abs(float(loss[b]) - ref_loss) / ref_loss < 1e-2
+
+
+@pytest.mark.parametrize("frames,height,width,text_len,batch", [(5, 40, 44, 300, 2), (5, 40, 42, 40, 1)])
+def test_block_with_key_split_tail(wan, frames, height, width, text_len, batch):
+    """Few work units (fewer than half the SMs), so every self-attention unit is split
+    over its key tiles (18 and 17 of them, L = 2200 and 2100) and the halves are merged;
+    all rows against the oracle."""
+    w = small_bf16(frames=frames, height=height, width=width, text_len=text_len, batch=batch)
+    r = Run(wan, w, zero_wx=False)
+    x = r.x.clone()
+    wan.dit_block_fwd(r.cfg, x, r.e, r.ctx, None, r.model.block_tables[0], r.ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(x)
+    for b in range(w.batch):
+        ref = O.dit_block(r.inp["x"][b], r.inp["e"][b], r.inp["blocks"][0], r.inp["ctx"][b], w.heads)
+        assert rel_err(got[b] - r.inp["x"][b], ref - r.inp["x"][b]) <= BF16_TOL

@@ -161,6 +161,30 @@ def test_attention(wan, dtype, B, Lq, Lk, H, logit_std):
         assert err <= tol, (b, err)
 
 
+@pytest.mark.parametrize("B,Lq,Lk,H", [(1, 200, 2100, 2), (2, 130, 2048, 1), (1, 1000, 2000, 1), (2, 1, 4000, 2),
+                                       (1, 600, 2500, 3), (1, 300, 1900, 1)])
+def test_attention_key_split(wan, B, Lq, Lk, H):
+    """With a workspace, units of a last wave that fills at most half of the SMs (here
+    every unit) are split over the key tiles (when there are 16 or more) and merged:
+    against the oracle, and close to the unsplit call; 1900 keys (15 tiles) stay
+    whole."""
+    d = 128
+    r = rng(Lq * 5 + Lk + H)
+    q, k, v = (_rb(a, "bf16") for a in _attn_case(r, B, Lq, Lk, H, d, 2.0))
+    cfg = _cfg(wan, "bf16", D=H * d, heads=H)
+    qd, kd, vd = dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16)
+    o = torch.empty(B, Lq, H * d, dtype=torch.bfloat16, device="cuda")
+    o2 = torch.empty_like(o)
+    ws = torch.empty(max(16, wan.attention_workspace_bytes(cfg, B, Lq)), dtype=torch.uint8, device="cuda")
+    wan.attention_fwd(cfg, qd, kd, vd, o, H, d, ws=ws)
+    wan.attention_fwd(cfg, qd, kd, vd, o2, H, d)
+    torch.cuda.synchronize()
+    got = host(o)
+    for b in range(B):
+        assert rel_err(got[b], O.attention(q[b], k[b], v[b], H)) <= BF16_TOL
+    assert rel_err(got, host(o2)) <= 1e-2
+
+
 def test_attention_planted_peak_and_strided_layout(wan):
     """Self-attention layout (q|k|v packed in one [B, L, 3D] buffer) writing into the
     right half of a [B, L, 2D] buffer; selected query rows get one key equal to 8 q."""

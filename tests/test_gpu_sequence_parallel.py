@@ -29,11 +29,16 @@ def test_sharded_self_attention(wan, P, frames, height, width):
     bw, mb, blk = r.model.block_tables[0], r.model.blocks[0]["mod_bias"], r.inp["blocks"][0]
     h = torch.empty(B, L, D, dtype=r.act, device="cuda")
     wan.adaln_modulate(r.cfg, r.x, r.e, mb, 0, h)
-    # unsharded reference through the ABI
-    x_ref = r.x.clone()
-    wan.self_attn_fwd(r.cfg, h, bw, r.e, x_ref, r.ws)
+    # unsharded reference through the single-kernel calls (attention without a workspace,
+    # so every work unit runs whole, as in the sharded attention)
+    blk_dev = r.model.blocks[0]
     qkv_full = torch.empty(B, L, 3 * D, dtype=r.act, device="cuda")
-    wan.linear_fwd(r.cfg, h, r.model.blocks[0]["w_qkv"], r.model.blocks[0]["b_qkv"], qkv_full, wan.EPI_STORE)
+    wan.linear_fwd(r.cfg, h, blk_dev["w_qkv"], blk_dev["b_qkv"], qkv_full, wan.EPI_STORE)
+    o_full = torch.empty(B, L, D, dtype=r.act, device="cuda")
+    wan.attention_fwd(r.cfg, qkv_full, qkv_full, qkv_full, o_full, w.heads, D // w.heads, 0, D, 2 * D, 0)
+    x_ref = r.x.clone()
+    wan.linear_fwd(r.cfg, o_full, blk_dev["w_o"], blk_dev["b_o"], x_ref, wan.EPI_RESIDUAL, gate=r.e[:, 2],
+                   gate_bias=mb[2], gate_batch_stride=6 * D, rows_per_batch=L)
     # sharded
     rows = [list(plan.rows(k)) for k in range(P)]
     h_shards = [h[:, rows[k]].contiguous() for k in range(P)]

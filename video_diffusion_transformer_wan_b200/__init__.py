@@ -17,7 +17,7 @@ __all__ = [
     "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights",
     "ImageMlpWeights", "StackWeights", "DiffusionCache", "Fp8Scales", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
     "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
-    "attention_fwd", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
+    "attention_fwd", "attention_workspace_bytes", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
     "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd",
     "fp8_quantize_rows", "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd",
     "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
@@ -99,7 +99,8 @@ def _load() -> ctypes.CDLL:
         "wan_flow_matching_input": (_i, [P(Config), _vp, _vp, _vp, _i, _i64, _vp, _vp, _vp]),
         "wan_flow_matching_loss": (_i, [P(Config), _vp, _vp, _vp, _i, _i64, _vp, _vp]),
         "wan_attention_fwd": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _i,
-                                   _i, _i, _i, _vp]),
+                                   _i, _i, _i, _vp, _sz, _vp]),
+        "wan_attention_workspace_bytes": (_sz, [P(Config), _i, _i]),
         "wan_linear_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i, _vp]),
         "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i, P(DiffusionCache)]),
         "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
@@ -213,7 +214,7 @@ def adaln_modulate(cfg, x, e, mod_bias, chunk, h_out, stream=None):
 
 
 def _ws(ws):
-    return _p(ws), ws.numel() * ws.element_size()
+    return (None, 0) if ws is None else (_p(ws), ws.numel() * ws.element_size())
 
 
 def self_attn_fwd(cfg, h, bw: BlockWeights, e, x_inout, ws, stream=None):
@@ -334,12 +335,17 @@ def sp_out_fwd(cfg, sp_size: int, o, bw: BlockWeights, e, x_inout, L: int, strea
                               o.shape[0], L, _stream(stream)), "wan_sp_out_fwd")
 
 
-def attention_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0, o_col0=0, stream=None):
-    """q [B, Lq, *], k/v [B, Lk, *], o [B, Lq, *] (contiguous rows)."""
+def attention_workspace_bytes(cfg: Config, B: int, Lq: int) -> int:
+    return int(_lib().wan_attention_workspace_bytes(ctypes.byref(cfg), B, Lq))
+
+
+def attention_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0, o_col0=0, stream=None, ws=None):
+    """q [B, Lq, *], k/v [B, Lk, *], o [B, Lq, *] (contiguous rows); ws: optional scratch
+    of attention_workspace_bytes (lets a last partial wave split over the keys)."""
     B, Lq, qs = q.shape
     Lk, ks = k.shape[1], k.shape[2]
     _check(_lib().wan_attention_fwd(ctypes.byref(cfg), _p(q), qs, q_col0, _p(k), ks, k_col0, _p(v), v.shape[2], v_col0,
-                                 _p(o), o.shape[2], o_col0, B, heads, Lq, Lk, head_dim, _stream(stream)),
+                                 _p(o), o.shape[2], o_col0, B, heads, Lq, Lk, head_dim, *_ws(ws), _stream(stream)),
            "wan_attention_fwd")
 
 

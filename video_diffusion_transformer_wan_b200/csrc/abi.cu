@@ -185,9 +185,20 @@ struct Layout {
   size_t big;      // region R, see below
   size_t x;        // [B, L, D] fp32 (stack)
   size_t e;        // [B, 6, D] fp32 (stack)
+  size_t split;    // partial outputs of key-split attention units (see attention())
+  size_t split_bytes;
   size_t total;
   size_t big_elems;
 };
+
+// Partial outputs for the attention units of a last, less-than-half-full wave that are
+// split over their key tiles: per split unit 2 halves x 2 query tiles x 128 rows x
+// (128 fp32 + max and sum). At most 74 units (half of 148 SMs) are ever split.
+constexpr size_t kSplitUnitBytes = 2 * 2 * 128 * (128 * 4 + 8);
+size_t split_bytes(const wan_dit_config* c, int B, int L) {
+  const int64_t units = static_cast<int64_t>(B) * c->heads * ((L + 255) / 256);
+  return static_cast<size_t>(units < 74 ? units : 74) * kSplitUnitBytes;
+}
 
 // Region R (act elements), reused by the three branches:
 //   self-attention: qkv [B*L, 3D] at 0, attention output [B*L, D] at 3*B*L*D
@@ -210,7 +221,9 @@ Layout layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
   l.big_elems = big;
   l.x = l.big + align_up(big * es);
   l.e = l.x + align_up(BL * D * 4);
-  l.total = l.e + align_up(static_cast<size_t>(B) * 6 * D * 4);
+  l.split = l.e + align_up(static_cast<size_t>(B) * 6 * D * 4);
+  l.split_bytes = c->dtype == WAN_BF16 ? split_bytes(c, B, L) : 0;
+  l.total = l.split + align_up(l.split_bytes);
   return l;
 }
 
@@ -225,8 +238,9 @@ int gemm(const wan_dit_config* c, const void* A, int64_t lda, const void* W, con
 }
 
 int attention(const wan_dit_config* c, AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t ors, int oc,
-              int B, int Lq, int Lk, cudaStream_t s) {
-  if (c->dtype == WAN_BF16) return launch_attn_tc(q, k, v, o, ors, oc, B, c->heads, Lq, Lk, s);
+              int B, int Lq, int Lk, cudaStream_t s, void* scratch = nullptr, size_t scratch_bytes = 0) {
+  if (c->dtype == WAN_BF16)
+    return launch_attn_tc(q, k, v, o, ors, oc, B, c->heads, Lq, Lk, s, nullptr, scratch, scratch_bytes);
   return launch_attn_simt(q, k, v, o, ors, oc, B, c->heads, Lq, Lk, c->head_dim, s);
 }
 
@@ -262,7 +276,8 @@ int self_attn_impl(const wan_dit_config* c, const void* h, const wan_block_weigh
   void* o = attn_kept ? attn_kept : R + static_cast<size_t>(3) * M * D * es;
   if (!(attn_kept && attn_reuse)) {
     WAN_TRY(gemm(c, h, D, w->w_qkv, w->b_qkv, qkv, M, 3 * D, D, 0, epi_store(3 * D), s));
-    WAN_TRY(attention(c, {qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, L, L, s));
+    WAN_TRY(attention(c, {qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, L, L, s,
+                      at(ws, ly.split), ly.split_bytes));
   }
   const float* gb = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
   return gemm(c, o, D, w->w_o, w->b_o, x, M, D, D, 0, epi_residual(D, e + 2 * D, gb, 6 * D, L), s);
@@ -288,13 +303,15 @@ int cross_attn_impl(const wan_dit_config* c, const void* h, const void* ctx, int
     kvt = const_cast<void*>(kvt_cached);
   else
     WAN_TRY(gemm(c, ctx, D, w->w_ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
-  WAN_TRY(attention(c, {q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, L, Lc, s));
+  void* scr = at(ws, ly.split);
+  const size_t scr_bytes = ly.split_bytes;
+  WAN_TRY(attention(c, {q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, L, Lc, s, scr, scr_bytes));
   if (with_img) {
     if (kvi_cached)
       kvi = const_cast<void*>(kvi_cached);
     else
       WAN_TRY(gemm(c, img, D, w->w_ckv_img, w->b_ckv_img, kvi, B * Li, 2 * D, D, 0, epi_store(2 * D), s));
-    WAN_TRY(attention(c, {q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, L, Li, s));
+    WAN_TRY(attention(c, {q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, L, Li, s, scr, scr_bytes));
     // (o_text + o_image) Wco^T as one reduction over [o_text | o_image] with Wco reused.
     return gemm(c, ocat, ow, w->w_co, w->b_co, x, M, D, 2 * D, D, epi_residual(D, nullptr, nullptr, 0, L), s);
   }
@@ -768,7 +785,10 @@ int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x, const float* e, c
   void* qkv = R;
   void* o = R + 3 * MD;
   WAN_TRY(e4m3_gemm(codes, scales, w->w_qkv, sc->qkv, w->b_qkv, qkv, M, 3 * D, D, epi_store(3 * D), s));
-  WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s));
+  void* scr = at(workspace, fl.base.split);
+  const size_t scr_bytes = fl.base.split_bytes;
+  WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s,
+                         nullptr, scr, scr_bytes));
   WAN_TRY(launch_quantize_rows(o, D, M, D, false, codes, scales, WAN_BF16, s));
   const float* gb_msa = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
   WAN_TRY(e4m3_gemm(codes, scales, w->w_o, sc->o, w->b_o, x, M, D, D, epi_residual(D, e + 2 * D, gb_msa, 6 * D, L), s));
@@ -782,12 +802,14 @@ int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x, const float* e, c
   WAN_TRY(launch_quantize_rows(ctx, D, B * Lc, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
   WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv, sc->ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, epi_store(2 * D), s));
   const int ow = with_img ? 2 * D : D;
-  WAN_TRY(launch_attn_tc({q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, cfg->heads, L, Lc, s));
+  WAN_TRY(launch_attn_tc({q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, cfg->heads, L, Lc, s, nullptr,
+                         scr, scr_bytes));
   if (with_img) {
     WAN_TRY(launch_quantize_rows(img_ctx, D, B * li, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
     WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv_img, sc->ckv_img, w->b_ckv_img, kvi, B * li, 2 * D, D,
                       epi_store(2 * D), s));
-    WAN_TRY(launch_attn_tc({q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, cfg->heads, L, li, s));
+    WAN_TRY(launch_attn_tc({q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, cfg->heads, L, li, s,
+                           nullptr, scr, scr_bytes));
   }
   // the text and image outputs are summed while quantised
   WAN_TRY(launch_quantize_rows(ocat, ow, M, D, with_img, codes, scales, WAN_BF16, s));
@@ -978,7 +1000,7 @@ int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void
 int wan_attention_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0, const void* k,
                       int64_t k_row_stride, int k_col0, const void* v, int64_t v_row_stride, int v_col0, void* o,
                       int64_t o_row_stride, int o_col0, int B, int heads, int Lq, int Lk, int head_dim,
-                      void* stream) {
+                      void* workspace, size_t ws_bytes, void* stream) {
   WAN_TRY(check_cfg(cfg, true));
   WAN_TRY(check_ptr(q));
   WAN_TRY(check_ptr(k));
@@ -992,8 +1014,14 @@ int wan_attention_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_st
                   o_col0 + need <= o_row_stride,
               WAN_ERR_SHAPE);
   if (cfg->dtype == WAN_F32) WAN_REQUIRE(Lk <= 8192, WAN_ERR_SHAPE);
+  if (workspace) WAN_TRY(check_ptr(workspace));
   return attention(cfg, {q, q_row_stride, q_col0}, {k, k_row_stride, k_col0}, {v, v_row_stride, v_col0}, o,
-                   o_row_stride, o_col0, B, Lq, Lk, as_stream(stream));
+                   o_row_stride, o_col0, B, Lq, Lk, as_stream(stream), workspace, workspace ? ws_bytes : 0);
+}
+
+size_t wan_attention_workspace_bytes(const wan_dit_config* cfg, int B, int Lq) {
+  if (check_cfg(cfg) != WAN_OK || B < 0 || Lq < 0) return 0;
+  return cfg->dtype == WAN_BF16 ? split_bytes(cfg, B, Lq) : 0;
 }
 
 int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, const void* bias, void* out, int M, int N,

@@ -26,6 +26,11 @@
 //               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
 //               base and p <= 256 stays well inside fp32 and bf16 range.
 // While one tile's softmax runs, the tensor core works on the other tile's MMAs.
+// Work units are (sample, head, pair of query tiles), one CTA each, in a 1D grid. When
+// the last wave would fill at most half of the SMs, its units are split over the key
+// tiles instead (two CTAs per unit, each over half of them); those CTAs write their
+// unnormalised output with each row's base and sum to a caller scratch, and
+// attn_combine_kernel merges the halves.
 // TMEM: S_0 (later P_0), S_1 (P_1), O_0, O_1 = 4 x 128 of the 512 columns.
 #include <cuda_bf16.h>
 
@@ -48,6 +53,7 @@ constexpr int kTileBytes = kTile * kHd * 2;    // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
 constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMinSplitKeyTiles = 16;          // see launch_attn_tc
 // Of every 8 exponentials, how many run on the FMA pipes (exp2_poly) instead of the
 // MUFU unit (0..4). Measured best at 0 for this kernel (1 and 2 were slower).
 #ifndef WAN_ATTN_POLY_EXP
@@ -64,6 +70,13 @@ struct AttnParams {
   int64_t o_batch_stride;
   int o_col0;
   SeqScatter sc;  // sc.ranks > 0: rows go to their owners' buffers
+  // Work units: (sample, head, pair of query tiles), unit = (b * H + h) * pairs + pair.
+  // CTAs [0, n_full) take one unit over all key tiles; the CTAs after them split the
+  // remaining units' key tiles in two halves (CTA n_full + 2u + half) and write
+  // unnormalised partial outputs to part_o / part_ml, merged by attn_combine_kernel.
+  int pairs, n_full;
+  float* part_o;   // [split CTA][tile][128 rows][128] fp32
+  float* part_ml;  // [split CTA][tile][128 rows][2] (row max, row sum) fp32
   int* err;
 };
 
@@ -90,10 +103,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (kQTiles * kTile);
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int nkv = (p.Lk + kTile - 1) / kTile;
+  const int nkv_all = (p.Lk + kTile - 1) / kTile;
+  int unit = blockIdx.x, kv0 = 0, kv1 = nkv_all, split = -1;
+  if (unit >= p.n_full) {
+    split = unit - p.n_full;
+    unit = p.n_full + (split >> 1);
+    kv0 = (split & 1) ? nkv_all / 2 : 0;
+    kv1 = (split & 1) ? nkv_all : nkv_all / 2;
+  }
+  const int nkv = kv1 - kv0;  // key tiles this CTA visits, from key tile kv0 on
+  const int bh = unit / p.pairs;
+  const int q0 = (unit - bh * p.pairs) * (kQTiles * kTile);
+  const int h = bh % p.H;
+  const int b = bh / p.H;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -152,8 +174,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int col = (is_v ? p.v_col0 : p.k_col0) + h * kHd;
         uint8_t* dst = sKV + stage * kTileBytes;
         mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
-        tma_load_3d(dst, map, &kv_full[stage], col, j * kTile, b);
-        tma_load_3d(dst + kHalfBytes, map, &kv_full[stage], col + 64, j * kTile, b);
+        tma_load_3d(dst, map, &kv_full[stage], col, (kv0 + j) * kTile, b);
+        tma_load_3d(dst + kHalfBytes, map, &kv_full[stage], col + 64, (kv0 + j) * kTile, b);
         ++issued;
       }
       mbar_wait(q_full, 0, p.err);
@@ -251,7 +273,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-      const int valid = p.Lk - j * kTile;  // keys of this tile that exist (mask the rest)
+      const int valid = p.Lk - (kv0 + j) * kTile;  // keys of this tile that exist (mask the rest)
       // The whole S row (128 fp32) is read with one wait; P is then packed in place into
       // the first 64 registers (pair i of the row lands in register i <= 2i, so the pass
       // never overwrites a value it still has to read) and stored over S in TMEM.
@@ -316,7 +338,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
-    if (ok && nkv > 0 && mbar_wait_warp(&o_final[t], 0, p.err)) {
+    const bool done = ok && nkv > 0 && mbar_wait_warp(&o_final[t], 0, p.err);
+    if (done && split >= 0) {
+      // Partial output of a key-split CTA: O unnormalised, with the row's base and sum.
+      tc_fence_after();
+      const int64_t slot = (static_cast<int64_t>(split) * kQTiles + t) * kTile + row;
+      float4* po = reinterpret_cast<float4*>(p.part_o + slot * kHd);
+#pragma unroll 1
+      for (int c = 0; c < kHd / 32; ++c) {
+        uint32_t r0[32];
+        tmem_ld32(o_row + c * 32, r0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          po[c * 8 + g] = make_float4(__uint_as_float(r0[4 * g]), __uint_as_float(r0[4 * g + 1]),
+                                      __uint_as_float(r0[4 * g + 2]), __uint_as_float(r0[4 * g + 3]));
+      }
+      reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_run, l_run);
+    } else if (done) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const int grow = q0 + t * kTile + row;
@@ -363,6 +402,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
+// Merge the two key halves of each split unit: with m = max(m0, m1) and
+// w_i = 2^((m_i - m) scale_log2), O = (w0 O0 + w1 O1) / (w0 l0 + w1 l1). One block per
+// (split unit, query tile); each warp takes rows, each lane 4 of the 128 columns.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+  const int u = blockIdx.x, t = blockIdx.y;
+  const int unit = p.n_full + u;
+  const int bh = unit / p.pairs;
+  const int q0 = (unit - bh * p.pairs) * (kQTiles * kTile) + t * kTile;
+  const int h = bh % p.H, b = bh / p.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int r = warp; r < kTile; r += 8) {
+    const int grow = q0 + r;
+    if (grow >= p.Lq) break;
+    const int64_t s0 = (static_cast<int64_t>(2 * u) * kQTiles + t) * kTile + r;
+    const int64_t s1 = (static_cast<int64_t>(2 * u + 1) * kQTiles + t) * kTile + r;
+    const float2 ml0 = reinterpret_cast<const float2*>(p.part_ml)[s0];
+    const float2 ml1 = reinterpret_cast<const float2*>(p.part_ml)[s1];
+    const float m = fmaxf(ml0.x, ml1.x);
+    const float w0 = exp2f((ml0.x - m) * p.scale_log2), w1 = exp2f((ml1.x - m) * p.scale_log2);
+    const float inv = 1.0f / (w0 * ml0.y + w1 * ml1.y);
+    const float4 a = reinterpret_cast<const float4*>(p.part_o + s0 * kHd)[lane];
+    const float4 c = reinterpret_cast<const float4*>(p.part_o + s1 * kHd)[lane];
+    uint2 v;
+    v.x = pack_bf16x2((w0 * a.x + w1 * c.x) * inv, (w0 * a.y + w1 * c.y) * inv);
+    v.y = pack_bf16x2((w0 * a.z + w1 * c.z) * inv, (w0 * a.w + w1 * c.w) * inv);
+    __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride + static_cast<int64_t>(grow) * p.o_row_stride +
+                          p.o_col0 + h * kHd;
+    reinterpret_cast<uint2*>(orow)[lane] = v;
+  }
+}
+
 bool make_operand_map(CUtensorMap* map, const AttnOperand& op, int B, int L) {
   const uint64_t dims[3] = {static_cast<uint64_t>(op.row_stride), static_cast<uint64_t>(L),
                             static_cast<uint64_t>(B)};
@@ -375,7 +445,7 @@ bool make_operand_map(CUtensorMap* map, const AttnOperand& op, int B, int L) {
 }  // namespace
 
 int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0, int B,
-                   int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc) {
+                   int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc, void* scratch, size_t scratch_bytes) {
   if (B == 0 || Lq == 0) return WAN_OK;
   if (Lk <= 0) return WAN_ERR_SHAPE;
   if (q.row_stride % 8 || k.row_stride % 8 || v.row_stride % 8 || o_row_stride % 8) return WAN_ERR_ALIGN;
@@ -407,10 +477,38 @@ int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t
     cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kAttnSmem));
   });
-  dim3 grid((Lq + kQTiles * kTile - 1) / (kQTiles * kTile), H, B);
+  // One CTA per unit. When the last wave would leave more than half of the SMs idle,
+  // its units are split over the key tiles instead (two CTAs each) and merged after.
+  p.pairs = (Lq + kQTiles * kTile - 1) / (kQTiles * kTile);
+  const int64_t units = static_cast<int64_t>(B) * H * p.pairs;
+  if (units >= (int64_t(1) << 31)) return WAN_ERR_SHAPE;
+  static int nsm_of[64] = {0};
+  if (nsm_of[dev & 63] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    nsm_of[dev & 63] = v > 0 ? v : 148;
+  }
+  const int nsm = nsm_of[dev & 63];
+  const int64_t rem = units % nsm;
+  const int nkv_all = (Lk + kTile - 1) / kTile;
+  const size_t part_o_bytes = static_cast<size_t>(2 * rem) * kQTiles * kTile * kHd * 4;
+  const size_t part_bytes = part_o_bytes + static_cast<size_t>(2 * rem) * kQTiles * kTile * 8;
+  // Only when a unit is long enough (16+ key tiles) for half of it to outweigh the
+  // partial-output traffic and the merge launch (at 4 key tiles, as in the text
+  // cross-attention, splitting measured 9 % slower).
+  const bool split = rem > 0 && 2 * rem <= nsm && nkv_all >= kMinSplitKeyTiles && !sc && scratch &&
+                     scratch_bytes >= part_bytes && (reinterpret_cast<uintptr_t>(scratch) & 15u) == 0;
+  p.n_full = static_cast<int>(split ? units - rem : units);
+  p.part_o = split ? static_cast<float*>(scratch) : nullptr;
+  p.part_ml = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + part_o_bytes) : nullptr;
+  const unsigned grid = static_cast<unsigned>(split ? units + rem : units);
   trace_launch_begin(WAN_KIND_ATTN, s, 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd);
   attn_fwd_tc_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(mq, mk, mv, p);
   int st = check_launch();
+  if (st == WAN_OK && split) {
+    attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);
+    st = check_launch();
+  }
   trace_launch_end(WAN_KIND_ATTN, s);
   return st;
 }

@@ -97,8 +97,11 @@ struct SeqScatter {
 };
 // bf16 tcgen05 flash attention, head_dim 128. With sc, o is ignored and each output row
 // is written to its owner's buffer (row stride o_row_stride, columns from o_col0).
+// scratch (16-byte aligned, device) lets the last partial wave of work units be split
+// over the key tiles; without it (or when too small) every unit runs whole.
 int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
-                   int B, int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc = nullptr);
+                   int B, int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc = nullptr,
+                   void* scratch = nullptr, size_t scratch_bytes = 0);
 // fp32 SIMT attention, head_dim <= 128, Lk <= 8192.
 int launch_attn_simt(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
                      int B, int H, int Lq, int Lk, int d, cudaStream_t s);
