@@ -339,9 +339,9 @@ def main():
 
     # ---------------- end to end through the C ABI with host buffers
     # Every step copies its inputs from pinned host memory and its velocity back. Two
-    # sets of device buffers and a copy stream let step k+1's inputs and step k-1's
-    # result cross PCIe while step k computes; the timed interval covers the first
-    # upload to the last download.
+    # sets of device buffers and an upload and a download stream let step k+1's inputs
+    # and step k-1's result cross PCIe while step k computes; the timed interval covers
+    # the first upload to the last download.
     lat_h = torch.empty(lat.shape, dtype=act, pin_memory=True)
     lat_h.copy_(lat.cpu())
     t_h = torch.from_numpy(t_host).pin_memory()
@@ -351,7 +351,7 @@ def main():
     h2d = lat_h.numel() * lat_h.element_size() + t_h.numel() * 4 + ctx_h.numel() * ctx_h.element_size()
     d2h = v_h.numel() * 4
     bufs = [(lat, t, ctx, v), (torch.empty_like(lat), torch.empty_like(t), torch.empty_like(ctx), torch.empty_like(v))]
-    copy = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     ready = [torch.cuda.Event() for _ in range(2)]      # inputs of the buffer set uploaded
     done = [torch.cuda.Event() for _ in range(2)]       # step on the buffer set finished
     drained = [torch.cuda.Event() for _ in range(2)]    # its velocity downloaded
@@ -360,29 +360,31 @@ def main():
         for k in range(n):
             i = k % 2
             lat_i, t_i, ctx_i, v_i = bufs[i]
-            with torch.cuda.stream(copy):
+            with torch.cuda.stream(up):
                 if k >= 2:
-                    copy.wait_event(drained[i])
+                    up.wait_event(drained[i])
                 lat_i.copy_(lat_h, non_blocking=True)
                 t_i.copy_(t_h, non_blocking=True)
                 ctx_i.copy_(ctx_h, non_blocking=True)
-                ready[i].record(copy)
+                ready[i].record(up)
             stream.wait_event(ready[i])
             wan.dit_stack_fwd(cfg, lat_i, t_i, model.stack_table, model.block_tables, ctx_i, img_ctx, v_i, ws)
             done[i].record(stream)
-            with torch.cuda.stream(copy):
-                copy.wait_event(done[i])
+            with torch.cuda.stream(down):
+                down.wait_event(done[i])
                 v_h.copy_(v_i, non_blocking=True)
-                drained[i].record(copy)
+                drained[i].record(down)
 
     e2e_run(2)
     barrier()
     torch.cuda.synchronize()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    copy.wait_event(e2)
+    up.wait_event(e2)
+    down.wait_event(e2)
     e2e_run(args.steps)
-    stream.wait_stream(copy)
+    stream.wait_stream(up)
+    stream.wait_stream(down)
     e3.record(stream)
     torch.cuda.synchronize()
     barrier()

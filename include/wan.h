@@ -129,6 +129,13 @@ size_t wan_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int 
  * out: WAN_OK, WAN_ERR_TIMEOUT, or WAN_ERR_CUDA if the sync itself failed. */
 int wan_device_status(void* stream);
 
+/* Exercises the failure path of the kernels' bounded waits: launches one thread that
+ * waits on a barrier nothing arrives at. The wait gives up after its limit (1 s) and
+ * records WAN_ERR_TIMEOUT in the device flag, which the next wan_device_status returns
+ * (and clears); the context stays usable. No fault, trap or hang is involved. Returns
+ * WAN_OK once launched (or WAN_ERR_CUDA). */
+int wan_wait_timeout_check(void* stream);
+
 /* ---- the hot path -------------------------------------------------------------- */
 
 /* Patchify [Wan 2.1 page, "Diffusion Transformer": 3D conv, kernel = stride = (1,2,2)].

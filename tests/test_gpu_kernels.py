@@ -329,3 +329,20 @@ def test_flow_matching(wan, dtype):
         ref_loss = np.mean((v[b] - O.flow_matching_target(x1[b], x0[b])) ** 2)
         assert abs(float(loss[b]) - ref_loss) / ref_loss < 1e-5
     assert np.allclose(t.cpu().numpy(), 1000 * u)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(wan):
+    """A wait on a barrier that nothing arrives at gives up after its limit; the host
+    reads WAN_ERR_TIMEOUT once, the flag clears, and the next kernel runs normally."""
+    assert wan.device_status() == 0
+    wan.wait_timeout_check()
+    assert wan.device_status() == -7
+    assert wan.device_status() == 0
+    cfg = _cfg(wan, "bf16", D=128, heads=1)
+    q = dev(rng(31).standard_normal((1, 130, 128)), torch.bfloat16)
+    o = torch.empty(1, 130, 128, dtype=torch.bfloat16, device="cuda")
+    wan.attention_fwd(cfg, q, q, q, o, 1, 128)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    ref = O.attention(host(q)[0], host(q)[0], host(q)[0], 1)
+    assert rel_err(host(o)[0], ref) <= BF16_TOL

@@ -14,13 +14,14 @@ from typing import Dict, Optional, Sequence
 
 __all__ = [
     "LIB_PATH", "lib", "WanError", "WAN_F32", "WAN_BF16", "EPI_STORE", "EPI_GELU", "EPI_RESIDUAL", "EPI_F32",
-    "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights",
-    "ImageMlpWeights", "StackWeights", "DiffusionCache", "Fp8Scales", "make_config", "workspace_bytes", "device_status", "patchify", "patchify_noalloc", "time_mlp",
-    "adaln_modulate", "self_attn_fwd", "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd",
-    "attention_fwd", "attention_workspace_bytes", "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input",
-    "flow_matching_loss", "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd",
-    "fp8_quantize_rows", "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd",
-    "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
+    "KIND_NORM", "KIND_GEMM", "KIND_ATTN", "KIND_SMALL", "Config", "BlockWeights", "TimeWeights", "ImageMlpWeights",
+    "StackWeights", "DiffusionCache", "Fp8Scales", "make_config", "workspace_bytes", "device_status",
+    "wait_timeout_check", "patchify", "patchify_noalloc", "time_mlp", "adaln_modulate", "self_attn_fwd",
+    "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd", "attention_fwd", "attention_workspace_bytes",
+    "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input", "flow_matching_loss",
+    "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd", "fp8_quantize_rows",
+    "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd", "launch_count",
+    "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
 LIB_PATH = os.environ.get("WAN_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "wan_status_string": (ctypes.c_char_p, [_i]),
         "wan_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i]),
         "wan_device_status": (_i, [_vp]),
+        "wan_wait_timeout_check": (_i, [_vp]),
         "wan_patchify": (_i, [P(Config), _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
         "wan_patchify_noalloc": (_i, [P(Config), _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
         "wan_time_mlp": (_i, [P(Config), _vp, _i, P(TimeWeights), _vp, _vp]),
@@ -187,6 +189,12 @@ def workspace_bytes(cfg: Config, B: int, L: int, Lc: int, Li: int = 0) -> int:
 
 def device_status(stream=None) -> int:
     return int(_lib().wan_device_status(_stream(stream)))
+
+
+def wait_timeout_check(stream=None) -> None:
+    """Launch the one-thread kernel whose bounded wait runs out (about 1 s); the next
+    device_status() returns WAN_ERR_TIMEOUT (-7)."""
+    _check(_lib().wan_wait_timeout_check(_stream(stream)), "wan_wait_timeout_check")
 
 
 def patchify(cfg, latent, w_p, b_p, x_out, ws, stream=None):

@@ -372,8 +372,9 @@ int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int 
   const int K = cfg->in_ch * 4;
   WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, patches, cfg->dtype, s));
   WAN_TRY(gemm(cfg, patches, K, sw->w_p, sw->b_p, x, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s));
+  // the hidden units of the time MLP go to region R, free once the patchify GEMM has run
   WAN_TRY(launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, sw->time.w_t1, sw->time.b_t1, sw->time.w_t2, sw->time.b_t2,
-                          e, cfg->dtype, s));
+                          e, cfg->dtype, s, reinterpret_cast<float*>(patches)));
   for (int i = 0; i < n_blocks; ++i)
     WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s, kvt ? kvt[i] : nullptr,
                        kvi ? kvi[i] : nullptr, attn_kept ? attn_kept[i] : nullptr, attn_reuse));
@@ -446,6 +447,8 @@ size_t wan_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int 
   if (check_cfg(cfg) != WAN_OK || B < 0 || L < 0 || Lc < 0 || Li < 0) return 0;
   return layout(cfg, B, L, Lc, Li).total;
 }
+
+int wan_wait_timeout_check(void* stream) { return launch_wait_timeout_probe(as_stream(stream)); }
 
 int wan_device_status(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return WAN_ERR_CUDA;

@@ -17,6 +17,8 @@ namespace wan {
 void trace_launch_begin(int kind, cudaStream_t s, double work = 0.0);
 void trace_launch_end(int kind, cudaStream_t s);
 int* device_error_flag();   // device address of the error flag of the current device
+// One-thread kernel whose bounded wait runs out (about 1 s) and sets the error flag.
+int launch_wait_timeout_probe(cudaStream_t s);
 
 // Returns WAN_ERR_CUDA if the last launch failed.
 inline int check_launch() {
@@ -110,7 +112,7 @@ int launch_attn_simt(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64
 int launch_patch_gather(const void* latent, int B, int C, int F, int H, int W, void* patches, int dtype,
                         cudaStream_t s);
 int launch_time_mlp(const float* t, int B, int D, int freq_dim, const void* w1, const void* b1, const void* w2,
-                    const void* b2, float* e_out, int dtype, cudaStream_t s);
+                    const void* b2, float* e_out, int dtype, cudaStream_t s, float* hid_scratch = nullptr);
 int launch_i2v_input(const void* noise, const void* cond, const uint8_t* keep, int B, int F, int H, int W,
                      void* out, int dtype, cudaStream_t s);
 int launch_flow_input(const void* x1, const void* x0, const float* u, int B, int64_t n, void* xt, float* t_out,

@@ -6,6 +6,7 @@
 #include <math.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace wan {
 namespace {
@@ -169,6 +170,70 @@ __global__ void __launch_bounds__(kTimeThreads) time_mlp_kernel(const float* __r
   }
 }
 
+// The same MLP in two launches when a scratch for the hidden units is available, so
+// that neither layer is recomputed per block and both spread over many SMs:
+// time_hidden_kernel writes hid[b, n] (kTimeSplitRows units per block),
+// time_out_kernel reads hid[b] into shared memory and writes kTimeSplitRows outputs.
+constexpr int kTimeSplitThreads = 256;
+constexpr int kTimeSplitRows = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(kTimeSplitThreads) time_hidden_kernel(const float* __restrict__ t, int D,
+                                                                        int freq_dim, const T* __restrict__ w1,
+                                                                        const T* __restrict__ b1,
+                                                                        float* __restrict__ hid) {
+  extern __shared__ float emb[];  // [freq_dim]
+  const int b = blockIdx.y;
+  const int half = freq_dim / 2;
+  const double tb = static_cast<double>(t[b]);
+  for (int k = threadIdx.x; k < half; k += kTimeSplitThreads) {
+    const double f = pow(10000.0, -static_cast<double>(k) / half);
+    emb[k] = static_cast<float>(cos(tb * f));
+    emb[half + k] = static_cast<float>(sin(tb * f));
+  }
+  __syncthreads();
+  constexpr int kWarps = kTimeSplitThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_end = min(D, (blockIdx.x + 1) * kTimeSplitRows);
+  for (int n0 = blockIdx.x * kTimeSplitRows + warp * kTimeRows; n0 < n_end; n0 += kWarps * kTimeRows) {
+    float acc[kTimeRows];
+    warp_dot_rows(w1, n0, D, freq_dim, emb, lane, acc);
+    if (lane < kTimeRows && n0 + lane < n_end) {
+      float a = acc[0];
+#pragma unroll
+      for (int r = 1; r < kTimeRows; ++r)
+        if (lane == r) a = acc[r];
+      const float z = a + ld(b1, n0 + lane);
+      hid[static_cast<int64_t>(b) * D + n0 + lane] = z / (1.0f + expf(-z));
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTimeSplitThreads) time_out_kernel(const float* __restrict__ hid, int D,
+                                                                     const T* __restrict__ w2,
+                                                                     const T* __restrict__ b2,
+                                                                     float* __restrict__ e) {
+  extern __shared__ float h[];  // [D]
+  const int b = blockIdx.y;
+  for (int n = threadIdx.x; n < D; n += kTimeSplitThreads) h[n] = hid[static_cast<int64_t>(b) * D + n];
+  __syncthreads();
+  constexpr int kWarps = kTimeSplitThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_end = min(6 * D, (blockIdx.x + 1) * kTimeSplitRows);
+  for (int m0 = blockIdx.x * kTimeSplitRows + warp * kTimeRows; m0 < m_end; m0 += kWarps * kTimeRows) {
+    float acc[kTimeRows];
+    warp_dot_rows(w2, m0, 6 * D, D, h, lane, acc);
+    if (lane < kTimeRows && m0 + lane < m_end) {
+      float a = acc[0];
+#pragma unroll
+      for (int r = 1; r < kTimeRows; ++r)
+        if (lane == r) a = acc[r];
+      e[static_cast<int64_t>(b) * 6 * D + m0 + lane] = a + ld(b2, m0 + lane);
+    }
+  }
+}
+
 // out[b, c, f, y, x]: c < 16 noise, c < 32 condition latent, c < 36 the frame mask,
 // where latent frame f, mask channel mc takes pixel frame 0 for f == 0 (the first frame
 // repeated 4 times) and pixel frame 4f + mc - 3 otherwise.
@@ -284,6 +349,15 @@ __global__ void euler_cfg_kernel(const float* __restrict__ v, int B, int64_t n, 
   }
 }
 
+// One thread waits on a barrier that nothing arrives at: the bounded wait gives up
+// after its limit and records the timeout in the device error flag.
+__global__ void wait_timeout_probe_kernel(int* err) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait(&bar, 0, err);
+}
+
 unsigned grid_for(int64_t total, int threads) {
   int64_t g = (total + threads - 1) / threads;
   if (g > 148 * 64) g = 148 * 64;
@@ -341,8 +415,28 @@ int launch_patch_gather(const void* latent, int B, int C, int F, int H, int W, v
 }
 
 int launch_time_mlp(const float* t, int B, int D, int freq_dim, const void* w1, const void* b1, const void* w2,
-                    const void* b2, float* e_out, int dtype, cudaStream_t s) {
+                    const void* b2, float* e_out, int dtype, cudaStream_t s, float* hid_scratch) {
   if (B == 0) return WAN_OK;
+  if (hid_scratch) {
+    if (static_cast<size_t>(D) * sizeof(float) > 48 * 1024) return WAN_ERR_SHAPE;
+    trace_launch_begin(WAN_KIND_SMALL, s);
+    const dim3 g1((D + kTimeSplitRows - 1) / kTimeSplitRows, B), g2((6 * D + kTimeSplitRows - 1) / kTimeSplitRows, B);
+    const size_t sm1 = static_cast<size_t>(freq_dim) * sizeof(float), sm2 = static_cast<size_t>(D) * sizeof(float);
+    if (dtype == WAN_BF16) {
+      time_hidden_kernel<__nv_bfloat16><<<g1, kTimeSplitThreads, sm1, s>>>(
+          t, D, freq_dim, static_cast<const __nv_bfloat16*>(w1), static_cast<const __nv_bfloat16*>(b1), hid_scratch);
+      time_out_kernel<__nv_bfloat16><<<g2, kTimeSplitThreads, sm2, s>>>(
+          hid_scratch, D, static_cast<const __nv_bfloat16*>(w2), static_cast<const __nv_bfloat16*>(b2), e_out);
+    } else {
+      time_hidden_kernel<float><<<g1, kTimeSplitThreads, sm1, s>>>(
+          t, D, freq_dim, static_cast<const float*>(w1), static_cast<const float*>(b1), hid_scratch);
+      time_out_kernel<float><<<g2, kTimeSplitThreads, sm2, s>>>(
+          hid_scratch, D, static_cast<const float*>(w2), static_cast<const float*>(b2), e_out);
+    }
+    const int st = check_launch();
+    trace_launch_end(WAN_KIND_SMALL, s);
+    return st;
+  }
   dim3 grid((6 * D + kTimeOutPerBlock - 1) / kTimeOutPerBlock, B);
   const size_t smem = static_cast<size_t>(freq_dim + D) * sizeof(float);
   if (smem > 48 * 1024) return WAN_ERR_SHAPE;
@@ -410,6 +504,11 @@ int launch_flow_loss(const float* v, const void* x1, const void* x0, int B, int6
   int st = check_launch();
   trace_launch_end(WAN_KIND_SMALL, s);
   return st;
+}
+
+int launch_wait_timeout_probe(cudaStream_t s) {
+  wait_timeout_probe_kernel<<<1, 1, 0, s>>>(device_error_flag());
+  return check_launch();
 }
 
 }  // namespace wan
