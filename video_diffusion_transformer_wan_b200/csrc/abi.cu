@@ -49,6 +49,8 @@ std::atomic<int64_t> g_launches{0};
 thread_local int tl_slot = -1;
 }  // namespace
 
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
 void trace_launch_begin(int kind, cudaStream_t s, double work) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   Trace& t = trace();

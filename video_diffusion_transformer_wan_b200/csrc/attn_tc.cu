@@ -507,6 +507,7 @@ int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t
   int st = check_launch();
   if (st == WAN_OK && split) {
     attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);
+    count_launches(1);
     st = check_launch();
   }
   trace_launch_end(WAN_KIND_ATTN, s);

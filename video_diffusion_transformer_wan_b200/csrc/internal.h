@@ -14,6 +14,9 @@ namespace wan {
 // Every kernel launch goes through trace_launch_begin/end: they count the launch and,
 // when tracing is on, bracket it with CUDA events on the launch stream.
 // `work`: algorithmic FLOPs (GEMM, attention) or bytes moved (other kernels).
+// Every kernel launch is counted (wan_launch_count): trace_launch_begin counts one;
+// launchers that issue more kernels inside one traced bracket, or none, add the rest.
+void count_launches(int n);
 void trace_launch_begin(int kind, cudaStream_t s, double work = 0.0);
 void trace_launch_end(int kind, cudaStream_t s);
 int* device_error_flag();   // device address of the error flag of the current device

@@ -433,6 +433,7 @@ int launch_time_mlp(const float* t, int B, int D, int freq_dim, const void* w1, 
       time_out_kernel<float><<<g2, kTimeSplitThreads, sm2, s>>>(
           hid_scratch, D, static_cast<const float*>(w2), static_cast<const float*>(b2), e_out);
     }
+    count_launches(1);  // two kernels in this bracket
     const int st = check_launch();
     trace_launch_end(WAN_KIND_SMALL, s);
     return st;
@@ -508,6 +509,7 @@ int launch_flow_loss(const float* v, const void* x1, const void* x0, int B, int6
 
 int launch_wait_timeout_probe(cudaStream_t s) {
   wait_timeout_probe_kernel<<<1, 1, 0, s>>>(device_error_flag());
+  count_launches(1);
   return check_launch();
 }
 
