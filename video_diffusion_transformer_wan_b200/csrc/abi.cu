@@ -1,7 +1,12 @@
-// The C ABI (include/wan.h): argument validation, workspace layout, and the order of
-// kernel launches for the Wan 2.1 DiT block and stack ("Wan: Open and Advanced
-// Large-Scale Video Generative Models", section "Diffusion Transformer"). The host only
-// enqueues work on the caller's stream; nothing here allocates device memory.
+// The C ABI (include/wan.h): argument validation, workspace layouts, and the order of
+// kernel launches for the Wan 2.1 DiT ("Wan: Open and Advanced Large-Scale Video
+// Generative Models"): the block and the stack (section "Diffusion Transformer"), I2V
+// and flow matching (sections "I2V 架构扩展", "训练方法"), and the inference paths of
+// section "Infra": the guided sampling loop with its diffusion cache, FP8 linear layers,
+// and Ulysses sequence parallelism. The host only enqueues work on the caller's stream;
+// nothing here allocates device memory. The file runs: device error flag, launch
+// trace, tensor maps, validation and workspace layouts, the branch / block / stack
+// implementations, then the exported calls.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
