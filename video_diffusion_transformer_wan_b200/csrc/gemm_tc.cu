@@ -11,10 +11,12 @@
 //             overlaps the main loop of the next;
 //   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).. (rows of the tile) and one
 //             half of the tile's columns with tcgen05.ld, applies bias / activation /
-//             gate and writes global memory. Two warps per lane quarter and column
-//             chunks taken in pairs (the fp32 residual of both chunks is loaded before
-//             either is updated) keep enough bytes in flight that the epilogue of one
-//             tile hides under the main loop of the next even when K is short.
+//             scale and writes global memory. The gated fp32 residual (its own
+//             instantiation) goes through a 32x32 shared-memory block per warp so that
+//             the read-modify-write of x moves whole 128-byte row segments; with the
+//             thread-per-row layout of the TMEM load it took 32 half-used sectors per
+//             instruction and the epilogue of the D x D projections did not hide under
+//             their short main loop.
 //
 // Tile order: the row blocks are cut into groups of group_m; within a group the row
 // block varies fastest, so the 148 tiles in flight share a slab of at most
@@ -38,14 +40,16 @@ constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 #define WAN_GEMM_SLAB_MB 32  // bytes of A (MiB) one tile group keeps resident in L2
 #endif
 
-template <int BN>
+template <int BN, bool kRes = false>
 struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int kABytes = kBM * 128;  // 128-byte rows: 64 bf16 or 128 E4M3 elements
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256;
+  // gated-residual instantiation: a 32x32 fp32 staging block per epilogue warp
+  static constexpr size_t kEpiStageBytes = kRes ? static_cast<size_t>(kEpiWarps) * 32 * 32 * 4 : 0;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kStageBytes + 256 + kEpiStageBytes;
 };
 
 struct GemmParams {
@@ -146,32 +150,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
     for (int g = 0; g < 8; ++g)
       if (n0 + g * 4 < p.N)
         reinterpret_cast<float4*>(o)[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-  } else if (kind == WAN_EPI_RESIDUAL) {
-    float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
-    const float* gate = p.epi.gate ? p.epi.gate + static_cast<int64_t>(row / p.epi.rows_per_batch) * p.epi.gate_bstride + n0
-                                   : nullptr;
-    const float* gb = p.epi.gate_bias ? p.epi.gate_bias + n0 : nullptr;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      if (n0 + g * 4 < p.N) {
-        float4 x = reinterpret_cast<float4*>(o)[g];
-        float gg[4] = {1.f, 1.f, 1.f, 1.f};
-        if (gate) {
-          float4 t = __ldg(reinterpret_cast<const float4*>(gate) + g);
-          gg[0] = t.x; gg[1] = t.y; gg[2] = t.z; gg[3] = t.w;
-          if (gb) {
-            float4 u = __ldg(reinterpret_cast<const float4*>(gb) + g);
-            gg[0] += u.x; gg[1] += u.y; gg[2] += u.z; gg[3] += u.w;
-          }
-        }
-        x.x += gg[0] * v[4 * g];
-        x.y += gg[1] * v[4 * g + 1];
-        x.z += gg[2] * v[4 * g + 2];
-        x.w += gg[3] * v[4 * g + 3];
-        reinterpret_cast<float4*>(o)[g] = x;
-      }
-    }
-  } else {  // kEpiHeadScatter: n = c*4 + ph*2 + pw, row = b*L + (f*Hh + i)*Wh + j
+  } else if (kind == kEpiHeadScatter) {  // n = c*4 + ph*2 + pw, row = b*L + (f*Hh + i)*Wh + j
     const int L = p.epi.rows_per_batch;
     const int b = row / L, l = row % L;
     const int Hh = p.epi.sc_H / 2, Wh = p.epi.sc_W / 2;
@@ -190,54 +169,72 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   }
 }
 
-// Two adjacent 32-column chunks [n0, n0+64) of one row. For the residual epilogue the
-// fp32 residual of both chunks is loaded before either is updated (16 loads in flight
-// per thread); other epilogues go chunk by chunk.
-__device__ __forceinline__ void epilogue_pair(const GemmParams& p, int row, int n0, const uint32_t (&r0)[32],
-                                              const uint32_t (&r1)[32]) {
-  if (p.epi.kind != WAN_EPI_RESIDUAL || row >= p.M || n0 + 64 > p.N) {
-    epilogue_chunk(p, row, n0, r0);
-    epilogue_chunk(p, row, n0 + 32, r1);
-    return;
-  }
-  float* o = static_cast<float*>(p.out) + static_cast<int64_t>(row) * p.epi.ldo + n0;
-  float4 x[16];
+// Gated residual epilogue through shared memory: for each 32-column chunk the warp
+// reads its 32 rows from TMEM (thread = row), scales and adds the bias, stages the
+// 32x32 block (16-byte units XOR-swizzled by row), then reads it back four rows per
+// instruction (8 threads x 16 bytes per row) so that every fp32 read-modify-write of x
+// moves whole 128-byte row segments.
+__device__ __forceinline__ void residual_staged(const GemmParams& p, float* stg, uint32_t t_row, int r0, int n0,
+                                                int lane, int chunks) {
+  const int row = r0 + lane;
+  const float sc = p.a_scale ? (row < p.M ? __ldg(p.a_scale + row) : 0.f) * __ldg(p.w_scale) : 1.0f;
+  const int sub = lane >> 3, cq = lane & 7;
+#pragma unroll 1
+  for (int c = 0; c < chunks; ++c) {
+    const int col0 = n0 + c * 32;
+    uint32_t r[32];
+    tmem_ld32(t_row + c * 32, r);
+    tmem_ld_wait();
 #pragma unroll
-  for (int g = 0; g < 16; ++g) x[g] = reinterpret_cast<const float4*>(o)[g];
-  const float* gate = p.epi.gate ? p.epi.gate + static_cast<int64_t>(row / p.epi.rows_per_batch) * p.epi.gate_bstride + n0
-                                 : nullptr;
-  const float* gb = p.epi.gate_bias ? p.epi.gate_bias + n0 : nullptr;
-  const float sc = p.a_scale ? __ldg(p.a_scale + row) * __ldg(p.w_scale) : 1.0f;
-#pragma unroll
-  for (int g = 0; g < 16; ++g) {
-    const uint32_t* rr = g < 8 ? r0 + 4 * g : r1 + 4 * (g - 8);
-    float v0 = __uint_as_float(rr[0]) * sc, v1 = __uint_as_float(rr[1]) * sc;
-    float v2 = __uint_as_float(rr[2]) * sc, v3 = __uint_as_float(rr[3]) * sc;
-    if (p.bias) {
-      const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.bias + n0) + g);
-      const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-      const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-      v0 += b01.x; v1 += b01.y; v2 += b23.x; v3 += b23.y;
-    }
-    if (gate) {
-      float4 t = __ldg(reinterpret_cast<const float4*>(gate) + g);
-      if (gb) {
-        const float4 u = __ldg(reinterpret_cast<const float4*>(gb) + g);
-        t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    for (int k = 0; k < 8; ++k) {
+      float4 v = make_float4(__uint_as_float(r[4 * k]) * sc, __uint_as_float(r[4 * k + 1]) * sc,
+                             __uint_as_float(r[4 * k + 2]) * sc, __uint_as_float(r[4 * k + 3]) * sc);
+      if (p.bias && col0 + 4 * k < p.N) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.bias + col0 + 4 * k));
+        const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v.x += b01.x; v.y += b01.y; v.z += b23.x; v.w += b23.y;
       }
-      v0 *= t.x; v1 *= t.y; v2 *= t.z; v3 *= t.w;
+      reinterpret_cast<float4*>(stg + lane * 32)[k ^ (lane & 7)] = v;
     }
-    x[g].x += v0;
-    x[g].y += v1;
-    x[g].z += v2;
-    x[g].w += v3;
-    reinterpret_cast<float4*>(o)[g] = x[g];
+    __syncwarp();
+    const int gcol = col0 + cq * 4;
+    float4 gb = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.epi.gate_bias && gcol < p.N) gb = __ldg(reinterpret_cast<const float4*>(p.epi.gate_bias + gcol));
+    float4 x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int grow = r0 + i * 4 + sub;
+      if (grow < p.M && gcol < p.N)
+        x[i] = *reinterpret_cast<const float4*>(static_cast<const float*>(p.out) + static_cast<int64_t>(grow) * p.epi.ldo +
+                                                gcol);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = i * 4 + sub;
+      const int grow = r0 + rr;
+      if (grow < p.M && gcol < p.N) {
+        const float4 v = reinterpret_cast<const float4*>(stg + rr * 32)[cq ^ (rr & 7)];
+        float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (p.epi.gate) {
+          g = __ldg(reinterpret_cast<const float4*>(
+              p.epi.gate + static_cast<int64_t>(grow / p.epi.rows_per_batch) * p.epi.gate_bstride + gcol));
+          if (p.epi.gate_bias) {
+            g.x += gb.x; g.y += gb.y; g.z += gb.z; g.w += gb.w;
+          }
+        }
+        float4 o = x[i];
+        o.x += g.x * v.x; o.y += g.y * v.y; o.z += g.z * v.z; o.w += g.w * v.w;
+        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.epi.ldo + gcol) = o;
+      }
+    }
+    __syncwarp();
   }
 }
 
-template <int BN, bool kF8>
+template <int BN, bool kF8, bool kRes>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, kRes>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -248,6 +245,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtenso
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  float* epi_stage = reinterpret_cast<float*>(sB + C::kStages * C::kBBytes + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -367,19 +365,17 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtenso
       const int row = m0 + quarter * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + colhalf * (BN / 2));
+      if constexpr (kRes) {
+        residual_staged(p, epi_stage + (warp - 2) * 1024, t_row, m0 + quarter * 32, n0, lane, kMine);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < kMine; c += 2) {
-        if (c + 1 < kMine) {
+        for (int c = 0; c < kMine; c += 2) {
           uint32_t r0[32], r1[32];
           tmem_ld32(t_row + c * 32, r0);
-          tmem_ld32(t_row + (c + 1) * 32, r1);
-          tmem_ld_wait();
-          epilogue_pair(p, row, n0 + c * 32, r0, r1);
-        } else {
-          uint32_t r0[32];
-          tmem_ld32(t_row + c * 32, r0);
+          if (c + 1 < kMine) tmem_ld32(t_row + (c + 1) * 32, r1);
           tmem_ld_wait();
           epilogue_chunk(p, row, n0 + c * 32, r0);
+          if (c + 1 < kMine) epilogue_chunk(p, row, n0 + (c + 1) * 32, r1);
         }
       }
       tc_fence_before();
@@ -393,18 +389,33 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtenso
   }
 }
 
-template <int BN>
+template <int BN, bool kRes>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const GemmParams p) {
-  gemm_body<BN, false>(mapA, mapB, p);
+  gemm_body<BN, false, kRes>(mapA, mapB, p);
 }
 
-template <int BN>
+template <int BN, bool kRes>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_e4m3_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                         const GemmParams p) {
-  gemm_body<BN, true>(mapA, mapB, p);
+  gemm_body<BN, true, kRes>(mapA, mapB, p);
+}
+
+// Launch one instantiation (the shared-memory opt-in is set once per device for each).
+template <int BN, bool kF8, bool kRes>
+int launch_inst(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p, int grid, cudaStream_t s) {
+  using C = GemmCfg<BN, kRes>;
+  auto kern = kF8 ? gemm_e4m3_tc_kernel<BN, kRes> : gemm_bf16_tc_kernel<BN, kRes>;
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev & 63],
+                 [kern] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(C::kSmemBytes)); });
+  kern<<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
+  return check_launch();
 }
 
 int sm_count() {
@@ -424,7 +435,6 @@ template <int BN, bool kF8>
 int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
               int w_k_period, const GemmEpi& epi, cudaStream_t s, const float* a_scale = nullptr,
               const float* w_scale = nullptr) {
-  using C = GemmCfg<BN>;
   constexpr int bk = kF8 ? 128 : 64;  // elements per 128-byte row
   constexpr int es = kF8 ? 1 : 2;
   CUtensorMap mapA, mapB;
@@ -458,24 +468,10 @@ int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void*
   p.out = out;
   p.epi = epi;
   p.err = device_error_flag();
-  static std::once_flag once[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::call_once(once[dev & 63], [] {
-    if (kF8)
-      cudaFuncSetAttribute(gemm_e4m3_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(C::kSmemBytes));
-    else
-      cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(C::kSmemBytes));
-  });
   const int tiles = p.m_blocks * p.n_blocks;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  if (kF8)
-    gemm_e4m3_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
-  else
-    gemm_bf16_tc_kernel<BN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(mapA, mapB, p);
-  return check_launch();
+  return epi.kind == WAN_EPI_RESIDUAL ? launch_inst<BN, kF8, true>(mapA, mapB, p, grid, s)
+                                      : launch_inst<BN, kF8, false>(mapA, mapB, p, grid, s);
 }
 
 }  // namespace
