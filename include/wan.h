@@ -308,6 +308,15 @@ int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x_inout, const float
                           const void* img_ctx, int Li, const wan_block_weights* w, const wan_fp8_scales* sc,
                           int B, int L, void* workspace, size_t ws_bytes, void* stream);
 
+/* wan_dit_stack_fwd with every block as in wan_dit_block_fp8_fwd: blocks hold E4M3 codes
+ * and scales is a HOST array of n_blocks weight-scale tables; patchify, the timestep
+ * MLP and the head stay bf16. Workspace: wan_fp8_workspace_bytes(cfg, B, L, Lc, Li). */
+int wan_dit_stack_fp8_fwd(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H,
+                          int W, const float* t, const wan_stack_weights* sw,
+                          const wan_block_weights* blocks, const wan_fp8_scales* scales, const void* ctx,
+                          int Lc, const void* img_ctx, int Li, float* v_out, void* workspace,
+                          size_t ws_bytes, void* stream);
+
 /* ---- sequence parallelism (Ulysses) ------------------------------------------ */
 
 /* Self-attention of one block split over P = sp_size ranks along the token axis, the
@@ -362,11 +371,12 @@ typedef struct {
   int cfg_start, cfg_interval;
 } wan_diffusion_cache;
 
-/* Device workspace (bytes) of wan_sample_euler_cfg for these sizes and cache (NULL =
- * no cache); 0 on a bad cfg. The cache adds n_blocks x 2B x L x D act elements of kept
- * attention outputs and B x out_ch x F x H x W fp32 of kept residual. */
+/* Device workspace (bytes) of wan_sample_euler_cfg for these sizes, cache (NULL = no
+ * cache) and precision (fp8 != 0: FP8 linear layers); 0 on a bad cfg. The cache adds
+ * n_blocks x 2B x L x D act elements of kept attention outputs and
+ * B x out_ch x F x H x W fp32 of kept residual. */
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W,
-                                  int Lc, int Li, const wan_diffusion_cache* cache);
+                                  int Lc, int Li, const wan_diffusion_cache* cache, int fp8);
 
 /* Generation loop with the DiT as the velocity model [Wan 2.1 page, "训练方法" (the
  * rectified-flow velocity) and "Infra" (a fixed number of sampling steps, about 50); the
@@ -387,7 +397,10 @@ size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B
  *   blocks: HOST array of n_blocks weight tables; sw: stack weights.
  *   Cross-attention K|V of both contexts are projected once per call and kept for all
  *   steps. cache: NULL (every step runs both passes in full) or the diffusion cache
- *   above. workspace >= wan_sample_workspace_bytes(...) device bytes (same cache).
+ *   above. fp8_scales: NULL (bf16 linear layers) or, with blocks holding E4M3 codes,
+ *   a HOST array of n_blocks weight-scale tables: every block runs as in
+ *   wan_dit_block_fp8_fwd (the K|V projections of the contexts too).
+ *   workspace >= wan_sample_workspace_bytes(...) device bytes (same cache, fp8).
  * Errors (before any launch): WAN_ERR_NULL, WAN_ERR_SHAPE (n_steps < 1, a guidance that
  * is not finite, out_ch > in_ch, Lc = 0, odd H or W, a cache interval < 1 or start < 0),
  * WAN_ERR_WORKSPACE, WAN_ERR_ALIGN.
@@ -397,7 +410,8 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
                          int W, int n_steps, float guidance, const wan_stack_weights* sw,
                          const wan_block_weights* blocks, const void* ctx_cond, const void* ctx_uncond,
                          int Lc, const void* img_ctx, int Li, const wan_diffusion_cache* cache,
-                         float* latent_out, void* workspace, size_t ws_bytes, void* stream);
+                         const wan_fp8_scales* fp8_scales, float* latent_out, void* workspace,
+                         size_t ws_bytes, void* stream);
 
 /* ---- single-kernel entry points (used by the branch calls; exposed for tests) --- */
 

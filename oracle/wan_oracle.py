@@ -353,19 +353,20 @@ def flow_matching_target(x1, x0) -> np.ndarray:
 
 def dit_stack(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, heads: int,
               eps: float = 1e-6, img_ctx=None, freq_dim: int = 256,
-              attn_caches: Optional[Sequence[Dict]] = None) -> np.ndarray:
+              attn_caches: Optional[Sequence[Dict]] = None, fp8: bool = False) -> np.ndarray:
     """Whole DiT on one sample [Wan-P2, "Diffusion Transformer"]: patchify -> the time
     MLP shared by all blocks -> N blocks (each with its own modulation bias) -> head ->
     unpatchify. ``weights`` holds ``w_p, b_p, w_t1, b_t1, w_t2, b_t2, w_head, b_head``.
-    ``attn_caches`` gives each block its attention cache (see ``dit_block``).
-    Returns the predicted velocity ``[out_ch, F, H, W]``."""
+    ``attn_caches`` gives each block its attention cache (see ``dit_block``); ``fp8``
+    runs the blocks' linear layers in FP8 (``dit_block``; patchify, the time MLP and
+    the head stay as they are). Returns the predicted velocity ``[out_ch, F, H, W]``."""
     lat = _f(latent)
     C, F, H, W = lat.shape
     x = patchify(lat, weights["w_p"], weights["b_p"])
     e = time_mlp(t, weights["w_t1"], weights["b_t1"], weights["w_t2"], weights["b_t2"], freq_dim)
     for i, blk in enumerate(blocks):
         x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx,
-                      attn_cache=None if attn_caches is None else attn_caches[i])
+                      attn_cache=None if attn_caches is None else attn_caches[i], fp8=fp8)
     y = head(x, weights["w_head"], weights["b_head"], eps)
     return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)
 
@@ -395,7 +396,7 @@ def euler_cfg(x0, n_steps: int, guidance: float, velocity_cond, velocity_uncond)
 
 def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks: Sequence[Dict], ctx_cond,
                      ctx_uncond, heads: int, eps: float = 1e-6, img_ctx=None, cond_channels=None,
-                     freq_dim: int = 256) -> np.ndarray:
+                     freq_dim: int = 256, fp8: bool = False) -> np.ndarray:
     """Generate a latent with the DiT as the velocity model: ``euler_cfg`` with
     ``v(x, t) = dit_stack(input(x), 1000 t, ...)`` under the text context (conditional)
     and the unconditional context. ``noise [16, F, H, W]`` is x at t = 0. For I2V,
@@ -407,7 +408,7 @@ def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks
 
     def vel(ctx):
         return lambda x, t: dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps,
-                                      img_ctx=img_ctx, freq_dim=freq_dim)
+                                      img_ctx=img_ctx, freq_dim=freq_dim, fp8=fp8)
     return euler_cfg(noise, n_steps, guidance, vel(ctx_cond), vel(ctx_uncond))
 
 

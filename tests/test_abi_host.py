@@ -130,8 +130,8 @@ def test_sampler_validation_and_workspace(wan):
 
     def call(n_steps=4, g=5.0, c=cfg, ctx_u=fake, ws=1 << 40, b=B, h=H, cache=None):
         return L.wan_sample_euler_cfg(ctypes.byref(c), 2, fake, b, F, h, W, n_steps, g, ctypes.byref(sw), bws, fake,
-                                      ctx_u, Lc, None, 0, None if cache is None else ctypes.byref(cache), fake, fake,
-                                      ws, None)
+                                      ctx_u, Lc, None, 0, None if cache is None else ctypes.byref(cache), None, fake,
+                                      fake, ws, None)
     assert call(n_steps=0) == -2
     assert call(g=float("nan")) == -2
     assert call(g=float("inf")) == -2

@@ -7,7 +7,8 @@ import pytest
 
 from oracle import wan_oracle as O
 from wan_inputs import WORKLOADS, make_inputs, round_bf16, sample_rows
-from gpu_util import FP8_TOL_MAX, FP8_TOL_RMS, dev, host, rel_err, rms_err, rng
+from gpu_util import (FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS, FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS, FP8_TOL_MAX,
+                      FP8_TOL_RMS, dev, host, rel_err, rms_err, rng)
 from test_gpu_block import Run, small_bf16
 
 torch = pytest.importorskip("torch")
@@ -142,3 +143,63 @@ def test_block_fp8_full_size_sampled_rows(wan):
     print(f"fp8 block 1.3B sampled rows: max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
     assert rel_err(d_got, d_ref) <= FP8_TOL_MAX
     assert rms_err(d_got, d_ref) <= FP8_TOL_RMS
+
+
+def _fp8_run(wan, i2v=False, batch=2, n_blocks=2):
+    from video_diffusion_transformer_wan_b200.model import Fp8Block
+    w = small_bf16(i2v=i2v, dim=512, heads=4, ffn=1024, n_blocks=n_blocks, batch=batch)
+    r = Run(wan, w, zero_wx=False, uncond=True)
+    fbs = [Fp8Block(r.cfg, b) for b in r.model.blocks]
+    return w, r, fbs
+
+
+@pytest.mark.parametrize("i2v", [False, True])
+def test_stack_fp8_matches_oracle(wan, i2v):
+    """Patchify, time MLP, two FP8 blocks, head: the velocity against the oracle's FP8 stack."""
+    w, r, fbs = _fp8_run(wan, i2v)
+    B, F, H, W = w.batch, w.frames, w.height, w.width
+    t = torch.from_numpy(r.inp["t"]).cuda()
+    lat = torch.from_numpy(r.inp["noise"]).cuda().to(r.act)
+    if i2v:
+        lat = torch.cat([lat, torch.zeros(B, 20, F, H, W, dtype=r.act, device="cuda")], dim=1).contiguous()
+    v = torch.empty(B, 16, F, H, W, dtype=torch.float32, device="cuda")
+    ws = torch.empty(wan.fp8_workspace_bytes(r.cfg, B, w.tokens, w.text_len, w.img_len if i2v else 0),
+                     dtype=torch.uint8, device="cuda")
+    wan.dit_stack_fp8_fwd(r.cfg, lat, t, r.model.stack_table, [f.table for f in fbs], [f.scale_table for f in fbs],
+                          r.ctx, r.img_ctx, v, ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(v)
+    for b in range(B):
+        lat_np = r.inp["noise"][b]
+        if i2v:
+            lat_np = np.concatenate([lat_np, np.zeros((20, F, H, W))], axis=0)
+        ref = O.dit_stack(lat_np, float(r.inp["t"][b]), r.inp, r.inp["blocks"], r.inp["ctx"][b], w.heads,
+                          img_ctx=None if r.img_np is None else r.img_np[b], fp8=True)
+        print(f"fp8 stack i2v={i2v} b={b}: max {rel_err(got[b], ref):.2e} rms {rms_err(got[b], ref):.2e}")
+        assert rel_err(got[b], ref) <= FP8_STACK_TOL_MAX
+        assert rms_err(got[b], ref) <= FP8_STACK_TOL_RMS
+
+
+def test_sampler_fp8_matches_oracle(wan):
+    """Three guided Euler steps with FP8 linear layers (including the cached context
+    K|V projections) against the oracle's FP8 loop."""
+    w, r, fbs = _fp8_run(wan)
+    B, F, H, W = w.batch, w.frames, w.height, w.width
+    inp = torch.from_numpy(r.inp["noise"]).cuda().to(r.act)
+    ws = torch.empty(wan.sample_workspace_bytes(r.cfg, 2, B, F, H, W, w.text_len, 0, None, fp8=True),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.full((B, 16, F, H, W), float("nan"), dtype=torch.float32, device="cuda")
+    wan.sample_euler_cfg(r.cfg, inp, 3, 5.0, r.model.stack_table, [f.table for f in fbs], r.ctx, r.ctx_uncond, None,
+                         out, ws, fp8_scales=[f.scale_table for f in fbs])
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(out)
+    for b in range(B):
+        x0 = r.inp["noise"][b]
+        ref = O.sample_euler_cfg(x0, 3, 5.0, r.inp, r.inp["blocks"], r.inp["ctx"][b], r.inp["ctx_uncond"][b],
+                                 w.heads, fp8=True)
+        d_got, d_ref = got[b] - x0, ref - x0
+        print(f"fp8 sampler b={b}: displacement max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
+        assert rel_err(d_got, d_ref) <= FP8_SAMPLE_TOL_MAX
+        assert rms_err(d_got, d_ref) <= FP8_SAMPLE_TOL_RMS

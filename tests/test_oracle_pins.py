@@ -460,6 +460,15 @@ def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
         xx = torch_block(xx, e, b, ctx, w.heads)
     ref2 = O.unpatchify(O.head(xx, inp["w_head"], inp["b_head"]), 16, w.frames, w.height, w.width)
     np.testing.assert_allclose(v2, ref2, rtol=1e-10, atol=1e-11)
+    # the FP8 stack == the torch re-expression of the FP8 block (torch's E4M3 conversion)
+    # applied twice; patchify, the time MLP and the head unchanged
+    v3 = O.dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads, fp8=True)
+    xx = x
+    for b in inp["blocks"]:
+        xx = torch_block(xx, e, b, ctx, w.heads, fp8=True)
+    ref3 = O.unpatchify(O.head(xx, inp["w_head"], inp["b_head"]), 16, w.frames, w.height, w.width)
+    np.testing.assert_allclose(v3, ref3, rtol=1e-9, atol=1e-10)
+    assert not np.allclose(v3, v2)
 
 
 def test_flow_matching_endpoints():

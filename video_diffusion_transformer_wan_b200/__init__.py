@@ -20,8 +20,8 @@ __all__ = [
     "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd", "attention_fwd", "attention_workspace_bytes",
     "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input", "flow_matching_loss",
     "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd", "fp8_quantize_rows",
-    "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd", "launch_count",
-    "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
+    "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd", "dit_stack_fp8_fwd",
+    "launch_count", "trace_enable", "trace_reset", "trace_read", "trace_launches", "status_string",
 ]
 
 LIB_PATH = os.environ.get("WAN_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
@@ -104,10 +104,12 @@ def _load() -> ctypes.CDLL:
                                    _i, _i, _i, _vp, _sz, _vp]),
         "wan_attention_workspace_bytes": (_sz, [P(Config), _i, _i]),
         "wan_linear_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i, _vp]),
-        "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i, P(DiffusionCache)]),
+        "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i, P(DiffusionCache), _i]),
         "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
-                                      P(BlockWeights), _vp, _vp, _i, _vp, _i, P(DiffusionCache), _vp, _vp, _sz,
-                                      _vp]),
+                                      P(BlockWeights), _vp, _vp, _i, _vp, _i, P(DiffusionCache), P(Fp8Scales), _vp,
+                                      _vp, _sz, _vp]),
+        "wan_dit_stack_fp8_fwd": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _vp, P(StackWeights), P(BlockWeights),
+                                       P(Fp8Scales), _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
         "wan_sp_qkv_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(BlockWeights), P(_vp), _vp]),
         "wan_sp_attn_fwd": (_i, [P(Config), _i, _i, _vp, _i, _i, P(_vp), _vp]),
         "wan_sp_out_fwd": (_i, [P(Config), _i, _vp, P(BlockWeights), _vp, _vp, _i, _i, _vp]),
@@ -267,23 +269,41 @@ def _cache_ref(cache: Optional[DiffusionCache]):
 
 
 def sample_workspace_bytes(cfg: Config, n_blocks: int, B: int, F: int, H: int, W: int, Lc: int, Li: int = 0,
-                           cache: Optional[DiffusionCache] = None) -> int:
-    return int(_lib().wan_sample_workspace_bytes(ctypes.byref(cfg), n_blocks, B, F, H, W, Lc, Li, _cache_ref(cache)))
+                           cache: Optional[DiffusionCache] = None, fp8: bool = False) -> int:
+    return int(_lib().wan_sample_workspace_bytes(ctypes.byref(cfg), n_blocks, B, F, H, W, Lc, Li, _cache_ref(cache),
+                                                 1 if fp8 else 0))
+
+
+def _scales_array(scales):
+    return None if scales is None else (Fp8Scales * max(1, len(scales)))(*scales)
 
 
 def sample_euler_cfg(cfg, inp, n_steps: int, guidance: float, sw: StackWeights, blocks: Sequence[BlockWeights],
                      ctx_cond, ctx_uncond, img_ctx, latent_out, ws, stream=None,
-                     cache: Optional[DiffusionCache] = None):
+                     cache: Optional[DiffusionCache] = None, fp8_scales: Optional[Sequence[Fp8Scales]] = None):
     """inp [B, in_ch, F, H, W]: the noise in its first out_ch channels (and, for I2V, the
-    fixed condition channels after them); latent_out [B, out_ch, F, H, W] fp32."""
+    fixed condition channels after them); latent_out [B, out_ch, F, H, W] fp32. With
+    fp8_scales (one table per block) the blocks hold E4M3 codes."""
     B, C, F, H, W = inp.shape
     arr = (BlockWeights * max(1, len(blocks)))(*blocks)
     Li = 0 if img_ctx is None else img_ctx.shape[1]
     _check(_lib().wan_sample_euler_cfg(ctypes.byref(cfg), len(blocks), _p(inp), B, F, H, W, n_steps, guidance,
                                     ctypes.byref(sw), arr, _p(ctx_cond), _p(ctx_uncond), ctx_cond.shape[1],
-                                    _p(img_ctx), Li, _cache_ref(cache), _p(latent_out), *_ws(ws),
-                                    _stream(stream)),
+                                    _p(img_ctx), Li, _cache_ref(cache), _scales_array(fp8_scales),
+                                    _p(latent_out), *_ws(ws), _stream(stream)),
            "wan_sample_euler_cfg")
+
+
+def dit_stack_fp8_fwd(cfg, latent, t, sw: StackWeights, blocks: Sequence[BlockWeights],
+                      scales: Sequence[Fp8Scales], ctx, img_ctx, v_out, ws, stream=None):
+    """wan_dit_stack_fwd with E4M3 block weights (blocks: code tables, scales: one per block)."""
+    B, C, F, H, W = latent.shape
+    arr = (BlockWeights * max(1, len(blocks)))(*blocks)
+    Li = 0 if img_ctx is None else img_ctx.shape[1]
+    _check(_lib().wan_dit_stack_fp8_fwd(ctypes.byref(cfg), len(blocks), _p(latent), B, F, H, W, _p(t),
+                                     ctypes.byref(sw), arr, _scales_array(scales), _p(ctx), ctx.shape[1],
+                                     _p(img_ctx), Li, _p(v_out), *_ws(ws), _stream(stream)),
+           "wan_dit_stack_fp8_fwd")
 
 
 def fp8_quantize_rows(cfg, x, q, scale, stream=None):

@@ -365,13 +365,121 @@ int head_impl(const wan_dit_config* c, const float* x, int B, int F, int H, int 
   return gemm(c, h, c->dim, w_head, b_head, v_out, B * L, c->out_ch * 4, c->dim, 0, ep, s);
 }
 
+// FP8 (E4M3) block
+// FP8 block workspace: the bf16 block's layout (its h region unused), then E4M3 codes
+// of the block inputs ([B*L, max(D, F)], reused by each linear layer in turn), codes of
+// the text / image context ([B*max(Lc, Li), D]) and the per-row scales of both.
+struct Fp8Layout {
+  Layout base;
+  size_t codes, ctx_codes, scales, ctx_scales, total;
+};
+Fp8Layout fp8_layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
+  Fp8Layout l;
+  l.base = layout(c, B, L, Lc, Li);
+  const size_t BL = static_cast<size_t>(B) * L;
+  const size_t Lx = static_cast<size_t>(B) * (Lc > Li ? Lc : Li);
+  const size_t wmax = c->ffn_dim > c->dim ? c->ffn_dim : c->dim;
+  l.codes = l.base.total;
+  l.ctx_codes = l.codes + align_up(BL * wmax);
+  l.scales = l.ctx_codes + align_up(Lx * c->dim);
+  l.ctx_scales = l.scales + align_up(BL * 4);
+  l.total = l.ctx_scales + align_up(Lx * 4);
+  return l;
+}
+
+int check_scales(const wan_fp8_scales* sc, bool with_img) {
+  WAN_REQUIRE(sc, WAN_ERR_NULL);
+  WAN_TRY(check_ptr_any(sc->qkv));
+  WAN_TRY(check_ptr_any(sc->o));
+  WAN_TRY(check_ptr_any(sc->cq));
+  WAN_TRY(check_ptr_any(sc->ckv));
+  WAN_TRY(check_ptr_any(sc->co));
+  WAN_TRY(check_ptr_any(sc->ffn1));
+  WAN_TRY(check_ptr_any(sc->ffn2));
+  if (with_img) WAN_TRY(check_ptr_any(sc->ckv_img));
+  return WAN_OK;
+}
+
+int e4m3_gemm(const void* A, const float* as, const void* W, const float* wsc, const void* bias, void* out, int M,
+              int N, int K, const GemmEpi& ep, cudaStream_t s) {
+  return launch_gemm_e4m3(A, K, as, W, wsc, bias, out, M, N, K, ep, s);
+}
+int block_fp8_impl(const wan_dit_config* cfg, float* x, const float* e, const void* ctx, int Lc, const void* img_ctx,
+                   int li, const wan_block_weights* w, const wan_fp8_scales* sc, int B, int L, void* workspace,
+                   const Fp8Layout& fl, cudaStream_t s, const void* kvt_cached = nullptr,
+                   const void* kvi_cached = nullptr, void* attn_kept = nullptr, bool attn_reuse = false) {
+  const bool with_img = img_ctx && li > 0;
+  const int D = cfg->dim, Fd = cfg->ffn_dim;
+  const int M = B * L;
+  const int64_t rows = M;
+  uint8_t* R = at(workspace, fl.base.big);
+  void* codes = at(workspace, fl.codes);
+  void* ctx_codes = at(workspace, fl.ctx_codes);
+  float* scales = reinterpret_cast<float*>(at(workspace, fl.scales));
+  float* ctx_scales = reinterpret_cast<float*>(at(workspace, fl.ctx_scales));
+  const size_t MD = static_cast<size_t>(M) * D * 2;  // bytes of one [M, D] bf16 slab
+  // self-attention
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 0, codes, scales, cfg->eps, s));
+  void* qkv = R;
+  void* o = attn_kept ? attn_kept : R + 3 * MD;
+  void* scr = at(workspace, fl.base.split);
+  const size_t scr_bytes = fl.base.split_bytes;
+  if (!(attn_kept && attn_reuse)) {
+    WAN_TRY(e4m3_gemm(codes, scales, w->w_qkv, sc->qkv, w->b_qkv, qkv, M, 3 * D, D, epi_store(3 * D), s));
+    WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s,
+                           nullptr, scr, scr_bytes));
+  }
+  WAN_TRY(launch_quantize_rows(o, D, M, D, false, codes, scales, WAN_BF16, s));
+  const float* gb_msa = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_o, sc->o, w->b_o, x, M, D, D, epi_residual(D, e + 2 * D, gb_msa, 6 * D, L), s));
+  // cross-attention
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, nullptr, nullptr, -1, codes, scales, cfg->eps, s));
+  void* q = R;
+  void* ocat = R + 3 * MD;
+  void* kvt = R + 5 * MD;
+  void* kvi = static_cast<uint8_t*>(kvt) + static_cast<size_t>(B) * Lc * 2 * D * 2;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_cq, sc->cq, w->b_cq, q, M, D, D, epi_store(D), s));
+  if (kvt_cached) {
+    kvt = const_cast<void*>(kvt_cached);
+  } else {
+    WAN_TRY(launch_quantize_rows(ctx, D, B * Lc, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
+    WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv, sc->ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, epi_store(2 * D),
+                      s));
+  }
+  const int ow = with_img ? 2 * D : D;
+  WAN_TRY(launch_attn_tc({q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, cfg->heads, L, Lc, s, nullptr,
+                         scr, scr_bytes));
+  if (with_img) {
+    if (kvi_cached) {
+      kvi = const_cast<void*>(kvi_cached);
+    } else {
+      WAN_TRY(launch_quantize_rows(img_ctx, D, B * li, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
+      WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv_img, sc->ckv_img, w->b_ckv_img, kvi, B * li, 2 * D, D,
+                        epi_store(2 * D), s));
+    }
+    WAN_TRY(launch_attn_tc({q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, cfg->heads, L, li, s,
+                           nullptr, scr, scr_bytes));
+  }
+  // the text and image outputs are summed while quantised
+  WAN_TRY(launch_quantize_rows(ocat, ow, M, D, with_img, codes, scales, WAN_BF16, s));
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_co, sc->co, w->b_co, x, M, D, D, epi_residual(D, nullptr, nullptr, 0, L), s));
+  // FFN
+  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 1, codes, scales, cfg->eps, s));
+  void* hid = R;
+  WAN_TRY(e4m3_gemm(codes, scales, w->w_1, sc->ffn1, w->b_1, hid, M, Fd, D, epi_store(Fd, WAN_EPI_GELU), s));
+  WAN_TRY(launch_quantize_rows(hid, Fd, M, Fd, false, codes, scales, WAN_BF16, s));
+  const float* gb_ffn = w->mod_bias ? w->mod_bias + 5 * D : nullptr;
+  return e4m3_gemm(codes, scales, w->w_2, sc->ffn2, w->b_2, x, M, D, Fd,
+                   epi_residual(D, e + 5 * D, gb_ffn, 6 * D, L), s);
+}
+
 // patchify -> timestep MLP -> blocks -> head. kvt/kvi: per-block cached cross-attention
 // K|V (arrays of n_blocks pointers) or NULL.
 int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H, int W,
                const float* t, const wan_stack_weights* sw, const wan_block_weights* blocks, const void* ctx, int Lc,
                const void* img_ctx, int li, float* v_out, void* workspace, const Layout& ly, cudaStream_t s,
                const void* const* kvt, const void* const* kvi, void* const* attn_kept = nullptr,
-               bool attn_reuse = false) {
+               bool attn_reuse = false, const wan_fp8_scales* fp8 = nullptr, const Fp8Layout* fl = nullptr) {
   const int L = F * (H / 2) * (W / 2);
   float* x = reinterpret_cast<float*>(at(workspace, ly.x));
   float* e = reinterpret_cast<float*>(at(workspace, ly.e));
@@ -382,9 +490,17 @@ int stack_impl(const wan_dit_config* cfg, int n_blocks, const void* latent, int 
   // the hidden units of the time MLP go to region R, free once the patchify GEMM has run
   WAN_TRY(launch_time_mlp(t, B, cfg->dim, cfg->freq_dim, sw->time.w_t1, sw->time.b_t1, sw->time.w_t2, sw->time.b_t2,
                           e, cfg->dtype, s, reinterpret_cast<float*>(patches)));
-  for (int i = 0; i < n_blocks; ++i)
-    WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s, kvt ? kvt[i] : nullptr,
-                       kvi ? kvi[i] : nullptr, attn_kept ? attn_kept[i] : nullptr, attn_reuse));
+  for (int i = 0; i < n_blocks; ++i) {
+    const void* kt = kvt ? kvt[i] : nullptr;
+    const void* ki = kvi ? kvi[i] : nullptr;
+    void* kept = attn_kept ? attn_kept[i] : nullptr;
+    if (fp8)
+      WAN_TRY(block_fp8_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], &fp8[i], B, L, workspace, *fl, s, kt, ki,
+                             kept, attn_reuse));
+    else
+      WAN_TRY(block_impl(cfg, x, e, ctx, Lc, img_ctx, li, &blocks[i], B, L, workspace, ly, s, kt, ki, kept,
+                         attn_reuse));
+  }
   return head_impl(cfg, x, B, F, H, W, sw->w_head, sw->b_head, v_out, at(workspace, ly.h), s);
 }
 
@@ -396,12 +512,12 @@ struct SampleLayout {
   size_t kvt_block, kvi_block, attn_block;  // bytes per block
 };
 SampleLayout sample_layout(const wan_dit_config* c, int n_blocks, int B, int F, int H, int W, int Lc, int Li,
-                           bool cache) {
+                           bool cache, bool fp8) {
   const size_t es = dtype_size(c->dtype);
   const int L = F * (H / 2) * (W / 2);
   const size_t fhw = static_cast<size_t>(F) * H * W;
   SampleLayout l;
-  l.in2 = align_up(layout(c, 2 * B, L, Lc, Li).total);
+  l.in2 = align_up(fp8 ? fp8_layout(c, 2 * B, L, Lc, Li).total : layout(c, 2 * B, L, Lc, Li).total);
   l.v = l.in2 + align_up(2 * static_cast<size_t>(B) * c->in_ch * fhw * es);
   l.t = l.v + align_up(2 * static_cast<size_t>(B) * c->out_ch * fhw * 4);
   l.kvt = l.t + align_up(2 * static_cast<size_t>(B) * 4);
@@ -671,47 +787,6 @@ int wan_sp_out_fwd(const wan_dit_config* cfg, int sp_size, const void* o, const 
               as_stream(stream));
 }
 
-// ------------------------------------------------------------------ FP8 (E4M3)
-namespace {
-// FP8 block workspace: the bf16 block's layout (its h region unused), then E4M3 codes
-// of the block inputs ([B*L, max(D, F)], reused by each linear layer in turn), codes of
-// the text / image context ([B*max(Lc, Li), D]) and the per-row scales of both.
-struct Fp8Layout {
-  Layout base;
-  size_t codes, ctx_codes, scales, ctx_scales, total;
-};
-Fp8Layout fp8_layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
-  Fp8Layout l;
-  l.base = layout(c, B, L, Lc, Li);
-  const size_t BL = static_cast<size_t>(B) * L;
-  const size_t Lx = static_cast<size_t>(B) * (Lc > Li ? Lc : Li);
-  const size_t wmax = c->ffn_dim > c->dim ? c->ffn_dim : c->dim;
-  l.codes = l.base.total;
-  l.ctx_codes = l.codes + align_up(BL * wmax);
-  l.scales = l.ctx_codes + align_up(Lx * c->dim);
-  l.ctx_scales = l.scales + align_up(BL * 4);
-  l.total = l.ctx_scales + align_up(Lx * 4);
-  return l;
-}
-
-int check_scales(const wan_fp8_scales* sc, bool with_img) {
-  WAN_REQUIRE(sc, WAN_ERR_NULL);
-  WAN_TRY(check_ptr_any(sc->qkv));
-  WAN_TRY(check_ptr_any(sc->o));
-  WAN_TRY(check_ptr_any(sc->cq));
-  WAN_TRY(check_ptr_any(sc->ckv));
-  WAN_TRY(check_ptr_any(sc->co));
-  WAN_TRY(check_ptr_any(sc->ffn1));
-  WAN_TRY(check_ptr_any(sc->ffn2));
-  if (with_img) WAN_TRY(check_ptr_any(sc->ckv_img));
-  return WAN_OK;
-}
-
-int e4m3_gemm(const void* A, const float* as, const void* W, const float* wsc, const void* bias, void* out, int M,
-              int N, int K, const GemmEpi& ep, cudaStream_t s) {
-  return launch_gemm_e4m3(A, K, as, W, wsc, bias, out, M, N, K, ep, s);
-}
-}  // namespace
 
 int wan_fp8_quantize_rows(const wan_dit_config* cfg, const void* x, int M, int K, void* q, float* scale,
                           void* stream) {
@@ -761,6 +836,7 @@ size_t wan_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, 
   return fp8_layout(cfg, B, L, Lc, Li).total;
 }
 
+
 int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x, const float* e, const void* ctx, int Lc,
                           const void* img_ctx, int Li, const wan_block_weights* w, const wan_fp8_scales* sc, int B,
                           int L, void* workspace, size_t ws_bytes, void* stream) {
@@ -780,73 +856,65 @@ int wan_dit_block_fp8_fwd(const wan_dit_config* cfg, float* x, const float* e, c
   const Fp8Layout fl = fp8_layout(cfg, B, L, Lc, li);
   WAN_REQUIRE(ws_bytes >= fl.total, WAN_ERR_WORKSPACE);
   if (B == 0 || L == 0) return WAN_OK;
-  cudaStream_t s = as_stream(stream);
-  const int D = cfg->dim, Fd = cfg->ffn_dim;
-  const int M = B * L;
-  const int64_t rows = M;
-  uint8_t* R = at(workspace, fl.base.big);
-  void* codes = at(workspace, fl.codes);
-  void* ctx_codes = at(workspace, fl.ctx_codes);
-  float* scales = reinterpret_cast<float*>(at(workspace, fl.scales));
-  float* ctx_scales = reinterpret_cast<float*>(at(workspace, fl.ctx_scales));
-  const size_t MD = static_cast<size_t>(M) * D * 2;  // bytes of one [M, D] bf16 slab
-  // self-attention
-  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 0, codes, scales, cfg->eps, s));
-  void* qkv = R;
-  void* o = R + 3 * MD;
-  WAN_TRY(e4m3_gemm(codes, scales, w->w_qkv, sc->qkv, w->b_qkv, qkv, M, 3 * D, D, epi_store(3 * D), s));
-  void* scr = at(workspace, fl.base.split);
-  const size_t scr_bytes = fl.base.split_bytes;
-  WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s,
-                         nullptr, scr, scr_bytes));
-  WAN_TRY(launch_quantize_rows(o, D, M, D, false, codes, scales, WAN_BF16, s));
-  const float* gb_msa = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
-  WAN_TRY(e4m3_gemm(codes, scales, w->w_o, sc->o, w->b_o, x, M, D, D, epi_residual(D, e + 2 * D, gb_msa, 6 * D, L), s));
-  // cross-attention
-  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, nullptr, nullptr, -1, codes, scales, cfg->eps, s));
-  void* q = R;
-  void* ocat = R + 3 * MD;
-  void* kvt = R + 5 * MD;
-  void* kvi = static_cast<uint8_t*>(kvt) + static_cast<size_t>(B) * Lc * 2 * D * 2;
-  WAN_TRY(e4m3_gemm(codes, scales, w->w_cq, sc->cq, w->b_cq, q, M, D, D, epi_store(D), s));
-  WAN_TRY(launch_quantize_rows(ctx, D, B * Lc, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
-  WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv, sc->ckv, w->b_ckv, kvt, B * Lc, 2 * D, D, epi_store(2 * D), s));
-  const int ow = with_img ? 2 * D : D;
-  WAN_TRY(launch_attn_tc({q, D, 0}, {kvt, 2 * D, 0}, {kvt, 2 * D, D}, ocat, ow, 0, B, cfg->heads, L, Lc, s, nullptr,
-                         scr, scr_bytes));
-  if (with_img) {
-    WAN_TRY(launch_quantize_rows(img_ctx, D, B * li, D, false, ctx_codes, ctx_scales, WAN_BF16, s));
-    WAN_TRY(e4m3_gemm(ctx_codes, ctx_scales, w->w_ckv_img, sc->ckv_img, w->b_ckv_img, kvi, B * li, 2 * D, D,
-                      epi_store(2 * D), s));
-    WAN_TRY(launch_attn_tc({q, D, 0}, {kvi, 2 * D, 0}, {kvi, 2 * D, D}, ocat, ow, D, B, cfg->heads, L, li, s,
-                           nullptr, scr, scr_bytes));
+  return block_fp8_impl(cfg, x, e, ctx, Lc, img_ctx, li, w, sc, B, L, workspace, fl, as_stream(stream));
+}
+
+int wan_dit_stack_fp8_fwd(const wan_dit_config* cfg, int n_blocks, const void* latent, int B, int F, int H, int W,
+                          const float* t, const wan_stack_weights* sw, const wan_block_weights* blocks,
+                          const wan_fp8_scales* scales, const void* ctx, int Lc, const void* img_ctx, int Li,
+                          float* v_out, void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_cfg(cfg, true));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  WAN_REQUIRE(sw && (n_blocks == 0 || (blocks && scales)), WAN_ERR_NULL);
+  WAN_REQUIRE(n_blocks >= 0 && B >= 0 && F >= 1 && H >= 2 && W >= 2 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(Lc > 0 && cfg->dim % 16 == 0 && cfg->ffn_dim % 16 == 0, WAN_ERR_SHAPE);
+  const bool with_img = img_ctx && Li > 0;
+  for (int i = 0; i < n_blocks; ++i) {
+    WAN_TRY(check_block_w(cfg, &blocks[i], with_img));
+    WAN_TRY(check_scales(&scales[i], with_img));
   }
-  // the text and image outputs are summed while quantised
-  WAN_TRY(launch_quantize_rows(ocat, ow, M, D, with_img, codes, scales, WAN_BF16, s));
-  WAN_TRY(e4m3_gemm(codes, scales, w->w_co, sc->co, w->b_co, x, M, D, D, epi_residual(D, nullptr, nullptr, 0, L), s));
-  // FFN
-  WAN_TRY(launch_layernorm_e4m3(x, rows, D, L, e, w->mod_bias, 1, codes, scales, cfg->eps, s));
-  void* hid = R;
-  WAN_TRY(e4m3_gemm(codes, scales, w->w_1, sc->ffn1, w->b_1, hid, M, Fd, D, epi_store(Fd, WAN_EPI_GELU), s));
-  WAN_TRY(launch_quantize_rows(hid, Fd, M, Fd, false, codes, scales, WAN_BF16, s));
-  const float* gb_ffn = w->mod_bias ? w->mod_bias + 5 * D : nullptr;
-  return e4m3_gemm(codes, scales, w->w_2, sc->ffn2, w->b_2, x, M, D, Fd,
-                   epi_residual(D, e + 5 * D, gb_ffn, 6 * D, L), s);
+  WAN_TRY(check_ptr(latent));
+  WAN_TRY(check_ptr(t));
+  WAN_TRY(check_ptr(ctx));
+  WAN_TRY(check_opt_ptr(img_ctx));
+  WAN_TRY(check_ptr(v_out));
+  WAN_TRY(check_ptr(sw->w_p));
+  WAN_TRY(check_opt_ptr(sw->b_p));
+  WAN_TRY(check_ptr(sw->w_head));
+  WAN_TRY(check_opt_ptr(sw->b_head));
+  WAN_TRY(check_ptr(sw->time.w_t1));
+  WAN_TRY(check_ptr(sw->time.w_t2));
+  WAN_TRY(check_ptr(sw->time.b_t1));
+  WAN_TRY(check_ptr(sw->time.b_t2));
+  WAN_TRY(check_ptr(workspace));
+  const int L = F * (H / 2) * (W / 2);
+  const int li = with_img ? Li : 0;
+  WAN_TRY(check_tokens(cfg, B, L, Lc, li));
+  const Fp8Layout fl = fp8_layout(cfg, B, L, Lc, li);
+  WAN_REQUIRE(ws_bytes >= fl.total, WAN_ERR_WORKSPACE);
+  if (B == 0) return WAN_OK;
+  return stack_impl(cfg, n_blocks, latent, B, F, H, W, t, sw, blocks, ctx, Lc, with_img ? img_ctx : nullptr, li, v_out,
+                    workspace, fl.base, as_stream(stream), nullptr, nullptr, nullptr, false, scales, &fl);
 }
 
 size_t wan_sample_workspace_bytes(const wan_dit_config* cfg, int n_blocks, int B, int F, int H, int W, int Lc,
-                                  int Li, const wan_diffusion_cache* cache) {
+                                  int Li, const wan_diffusion_cache* cache, int fp8) {
   if (check_cfg(cfg) != WAN_OK || n_blocks < 0 || B < 0 || F < 0 || H < 0 || W < 0 || Lc < 0 || Li < 0) return 0;
-  return sample_layout(cfg, n_blocks, B, F, H, W, Lc, Li, cache != nullptr).total;
+  return sample_layout(cfg, n_blocks, B, F, H, W, Lc, Li, cache != nullptr, fp8 != 0).total;
 }
 
 int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* input, int B, int F, int H, int W,
                          int n_steps, float guidance, const wan_stack_weights* sw, const wan_block_weights* blocks,
                          const void* ctx_cond, const void* ctx_uncond, int Lc, const void* img_ctx, int Li,
-                         const wan_diffusion_cache* cache, float* latent_out, void* workspace, size_t ws_bytes,
-                         void* stream) {
+                         const wan_diffusion_cache* cache, const wan_fp8_scales* fp8_scales, float* latent_out,
+                         void* workspace, size_t ws_bytes, void* stream) {
   WAN_TRY(check_cfg(cfg, true));
   WAN_REQUIRE(sw && (blocks || n_blocks == 0), WAN_ERR_NULL);
+  const bool fp8 = fp8_scales != nullptr;
+  if (fp8) {
+    if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+    WAN_REQUIRE(cfg->dim % 16 == 0 && cfg->ffn_dim % 16 == 0, WAN_ERR_SHAPE);
+  }
   if (cache)
     WAN_REQUIRE(cache->attn_start >= 0 && cache->attn_interval >= 1 && cache->cfg_start >= 0 &&
                     cache->cfg_interval >= 1,
@@ -855,7 +923,10 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
   WAN_REQUIRE(B >= 0 && F >= 1 && H >= 2 && W >= 2 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
   WAN_REQUIRE(cfg->out_ch <= cfg->in_ch && Lc > 0, WAN_ERR_SHAPE);
   const bool with_img = img_ctx && Li > 0;
-  for (int i = 0; i < n_blocks; ++i) WAN_TRY(check_block_w(cfg, &blocks[i], with_img));
+  for (int i = 0; i < n_blocks; ++i) {
+    WAN_TRY(check_block_w(cfg, &blocks[i], with_img));
+    if (fp8) WAN_TRY(check_scales(&fp8_scales[i], with_img));
+  }
   WAN_TRY(check_ptr(input));
   WAN_TRY(check_ptr(ctx_cond));
   WAN_TRY(check_ptr(ctx_uncond));
@@ -873,7 +944,7 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
   const int L = F * (H / 2) * (W / 2);
   const int li = with_img ? Li : 0;
   WAN_TRY(check_tokens(cfg, 2 * B, L, Lc, li));
-  const SampleLayout sl = sample_layout(cfg, n_blocks, B, F, H, W, Lc, li, cache != nullptr);
+  const SampleLayout sl = sample_layout(cfg, n_blocks, B, F, H, W, Lc, li, cache != nullptr, fp8);
   WAN_REQUIRE(ws_bytes >= sl.total, WAN_ERR_WORKSPACE);
   if (B == 0) return WAN_OK;
   cudaStream_t s = as_stream(stream);
@@ -885,21 +956,30 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
   float* v = reinterpret_cast<float*>(at(workspace, sl.v));
   float* t = reinterpret_cast<float*>(at(workspace, sl.t));
   WAN_TRY(launch_sampler_init(input, B, n, in_stride, latent_out, in2, t, cfg->dtype, s));
-  // Cross-attention K|V of both contexts, once per block for all steps.
+  // Cross-attention K|V of both contexts, once per block for all steps (E4M3 projections
+  // on the FP8 path, the context quantised per row in the stack workspace's code area).
+  const Fp8Layout fl = fp8_layout(cfg, 2 * B, L, Lc, li);
+  auto kv_proj = [&](const void* src, int rows, const void* wk, const void* bk, const float* wsc, void* dst) -> int {
+    if (!fp8) return gemm(cfg, src, D, wk, bk, dst, rows, 2 * D, D, 0, epi_store(2 * D), s);
+    void* codes = at(workspace, fl.ctx_codes);
+    float* scl = reinterpret_cast<float*>(at(workspace, fl.ctx_scales));
+    WAN_TRY(launch_quantize_rows(src, D, rows, D, false, codes, scl, WAN_BF16, s));
+    return e4m3_gemm(codes, scl, wk, wsc, bk, dst, rows, 2 * D, D, epi_store(2 * D), s);
+  };
   std::vector<const void*> kvt(n_blocks), kvi(n_blocks, nullptr);
   for (int i = 0; i < n_blocks; ++i) {
     uint8_t* ct = at(workspace, sl.kvt + i * sl.kvt_block);
     const size_t half_t = static_cast<size_t>(B) * Lc * 2 * D * es;
-    WAN_TRY(gemm(cfg, ctx_cond, D, blocks[i].w_ckv, blocks[i].b_ckv, ct, B * Lc, 2 * D, D, 0, epi_store(2 * D), s));
-    WAN_TRY(gemm(cfg, ctx_uncond, D, blocks[i].w_ckv, blocks[i].b_ckv, ct + half_t, B * Lc, 2 * D, D, 0,
-                 epi_store(2 * D), s));
+    const float* s_ckv = fp8 ? fp8_scales[i].ckv : nullptr;
+    WAN_TRY(kv_proj(ctx_cond, B * Lc, blocks[i].w_ckv, blocks[i].b_ckv, s_ckv, ct));
+    WAN_TRY(kv_proj(ctx_uncond, B * Lc, blocks[i].w_ckv, blocks[i].b_ckv, s_ckv, ct + half_t));
     kvt[i] = ct;
     if (with_img) {
       uint8_t* ci = at(workspace, sl.kvi + i * sl.kvi_block);
       const size_t half_i = static_cast<size_t>(B) * li * 2 * D * es;
       for (int h = 0; h < 2; ++h)
-        WAN_TRY(gemm(cfg, img_ctx, D, blocks[i].w_ckv_img, blocks[i].b_ckv_img, ci + h * half_i, B * li, 2 * D, D,
-                     0, epi_store(2 * D), s));
+        WAN_TRY(kv_proj(img_ctx, B * li, blocks[i].w_ckv_img, blocks[i].b_ckv_img,
+                        fp8 ? fp8_scales[i].ckv_img : nullptr, ci + h * half_i));
       kvi[i] = ci;
     }
   }
@@ -911,7 +991,7 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
     for (int i = 0; i < n_blocks; ++i) kept.push_back(at(workspace, sl.attn + i * sl.attn_block));
     delta = reinterpret_cast<float*>(at(workspace, sl.delta));
   }
-  const Layout ly = layout(cfg, 2 * B, L, Lc, li);
+  const Layout ly = fp8 ? fl.base : layout(cfg, 2 * B, L, Lc, li);
   const float dt = 1.0f / static_cast<float>(n_steps);
   for (int k = 0; k < n_steps; ++k) {
     bool reuse = false, skip = false;
@@ -923,7 +1003,7 @@ int wan_sample_euler_cfg(const wan_dit_config* cfg, int n_blocks, const void* in
     WAN_TRY(stack_impl(cfg, n_blocks, in2, Bp, F, H, W, t, sw, blocks, ctx_cond, Lc,
                        with_img ? img_ctx : nullptr, li, v, workspace, ly, s,
                        n_blocks ? kvt.data() : nullptr, with_img && n_blocks ? kvi.data() : nullptr,
-                       cache && n_blocks ? kept.data() : nullptr, reuse));
+                       cache && n_blocks ? kept.data() : nullptr, reuse, fp8 ? fp8_scales : nullptr, &fl));
     const float t_next = static_cast<float>(1000.0 * (k + 1) / n_steps);
     WAN_TRY(launch_euler_cfg(v, B, n, in_stride, dt, guidance, latent_out, in2, t, t_next, cfg->dtype, s, delta,
                              skip));

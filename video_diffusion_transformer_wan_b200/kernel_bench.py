@@ -50,16 +50,20 @@ def _sample(a) -> dict:
     ctx, ctx_u = to_device(inp["ctx"], model.act), to_device(inp["ctx_uncond"], model.act)
     out = torch.empty(B, w.out_ch, F, H, W, dtype=torch.float32, device="cuda")
     cache = wan.DiffusionCache(*[int(v) for v in a.cache.split(",")]) if a.cache else None
-    ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len, 0, cache), dtype=torch.uint8,
-                     device="cuda")
-    ms = _time(lambda: wan.sample_euler_cfg(cfg, noise, a.steps, a.guidance, model.stack_table,
-                                            model.block_tables, ctx, ctx_u, None, out, ws, cache=cache),
-               a.iters, a.warmup)
+    tables, scales = model.block_tables, None
+    if a.fp8:
+        from .model import Fp8Block
+        fbs = [Fp8Block(cfg, b) for b in model.blocks]
+        tables, scales = [f.table for f in fbs], [f.scale_table for f in fbs]
+    ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len, 0, cache, fp8=a.fp8),
+                     dtype=torch.uint8, device="cuda")
+    ms = _time(lambda: wan.sample_euler_cfg(cfg, noise, a.steps, a.guidance, model.stack_table, tables, ctx, ctx_u,
+                                            None, out, ws, cache=cache, fp8_scales=scales), a.iters, a.warmup)
     Lc, Fd = w.text_len, w.ffn
     # per step; the text K|V projections are made once per call and not counted
     block = 2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * L * Lc * D + 4 * L * D * Fd
     flops_step = 2 * B * (a.blocks * block + 2 * L * D * 64 * 2)
-    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, cache=a.cache or None, ms_per_call=ms,
+    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, cache=a.cache or None, fp8=a.fp8, ms_per_call=ms,
                 ms_per_euler_step=ms / a.steps,
                 latent_tokens_per_s=B * L * a.steps / (ms / 1e3),
                 tflops_uncached_equivalent=flops_step * a.steps / ms / 1e9)
@@ -96,7 +100,7 @@ def _block(a) -> dict:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block"])
-    ap.add_argument("--fp8", action="store_true", help="gemm / block: E4M3 operands (kind::f8f6f4)")
+    ap.add_argument("--fp8", action="store_true", help="gemm / block / sample: E4M3 operands (kind::f8f6f4)")
     ap.add_argument("--no-split", action="store_true",
                     help="attention: no workspace, so a partial last wave is not split over the keys")
     ap.add_argument("--workload", default="wan13b_480p_block", help="block: workload name")
