@@ -151,3 +151,16 @@ def test_sampler_validation_and_workspace(wan):
 
 def test_trace_read_without_events(wan):
     assert wan.trace_read(wan.KIND_ATTN) == (0.0, 0)
+
+
+def test_binding_refuses_strided_views(wan):
+    """The C calls take dense row-major arrays; a strided view is refused before the
+    call instead of being read with the wrong layout."""
+    import torch
+    t = torch.zeros(4, 6)
+    assert wan._p(t) == t.data_ptr()
+    with pytest.raises(ValueError):
+        wan._p(t.t())
+    with pytest.raises(ValueError):
+        wan._p(t[:, 1:3])
+    assert wan._p_strided(t[:, 2]) == t[:, 2].data_ptr()

@@ -159,12 +159,21 @@ def _check(status: int, where: str) -> None:
 
 
 def _p(t) -> Optional[int]:
-    """Device pointer of a tensor (or None)."""
+    """Device pointer of a contiguous tensor (or None, or a raw address). The C calls take
+    dense row-major arrays, so a strided view is refused here rather than misread."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got shape {tuple(t.shape)} strides {t.stride()}")
     return t.data_ptr()
+
+
+def _p_strided(t) -> Optional[int]:
+    """Device pointer of a tensor whose layout the call describes with explicit strides
+    (the residual epilogue's gate rows)."""
+    return None if t is None else (t if isinstance(t, int) else t.data_ptr())
 
 
 def _stream(stream=None) -> Optional[int]:
@@ -325,8 +334,8 @@ def linear_fp8_fwd(cfg, A, a_scale, W, w_scale, bias, out, epilogue, gate=None, 
     M = A.numel() // K
     N = W.shape[0]
     _check(_lib().wan_linear_fp8_fwd(ctypes.byref(cfg), _p(A), _p(a_scale), _p(W), _p(w_scale), _p(bias), _p(out),
-                                  M, N, K, epilogue, _p(gate), _p(gate_bias), gate_batch_stride, rows_per_batch,
-                                  _stream(stream)), "wan_linear_fp8_fwd")
+                                  M, N, K, epilogue, _p_strided(gate), _p(gate_bias), gate_batch_stride,
+                                  rows_per_batch, _stream(stream)), "wan_linear_fp8_fwd")
 
 
 def fp8_workspace_bytes(cfg: Config, B: int, L: int, Lc: int, Li: int = 0) -> int:
@@ -382,8 +391,9 @@ def linear_fwd(cfg, A, W, bias, out, epilogue, gate=None, gate_bias=None, gate_b
     K = A.shape[-1]
     M = A.numel() // K
     N = W.shape[0]
-    _check(_lib().wan_linear_fwd(ctypes.byref(cfg), _p(A), _p(W), _p(bias), _p(out), M, N, K, epilogue, _p(gate),
-                              _p(gate_bias), gate_batch_stride, rows_per_batch, _stream(stream)), "wan_linear_fwd")
+    _check(_lib().wan_linear_fwd(ctypes.byref(cfg), _p(A), _p(W), _p(bias), _p(out), M, N, K, epilogue,
+                              _p_strided(gate), _p(gate_bias), gate_batch_stride, rows_per_batch, _stream(stream)),
+           "wan_linear_fwd")
 
 
 def head_fwd(cfg, x, F, H, W, w_head, b_head, v_out, ws, stream=None):
