@@ -164,3 +164,23 @@ def test_binding_refuses_strided_views(wan):
     with pytest.raises(ValueError):
         wan._p(t[:, 1:3])
     assert wan._p_strided(t[:, 2]) == t[:, 2].data_ptr()
+
+
+def test_empty_inputs_launch_nothing(wan):
+    """Zero samples or zero tokens are valid and do nothing: status 0, no launch (which is
+    why this runs without a GPU)."""
+    L = wan.lib
+    cfg = _cfg(wan)
+    fake = 1 << 20
+    bw = wan.BlockWeights(*([fake] * 17))
+    n = wan.launch_count()
+    for B, T in [(0, 32), (1, 0), (0, 0)]:
+        assert L.wan_dit_block_fwd(ctypes.byref(cfg), fake, fake, fake, 512, None, 0, ctypes.byref(bw), B, T, fake,
+                                   1 << 40, None) == 0
+        assert L.wan_self_attn_fwd(ctypes.byref(cfg), fake, ctypes.byref(bw), fake, fake, B, T, fake, 1 << 40,
+                                   None) == 0
+        assert L.wan_ffn_fwd(ctypes.byref(cfg), fake, ctypes.byref(bw), fake, fake, B, T, fake, 1 << 40, None) == 0
+    assert L.wan_attention_fwd(ctypes.byref(cfg), fake, 4608, 0, fake, 4608, 1536, fake, 4608, 3072, fake, 1536, 0,
+                               0, 12, 32, 32, 128, None, 0, None) == 0
+    assert L.wan_linear_fwd(ctypes.byref(cfg), fake, fake, None, fake, 0, 64, 64, 0, None, None, 0, 1, None) == 0
+    assert wan.launch_count() == n

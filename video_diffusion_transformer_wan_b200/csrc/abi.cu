@@ -295,6 +295,7 @@ int self_attn_impl(const wan_dit_config* c, const void* h, const wan_block_weigh
 int cross_attn_impl(const wan_dit_config* c, const void* h, const void* ctx, int Lc, const void* img, int Li,
                     const wan_block_weights* w, float* x, int B, int L, void* ws, const Layout& ly, cudaStream_t s,
                     const void* kvt_cached = nullptr, const void* kvi_cached = nullptr) {
+  if (B == 0 || L == 0) return WAN_OK;  // no query rows: nothing to add to x
   const int D = c->dim;
   const size_t es = dtype_size(c->dtype);
   const int M = B * L;
@@ -339,6 +340,7 @@ int block_impl(const wan_dit_config* c, float* x, const float* e, const void* ct
                const wan_block_weights* w, int B, int L, void* ws, const Layout& ly, cudaStream_t s,
                const void* kvt_cached = nullptr, const void* kvi_cached = nullptr, void* attn_kept = nullptr,
                bool attn_reuse = false) {
+  if (B == 0 || L == 0) return WAN_OK;
   void* h = at(ws, ly.h);
   const int64_t rows = static_cast<int64_t>(B) * L;
   WAN_TRY(launch_layernorm(x, rows, c->dim, L, e, w->mod_bias, 0, h, c->dtype, c->eps, s));
