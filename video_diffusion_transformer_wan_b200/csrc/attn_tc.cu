@@ -54,12 +54,6 @@ constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
 constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMinSplitKeyTiles = 16;          // see launch_attn_tc
-// Of every 8 exponentials, how many run on the FMA pipes (exp2_poly) instead of the
-// MUFU unit (0..4). Measured best at 0 for this kernel (1 and 2 were slower).
-#ifndef WAN_ATTN_POLY_EXP
-#define WAN_ATTN_POLY_EXP 0
-#endif
-constexpr int kPolyExp = WAN_ATTN_POLY_EXP;
 
 struct AttnParams {
   int Lq, Lk, H;
@@ -313,7 +307,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float x0 = fmaf(__uint_as_float(r[2 * i]), sl2, nb);
         const float x1 = fmaf(__uint_as_float(r[2 * i + 1]), sl2, nb);
         const float e0 = ex2_approx(x0);
-        const float e1 = ((i & 3) < kPolyExp) ? exp2_poly(x1) : ex2_approx(x1);
+        const float e1 = ex2_approx(x1);
         rs8[i & 7] += e0 + e1;
         r[i] = pack_bf16x2(e0, e1);
       }

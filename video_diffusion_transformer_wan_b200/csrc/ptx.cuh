@@ -239,23 +239,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA/ALU pipes, leaving the MUFU unit to other exponentials. Cody-Waite
-// range reduction (W. J. Cody and W. Waite, "Software Manual for the Elementary
-// Functions", 1980): x = n + f with n = round(x) (the 1.5 * 2^23 addition puts n in the
-// low mantissa bits) and f in [-0.5, 0.5]; 2^f from a degree-3 polynomial whose
-// coefficients were fitted here for minimum relative error on [-0.5, 0.5] (max relative
-// error 7.5e-5, 13.7 bits - above the 8 bits of the bf16 P it feeds); 2^n is added to
-// the exponent field. Inputs below -125 are clamped (result ~2e-38, i.e. zero weight).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const int n = __float_as_int(t) - 0x4B400000;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.055171143263578415f, f, 0.24260996282100677f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999281167984009f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
