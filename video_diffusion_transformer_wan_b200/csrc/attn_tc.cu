@@ -18,7 +18,9 @@
 //               values are read from TMEM with a single wait (the wait covers every
 //               outstanding TMEM load, so reading in pieces would expose its latency
 //               once per piece); fp32 max and sum, ex2, the ragged last key tile
-//               masked only on that tile. P is rounded to bf16, packed in place and
+//               masked only on that tile. Scaling and row sums run on packed f32x2
+//               pairs (one instruction per pair), which leaves more issue slots to the
+//               other tile's softmax warp and the MMA warp on the same SM sub-partition. P is rounded to bf16, packed in place and
 //               written back into tensor memory over the S columns already read (two
 //               bf16 per 32-bit column, the layout of a K-major MMA operand), so P
 //               never touches shared memory.
@@ -182,31 +184,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(kTile, kHd, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t kv_addr = smem_u32(sKV);
+      // Shared-memory descriptors are built once: every operand below sits at a fixed
+      // byte offset from sQ or sKV, and an offset moves only the 14-bit address field
+      // (offset >> 4, no carry out of it since shared addresses stay below 256 KB). The
+      // single issuing thread then spends one add per operand on each MMA.
+      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(smem_u32(sKV), 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(sKV), kHalfBytes, 1024);
       auto wait_pos = [&](int pos) {
         return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
       };
       auto pv = [&](int t, int i, int vstage) {
         // A = P_t in TMEM: bf16 pairs packed in the first 64 columns of S_t's region.
         const uint32_t p_tmem = tmem_base + t * kTile;
-        const uint32_t va = kv_addr + vstage * kTileBytes;
+        const uint64_t vd = v_desc + static_cast<uint32_t>((vstage * kTileBytes) >> 4);
         const uint32_t o_tmem = tmem_base + 256 + t * kTile;
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k) {
-          const uint64_t bd = sdesc_sw128(va + k * 16 * 128, kHalfBytes, 1024);
-          tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, bd, idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < kTile / 16; ++k)
+          tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
       };
       auto qk = [&](int t, int kstage) {
-        const uint32_t qa = q_addr + t * kTileBytes;
-        const uint32_t ka = kv_addr + kstage * kTileBytes;
+        const uint64_t qd = q_desc + static_cast<uint32_t>((t * kTileBytes) >> 4);
+        const uint64_t kd = k_desc + static_cast<uint32_t>((kstage * kTileBytes) >> 4);
         const uint32_t s_tmem = tmem_base + t * kTile;
 #pragma unroll
         for (int k = 0; k < kHd / 16; ++k) {
-          const uint32_t off = (k >> 2) * kHalfBytes + (k & 3) * 32;
-          tc_mma_bf16(s_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc_qk,
-                      k > 0 ? 1u : 0u);
+          const uint32_t off = ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4;
+          tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(q_full, 0, p.err);
@@ -286,7 +290,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(r[a]);
 #pragma unroll
-      for (int i = 8; i < kTile; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], __uint_as_float(r[i]));
+      for (int i = 8; i < kTile; i += 2)
+        mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const bool grow = (mx - m_run) * sl2 > kRescaleLog2;
@@ -301,14 +306,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         rescale = true;
       }
       const float nb = -m_run * sl2;
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const unsigned long long sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
+      unsigned long long rs4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int i = 0; i < kTile / 2; ++i) {
-        const float x0 = fmaf(__uint_as_float(r[2 * i]), sl2, nb);
-        const float x1 = fmaf(__uint_as_float(r[2 * i + 1]), sl2, nb);
-        const float e0 = ex2_approx(x0);
-        const float e1 = ex2_approx(x1);
-        rs8[i & 7] += e0 + e1;
+        const unsigned long long s2 = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        const float2 x = f2_unpack(f2_fma(s2, sl2x2, nbx2));
+        const float e0 = ex2_approx(x.x);
+        const float e1 = ex2_approx(x.y);
+        rs4[i & 3] = f2_add(rs4[i & 3], f2_pack(e0, e1));
         r[i] = pack_bf16x2(e0, e1);
       }
       tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
@@ -327,7 +333,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         l_run *= alpha;
       }
-      l_run += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      {
+        const float2 s01 = f2_unpack(f2_add(rs4[0], rs4[1])), s23 = f2_unpack(f2_add(rs4[2], rs4[3]));
+        l_run += (s01.x + s01.y) + (s23.x + s23.y);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
