@@ -538,3 +538,33 @@ def linear_fp8(x, weight, bias=None) -> np.ndarray:
     qw, sw = quantize_e4m3(weight)
     y = (qx @ qw.T) * sx.astype(np.float64) * np.float64(sw)
     return y if bias is None else y + _f(bias)
+
+
+def attention_fp8(q, k, v, heads: int) -> np.ndarray:
+    """8-bit attention [Wan-P2, "Infra", inference optimisation: 8-bit FlashAttention,
+    INT8 for q k^T and FP8 for the product with v]. reading: E4M3 for both products (the
+    8-bit format of the tensor cores' f8 kind), with these scales, each an amax / 448
+    as in ``quantize_e4m3``:
+
+    * q: one scale per (token, head) -- the per-token activation scale, per head since
+      each head's q k^T is a separate product;
+    * k and v: one scale per head over all key rows, so a key's scale does not vary
+      along a row of the score matrix;
+    * the probabilities ``p = exp(s - max_j s)`` (in (0, 1]) are rounded to E4M3
+      without a scale, for the product with v; the normaliser is the sum of the
+      unrounded p.
+
+    Per head: ``s = (q^ k^T) sq sk / sqrt(d)``, ``o = sv (E4M3(p) v^) / sum_j p``."""
+    q, k, v = (np.asarray(a, dtype=np.float32) for a in (q, k, v))
+    Lq, D = q.shape
+    d = D // heads
+    out = np.empty((Lq, D), dtype=F64)
+    for hh in range(heads):
+        sl = slice(hh * d, (hh + 1) * d)
+        qq, sq = quantize_e4m3(q[:, sl], axis=-1)
+        kq, sk = quantize_e4m3(k[:, sl])
+        vq, sv = quantize_e4m3(v[:, sl])
+        s = (qq @ kq.T) * sq.astype(F64) * F64(sk) / math.sqrt(d)
+        p = np.exp(s - s.max(axis=-1, keepdims=True))
+        out[:, sl] = F64(sv) * (round_e4m3(p) @ vq) / p.sum(axis=-1, keepdims=True)
+    return out

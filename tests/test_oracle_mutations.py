@@ -224,3 +224,30 @@ def test_fp8_mutations_are_caught(monkeypatch):
     monkeypatch.setattr(O, "quantize_e4m3", tensor_scales)
     _fails(P.check_block_fp8_vs_torch, O.dit_block)
     monkeypatch.undo()
+
+
+def _attention_fp8_variant(q_axis=-1, round_p=True, norm_rounded=False, v_axis=None):
+    def f(q, k, v, heads):
+        q, k, v = (np.asarray(a, dtype=np.float32) for a in (q, k, v))
+        d = q.shape[1] // heads
+        out = np.empty(q.shape)
+        for hh in range(heads):
+            sl = slice(hh * d, (hh + 1) * d)
+            qq, sq = O.quantize_e4m3(q[:, sl], axis=q_axis)
+            kq, sk = O.quantize_e4m3(k[:, sl])
+            vq, sv = O.quantize_e4m3(v[:, sl], axis=v_axis)
+            s = (qq @ kq.T) * np.asarray(sq, np.float64) * np.float64(sk) / math.sqrt(d)
+            p = np.exp(s - s.max(axis=-1, keepdims=True))
+            pr = O.round_e4m3(p) if round_p else p
+            vv = vq * np.asarray(sv, np.float64)
+            out[:, sl] = (pr @ vv) / (pr if norm_rounded else p).sum(axis=-1, keepdims=True)
+        return out
+    return f
+
+
+def test_attention_fp8_mutations_are_caught():
+    _fails(P.check_attention_fp8, _attention_fp8_variant(q_axis=None))          # one q scale per head
+    _fails(P.check_attention_fp8, _attention_fp8_variant(round_p=False))        # p kept exact
+    _fails(P.check_attention_fp8, _attention_fp8_variant(norm_rounded=True))    # normaliser from rounded p
+    _fails(P.check_attention_fp8, _attention_fp8_variant(v_axis=-1))            # a v scale per key row
+    P.check_attention_fp8(_attention_fp8_variant())                              # the unmutated restatement passes

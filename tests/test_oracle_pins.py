@@ -716,3 +716,59 @@ def check_block_fp8_vs_torch(dit_block):
 
 def test_block_fp8_matches_library_reexpression():
     check_block_fp8_vs_torch(O.dit_block)
+
+
+# ----------------------------------------------------------------------------------------
+# 8-bit attention
+# ----------------------------------------------------------------------------------------
+
+def torch_attention_fp8(q, k, v, heads):
+    """The same definition through torch's float8_e4m3fn conversion (float32 scales and
+    divisions, as in the kernels' quantisers)."""
+    q, k, v = (torch.from_numpy(np.asarray(a, dtype=np.float32)) for a in (q, k, v))
+    d = q.shape[1] // heads
+    f8 = torch.float8_e4m3fn
+
+    def scale(a, dim=None):
+        m = a.abs().amax(dim=dim, keepdim=dim is not None)
+        return torch.where(m > 0, m / 448.0, torch.ones_like(m))
+    outs = []
+    for h in range(heads):
+        qh, kh, vh = (a[:, h * d:(h + 1) * d] for a in (q, k, v))
+        sq, sk, sv = scale(qh, 1), scale(kh), scale(vh)
+        qc, kc, vc = ((a / s).to(f8).double() for a, s in ((qh, sq), (kh, sk), (vh, sv)))
+        s = (qc @ kc.T) * sq.double() * sk.double() / math.sqrt(d)
+        p = torch.exp(s - s.amax(1, keepdim=True))
+        outs.append(sv.double() * (p.to(f8).double() @ vc) / p.sum(1, keepdim=True))
+    return torch.cat(outs, 1).numpy()
+
+
+def check_attention_fp8(attention_fp8):
+    rng = RNG(31)
+    for Lq, Lk, H, d in [(5, 7, 2, 16), (9, 40, 3, 8), (4, 1, 1, 32)]:
+        q = rng.standard_normal((Lq, H * d)) * np.exp2(rng.integers(-3, 4, (Lq, 1)))
+        k = rng.standard_normal((Lk, H * d)) * 2
+        v = rng.standard_normal((Lk, H * d))
+        got = attention_fp8(q, k, v, H)
+        np.testing.assert_allclose(got, torch_attention_fp8(q, k, v, H), rtol=1e-12, atol=1e-13)
+        exact = O.attention(q.astype(np.float32), k.astype(np.float32), v.astype(np.float32), H)
+        assert np.abs(got - exact).max() < 0.15 * np.abs(exact).max()        # an approximation of it
+    # values on the E4M3 grid with a power-of-two scale are represented exactly:
+    # one key gives that key's value, equal keys give the mean of the values
+    grid = np.array([O.e4m3_decode(c) for c in range(0x7F)])
+    v = rng.choice(grid, (6, 16)) * rng.choice([-1.0, 1.0], (6, 16)) / 16.0
+    v[0, 0] = 448.0 / 16.0                                                   # scale 2^-4 for both heads
+    v[0, 8] = -448.0 / 16.0
+    q = rng.standard_normal((4, 16))
+    np.testing.assert_array_equal(attention_fp8(q, rng.standard_normal((1, 16)), v[:1], 2), np.repeat(v[:1], 4, 0))
+    k = np.repeat(rng.standard_normal((1, 16)), 6, 0)
+    np.testing.assert_allclose(attention_fp8(q, k, v, 2), np.repeat(v.mean(0, keepdims=True), 4, 0),
+                               rtol=1e-15, atol=1e-15)
+    # keys and values permuted together: same output
+    k, v = rng.standard_normal((11, 16)), rng.standard_normal((11, 16))
+    perm = rng.permutation(11)
+    np.testing.assert_allclose(attention_fp8(q, k[perm], v[perm], 2), attention_fp8(q, k, v, 2), rtol=1e-12)
+
+
+def test_attention_fp8_pins():
+    check_attention_fp8(O.attention_fp8)
