@@ -550,11 +550,14 @@ def attention_fp8(q, k, v, heads: int) -> np.ndarray:
       each head's q k^T is a separate product;
     * k and v: one scale per head over all key rows, so a key's scale does not vary
       along a row of the score matrix;
-    * the probabilities ``p = exp(s - max_j s)`` (in (0, 1]) are rounded to E4M3
-      without a scale, for the product with v; the normaliser is the sum of the
-      unrounded p.
+    * the probabilities, taken against a power-of-two base, ``p = 2^(x - ceil(max_j x))``
+      with ``x`` the logit in log2 units (so the row's largest p lies in (1/2, 1]), are
+      rounded to E4M3 without a further scale for the product with v; the normaliser
+      is the sum of the unrounded p. (Softmax does not depend on the base; a power-of-
+      two base makes the rounding of p the same for any base a whole power of two
+      away, which a one-pass kernel with a running base can reproduce.)
 
-    Per head: ``s = (q^ k^T) sq sk / sqrt(d)``, ``o = sv (E4M3(p) v^) / sum_j p``."""
+    Per head: ``x = (q^ k^T) sq sk / (sqrt(d) ln 2)``, ``o = sv (E4M3(p) v^) / sum_j p``."""
     q, k, v = (np.asarray(a, dtype=np.float32) for a in (q, k, v))
     Lq, D = q.shape
     d = D // heads
@@ -564,7 +567,7 @@ def attention_fp8(q, k, v, heads: int) -> np.ndarray:
         qq, sq = quantize_e4m3(q[:, sl], axis=-1)
         kq, sk = quantize_e4m3(k[:, sl])
         vq, sv = quantize_e4m3(v[:, sl])
-        s = (qq @ kq.T) * sq.astype(F64) * F64(sk) / math.sqrt(d)
-        p = np.exp(s - s.max(axis=-1, keepdims=True))
+        x = (qq @ kq.T) * sq.astype(F64) * F64(sk) / (math.sqrt(d) * math.log(2.0))
+        p = np.exp2(x - np.ceil(x.max(axis=-1, keepdims=True)))
         out[:, sl] = F64(sv) * (round_e4m3(p) @ vq) / p.sum(axis=-1, keepdims=True)
     return out

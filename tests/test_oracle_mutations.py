@@ -226,7 +226,7 @@ def test_fp8_mutations_are_caught(monkeypatch):
     monkeypatch.undo()
 
 
-def _attention_fp8_variant(q_axis=-1, round_p=True, norm_rounded=False, v_axis=None):
+def _attention_fp8_variant(q_axis=-1, round_p=True, norm_rounded=False, v_axis=None, int_base=True):
     def f(q, k, v, heads):
         q, k, v = (np.asarray(a, dtype=np.float32) for a in (q, k, v))
         d = q.shape[1] // heads
@@ -236,8 +236,9 @@ def _attention_fp8_variant(q_axis=-1, round_p=True, norm_rounded=False, v_axis=N
             qq, sq = O.quantize_e4m3(q[:, sl], axis=q_axis)
             kq, sk = O.quantize_e4m3(k[:, sl])
             vq, sv = O.quantize_e4m3(v[:, sl], axis=v_axis)
-            s = (qq @ kq.T) * np.asarray(sq, np.float64) * np.float64(sk) / math.sqrt(d)
-            p = np.exp(s - s.max(axis=-1, keepdims=True))
+            x = (qq @ kq.T) * np.asarray(sq, np.float64) * np.float64(sk) / (math.sqrt(d) * math.log(2.0))
+            m = x.max(axis=-1, keepdims=True)
+            p = np.exp2(x - (np.ceil(m) if int_base else m))
             pr = O.round_e4m3(p) if round_p else p
             vv = vq * np.asarray(sv, np.float64)
             out[:, sl] = (pr @ vv) / (pr if norm_rounded else p).sum(axis=-1, keepdims=True)
@@ -250,4 +251,5 @@ def test_attention_fp8_mutations_are_caught():
     _fails(P.check_attention_fp8, _attention_fp8_variant(round_p=False))        # p kept exact
     _fails(P.check_attention_fp8, _attention_fp8_variant(norm_rounded=True))    # normaliser from rounded p
     _fails(P.check_attention_fp8, _attention_fp8_variant(v_axis=-1))            # a v scale per key row
+    _fails(P.check_attention_fp8, _attention_fp8_variant(int_base=False))       # base at the row max itself
     P.check_attention_fp8(_attention_fp8_variant())                              # the unmutated restatement passes

@@ -737,8 +737,8 @@ def torch_attention_fp8(q, k, v, heads):
         qh, kh, vh = (a[:, h * d:(h + 1) * d] for a in (q, k, v))
         sq, sk, sv = scale(qh, 1), scale(kh), scale(vh)
         qc, kc, vc = ((a / s).to(f8).double() for a, s in ((qh, sq), (kh, sk), (vh, sv)))
-        s = (qc @ kc.T) * sq.double() * sk.double() / math.sqrt(d)
-        p = torch.exp(s - s.amax(1, keepdim=True))
+        x = (qc @ kc.T) * sq.double() * sk.double() / math.sqrt(d) / math.log(2.0)
+        p = torch.exp2(x - torch.ceil(x.amax(1, keepdim=True)))
         outs.append(sv.double() * (p.to(f8).double() @ vc) / p.sum(1, keepdim=True))
     return torch.cat(outs, 1).numpy()
 
@@ -753,17 +753,18 @@ def check_attention_fp8(attention_fp8):
         np.testing.assert_allclose(got, torch_attention_fp8(q, k, v, H), rtol=1e-12, atol=1e-13)
         exact = O.attention(q.astype(np.float32), k.astype(np.float32), v.astype(np.float32), H)
         assert np.abs(got - exact).max() < 0.15 * np.abs(exact).max()        # an approximation of it
-    # values on the E4M3 grid with a power-of-two scale are represented exactly:
-    # one key gives that key's value, equal keys give the mean of the values
+    # values on the E4M3 grid with a power-of-two scale are represented exactly, and a
+    # zero query makes every logit 0, so p = 1 exactly: one key gives that key's value,
+    # several keys the mean of the values
     grid = np.array([O.e4m3_decode(c) for c in range(0x7F)])
     v = rng.choice(grid, (6, 16)) * rng.choice([-1.0, 1.0], (6, 16)) / 16.0
     v[0, 0] = 448.0 / 16.0                                                   # scale 2^-4 for both heads
     v[0, 8] = -448.0 / 16.0
+    q0 = np.zeros((4, 16))
+    np.testing.assert_array_equal(attention_fp8(q0, rng.standard_normal((1, 16)), v[:1], 2), np.repeat(v[:1], 4, 0))
+    np.testing.assert_allclose(attention_fp8(q0, rng.standard_normal((6, 16)), v, 2),
+                               np.repeat(v.mean(0, keepdims=True), 4, 0), rtol=1e-15, atol=1e-15)
     q = rng.standard_normal((4, 16))
-    np.testing.assert_array_equal(attention_fp8(q, rng.standard_normal((1, 16)), v[:1], 2), np.repeat(v[:1], 4, 0))
-    k = np.repeat(rng.standard_normal((1, 16)), 6, 0)
-    np.testing.assert_allclose(attention_fp8(q, k, v, 2), np.repeat(v.mean(0, keepdims=True), 4, 0),
-                               rtol=1e-15, atol=1e-15)
     # keys and values permuted together: same output
     k, v = rng.standard_normal((11, 16)), rng.standard_normal((11, 16))
     perm = rng.permutation(11)
