@@ -440,6 +440,42 @@ int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, cons
                    const float* gate, const float* gate_bias, int64_t gate_batch_stride,
                    int rows_per_batch, void* stream);
 
+/* ---- 8-bit attention --------------------------------------------------------------- */
+
+/* 8-bit attention [Wan 2.1 page, "Infra", inference optimisation: 8-bit FlashAttention,
+ * INT8 for q k^T and FP8 for the product with v], here with E4M3 for both products
+ * (the tensor cores' f8 kind; tcgen05 kind::f8f6f4). Scales (each amax / 448 as above,
+ * IEEE float32): q per (sample, token, head); k and v per (sample, head) over all key
+ * rows. The probabilities p = 2^(s log2e / sqrt(d) - base) are rounded to E4M3 for the
+ * product with v; the normaliser is the fp32 sum of the unrounded p. The base of a row
+ * is its running max, moved only when the max grows by more than 2^8 (p <= 256). */
+
+/* The quantisation step alone. Inputs as in wan_attention_fwd (bf16, head_dim 128).
+ * Outputs (device, caller-owned): q_codes [B, Lq, H*128] E4M3 bytes; q_scale
+ * [B, Lq, H] fp32; k_codes [B, Lk, H*128]; vt_codes [B, H*128, vt_stride] (v
+ * transposed: row = head dim, column = key; vt_stride % 64 == 0, vt_stride >= Lk;
+ * columns from Lk to the next multiple of 64 are written as code 0); kv_scale [B, H, 2]
+ * fp32 = (k scale, v scale), also used as scratch while the work runs. Five kernels. */
+int wan_attention_fp8_quantize(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0,
+                               const void* k, int64_t k_row_stride, int k_col0,
+                               const void* v, int64_t v_row_stride, int v_col0,
+                               int B, int heads, int Lq, int Lk, int head_dim,
+                               void* q_codes, float* q_scale, void* k_codes, void* vt_codes, int64_t vt_stride,
+                               float* kv_scale, void* stream);
+
+/* softmax(q k^T / sqrt(d)) v on the E4M3 operands above: the same arguments and output
+ * as wan_attention_fwd; the workspace (required, wan_attention_fp8_workspace_bytes)
+ * holds the codes and scales, and the key-split scratch of a partial last wave. */
+int wan_attention_fp8_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0,
+                          const void* k, int64_t k_row_stride, int k_col0,
+                          const void* v, int64_t v_row_stride, int v_col0,
+                          void* o, int64_t o_row_stride, int o_col0,
+                          int B, int heads, int Lq, int Lk, int head_dim, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/* Bytes of the wan_attention_fp8_fwd workspace for B samples, Lq queries, Lk keys. */
+size_t wan_attention_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int Lq, int Lk);
+
 /* ---- tracing ------------------------------------------------------------------- */
 
 /* Total number of kernels this library has launched in this process. */

@@ -20,6 +20,16 @@ FP8_TOL_RMS = 2.5e-2
 # and 4.5 % apart).
 FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS = 1e-2, 8e-3
 FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
+# 8-bit attention against the oracle's. The kernel takes each row's probabilities
+# against its running max (moved only when the max grows past 2^8), rounded up to a
+# whole power of two; the oracle against the row's final max. Whole powers of two leave
+# E4M3 codes unchanged up to that factor, except in the subnormal and flush range, where
+# a lower running base keeps small probabilities the oracle rounds away. Emulating the
+# kernel's running base in the oracle (per 128-key tile, per 32-row warp) moves the
+# result by at most 5.3 % (max-norm) and 2.0 % (RMS) over logit standard deviations 0.6,
+# 1 and 4, 700 to 32760 keys, whole and key-split; bars 1.5x: 8e-2 and 3e-2. (8-bit
+# attention itself is 4-10 % (max) and 4-11 % (RMS) away from exact attention there.)
+FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS = 8e-2, 3e-2
 
 
 def rel_err(got, ref) -> float:

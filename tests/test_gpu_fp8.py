@@ -1,14 +1,15 @@
 """FP8 (E4M3) path through the C ABI against the oracle: quantisation codes and scales
 bit-exact (same float32 input, same float32 decision), the kind::f8f6f4 GEMM against
-the product of the codes, and the FP8 block against the oracle's FP8 block (T2V, I2V,
-and the 1.3B 480P block on sampled rows)."""
+the product of the codes, the FP8 block against the oracle's FP8 block (T2V, I2V,
+and the 1.3B 480P block on sampled rows), and 8-bit attention (operand codes bit-exact,
+output within the derived bars)."""
 import numpy as np
 import pytest
 
 from oracle import wan_oracle as O
 from wan_inputs import WORKLOADS, make_inputs, round_bf16, sample_rows
-from gpu_util import (FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS, FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS, FP8_TOL_MAX,
-                      FP8_TOL_RMS, dev, host, rel_err, rms_err, rng)
+from gpu_util import (FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS, FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS, FP8_STACK_TOL_MAX,
+                      FP8_STACK_TOL_RMS, FP8_TOL_MAX, FP8_TOL_RMS, dev, host, rel_err, rms_err, rng)
 from test_gpu_block import Run, small_bf16
 
 torch = pytest.importorskip("torch")
@@ -203,3 +204,87 @@ def test_sampler_fp8_matches_oracle(wan):
         print(f"fp8 sampler b={b}: displacement max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
         assert rel_err(d_got, d_ref) <= FP8_SAMPLE_TOL_MAX
         assert rms_err(d_got, d_ref) <= FP8_SAMPLE_TOL_RMS
+
+
+# ----------------------------------------------------------------------------------------
+# 8-bit attention
+# ----------------------------------------------------------------------------------------
+
+def _qkv(seed, B, Lq, Lk, H, logit_std):
+    r = rng(seed)
+    s = np.sqrt(logit_std)
+    D = H * 128
+    q = round_bf16(r.standard_normal((B, Lq, D)) * s * np.exp2(r.integers(-3, 4, (B, Lq, 1))))
+    k = round_bf16(r.standard_normal((B, Lk, D)) * s)
+    v = round_bf16(r.standard_normal((B, Lk, D)))
+    return q, k, v
+
+
+def _attn_cfg(wan, H):
+    return wan.make_config(H * 128, H, 4 * H * 128)
+
+
+@pytest.mark.parametrize("B,Lq,Lk,H", [(2, 300, 700, 2), (1, 1, 65, 1), (1, 129, 1, 3)])
+def test_attention_fp8_quantize_bit_exact(wan, B, Lq, Lk, H):
+    q, k, v = _qkv(B * Lq + Lk, B, Lq, Lk, H, 1.0)
+    q[0, 0, :128] = 0.0                                  # a zero (row, head): scale 1
+    D = H * 128
+    S = (Lk + 63) // 64 * 64
+    qc = torch.empty(B, Lq, D, dtype=torch.uint8, device="cuda")
+    qs = torch.empty(B, Lq, H, dtype=torch.float32, device="cuda")
+    kc = torch.empty(B, Lk, D, dtype=torch.uint8, device="cuda")
+    vt = torch.full((B, D, S), 0xAB, dtype=torch.uint8, device="cuda")
+    kvs = torch.empty(B, H, 2, dtype=torch.float32, device="cuda")
+    bf = torch.bfloat16
+    wan.attention_fp8_quantize(_attn_cfg(wan, H), dev(q, bf), dev(k, bf), dev(v, bf), H, 128, qc, qs, kc, vt, kvs)
+    torch.cuda.synchronize()
+    qc, qs, kc, vt, kvs = (t.cpu().numpy() for t in (qc, qs, kc, vt, kvs))
+    for b in range(B):
+        for h in range(H):
+            sl = slice(h * 128, (h + 1) * 128)
+            rq, rs = O.quantize_e4m3(np.asarray(q[b][:, sl], np.float32), axis=-1)
+            assert np.array_equal(E4M3[qc[b][:, sl]], rq) and np.array_equal(qs[b][:, h], rs[:, 0])
+            rk, sk = O.quantize_e4m3(np.asarray(k[b][:, sl], np.float32))
+            assert np.array_equal(E4M3[kc[b][:, sl]], rk) and kvs[b, h, 0] == sk
+            rv, sv = O.quantize_e4m3(np.asarray(v[b][:, sl], np.float32))
+            assert np.array_equal(E4M3[vt[b][sl, :Lk]], rv.T) and kvs[b, h, 1] == sv
+            assert not vt[b][sl, Lk:].any()              # keys past Lk are code 0 up to the 64-multiple
+
+
+def _attention_fp8_case(wan, B, Lq, Lk, H, logit_std, seed, rows=None):
+    q, k, v = _qkv(seed, B, Lq, Lk, H, logit_std)
+    D = H * 128
+    cfg = _attn_cfg(wan, H)
+    bf = torch.bfloat16
+    o = torch.full((B, Lq, D), float("nan"), dtype=bf, device="cuda")
+    ws = torch.empty(wan.attention_fp8_workspace_bytes(cfg, B, Lq, Lk), dtype=torch.uint8, device="cuda")
+    wan.attention_fp8_fwd(cfg, dev(q, bf), dev(k, bf), dev(v, bf), o, H, 128, ws=ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(o)
+    for b in range(B):
+        r = np.arange(Lq) if rows is None else rows
+        ref = O.attention_fp8(q[b][r], k[b], v[b], H)
+        assert rel_err(got[b][r], ref) <= FP8_ATTN_TOL_MAX
+        assert rms_err(got[b][r], ref) <= FP8_ATTN_TOL_RMS
+    return got, q, k, v
+
+
+@pytest.mark.parametrize("B,Lq,Lk,H,logit_std", [
+    (1, 300, 700, 2, 1.0),        # two query-tile pairs, ragged; 6 key tiles, ragged
+    (1, 300, 700, 2, 4.0),        # peaked rows: the running base moves
+    (2, 257, 2100, 2, 1.0),       # 17 key tiles: the partial last wave is split over the keys
+    (1, 130, 1, 1, 1.0),          # one key
+    (1, 1, 300, 2, 0.36),         # one query
+])
+def test_attention_fp8_parity(wan, B, Lq, Lk, H, logit_std):
+    _attention_fp8_case(wan, B, Lq, Lk, H, logit_std, seed=Lq * 7 + Lk)
+
+
+def test_attention_fp8_full_size_sampled_rows(wan):
+    """1.3B self-attention shape (32760 tokens, 12 heads) on 256 sampled query rows."""
+    L = 32760
+    rows = sample_rows(L)
+    got, q, k, v = _attention_fp8_case(wan, 1, L, L, 12, 1.0, seed=5, rows=rows)
+    exact = O.attention(q[0][rows], k[0], v[0], 12)
+    assert rms_err(got[0][rows], exact) > FP8_ATTN_TOL_RMS / 3           # it is the 8-bit path, not bf16

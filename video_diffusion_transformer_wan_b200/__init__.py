@@ -18,6 +18,7 @@ __all__ = [
     "StackWeights", "DiffusionCache", "Fp8Scales", "make_config", "workspace_bytes", "device_status",
     "wait_timeout_check", "patchify", "patchify_noalloc", "time_mlp", "adaln_modulate", "self_attn_fwd",
     "cross_attn_fwd", "ffn_fwd", "dit_block_fwd", "dit_stack_fwd", "attention_fwd", "attention_workspace_bytes",
+    "attention_fp8_fwd", "attention_fp8_quantize", "attention_fp8_workspace_bytes",
     "linear_fwd", "head_fwd", "i2v_input", "image_context_fwd", "flow_matching_input", "flow_matching_loss",
     "sample_workspace_bytes", "sample_euler_cfg", "sp_qkv_fwd", "sp_attn_fwd", "sp_out_fwd", "fp8_quantize_rows",
     "fp8_quantize_tensor", "linear_fp8_fwd", "fp8_workspace_bytes", "dit_block_fp8_fwd", "dit_stack_fp8_fwd",
@@ -103,6 +104,11 @@ def _load() -> ctypes.CDLL:
         "wan_attention_fwd": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _i,
                                    _i, _i, _i, _vp, _sz, _vp]),
         "wan_attention_workspace_bytes": (_sz, [P(Config), _i, _i]),
+        "wan_attention_fp8_quantize": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i, _i, _i, _i,
+                                            _i, _vp, _vp, _vp, _vp, _i64, _vp, _vp]),
+        "wan_attention_fp8_fwd": (_i, [P(Config), _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _i,
+                                       _i, _i, _i, _i, _vp, _sz, _vp]),
+        "wan_attention_fp8_workspace_bytes": (_sz, [P(Config), _i, _i, _i]),
         "wan_linear_fwd": (_i, [P(Config), _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _i64, _i, _vp]),
         "wan_sample_workspace_bytes": (_sz, [P(Config), _i, _i, _i, _i, _i, _i, _i, P(DiffusionCache), _i]),
         "wan_sample_euler_cfg": (_i, [P(Config), _i, _vp, _i, _i, _i, _i, _i, ctypes.c_float, P(StackWeights),
@@ -384,6 +390,34 @@ def attention_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0
     _check(_lib().wan_attention_fwd(ctypes.byref(cfg), _p(q), qs, q_col0, _p(k), ks, k_col0, _p(v), v.shape[2], v_col0,
                                  _p(o), o.shape[2], o_col0, B, heads, Lq, Lk, head_dim, *_ws(ws), _stream(stream)),
            "wan_attention_fwd")
+
+
+def attention_fp8_workspace_bytes(cfg: Config, B: int, Lq: int, Lk: int) -> int:
+    return int(_lib().wan_attention_fp8_workspace_bytes(ctypes.byref(cfg), B, Lq, Lk))
+
+
+def attention_fp8_fwd(cfg, q, k, v, o, heads, head_dim, q_col0=0, k_col0=0, v_col0=0, o_col0=0, ws=None,
+                      stream=None):
+    """8-bit attention: the operands of attention_fwd; ws (required) of
+    attention_fp8_workspace_bytes holds the E4M3 codes and scales."""
+    B, Lq, qs = q.shape
+    Lk, ks = k.shape[1], k.shape[2]
+    _check(_lib().wan_attention_fp8_fwd(ctypes.byref(cfg), _p(q), qs, q_col0, _p(k), ks, k_col0, _p(v), v.shape[2],
+                                     v_col0, _p(o), o.shape[2], o_col0, B, heads, Lq, Lk, head_dim, *_ws(ws),
+                                     _stream(stream)), "wan_attention_fp8_fwd")
+
+
+def attention_fp8_quantize(cfg, q, k, v, heads, head_dim, q_codes, q_scale, k_codes, vt_codes, kv_scale, q_col0=0,
+                           k_col0=0, v_col0=0, stream=None):
+    """E4M3 operands of attention_fp8_fwd into caller tensors: q_codes [B, Lq, H*d] and
+    k_codes [B, Lk, H*d] uint8, vt_codes [B, H*d, S] uint8 (S % 64 == 0, S >= Lk),
+    q_scale [B, Lq, H] and kv_scale [B, H, 2] float32."""
+    B, Lq, qs = q.shape
+    Lk, ks = k.shape[1], k.shape[2]
+    _check(_lib().wan_attention_fp8_quantize(ctypes.byref(cfg), _p(q), qs, q_col0, _p(k), ks, k_col0, _p(v),
+                                          v.shape[2], v_col0, B, heads, Lq, Lk, head_dim, _p(q_codes), _p(q_scale),
+                                          _p(k_codes), _p(vt_codes), vt_codes.shape[2], _p(kv_scale),
+                                          _stream(stream)), "wan_attention_fp8_quantize")
 
 
 def linear_fwd(cfg, A, W, bias, out, epilogue, gate=None, gate_bias=None, gate_batch_stride=0, rows_per_batch=1,

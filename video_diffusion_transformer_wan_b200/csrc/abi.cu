@@ -1136,6 +1136,89 @@ int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, cons
   return gemm(cfg, A, K, W, bias, out, M, N, K, 0, ep, as_stream(stream));
 }
 
+// 8-bit attention workspace: q codes, q scales, k codes, v^T codes, k/v scales, and the
+// key-split scratch of a partial last wave.
+struct AttnF8Layout {
+  size_t qc, qs, kc, vt, kvs, split, split_bytes, total;
+  int64_t vt_stride;
+};
+AttnF8Layout attn_f8_layout(const wan_dit_config* c, int B, int Lq, int Lk) {
+  const size_t D = c->dim, H = c->heads;
+  AttnF8Layout l;
+  l.vt_stride = (static_cast<int64_t>(Lk) + 63) / 64 * 64;
+  l.qc = 0;
+  l.qs = l.qc + align_up(static_cast<size_t>(B) * Lq * D);
+  l.kc = l.qs + align_up(static_cast<size_t>(B) * Lq * H * 4);
+  l.vt = l.kc + align_up(static_cast<size_t>(B) * Lk * D);
+  l.kvs = l.vt + align_up(static_cast<size_t>(B) * D * l.vt_stride);
+  l.split = l.kvs + align_up(static_cast<size_t>(B) * H * 2 * 4);
+  l.split_bytes = split_bytes(c, B, Lq);
+  l.total = l.split + align_up(l.split_bytes);
+  return l;
+}
+
+int check_attn_fp8_args(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0, const void* k,
+                        int64_t k_row_stride, int k_col0, const void* v, int64_t v_row_stride, int v_col0, int B,
+                        int heads, int Lq, int Lk, int head_dim) {
+  WAN_TRY(check_cfg(cfg, true));
+  if (cfg->dtype != WAN_BF16) return WAN_ERR_UNSUPPORTED;
+  WAN_TRY(check_ptr(q));
+  WAN_TRY(check_ptr(k));
+  WAN_TRY(check_ptr(v));
+  WAN_REQUIRE(heads == cfg->heads && head_dim == cfg->head_dim, WAN_ERR_SHAPE);
+  WAN_REQUIRE(B >= 0 && Lq >= 0 && Lk > 0, WAN_ERR_SHAPE);
+  const int64_t need = static_cast<int64_t>(heads) * head_dim;
+  WAN_REQUIRE(q_col0 >= 0 && k_col0 >= 0 && v_col0 >= 0, WAN_ERR_SHAPE);
+  WAN_REQUIRE(q_col0 + need <= q_row_stride && k_col0 + need <= k_row_stride && v_col0 + need <= v_row_stride,
+              WAN_ERR_SHAPE);
+  return WAN_OK;
+}
+
+int wan_attention_fp8_quantize(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0,
+                               const void* k, int64_t k_row_stride, int k_col0, const void* v, int64_t v_row_stride,
+                               int v_col0, int B, int heads, int Lq, int Lk, int head_dim, void* q_codes,
+                               float* q_scale, void* k_codes, void* vt_codes, int64_t vt_stride, float* kv_scale,
+                               void* stream) {
+  WAN_TRY(check_attn_fp8_args(cfg, q, q_row_stride, q_col0, k, k_row_stride, k_col0, v, v_row_stride, v_col0, B,
+                              heads, Lq, Lk, head_dim));
+  WAN_TRY(check_ptr_any(q_codes));
+  WAN_TRY(check_ptr_any(q_scale));
+  WAN_TRY(check_ptr(k_codes));
+  WAN_TRY(check_ptr(vt_codes));
+  WAN_TRY(check_ptr_any(kv_scale));
+  WAN_REQUIRE(vt_stride >= Lk && vt_stride % 64 == 0, WAN_ERR_SHAPE);
+  return launch_attn_fp8_quantize(q, q_row_stride, q_col0, k, k_row_stride, k_col0, v, v_row_stride, v_col0, B, heads,
+                                  Lq, Lk, q_codes, q_scale, k_codes, vt_codes, vt_stride, kv_scale,
+                                  as_stream(stream));
+}
+
+int wan_attention_fp8_fwd(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0, const void* k,
+                          int64_t k_row_stride, int k_col0, const void* v, int64_t v_row_stride, int v_col0, void* o,
+                          int64_t o_row_stride, int o_col0, int B, int heads, int Lq, int Lk, int head_dim,
+                          void* workspace, size_t ws_bytes, void* stream) {
+  WAN_TRY(check_attn_fp8_args(cfg, q, q_row_stride, q_col0, k, k_row_stride, k_col0, v, v_row_stride, v_col0, B,
+                              heads, Lq, Lk, head_dim));
+  WAN_TRY(check_ptr(o));
+  WAN_REQUIRE(o_col0 >= 0 && o_col0 + static_cast<int64_t>(heads) * head_dim <= o_row_stride, WAN_ERR_SHAPE);
+  WAN_TRY(check_ptr(workspace));
+  const AttnF8Layout l = attn_f8_layout(cfg, B, Lq, Lk);
+  WAN_REQUIRE(ws_bytes >= l.total, WAN_ERR_WORKSPACE);
+  if (B == 0 || Lq == 0) return WAN_OK;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  float* qs = reinterpret_cast<float*>(w + l.qs);
+  float* kvs = reinterpret_cast<float*>(w + l.kvs);
+  cudaStream_t s = as_stream(stream);
+  WAN_TRY(launch_attn_fp8_quantize(q, q_row_stride, q_col0, k, k_row_stride, k_col0, v, v_row_stride, v_col0, B,
+                                   heads, Lq, Lk, w + l.qc, qs, w + l.kc, w + l.vt, l.vt_stride, kvs, s));
+  return launch_attn_tc_fp8(w + l.qc, qs, w + l.kc, w + l.vt, l.vt_stride, kvs, o, o_row_stride, o_col0, B, heads,
+                            Lq, Lk, s, w + l.split, l.split_bytes);
+}
+
+size_t wan_attention_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int Lq, int Lk) {
+  if (check_cfg(cfg) != WAN_OK || cfg->dtype != WAN_BF16 || B < 0 || Lq < 0 || Lk <= 0) return 0;
+  return attn_f8_layout(cfg, B, Lq, Lk).total;
+}
+
 int64_t wan_launch_count(void) { return g_launches.load(); }
 
 int wan_trace_enable(int on) {

@@ -50,10 +50,19 @@ constexpr int kAttnThreads = 320;
 constexpr int kTile = 128;                     // query rows per tile = key rows per tile
 constexpr int kHd = 128;                       // head dim
 constexpr int kQTiles = 2;                     // query tiles per CTA
-constexpr int kStages = 5;                     // K/V ring depth
-constexpr int kTileBytes = kTile * kHd * 2;    // 32 KB
-constexpr int kHalfBytes = kTileBytes / 2;     // one 64-column half
-constexpr size_t kAttnSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
+constexpr int kHalfBytes = kTile * 128;        // 128 rows of one 128-byte swizzled span
+
+// Operand shapes: bf16 tiles are two 64-column spans (32 KB), E4M3 tiles one span of
+// 128 codes (16 KB). K of one MMA is 16 (bf16) or 32 (E4M3), so a 128-deep product
+// takes 8 or 4 instructions. The 16 KB tiles leave room for a deeper K/V ring.
+template <bool kF8>
+struct AttnShape {
+  static constexpr int kTileBytes = kTile * (kF8 ? 128 : 256);
+  static constexpr int kSpans = kF8 ? 1 : 2;
+  static constexpr int kStages = kF8 ? 8 : 5;
+  static constexpr int kMmas = kF8 ? 4 : 8;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
+};
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMinSplitKeyTiles = 16;          // see launch_attn_tc
 
@@ -73,6 +82,10 @@ struct AttnParams {
   int pairs, n_full;
   float* part_o;   // [split CTA][tile][128 rows][128] fp32
   float* part_ml;  // [split CTA][tile][128 rows][2] (row max, row sum) fp32
+  // E4M3 operands only: q scale per (sample, query row, head) [B, Lq, H]; k and v scale
+  // per (sample, head) [B, H, 2]. V is stored transposed ([B, H*128 dims, keys]).
+  const float* q_scale;
+  const float* kv_scale;
   int* err;
 };
 
@@ -80,13 +93,18 @@ struct AttnParams {
 __device__ __forceinline__ int pos_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int pos_v(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 * j + 2; }
 
+template <bool kF8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const AttnParams p) {
+  constexpr int kTileBytes = AttnShape<kF8>::kTileBytes;
+  constexpr int kStages = AttnShape<kF8>::kStages;
+  constexpr int kSpans = AttnShape<kF8>::kSpans;
+  constexpr int kMmas = AttnShape<kF8>::kMmas;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                  // [2][32 KB]
-  uint8_t* sKV = sQ + kQTiles * kTileBytes;            // [kStages][32 KB]
+  uint8_t* sQ = smem;                                  // [2][tile]
+  uint8_t* sKV = sQ + kQTiles * kTileBytes;            // [kStages][tile]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * kTileBytes);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
@@ -145,10 +163,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, kQTiles * kTileBytes);
       const int qc = p.q_col0 + h * kHd;
-      for (int t = 0; t < kQTiles; ++t) {
-        tma_load_3d(sQ + t * kTileBytes, &mapQ, q_full, qc, q0 + t * kTile, b);
-        tma_load_3d(sQ + t * kTileBytes + kHalfBytes, &mapQ, q_full, qc + 64, q0 + t * kTile, b);
-      }
+      for (int t = 0; t < kQTiles; ++t)
+        for (int c = 0; c < kSpans; ++c)
+          tma_load_3d(sQ + t * kTileBytes + c * kHalfBytes, &mapQ, q_full, qc + 64 * c, q0 + t * kTile, b);
       const int n_loads = 2 * nkv;
       int issued = 0;
       for (int ld = 0; ld < n_loads; ++ld) {
@@ -170,8 +187,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int col = (is_v ? p.v_col0 : p.k_col0) + h * kHd;
         uint8_t* dst = sKV + stage * kTileBytes;
         mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
-        tma_load_3d(dst, map, &kv_full[stage], col, (kv0 + j) * kTile, b);
-        tma_load_3d(dst + kHalfBytes, map, &kv_full[stage], col + 64, (kv0 + j) * kTile, b);
+        if (kF8 && is_v) {  // V^T: 128 dims (rows) x 128 keys (x)
+          tma_load_3d(dst, map, &kv_full[stage], (kv0 + j) * kTile, p.v_col0 + h * kHd, b);
+        } else {
+          for (int c = 0; c < kSpans; ++c)
+            tma_load_3d(dst + c * kHalfBytes, map, &kv_full[stage], col + 64 * c, (kv0 + j) * kTile, b);
+        }
         ++issued;
       }
       mbar_wait(q_full, 0, p.err);
@@ -182,35 +203,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(kTile, kHd, 0, 1);
+      const uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(kTile, kTile) : idesc_bf16_f32(kTile, kTile, 0, 0);
+      // PV: bf16 V is an MN-major operand; E4M3 V arrives transposed, so K-major.
+      const uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(kTile, kHd) : idesc_bf16_f32(kTile, kHd, 0, 1);
       // Shared-memory descriptors are built once: every operand below sits at a fixed
       // byte offset from sQ or sKV, and an offset moves only the 14-bit address field
       // (offset >> 4, no carry out of it since shared addresses stay below 256 KB). The
       // single issuing thread then spends one add per operand on each MMA.
       const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t k_desc = sdesc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t v_desc = sdesc_sw128(smem_u32(sKV), kHalfBytes, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(sKV), kF8 ? 16 : kHalfBytes, 1024);
       auto wait_pos = [&](int pos) {
         return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
       };
       auto pv = [&](int t, int i, int vstage) {
-        // A = P_t in TMEM: bf16 pairs packed in the first 64 columns of S_t's region.
+        // A = P_t in TMEM, packed from the first column of S_t's region (bf16 pairs or
+        // E4M3 quads per column, so 8 columns per MMA either way).
         const uint32_t p_tmem = tmem_base + t * kTile;
         const uint64_t vd = v_desc + static_cast<uint32_t>((vstage * kTileBytes) >> 4);
         const uint32_t o_tmem = tmem_base + 256 + t * kTile;
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < kMmas; ++k) {
+          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+          if constexpr (kF8)
+            tc_mma_e4m3_ts(o_tmem, p_tmem + k * 8, vd + ((k * 32) >> 4), idesc_pv, acc);
+          else
+            tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, acc);
+        }
       };
       auto qk = [&](int t, int kstage) {
         const uint64_t qd = q_desc + static_cast<uint32_t>((t * kTileBytes) >> 4);
         const uint64_t kd = k_desc + static_cast<uint32_t>((kstage * kTileBytes) >> 4);
         const uint32_t s_tmem = tmem_base + t * kTile;
 #pragma unroll
-        for (int k = 0; k < kHd / 16; ++k) {
-          const uint32_t off = ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4;
-          tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
+        for (int k = 0; k < kMmas; ++k) {
+          const uint32_t off = ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4;  // 32 bytes of K per MMA
+          if constexpr (kF8)
+            tc_mma_e4m3(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
+          else
+            tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(q_full, 0, p.err);
@@ -261,7 +292,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_row = tmem_base + lane_off + t * kTile;
     const uint32_t o_row = tmem_base + lane_off + 256 + t * kTile;
-    const float sl2 = p.scale_log2;
+    float sl2 = p.scale_log2;
+    float v_scale = 1.0f;
+    if constexpr (kF8) {
+      // Logit = S q_scale k_scale / sqrt(d): the row's scales fold into its log2 scale;
+      // the v scale multiplies the output.
+      const float* kvs = p.kv_scale + 2 * (static_cast<int64_t>(b) * p.H + h);
+      const int grow0 = q0 + t * kTile + row;
+      sl2 *= kvs[0] * (grow0 < p.Lq ? p.q_scale[(static_cast<int64_t>(b) * p.Lq + grow0) * p.H + h] : 1.0f);
+      v_scale = kvs[1];
+    }
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -301,24 +341,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         m_run = mx;
       } else if (__any_sync(0xffffffffu, grow)) {
         const float m_new = fmaxf(m_run, mx);
-        alpha = ex2_approx((m_run - m_new) * sl2);
+        // E4M3 P: bases are whole powers of two (see below), so alpha is one as well.
+        alpha = kF8 ? pow2i(static_cast<int>(ceilf(m_run * sl2) - ceilf(m_new * sl2)))
+                    : ex2_approx((m_run - m_new) * sl2);
         m_run = m_new;
         rescale = true;
       }
-      const float nb = -m_run * sl2;
+      // E4M3 P is taken against the base rounded up to a whole power of two: p <= 2^8
+      // still, and its codes are those of the exact-max base times an exact power of two
+      // (outside the subnormal range), whatever this row's running max is.
+      const float nb = kF8 ? -ceilf(m_run * sl2) : -m_run * sl2;
       const unsigned long long sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
       unsigned long long rs4[4] = {0ull, 0ull, 0ull, 0ull};
+      if constexpr (kF8) {
+        // E4M3 P: four codes per register (quad i of the row lands in register i <= 4i).
 #pragma unroll
-      for (int i = 0; i < kTile / 2; ++i) {
-        const unsigned long long s2 = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        const float2 x = f2_unpack(f2_fma(s2, sl2x2, nbx2));
-        const float e0 = ex2_approx(x.x);
-        const float e1 = ex2_approx(x.y);
-        rs4[i & 3] = f2_add(rs4[i & 3], f2_pack(e0, e1));
-        r[i] = pack_bf16x2(e0, e1);
+        for (int i = 0; i < kTile / 4; ++i) {
+          const unsigned long long s01 = f2_pack(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+          const unsigned long long s23 = f2_pack(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          const float2 x01 = f2_unpack(f2_fma(s01, sl2x2, nbx2));
+          const float2 x23 = f2_unpack(f2_fma(s23, sl2x2, nbx2));
+          const float e0 = ex2_approx(x01.x), e1 = ex2_approx(x01.y);
+          const float e2 = ex2_approx(x23.x), e3 = ex2_approx(x23.y);
+          rs4[(2 * i) & 3] = f2_add(rs4[(2 * i) & 3], f2_pack(e0, e1));
+          rs4[(2 * i + 1) & 3] = f2_add(rs4[(2 * i + 1) & 3], f2_pack(e2, e3));
+          r[i] = pack_e4m3x4(e0, e1, e2, e3);
+        }
+        tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTile / 2; ++i) {
+          const unsigned long long s2 = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          const float2 x = f2_unpack(f2_fma(s2, sl2x2, nbx2));
+          const float e0 = ex2_approx(x.x);
+          const float e1 = ex2_approx(x.y);
+          rs4[i & 3] = f2_add(rs4[i & 3], f2_pack(e0, e1));
+          r[i] = pack_bf16x2(e0, e1);
+        }
+        tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_st32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
       }
-      tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
-      tmem_st32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
       if (rescale) {
         // S_t(j) ready implies PV_t(j-1) completed, and PV_t(j) waits for this thread's
         // arrival below: O_t is current and idle while it is rescaled here.
@@ -357,10 +419,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           po[c * 8 + g] = make_float4(__uint_as_float(r0[4 * g]), __uint_as_float(r0[4 * g + 1]),
                                       __uint_as_float(r0[4 * g + 2]), __uint_as_float(r0[4 * g + 3]));
       }
-      reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_run, l_run);
+      // E4M3: the whole-power-of-two base itself (the merge then uses scale 1).
+      const float m_common = kF8 ? ceilf(m_run * sl2) : m_run;
+      reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_common, l_run);
     } else if (done) {
       tc_fence_after();
-      const float inv = 1.0f / l_run;
+      const float inv = v_scale / l_run;
       const int grow = q0 + t * kTile + row;
       __nv_bfloat16* orow;
       if (p.sc.ranks > 0) {
@@ -423,8 +487,10 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
     const float2 ml0 = reinterpret_cast<const float2*>(p.part_ml)[s0];
     const float2 ml1 = reinterpret_cast<const float2*>(p.part_ml)[s1];
     const float m = fmaxf(ml0.x, ml1.x);
-    const float w0 = exp2f((ml0.x - m) * p.scale_log2), w1 = exp2f((ml1.x - m) * p.scale_log2);
-    const float inv = 1.0f / (w0 * ml0.y + w1 * ml1.y);
+    const float ms = p.kv_scale ? 1.0f : p.scale_log2;  // E4M3 partials carry log2 bases
+    const float w0 = exp2f((ml0.x - m) * ms), w1 = exp2f((ml1.x - m) * ms);
+    const float v_scale = p.kv_scale ? p.kv_scale[2 * (static_cast<int64_t>(b) * p.H + h) + 1] : 1.0f;
+    const float inv = v_scale / (w0 * ml0.y + w1 * ml1.y);
     const float4 a = reinterpret_cast<const float4*>(p.part_o + s0 * kHd)[lane];
     const float4 c = reinterpret_cast<const float4*>(p.part_o + s1 * kHd)[lane];
     uint2 v;
@@ -444,6 +510,57 @@ bool make_operand_map(CUtensorMap* map, const AttnOperand& op, int B, int L) {
   const uint32_t box[3] = {64, kTile, 1};
   return make_tmap_bf16(map, op.ptr, 3, dims, strides, box);
 }
+
+// Grid, optional key split of a partial last wave, launch and merge (both operand kinds).
+template <bool kF8>
+int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, AttnParams& p, int B, int H,
+                 int Lq, int Lk, cudaStream_t s, bool has_sc, void* scratch, size_t scratch_bytes) {
+  p.err = device_error_flag();
+  constexpr size_t kSmem = AttnShape<kF8>::kSmem;
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev & 63], [] {
+    cudaFuncSetAttribute(attn_fwd_tc_kernel<kF8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kSmem));
+  });
+  // One CTA per unit. When the last wave would leave more than half of the SMs idle,
+  // its units are split over the key tiles instead (two CTAs each) and merged after.
+  p.pairs = (Lq + kQTiles * kTile - 1) / (kQTiles * kTile);
+  const int64_t units = static_cast<int64_t>(B) * H * p.pairs;
+  if (units >= (int64_t(1) << 31)) return WAN_ERR_SHAPE;
+  static int nsm_of[64] = {0};
+  if (nsm_of[dev & 63] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    nsm_of[dev & 63] = v > 0 ? v : 148;
+  }
+  const int nsm = nsm_of[dev & 63];
+  const int64_t rem = units % nsm;
+  const int nkv_all = (Lk + kTile - 1) / kTile;
+  const size_t part_o_bytes = static_cast<size_t>(2 * rem) * kQTiles * kTile * kHd * 4;
+  const size_t part_bytes = part_o_bytes + static_cast<size_t>(2 * rem) * kQTiles * kTile * 8;
+  // Only when a unit is long enough (16+ key tiles) for half of it to outweigh the
+  // partial-output traffic and the merge launch (at 4 key tiles, as in the text
+  // cross-attention, splitting measured 9 % slower).
+  const bool split = rem > 0 && 2 * rem <= nsm && nkv_all >= kMinSplitKeyTiles && !has_sc && scratch &&
+                     scratch_bytes >= part_bytes && (reinterpret_cast<uintptr_t>(scratch) & 15u) == 0;
+  p.n_full = static_cast<int>(split ? units - rem : units);
+  p.part_o = split ? static_cast<float*>(scratch) : nullptr;
+  p.part_ml = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + part_o_bytes) : nullptr;
+  const unsigned grid = static_cast<unsigned>(split ? units + rem : units);
+  trace_launch_begin(WAN_KIND_ATTN, s, 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd);
+  attn_fwd_tc_kernel<kF8><<<grid, kAttnThreads, kSmem, s>>>(mq, mk, mv, p);
+  int st = check_launch();
+  if (st == WAN_OK && split) {
+    attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);
+    count_launches(1);
+    st = check_launch();
+  }
+  trace_launch_end(WAN_KIND_ATTN, s);
+  return st;
+}
+
 
 }  // namespace
 
@@ -472,49 +589,46 @@ int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t
   if (sc && (sc->ranks < 1 || sc->ranks > kMaxSeqRanks || sc->rows_local < 1 ||
              static_cast<int64_t>(sc->rows_local) * sc->ranks < Lq))
     return WAN_ERR_SHAPE;
-  p.err = device_error_flag();
-  static std::once_flag once[64];
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::call_once(once[dev & 63], [] {
-    cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kAttnSmem));
-  });
-  // One CTA per unit. When the last wave would leave more than half of the SMs idle,
-  // its units are split over the key tiles instead (two CTAs each) and merged after.
-  p.pairs = (Lq + kQTiles * kTile - 1) / (kQTiles * kTile);
-  const int64_t units = static_cast<int64_t>(B) * H * p.pairs;
-  if (units >= (int64_t(1) << 31)) return WAN_ERR_SHAPE;
-  static int nsm_of[64] = {0};
-  if (nsm_of[dev & 63] == 0) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    nsm_of[dev & 63] = v > 0 ? v : 148;
-  }
-  const int nsm = nsm_of[dev & 63];
-  const int64_t rem = units % nsm;
-  const int nkv_all = (Lk + kTile - 1) / kTile;
-  const size_t part_o_bytes = static_cast<size_t>(2 * rem) * kQTiles * kTile * kHd * 4;
-  const size_t part_bytes = part_o_bytes + static_cast<size_t>(2 * rem) * kQTiles * kTile * 8;
-  // Only when a unit is long enough (16+ key tiles) for half of it to outweigh the
-  // partial-output traffic and the merge launch (at 4 key tiles, as in the text
-  // cross-attention, splitting measured 9 % slower).
-  const bool split = rem > 0 && 2 * rem <= nsm && nkv_all >= kMinSplitKeyTiles && !sc && scratch &&
-                     scratch_bytes >= part_bytes && (reinterpret_cast<uintptr_t>(scratch) & 15u) == 0;
-  p.n_full = static_cast<int>(split ? units - rem : units);
-  p.part_o = split ? static_cast<float*>(scratch) : nullptr;
-  p.part_ml = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + part_o_bytes) : nullptr;
-  const unsigned grid = static_cast<unsigned>(split ? units + rem : units);
-  trace_launch_begin(WAN_KIND_ATTN, s, 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd);
-  attn_fwd_tc_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(mq, mk, mv, p);
-  int st = check_launch();
-  if (st == WAN_OK && split) {
-    attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);
-    count_launches(1);
-    st = check_launch();
-  }
-  trace_launch_end(WAN_KIND_ATTN, s);
-  return st;
+  p.q_scale = nullptr;
+  p.kv_scale = nullptr;
+  return launch_units<false>(mq, mk, mv, p, B, H, Lq, Lk, s, sc != nullptr, scratch, scratch_bytes);
+}
+
+int launch_attn_tc_fp8(const void* q_codes, const float* q_scale, const void* k_codes, const void* vt_codes,
+                       int64_t vt_row_stride, const float* kv_scale, void* o, int64_t o_row_stride, int o_col0, int B,
+                       int H, int Lq, int Lk, cudaStream_t s, void* scratch, size_t scratch_bytes) {
+  if (B == 0 || Lq == 0) return WAN_OK;
+  if (Lk <= 0) return WAN_ERR_SHAPE;
+  if (vt_row_stride % 16 || vt_row_stride < Lk || o_row_stride % 8 || o_col0 % 8) return WAN_ERR_ALIGN;
+  const uint64_t D = static_cast<uint64_t>(H) * kHd;
+  // Codes: q [B, Lq, D] and k [B, Lk, D] row-major; v^T [B, D, vt_row_stride] (keys along x).
+  CUtensorMap mq, mk, mv;
+  const uint64_t dq[3] = {D, static_cast<uint64_t>(Lq), static_cast<uint64_t>(B)};
+  const uint64_t sq[2] = {D, D * static_cast<uint64_t>(Lq)};
+  const uint64_t dk[3] = {D, static_cast<uint64_t>(Lk), static_cast<uint64_t>(B)};
+  const uint64_t sk[2] = {D, D * static_cast<uint64_t>(Lk)};
+  const uint64_t dv[3] = {static_cast<uint64_t>(Lk), D, static_cast<uint64_t>(B)};
+  const uint64_t sv[2] = {static_cast<uint64_t>(vt_row_stride), static_cast<uint64_t>(vt_row_stride) * D};
+  const uint32_t box[3] = {128, kTile, 1};
+  if (!make_tmap_u8(&mq, q_codes, 3, dq, sq, box) || !make_tmap_u8(&mk, k_codes, 3, dk, sk, box) ||
+      !make_tmap_u8(&mv, vt_codes, 3, dv, sv, box))
+    return WAN_ERR_CUDA;
+  AttnParams p;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.H = H;
+  p.q_col0 = 0;
+  p.k_col0 = 0;
+  p.v_col0 = 0;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(kHd)));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_row_stride = o_row_stride;
+  p.o_batch_stride = o_row_stride * Lq;
+  p.o_col0 = o_col0;
+  p.sc = SeqScatter{};
+  p.q_scale = q_scale;
+  p.kv_scale = kv_scale;
+  return launch_units<true>(mq, mk, mv, p, B, H, Lq, Lk, s, false, scratch, scratch_bytes);
 }
 
 }  // namespace wan

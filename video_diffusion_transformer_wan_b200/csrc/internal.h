@@ -107,6 +107,18 @@ struct SeqScatter {
 int launch_attn_tc(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
                    int B, int H, int Lq, int Lk, cudaStream_t s, const SeqScatter* sc = nullptr,
                    void* scratch = nullptr, size_t scratch_bytes = 0);
+// 8-bit attention operands from bf16 q, k, v (head_dim 128): q codes [B, Lq, H*128] with
+// a scale per (sample, row, head) [B, Lq, H]; k codes [B, Lk, H*128]; v^T codes
+// [B, H*128, vt_stride] (vt_stride a multiple of 64, >= Lk; keys past Lk are code 0);
+// kv_scale [B, H, 2] = (k scale, v scale). Five kernels.
+int launch_attn_fp8_quantize(const void* q, int64_t q_row_stride, int q_col0, const void* k, int64_t k_row_stride,
+                             int k_col0, const void* v, int64_t v_row_stride, int v_col0, int B, int H, int Lq, int Lk,
+                             void* q_codes, float* q_scale, void* k_codes, void* vt_codes, int64_t vt_stride,
+                             float* kv_scale, cudaStream_t s);
+// Tensor-core attention over those operands (E4M3 products, E4M3 P); bf16 output.
+int launch_attn_tc_fp8(const void* q_codes, const float* q_scale, const void* k_codes, const void* vt_codes,
+                       int64_t vt_row_stride, const float* kv_scale, void* o, int64_t o_row_stride, int o_col0, int B,
+                       int H, int Lq, int Lk, cudaStream_t s, void* scratch = nullptr, size_t scratch_bytes = 0);
 // fp32 SIMT attention, head_dim <= 128, Lk <= 8192.
 int launch_attn_simt(AttnOperand q, AttnOperand k, AttnOperand v, void* o, int64_t o_row_stride, int o_col0,
                      int B, int H, int Lq, int Lk, int d, cudaStream_t s);

@@ -163,6 +163,18 @@ __device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
+// Same with A read from tensor memory (four E4M3 codes per 32-bit column, row m in
+// lane m): D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f8f6f4, K = 32 per instruction.
+__device__ __forceinline__ void tc_mma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 D.
 // Bits: [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
 // 15 A major (0 = K-major, 1 = MN-major), 16 B major, [17,23) N >> 3, [24,29) M >> 4.
@@ -239,6 +251,8 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^n for an integer n, exactly (0 below the normal range).
+__device__ __forceinline__ float pow2i(int n) { return n < -126 ? 0.0f : __int_as_float((min(n, 127) + 127) << 23); }
 // Largest of three floats in one instruction (the three-input form of max, sm_100+).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float y;

@@ -100,7 +100,7 @@ def _block(a) -> dict:
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block"])
-    ap.add_argument("--fp8", action="store_true", help="gemm / block / sample: E4M3 operands (kind::f8f6f4)")
+    ap.add_argument("--fp8", action="store_true", help="attention / gemm / block / sample: E4M3 operands (kind::f8f6f4)")
     ap.add_argument("--no-split", action="store_true",
                     help="attention: no workspace, so a partial last wave is not split over the keys")
     ap.add_argument("--workload", default="wan13b_480p_block", help="block: workload name")
@@ -134,11 +134,17 @@ def main(argv=None):
             k = v = torch.randn(1, Lk, 2 * D, device="cuda", generator=g).to(torch.bfloat16)
             cols = (0, 0, D)
         o = torch.empty(1, a.L, D, dtype=torch.bfloat16, device="cuda")
-        ws = None if a.no_split else torch.empty(max(16, wan.attention_workspace_bytes(cfg, 1, a.L)),
-                                                 dtype=torch.uint8, device="cuda")
-        ms = _time(lambda: wan.attention_fwd(cfg, q, k, v, o, a.heads, 128, *cols, 0, ws=ws), a.iters, a.warmup)
+        if a.fp8:
+            # quantisation of q, k, v (five small kernels) included, as a caller sees it
+            ws = torch.empty(wan.attention_fp8_workspace_bytes(cfg, 1, a.L, Lk), dtype=torch.uint8, device="cuda")
+            ms = _time(lambda: wan.attention_fp8_fwd(cfg, q, k, v, o, a.heads, 128, *cols, 0, ws=ws), a.iters,
+                       a.warmup)
+        else:
+            ws = None if a.no_split else torch.empty(max(16, wan.attention_workspace_bytes(cfg, 1, a.L)),
+                                                     dtype=torch.uint8, device="cuda")
+            ms = _time(lambda: wan.attention_fwd(cfg, q, k, v, o, a.heads, 128, *cols, 0, ws=ws), a.iters, a.warmup)
         flops = 4.0 * a.L * Lk * D
-        out.update(L=a.L, Lk=Lk, heads=a.heads, split=not a.no_split, ms=ms, tflops=flops / ms / 1e9)
+        out.update(L=a.L, Lk=Lk, heads=a.heads, split=not a.no_split, fp8=a.fp8, ms=ms, tflops=flops / ms / 1e9)
     elif a.kernel == "gemm":
         cfg = wan.make_config(128, 1, 128)
         A = torch.randn(a.M, a.K, device="cuda", generator=g).to(torch.bfloat16)
