@@ -271,9 +271,13 @@ int wan_flow_matching_loss(const wan_dit_config* cfg, const float* v, const void
  * tensor), computed in IEEE float32. Requires a bf16 config; E4M3 arrays are bytes. */
 
 /* Per-tensor scales (device fp32 scalars) of a block's E4M3 weights. ckv_img may be
- * NULL for T2V. */
+ * NULL for T2V. attention_fp8 nonzero: the block's self-attention also runs on E4M3
+ * operands (the 8-bit attention of wan_attention_fp8_fwd, below); the text and image
+ * cross-attention stay bf16 (with 512 or 257 keys, quantising their queries costs more
+ * than the 8-bit products save). */
 typedef struct {
   const float *qkv, *o, *cq, *ckv, *co, *ckv_img, *ffn1, *ffn2;
+  int attention_fp8;
 } wan_fp8_scales;
 
 /* Codes of x [M, K] act, one scale per row: q [M, K] E4M3, scale [M] fp32 (device).

@@ -184,11 +184,15 @@ def attention(q, k, v, heads: int) -> np.ndarray:
 # Block branches
 # --------------------------------------------------------------------------------------
 
-def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None, fp8: bool = False) -> np.ndarray:
+def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None, fp8: bool = False,
+                        fp8_attention: bool = False) -> np.ndarray:
     """The attention output ``attn(h Wq, h Wk, h Wv)`` before the output projection.
     The fused QKV weight ``w_qkv [3D, D]`` is stacked (q, k, v). ``kv_source`` (all rows
     of h) lets the caller evaluate only some query rows; by default it is ``h``. With
-    ``fp8`` the projection is ``linear_fp8`` of the fused weight (one weight scale)."""
+    ``fp8`` the projection is ``linear_fp8`` of the fused weight (one weight scale); with
+    ``fp8_attention`` the attention is ``attention_fp8`` (its q scales are per row, its
+    k and v scales over all key rows, so a subset of query rows stays exact)."""
+    attn = attention_fp8 if fp8_attention else attention
     h = _f(h)
     D = h.shape[-1]
     src = h if kv_source is None else _f(kv_source)
@@ -196,11 +200,11 @@ def self_attention_core(h, w: Dict[str, np.ndarray], heads: int, kv_source=None,
     if fp8:
         q = linear_fp8(h, wqkv, bqkv)[:, :D]
         kv = linear_fp8(src, wqkv, bqkv)
-        return attention(q, kv[:, D:2 * D], kv[:, 2 * D:], heads)
+        return attn(q, kv[:, D:2 * D], kv[:, 2 * D:], heads)
     q = linear(h, wqkv[:D], bqkv[:D])
     k = linear(src, wqkv[D:2 * D], bqkv[D:2 * D])
     v = linear(src, wqkv[2 * D:], bqkv[2 * D:])
-    return attention(q, k, v, heads)
+    return attn(q, k, v, heads)
 
 
 def self_attention_branch(h, w: Dict[str, np.ndarray], heads: int,
@@ -241,7 +245,8 @@ def ffn_branch(h, w: Dict[str, np.ndarray], fp8: bool = False) -> np.ndarray:
 
 def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6,
               img_ctx=None, rows: Optional[Sequence[int]] = None,
-              return_parts: bool = False, attn_cache: Optional[Dict] = None, fp8: bool = False):
+              return_parts: bool = False, attn_cache: Optional[Dict] = None, fp8: bool = False,
+              fp8_attention: bool = False):
     """One DiT block [Wan-P2, "Diffusion Transformer"]:
 
     1. ``x += gate_msa * SelfAttn(LN(x) (1 + scale_msa) + shift_msa)``
@@ -266,7 +271,8 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
 
     ``fp8`` runs every linear layer of the block as ``linear_fp8`` (per-token input
     codes, per-tensor weight codes; the sum of the text and image attention outputs is
-    quantised as one input).
+    quantised as one input); ``fp8_attention`` also runs the self-attention as
+    ``attention_fp8`` (the cross-attention keeps exact attention).
     """
     x = _f(x)
     mod = block_modulation(e, w["mod_bias"])
@@ -281,7 +287,7 @@ def dit_block(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6
     if attn_cache is not None and attn_cache.get("reuse"):
         sa = self_attention_branch(hr, w, heads, o=attn_cache["o"], fp8=fp8)
     else:
-        o = self_attention_core(hr, w, heads, kv_source=h_all, fp8=fp8)
+        o = self_attention_core(hr, w, heads, kv_source=h_all, fp8=fp8, fp8_attention=fp8_attention)
         if attn_cache is not None:
             attn_cache["o"] = o
         sa = self_attention_branch(hr, w, heads, o=o, fp8=fp8)
@@ -353,20 +359,23 @@ def flow_matching_target(x1, x0) -> np.ndarray:
 
 def dit_stack(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, heads: int,
               eps: float = 1e-6, img_ctx=None, freq_dim: int = 256,
-              attn_caches: Optional[Sequence[Dict]] = None, fp8: bool = False) -> np.ndarray:
+              attn_caches: Optional[Sequence[Dict]] = None, fp8: bool = False,
+              fp8_attention: bool = False) -> np.ndarray:
     """Whole DiT on one sample [Wan-P2, "Diffusion Transformer"]: patchify -> the time
     MLP shared by all blocks -> N blocks (each with its own modulation bias) -> head ->
     unpatchify. ``weights`` holds ``w_p, b_p, w_t1, b_t1, w_t2, b_t2, w_head, b_head``.
     ``attn_caches`` gives each block its attention cache (see ``dit_block``); ``fp8``
-    runs the blocks' linear layers in FP8 (``dit_block``; patchify, the time MLP and
-    the head stay as they are). Returns the predicted velocity ``[out_ch, F, H, W]``."""
+    runs the blocks' linear layers in FP8 and ``fp8_attention`` their self-attention
+    (``dit_block``; patchify, the time MLP and the head stay as they are). Returns the
+    predicted velocity ``[out_ch, F, H, W]``."""
     lat = _f(latent)
     C, F, H, W = lat.shape
     x = patchify(lat, weights["w_p"], weights["b_p"])
     e = time_mlp(t, weights["w_t1"], weights["b_t1"], weights["w_t2"], weights["b_t2"], freq_dim)
     for i, blk in enumerate(blocks):
         x = dit_block(x, e, blk, ctx, heads, eps, img_ctx=img_ctx,
-                      attn_cache=None if attn_caches is None else attn_caches[i], fp8=fp8)
+                      attn_cache=None if attn_caches is None else attn_caches[i], fp8=fp8,
+                      fp8_attention=fp8_attention)
     y = head(x, weights["w_head"], weights["b_head"], eps)
     return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)
 
@@ -396,7 +405,7 @@ def euler_cfg(x0, n_steps: int, guidance: float, velocity_cond, velocity_uncond)
 
 def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks: Sequence[Dict], ctx_cond,
                      ctx_uncond, heads: int, eps: float = 1e-6, img_ctx=None, cond_channels=None,
-                     freq_dim: int = 256, fp8: bool = False) -> np.ndarray:
+                     freq_dim: int = 256, fp8: bool = False, fp8_attention: bool = False) -> np.ndarray:
     """Generate a latent with the DiT as the velocity model: ``euler_cfg`` with
     ``v(x, t) = dit_stack(input(x), 1000 t, ...)`` under the text context (conditional)
     and the unconditional context. ``noise [16, F, H, W]`` is x at t = 0. For I2V,
@@ -408,7 +417,7 @@ def sample_euler_cfg(noise, n_steps: int, guidance: float, weights: Dict, blocks
 
     def vel(ctx):
         return lambda x, t: dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps,
-                                      img_ctx=img_ctx, freq_dim=freq_dim, fp8=fp8)
+                                      img_ctx=img_ctx, freq_dim=freq_dim, fp8=fp8, fp8_attention=fp8_attention)
     return euler_cfg(noise, n_steps, guidance, vel(ctx_cond), vel(ctx_uncond))
 
 

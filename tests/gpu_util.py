@@ -30,6 +30,11 @@ FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
 # 1 and 4, 700 to 32760 keys, whole and key-split; bars 1.5x: 8e-2 and 3e-2. (8-bit
 # attention itself is 4-10 % (max) and 4-11 % (RMS) away from exact attention there.)
 FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS = 8e-2, 3e-2
+# The FP8 block with 8-bit self-attention: the derivation of FP8_TOL_* with q, k and v
+# also moved by +-2^-9 and the running base emulated in the 8-bit attention moves the
+# block by at most 2.8 % (max) and 2.1 % (RMS) (960-token T2V and I2V blocks, 6 trials
+# each; the 1.3B block on 256 sampled rows, 2 trials); bars 1.5x, rounded: 5e-2, 3.2e-2.
+FP8A_BLOCK_TOL_MAX, FP8A_BLOCK_TOL_RMS = 5e-2, 3.2e-2
 
 
 def rel_err(got, ref) -> float:

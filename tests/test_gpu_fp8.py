@@ -8,7 +8,7 @@ import pytest
 
 from oracle import wan_oracle as O
 from wan_inputs import WORKLOADS, make_inputs, round_bf16, sample_rows
-from gpu_util import (FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS, FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS, FP8_STACK_TOL_MAX,
+from gpu_util import (FP8A_BLOCK_TOL_MAX, FP8A_BLOCK_TOL_RMS, FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS, FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS, FP8_STACK_TOL_MAX,
                       FP8_STACK_TOL_RMS, FP8_TOL_MAX, FP8_TOL_RMS, dev, host, rel_err, rms_err, rng)
 from test_gpu_block import Run, small_bf16
 
@@ -288,3 +288,62 @@ def test_attention_fp8_full_size_sampled_rows(wan):
     got, q, k, v = _attention_fp8_case(wan, 1, L, L, 12, 1.0, seed=5, rows=rows)
     exact = O.attention(q[0][rows], k[0], v[0], 12)
     assert rms_err(got[0][rows], exact) > FP8_ATTN_TOL_RMS / 3           # it is the 8-bit path, not bf16
+
+
+@pytest.mark.parametrize("i2v", [False, True])
+def test_block_fp8_attention_matches_oracle(wan, i2v):
+    """FP8 block with 8-bit self-attention (960 tokens: 8 key tiles, so the running base
+    moves) against the oracle's; the 8-bit attention path is the one that ran (its five
+    quantiser launches)."""
+    from video_diffusion_transformer_wan_b200.model import Fp8Block
+    w = small_bf16(i2v=i2v, frames=5, height=24, width=32, dim=512, heads=4, ffn=1024)
+    r = Run(wan, w, zero_wx=False)
+    ws = torch.empty(wan.fp8_workspace_bytes(r.cfg, w.batch, w.tokens, w.text_len, w.img_len if i2v else 0),
+                     dtype=torch.uint8, device="cuda")
+    launches = {}
+    outs = {}
+    for fa in (False, True):
+        fb = Fp8Block(r.cfg, r.model.blocks[0], attention_fp8=fa)
+        x = r.x.clone()
+        torch.cuda.synchronize()
+        n0 = wan.launch_count()
+        wan.dit_block_fp8_fwd(r.cfg, x, r.e, r.ctx, r.img_ctx, fb.table, fb.scale_table, ws)
+        launches[fa] = wan.launch_count() - n0
+        torch.cuda.synchronize()
+        assert wan.device_status() == 0
+        outs[fa] = host(x)
+    assert launches[True] - launches[False] == 5
+    for b in range(w.batch):
+        img = None if r.img_np is None else r.img_np[b]
+        ref = O.dit_block(r.inp["x"][b], r.inp["e"][b], r.inp["blocks"][0], r.inp["ctx"][b], w.heads, img_ctx=img,
+                          fp8=True, fp8_attention=True)
+        d_got, d_ref = outs[True][b] - r.inp["x"][b], ref - r.inp["x"][b]
+        print(f"fp8 block + 8-bit attention i2v={i2v}: max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
+        assert rel_err(d_got, d_ref) <= FP8A_BLOCK_TOL_MAX
+        assert rms_err(d_got, d_ref) <= FP8A_BLOCK_TOL_RMS
+
+
+def test_block_fp8_attention_full_size_sampled_rows(wan):
+    """The 1.3B 480P block with FP8 linears and 8-bit self-attention, 256 sampled rows."""
+    from video_diffusion_transformer_wan_b200.model import DitModel, Fp8Block, config_for, to_device
+    w = WORKLOADS["wan13b_480p_block"]
+    inp = make_inputs(w, seed=0)
+    cfg = config_for(w)
+    model = DitModel(cfg, inp)
+    fb = Fp8Block(cfg, model.blocks[0], attention_fp8=True)
+    x = to_device(inp["x"], torch.float32)
+    e = to_device(inp["e"], torch.float32)
+    ctx = to_device(inp["ctx"], torch.bfloat16)
+    ws = torch.empty(wan.fp8_workspace_bytes(cfg, 1, w.tokens, w.text_len), dtype=torch.uint8, device="cuda")
+    wan.dit_block_fp8_fwd(cfg, x, e, ctx, None, fb.table, fb.scale_table, ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    rows = sample_rows(w.tokens)
+    got = x[0].cpu().numpy().astype(np.float64)[rows]
+    ref = O.dit_block(inp["x"][0], inp["e"][0], inp["blocks"][0], inp["ctx"][0], w.heads, rows=rows, fp8=True,
+                      fp8_attention=True)
+    d_got, d_ref = got - inp["x"][0][rows], ref - inp["x"][0][rows]
+    print(f"fp8 block + 8-bit attention 1.3B sampled rows: max {rel_err(d_got, d_ref):.2e} "
+          f"rms {rms_err(d_got, d_ref):.2e}")
+    assert rel_err(d_got, d_ref) <= FP8A_BLOCK_TOL_MAX
+    assert rms_err(d_got, d_ref) <= FP8A_BLOCK_TOL_RMS

@@ -305,10 +305,11 @@ def torch_fp8_linear(t, W, b):
     return (qx @ qw.T) * sx * sw + b
 
 
-def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None, fp8=False):
+def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None, fp8=False, fp8_attention=False):
     """The block re-expressed with torch library routines (layer_norm, linear,
     scaled_dot_product_attention, gelu) in float64; with ``fp8`` every linear layer
-    uses torch's E4M3 conversion (``torch_fp8_linear``)."""
+    uses torch's E4M3 conversion (``torch_fp8_linear``), with ``fp8_attention`` the
+    self-attention is ``torch_attention_fp8``."""
     X, E, C = t64(x), t64(e) + t64(w["mod_bias"]), t64(ctx)
     lin = torch_fp8_linear if fp8 else tF.linear
     D = X.shape[-1]
@@ -325,7 +326,9 @@ def torch_block(x, e, w, ctx, heads, eps=1e-6, img_ctx=None, fp8=False):
     ln = lambda t: tF.layer_norm(t, (D,), eps=eps)  # noqa: E731
     h = ln(X) * (1 + E[1]) + E[0]
     qkv = lin(h, W["w_qkv"], W["b_qkv"])
-    X = X + E[2] * lin(mha(qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:]), W["w_o"], W["b_o"])
+    sa_in = (qkv[:, :D], qkv[:, D:2 * D], qkv[:, 2 * D:])
+    o_sa = t64(torch_attention_fp8(*(a.numpy() for a in sa_in), heads)) if fp8_attention else mha(*sa_in)
+    X = X + E[2] * lin(o_sa, W["w_o"], W["b_o"])
     hc = ln(X)
     q = lin(hc, W["w_cq"], W["b_cq"])
     kv = lin(C, W["w_ckv"], W["b_ckv"])
@@ -699,15 +702,17 @@ def test_linear_fp8_is_the_dequantised_product():
 
 
 def check_block_fp8_vs_torch(dit_block):
-    for i2v in (False, True):
+    for i2v, fa in ((False, False), (True, False), (False, True), (True, True)):
         w, inp = _tiny_block_inputs(i2v, seed=6)
         blk = inp["blocks"][0]
         img = None
         if i2v:
             img = O.image_context_mlp(inp["img_feat"][0], inp["w_i1"], inp["b_i1"], inp["w_i2"],
                                       inp["b_i2"], inp["w_i3"], inp["b_i3"])
-        got = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True)
-        ref = torch_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True)
+        got = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True,
+                        fp8_attention=fa)
+        ref = torch_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img, fp8=True,
+                          fp8_attention=fa)
         np.testing.assert_allclose(got - inp["x"][0], ref - inp["x"][0], rtol=1e-9, atol=1e-10)
         plain = dit_block(inp["x"][0], inp["e"][0], blk, inp["ctx"][0], w.heads, img_ctx=img)
         d, dp = got - inp["x"][0], plain - inp["x"][0]

@@ -66,8 +66,10 @@ class DiffusionCache(ctypes.Structure):
 
 
 class Fp8Scales(ctypes.Structure):
-    """Device pointers of the per-tensor scales of a block's E4M3 weights."""
-    _fields_ = [(n, _vp) for n in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]]
+    """Device pointers of the per-tensor scales of a block's E4M3 weights; with
+    attention_fp8 = 1 the block's self-attention also runs on E4M3 operands."""
+    _fields_ = [(n, _vp) for n in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]] + \
+        [("attention_fp8", _i)]
 
 
 class WanError(RuntimeError):

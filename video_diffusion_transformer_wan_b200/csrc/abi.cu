@@ -371,9 +371,31 @@ int head_impl(const wan_dit_config* c, const float* x, int B, int F, int H, int 
 // FP8 block workspace: the bf16 block's layout (its h region unused), then E4M3 codes
 // of the block inputs ([B*L, max(D, F)], reused by each linear layer in turn), codes of
 // the text / image context ([B*max(Lc, Li), D]) and the per-row scales of both.
+// 8-bit attention workspace: q codes, q scales, k codes, v^T codes, k/v scales, and the
+// key-split scratch of a partial last wave.
+struct AttnF8Layout {
+  size_t qc, qs, kc, vt, kvs, split, split_bytes, total;
+  int64_t vt_stride;
+};
+AttnF8Layout attn_f8_layout(const wan_dit_config* c, int B, int Lq, int Lk) {
+  const size_t D = c->dim, H = c->heads;
+  AttnF8Layout l;
+  l.vt_stride = (static_cast<int64_t>(Lk) + 63) / 64 * 64;
+  l.qc = 0;
+  l.qs = l.qc + align_up(static_cast<size_t>(B) * Lq * D);
+  l.kc = l.qs + align_up(static_cast<size_t>(B) * Lq * H * 4);
+  l.vt = l.kc + align_up(static_cast<size_t>(B) * Lk * D);
+  l.kvs = l.vt + align_up(static_cast<size_t>(B) * D * l.vt_stride);
+  l.split = l.kvs + align_up(static_cast<size_t>(B) * H * 2 * 4);
+  l.split_bytes = split_bytes(c, B, Lq);
+  l.total = l.split + align_up(l.split_bytes);
+  return l;
+}
+
 struct Fp8Layout {
   Layout base;
-  size_t codes, ctx_codes, scales, ctx_scales, total;
+  size_t codes, ctx_codes, scales, ctx_scales, attn, total;
+  AttnF8Layout attn_parts;  // offsets relative to `attn` (its own key-split scratch unused)
 };
 Fp8Layout fp8_layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
   Fp8Layout l;
@@ -385,7 +407,10 @@ Fp8Layout fp8_layout(const wan_dit_config* c, int B, int L, int Lc, int Li) {
   l.ctx_codes = l.codes + align_up(BL * wmax);
   l.scales = l.ctx_codes + align_up(Lx * c->dim);
   l.ctx_scales = l.scales + align_up(BL * 4);
-  l.total = l.ctx_scales + align_up(Lx * 4);
+  // operands of 8-bit self-attention (used when the scales ask for it)
+  l.attn = l.ctx_scales + align_up(Lx * 4);
+  l.attn_parts = attn_f8_layout(c, B, L, L);
+  l.total = l.attn + align_up(l.attn_parts.split);
   return l;
 }
 
@@ -428,8 +453,19 @@ int block_fp8_impl(const wan_dit_config* cfg, float* x, const float* e, const vo
   const size_t scr_bytes = fl.base.split_bytes;
   if (!(attn_kept && attn_reuse)) {
     WAN_TRY(e4m3_gemm(codes, scales, w->w_qkv, sc->qkv, w->b_qkv, qkv, M, 3 * D, D, epi_store(3 * D), s));
-    WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s,
-                           nullptr, scr, scr_bytes));
+    if (sc->attention_fp8) {
+      const AttnF8Layout& a = fl.attn_parts;
+      uint8_t* A = at(workspace, fl.attn);
+      float* qs = reinterpret_cast<float*>(A + a.qs);
+      float* kvs = reinterpret_cast<float*>(A + a.kvs);
+      WAN_TRY(launch_attn_fp8_quantize(qkv, 3 * D, 0, qkv, 3 * D, D, qkv, 3 * D, 2 * D, B, cfg->heads, L, L, A + a.qc,
+                                       qs, A + a.kc, A + a.vt, a.vt_stride, kvs, s));
+      WAN_TRY(launch_attn_tc_fp8(A + a.qc, qs, A + a.kc, A + a.vt, a.vt_stride, kvs, o, D, 0, B, cfg->heads, L, L, s,
+                                 scr, scr_bytes));
+    } else {
+      WAN_TRY(launch_attn_tc({qkv, 3 * D, 0}, {qkv, 3 * D, D}, {qkv, 3 * D, 2 * D}, o, D, 0, B, cfg->heads, L, L, s,
+                             nullptr, scr, scr_bytes));
+    }
   }
   WAN_TRY(launch_quantize_rows(o, D, M, D, false, codes, scales, WAN_BF16, s));
   const float* gb_msa = w->mod_bias ? w->mod_bias + 2 * D : nullptr;
@@ -1134,27 +1170,6 @@ int wan_linear_fwd(const wan_dit_config* cfg, const void* A, const void* W, cons
   GemmEpi ep = epilogue == WAN_EPI_RESIDUAL ? epi_residual(N, gate, gate_bias, gate_batch_stride, rows_per_batch)
                                             : epi_store(N, epilogue);
   return gemm(cfg, A, K, W, bias, out, M, N, K, 0, ep, as_stream(stream));
-}
-
-// 8-bit attention workspace: q codes, q scales, k codes, v^T codes, k/v scales, and the
-// key-split scratch of a partial last wave.
-struct AttnF8Layout {
-  size_t qc, qs, kc, vt, kvs, split, split_bytes, total;
-  int64_t vt_stride;
-};
-AttnF8Layout attn_f8_layout(const wan_dit_config* c, int B, int Lq, int Lk) {
-  const size_t D = c->dim, H = c->heads;
-  AttnF8Layout l;
-  l.vt_stride = (static_cast<int64_t>(Lk) + 63) / 64 * 64;
-  l.qc = 0;
-  l.qs = l.qc + align_up(static_cast<size_t>(B) * Lq * D);
-  l.kc = l.qs + align_up(static_cast<size_t>(B) * Lq * H * 4);
-  l.vt = l.kc + align_up(static_cast<size_t>(B) * Lk * D);
-  l.kvs = l.vt + align_up(static_cast<size_t>(B) * D * l.vt_stride);
-  l.split = l.kvs + align_up(static_cast<size_t>(B) * H * 2 * 4);
-  l.split_bytes = split_bytes(c, B, Lq);
-  l.total = l.split + align_up(l.split_bytes);
-  return l;
 }
 
 int check_attn_fp8_args(const wan_dit_config* cfg, const void* q, int64_t q_row_stride, int q_col0, const void* k,

@@ -53,7 +53,7 @@ def _sample(a) -> dict:
     tables, scales = model.block_tables, None
     if a.fp8:
         from .model import Fp8Block
-        fbs = [Fp8Block(cfg, b) for b in model.blocks]
+        fbs = [Fp8Block(cfg, b, attention_fp8=a.fp8_attention) for b in model.blocks]
         tables, scales = [f.table for f in fbs], [f.scale_table for f in fbs]
     ws = torch.empty(wan.sample_workspace_bytes(cfg, a.blocks, B, F, H, W, w.text_len, 0, cache, fp8=a.fp8),
                      dtype=torch.uint8, device="cuda")
@@ -63,7 +63,8 @@ def _sample(a) -> dict:
     # per step; the text K|V projections are made once per call and not counted
     block = 2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * L * Lc * D + 4 * L * D * Fd
     flops_step = 2 * B * (a.blocks * block + 2 * L * D * 64 * 2)
-    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, cache=a.cache or None, fp8=a.fp8, ms_per_call=ms,
+    return dict(workload=w.name, blocks=a.blocks, euler_steps=a.steps, cache=a.cache or None, fp8=a.fp8,
+                fp8_attention=a.fp8 and a.fp8_attention, ms_per_call=ms,
                 ms_per_euler_step=ms / a.steps,
                 latent_tokens_per_s=B * L * a.steps / (ms / 1e3),
                 tflops_uncached_equivalent=flops_step * a.steps / ms / 1e9)
@@ -84,7 +85,7 @@ def _block(a) -> dict:
     x = x0.clone()
     B, L = w.batch, w.tokens
     if a.fp8:
-        fb = Fp8Block(cfg, model.blocks[0])
+        fb = Fp8Block(cfg, model.blocks[0], attention_fp8=a.fp8_attention)
         ws = torch.empty(wan.fp8_workspace_bytes(cfg, B, L, w.text_len), dtype=torch.uint8, device="cuda")
         ms = _time(lambda: wan.dit_block_fp8_fwd(cfg, x, e, ctx, None, fb.table, fb.scale_table, ws), a.iters,
                    a.warmup)
@@ -94,13 +95,16 @@ def _block(a) -> dict:
     D, F, Lc = w.dim, w.ffn, w.text_len
     flops = B * (2 * L * D * 3 * D + 4 * L * L * D + 3 * 2 * L * D * D + 4 * Lc * D * D + 4 * L * Lc * D
                  + 4 * L * D * F)
-    return dict(workload=w.name, fp8=a.fp8, ms=ms, tokens_per_s=B * L / (ms / 1e3), tflops=flops / ms / 1e9)
+    return dict(workload=w.name, fp8=a.fp8, fp8_attention=a.fp8 and a.fp8_attention, ms=ms,
+                tokens_per_s=B * L / (ms / 1e3), tflops=flops / ms / 1e9)
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block"])
     ap.add_argument("--fp8", action="store_true", help="attention / gemm / block / sample: E4M3 operands (kind::f8f6f4)")
+    ap.add_argument("--fp8-attention", action="store_true",
+                    help="block / sample with --fp8: the self-attention on E4M3 operands as well")
     ap.add_argument("--no-split", action="store_true",
                     help="attention: no workspace, so a partial last wave is not split over the keys")
     ap.add_argument("--workload", default="wan13b_480p_block", help="block: workload name")

@@ -69,9 +69,10 @@ FP8_WEIGHTS = {"w_qkv": "qkv", "w_o": "o", "w_cq": "cq", "w_ckv": "ckv", "w_co":
 class Fp8Block:
     """A block's weights as E4M3 codes with per-tensor scales, quantised on the GPU by
     ``wan_fp8_quantize_tensor`` from the bf16 device weights; biases and ``mod_bias``
-    are shared with the bf16 block."""
+    are shared with the bf16 block. ``attention_fp8``: the block's self-attention runs on
+    E4M3 operands too."""
 
-    def __init__(self, cfg: Config, block: Dict[str, torch.Tensor]):
+    def __init__(self, cfg: Config, block: Dict[str, torch.Tensor], attention_fp8: bool = False):
         self.codes: Dict[str, torch.Tensor] = {}
         self.scales: Dict[str, torch.Tensor] = {}
         for name, key in FP8_WEIGHTS.items():
@@ -86,4 +87,5 @@ class Fp8Block:
         tables.update(self.codes)
         self.table = block_weights(tables)
         self.scale_table = Fp8Scales(*(self.scales[k].data_ptr() if k in self.scales else None
-                                       for k in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]))
+                                       for k in ["qkv", "o", "cq", "ckv", "co", "ckv_img", "ffn1", "ffn2"]),
+                                     1 if attention_fp8 else 0)
