@@ -34,6 +34,16 @@
 // unnormalised output with each row's base and sum to a caller scratch, and
 // attn_combine_kernel merges the halves.
 // TMEM: S_0 (later P_0), S_1 (P_1), O_0, O_1 = 4 x 128 of the 512 columns.
+//
+// The E4M3 instantiation (kF8; the 8-bit attention of the same page's section "Infra",
+// inference optimisation, here with E4M3 for both products) runs the same protocol on
+// E4M3 codes: 16 KB tiles (128 codes per 128-byte swizzled row), an 8-stage ring, four
+// kind::f8f6f4 MMAs of K = 32 per product, P as four E4M3 codes per TMEM column, and V
+// stored transposed so that both products take K-major operands. A row's q scale and
+// its head's k scale fold into the row's log2 scale, the v scale into the output. The
+// running base is rounded up to a whole power of two, so that P's codes equal those of
+// the final base times an exact power of two (outside E4M3's subnormal range) and every
+// rescale factor is exact.
 #include <cuda_bf16.h>
 
 #include <math.h>
