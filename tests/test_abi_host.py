@@ -184,3 +184,38 @@ def test_empty_inputs_launch_nothing(wan):
                                0, 12, 32, 32, 128, None, 0, None) == 0
     assert L.wan_linear_fwd(ctypes.byref(cfg), fake, fake, None, fake, 0, 64, 64, 0, None, None, 0, 1, None) == 0
     assert wan.launch_count() == n
+
+
+def test_attention_fp8_validation_and_workspace(wan):
+    """8-bit attention: workspace = q codes + q scales + k codes + v^T codes (keys padded
+    to a multiple of 64) + k/v scales + the key-split scratch, each 256-aligned; bad
+    arguments are refused before any launch."""
+    L = wan.lib
+    cfg = _cfg(wan)
+    B, Lq, Lk, H, D = 1, 32760, 32760, 12, 1536
+    n = wan.attention_fp8_workspace_bytes(cfg, B, Lq, Lk)
+    S = (Lk + 63) // 64 * 64
+    split = min(B * H * ((Lq + 255) // 256), 74) * 2 * 2 * 128 * 520
+    lower = B * Lq * D + 4 * B * Lq * H + B * Lk * D + B * D * S + 8 * B * H + split
+    assert lower <= n <= lower + 6 * 256
+    assert wan.attention_fp8_workspace_bytes(_cfg(wan, dtype="f32"), B, Lq, Lk) == 0
+    assert wan.attention_fp8_workspace_bytes(cfg, B, Lq, 0) == 0
+    fake = 1 << 20
+    n0 = wan.launch_count()
+
+    def fwd(c=cfg, ws_bytes=1 << 40, heads=H, hd=128, lk=Lk, q_col0=0, ws=fake):
+        return L.wan_attention_fp8_fwd(ctypes.byref(c), fake, 3 * D, q_col0, fake, 3 * D, D, fake, 3 * D, 2 * D, fake,
+                                       D, 0, B, heads, Lq, lk, hd, ws, ws_bytes, None)
+    assert fwd(ws_bytes=n - 1) == -5                     # workspace too small
+    assert fwd(ws=None) == -1                            # workspace required
+    assert fwd(c=_cfg(wan, dtype="f32")) == -8           # bf16 only
+    assert fwd(heads=8) == -2 and fwd(hd=64) == -2       # heads / head_dim differ from the config
+    assert fwd(lk=0) == -2                               # no keys
+    assert fwd(q_col0=3 * D) == -2                       # head columns past the row
+    q = L.wan_attention_fp8_quantize
+    args = (ctypes.byref(cfg), fake, 3 * D, 0, fake, 3 * D, D, fake, 3 * D, 2 * D, B, H, Lq, Lk, 128, fake, fake,
+            fake, fake)
+    assert q(*args, S - 1, fake, None) == -2             # v^T row stride not a multiple of 64
+    assert q(*args, S - 64, fake, None) == -2            # shorter than the keys
+    assert q(*args[:-1], fake + 8, S, fake, None) == -4  # v^T codes not 16-byte aligned
+    assert wan.launch_count() == n0
