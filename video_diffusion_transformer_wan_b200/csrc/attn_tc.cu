@@ -43,7 +43,8 @@
 // its head's k scale fold into the row's log2 scale, the v scale into the output. The
 // running base is rounded up to a whole power of two, so that P's codes equal those of
 // the final base times an exact power of two (outside E4M3's subnormal range) and every
-// rescale factor is exact.
+// rescale factor is exact. With the products at twice the rate the exponentials are the
+// busier unit, so one in eight runs on the FMA pipes (exp2_poly).
 #include <cuda_bf16.h>
 
 #include <math.h>
@@ -372,7 +373,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float2 x01 = f2_unpack(f2_fma(s01, sl2x2, nbx2));
           const float2 x23 = f2_unpack(f2_fma(s23, sl2x2, nbx2));
           const float e0 = ex2_approx(x01.x), e1 = ex2_approx(x01.y);
-          const float e2 = ex2_approx(x23.x), e3 = ex2_approx(x23.y);
+          // one exponential in eight on the FMA pipes (MUFU is the busier unit here)
+          const float e2 = ex2_approx(x23.x);
+          const float e3 = (i & 1) == 0 ? exp2_poly(x23.y) : ex2_approx(x23.y);
           rs4[(2 * i) & 3] = f2_add(rs4[(2 * i) & 3], f2_pack(e0, e1));
           rs4[(2 * i + 1) & 3] = f2_add(rs4[(2 * i + 1) & 3], f2_pack(e2, e3));
           r[i] = pack_e4m3x4(e0, e1, e2, e3);

@@ -259,6 +259,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
   return y;
 }
+// 2^x on the FMA pipes for a share of the exponentials: Cody-Waite range reduction
+// (W. J. Cody and W. Waite, "Software Manual for the Elementary Functions", 1980),
+// x = n + f, n = round(x), f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted for
+// minimum relative error on [-0.5, 0.5] (7.5e-5); 2^n added to the exponent field.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const int n = __float_as_int(t) - 0x4B400000;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(0.055171143263578415f, f, 0.24260996282100677f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999281167984009f);
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
