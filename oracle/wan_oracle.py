@@ -470,11 +470,11 @@ def euler_cfg_cached(x0, n_steps: int, guidance: float, velocity_cond, velocity_
 
 def sample_euler_cfg_cached(noise, n_steps: int, guidance: float, weights: Dict, blocks: Sequence[Dict], ctx_cond,
                             ctx_uncond, heads: int, schedule, eps: float = 1e-6, img_ctx=None, cond_channels=None,
-                            freq_dim: int = 256) -> np.ndarray:
+                            freq_dim: int = 256, fp8: bool = False, fp8_attention: bool = False) -> np.ndarray:
     """``sample_euler_cfg`` with the diffusion cache of ``schedule``
     (``diffusion_cache_schedule``). Each branch keeps its own per-block attention
     outputs: a branch that reuses attention takes the outputs of the last step on which
-    that branch computed it."""
+    that branch computed it. ``fp8`` / ``fp8_attention`` as in ``dit_stack``."""
     caches = {"c": [{} for _ in blocks], "u": [{} for _ in blocks]}
 
     def make_input(x):
@@ -485,7 +485,7 @@ def sample_euler_cfg_cached(noise, n_steps: int, guidance: float, weights: Dict,
             for c in caches[key]:
                 c["reuse"] = reuse
             return dit_stack(make_input(x), 1000.0 * t, weights, blocks, ctx, heads, eps, img_ctx=img_ctx,
-                             freq_dim=freq_dim, attn_caches=caches[key])
+                             freq_dim=freq_dim, attn_caches=caches[key], fp8=fp8, fp8_attention=fp8_attention)
         return f
     return euler_cfg_cached(noise, n_steps, guidance, vel(ctx_cond, "c"), vel(ctx_uncond, "u"), schedule)
 
