@@ -14,11 +14,12 @@ F32_TOL = 1e-4    # same, fp32 path
 FP8_TOL_MAX = 5e-2
 FP8_TOL_RMS = 2.5e-2
 # The same derivation for outputs further from the quantisers: the FP8 stack's velocity
-# (two blocks, LN, head) moves by at most 0.61 % (max) and 0.52 % (RMS) under those
-# perturbations (8 trials), a 3-step guided FP8 sampling displacement by at most 1.31 %
-# and 1.0 % (4 trials); bars 1.5x, rounded up. Both still separate FP8 from bf16 (1.5 %
-# and 4.5 % apart).
-FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS = 1e-2, 8e-3
+# (two blocks, LN, head) moves by at most 0.84 % (max) and 0.54 % (RMS) under those
+# perturbations (8 trials for each of the two samples, T2V and I2V, with and without
+# 8-bit self-attention), a 3-step guided FP8 sampling displacement by at most 1.31 %
+# and 1.0 % (4 trials); bars 1.5x, rounded up. The sampler bars separate FP8 from bf16
+# (4.5 % apart); at the stack the RMS bar does (1.5 % apart).
+FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS = 1.3e-2, 8.5e-3
 FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
 # 8-bit attention against the oracle's. The kernel takes each row's probabilities
 # against its running max (moved only when the max grows past 2^8), rounded up to a
