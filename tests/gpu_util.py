@@ -8,11 +8,12 @@ F32_TOL = 1e-4    # same, fp32 path
 # probability ~1/64 and then by a whole code. The GPU's quantiser inputs (attention
 # output, FFN hidden) are bf16 tensors whose values differ from the oracle's float64
 # ones at that level. Perturbing exactly those tensors by +-2^-9 in the oracle moves its
-# FP8 block by at most 3.3 % (max-norm) and 1.6 % (RMS) over 16 seeded trials (T2V and
-# I2V), so the bars are 1.5x those: 5e-2 and 2.5e-2. The RMS bar also separates the FP8
-# block from the bf16 one, which is 5 % RMS away.
+# FP8 block by at most 3.3 % (max-norm) and 1.6 % (RMS) over 16 seeded trials (small T2V
+# and I2V blocks) and by 2.1 % / 2.1 % on 256 sampled rows of the 1.3B block (3 trials),
+# so the bars are 1.5x the worst: 5e-2 and 3.2e-2. The RMS bar also separates the FP8
+# block from the bf16 one, which is 5 % (small) and 5.4 % (1.3B) RMS away.
 FP8_TOL_MAX = 5e-2
-FP8_TOL_RMS = 2.5e-2
+FP8_TOL_RMS = 3.2e-2
 # The same derivation for outputs further from the quantisers: the FP8 stack's velocity
 # (two blocks, LN, head) moves by at most 0.84 % (max) and 0.54 % (RMS) under those
 # perturbations (8 trials for each of the two samples, T2V and I2V, with and without
