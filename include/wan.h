@@ -298,7 +298,9 @@ int wan_linear_fp8_fwd(const wan_dit_config* cfg, const void* A, const float* a_
                        const float* gate, const float* gate_bias, int64_t gate_batch_stride,
                        int rows_per_batch, void* stream);
 
-/* Workspace (bytes) of wan_dit_block_fp8_fwd. */
+/* Workspace (bytes) of wan_dit_block_fp8_fwd: the bf16 block's workspace, the E4M3 codes
+ * and row scales of the activations and the context, and the operands of the 8-bit
+ * self-attention (used only with attention_fp8; about 3 B*L*dim bytes). */
 size_t wan_fp8_workspace_bytes(const wan_dit_config* cfg, int B, int L, int Lc, int Li);
 
 /* wan_dit_block_fwd with every linear layer in FP8: w holds E4M3 codes for the eight
