@@ -28,10 +28,11 @@ FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
 # E4M3 codes unchanged up to that factor, except in the subnormal and flush range, where
 # a lower running base keeps small probabilities the oracle rounds away. Emulating the
 # kernel's running base in the oracle (per 128-key tile, per 32-row warp) moves the
-# result by at most 5.3 % (max-norm) and 2.0 % (RMS) over logit standard deviations 0.6,
-# 1 and 4, 700 to 32760 keys, whole and key-split; bars 1.5x: 8e-2 and 3e-2. (8-bit
-# attention itself is 4-10 % (max) and 4-11 % (RMS) away from exact attention there.)
-FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS = 8e-2, 3e-2
+# result by at most 5.3 % (max-norm) and 2.4 % (RMS) over logit standard deviations 0.6,
+# 1 and 4, 700 to 75600 keys, whole and key-split (the RMS grows with the key count:
+# 2.0 % at 32760, 2.4 % at 75600); bars 1.5x: 8e-2 and 3.7e-2. (8-bit attention itself
+# is 4-18 % (max) and 4-12 % (RMS) away from exact attention there.)
+FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS = 8e-2, 3.7e-2
 # The FP8 block with 8-bit self-attention: the derivation of FP8_TOL_* with q, k and v
 # also moved by +-2^-9 and the running base emulated in the 8-bit attention moves the
 # block by at most 2.8 % (max) and 2.1 % (RMS) (960-token T2V and I2V blocks, 6 trials

@@ -287,12 +287,13 @@ def test_attention_fp8_parity(wan, B, Lq, Lk, H, logit_std):
     _attention_fp8_case(wan, B, Lq, Lk, H, logit_std, seed=Lq * 7 + Lk)
 
 
-def test_attention_fp8_full_size_sampled_rows(wan):
-    """1.3B self-attention shape (32760 tokens, 12 heads) on 256 sampled query rows."""
-    L = 32760
+@pytest.mark.parametrize("L,H", [(32760, 12), (75600, 40)])
+def test_attention_fp8_full_size_sampled_rows(wan, L, H):
+    """1.3B (32760 tokens, 12 heads) and 14B (75600 tokens, 40 heads) self-attention
+    shapes on 256 sampled query rows."""
     rows = sample_rows(L)
-    got, q, k, v = _attention_fp8_case(wan, 1, L, L, 12, 1.0, seed=5, rows=rows)
-    exact = O.attention(q[0][rows], k[0], v[0], 12)
+    got, q, k, v = _attention_fp8_case(wan, 1, L, L, H, 1.0, seed=5, rows=rows)
+    exact = O.attention(q[0][rows], k[0], v[0], H)
     assert rms_err(got[0][rows], exact) > FP8_ATTN_TOL_RMS / 3           # it is the 8-bit path, not bf16
 
 
