@@ -219,3 +219,19 @@ def test_attention_fp8_validation_and_workspace(wan):
     assert q(*args, S - 64, fake, None) == -2            # shorter than the keys
     assert q(*args[:-1], fake + 8, S, fake, None) == -4  # v^T codes not 16-byte aligned
     assert wan.launch_count() == n0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """With the CUDA library absent, the first call raises: there is no CPU fallback."""
+    import subprocess
+    import sys
+    code = ("import video_diffusion_transformer_wan_b200 as w\n"
+            "try:\n"
+            "    w.status_string(0)\n"
+            "except ImportError as e:\n"
+            "    print('refused:', e)\n"
+            "    raise SystemExit(3)\n")
+    env = dict(os.environ, WAN_B200_LIB=str(tmp_path / "absent.so"))
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 3 and "refused:" in r.stdout
