@@ -385,3 +385,26 @@ def test_cached_sampler_fp8_matches_oracle(wan, fa):
         print(f"cached fp8 sampler attn8={fa} b={b}: max {rel_err(d_got, d_ref):.2e} rms {rms_err(d_got, d_ref):.2e}")
         assert rel_err(d_got, d_ref) <= FP8_SAMPLE_TOL_MAX
         assert rms_err(d_got, d_ref) <= FP8_SAMPLE_TOL_RMS
+
+
+def test_attention_fp8_fused_qkv_layout(wan):
+    """q, k and v as column slices of one [B, L, 3D] projection (row stride 3D, head
+    columns from 0, D and 2D), and the output into a wider buffer at a column offset."""
+    B, L, H = 2, 700, 2
+    D = H * 128
+    q, k, v = _qkv(11, B, L, L, H, 1.0)
+    qkv = np.concatenate([q, k, v], axis=2)
+    cfg = _attn_cfg(wan, H)
+    bf = torch.bfloat16
+    o = torch.full((B, L, D + 64), float("nan"), dtype=bf, device="cuda")
+    ws = torch.empty(wan.attention_fp8_workspace_bytes(cfg, B, L, L), dtype=torch.uint8, device="cuda")
+    t = dev(qkv, bf)
+    wan.attention_fp8_fwd(cfg, t, t, t, o, H, 128, 0, D, 2 * D, 64, ws=ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = host(o)
+    assert np.isnan(got[:, :, :64]).all()                                 # columns before o_col0 untouched
+    for b in range(B):
+        ref = O.attention_fp8(q[b], k[b], v[b], H)
+        assert rel_err(got[b][:, 64:], ref) <= FP8_ATTN_TOL_MAX
+        assert rms_err(got[b][:, 64:], ref) <= FP8_ATTN_TOL_RMS
