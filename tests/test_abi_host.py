@@ -235,3 +235,19 @@ def test_missing_library_fails_loudly(tmp_path):
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=120)
     assert r.returncode == 3 and "refused:" in r.stdout
+
+
+def test_fp8_workspace_holds_the_bf16_workspace_codes_and_attention_operands(wan):
+    """FP8 block workspace = the bf16 block's + E4M3 codes of the widest activation
+    (F or D per row) and of the context + their row scales + the 8-bit self-attention's
+    operands (its own key-split scratch excluded: the block's is reused), each region
+    256-aligned; the FP8 sampler's is larger than the bf16 sampler's by that much."""
+    cfg = _cfg(wan)
+    B, L, Lc, H, D, F = 1, 32760, 512, 12, 1536, 8960
+    base = wan.workspace_bytes(cfg, B, L, Lc)
+    S = (L + 63) // 64 * 64
+    attn = B * L * D + 4 * B * L * H + B * L * D + B * D * S + 8 * B * H
+    extra = B * L * max(F, D) + B * Lc * D + 4 * B * L + 4 * B * Lc + attn
+    n = wan.fp8_workspace_bytes(cfg, B, L, Lc)
+    assert base + extra <= n <= base + extra + 10 * 256
+    assert wan.fp8_workspace_bytes(_cfg(wan, heads=7), B, 10, 10) == 0
