@@ -580,3 +580,143 @@ def attention_fp8(q, k, v, heads: int) -> np.ndarray:
         p = np.exp2(x - np.ceil(x.max(axis=-1, keepdims=True)))
         out[:, sl] = F64(sv) * (round_e4m3(p) @ vq) / p.sum(axis=-1, keepdims=True)
     return out
+
+
+# --------------------------------------------------------------------------------------
+# Full-size stack evaluation: float32 products, float64 reductions
+# --------------------------------------------------------------------------------------
+# The 30-block 1.3B stack at 480P (32760 tokens) is ~283 TFLOP; in float64 numpy it would
+# take hours on a host. This variant computes the same definition (``dit_stack``, the
+# flow-matching input of [Wan-P2, "训练方法"]) with every matrix product in float32 (the
+# products of float32 numbers accumulate in float32 inside the BLAS) and everything else
+# in float64: the residual stream, LayerNorm (mean and variance), modulation, GELU,
+# biases, the softmax row maximum and the row sum. The softmax exponentials are float32
+# values of the float32 logits. Its distance from the float64 definition (~1e-6 relative)
+# is pinned against ``dit_stack`` at small sizes. torch's CPU ops serve as the library
+# steps (multi-threaded matmul, exp and sum), nothing else.
+
+def _t32(a):
+    import torch
+    if isinstance(a, torch.Tensor):
+        return a.to(torch.float32).contiguous()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+
+
+def _t64(a):
+    import torch
+    if isinstance(a, torch.Tensor):
+        return a.to(torch.float64)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+
+
+def linear_f32(x, weight, bias=None):
+    """``x W^T`` as a float32 product, plus the bias in float64; returns float64."""
+    import torch
+    y = (_t32(x) @ _t32(weight).T).to(torch.float64)
+    return y if bias is None else y + _t64(bias)
+
+
+def layer_norm_f64(x, eps: float = 1e-6):
+    """``layer_norm`` on a torch float64 tensor (same definition)."""
+    x = _t64(x)
+    mu = x.mean(dim=-1, keepdim=True)
+    var = ((x - mu) ** 2).mean(dim=-1, keepdim=True)
+    return (x - mu) / (var + eps).sqrt()
+
+
+def attention_f32(q, k, v, heads: int, chunk: int = 2048):
+    """``attention`` with the two products in float32: per head and per block of query
+    rows, ``s = q k^T`` (float32), ``p = exp((s - max_j s) / sqrt(d))`` (float32
+    exponentials), ``l = sum_j p`` (float64 over float32 partial sums of 128
+    consecutive keys), ``o = (p v) / l`` (the product in float32)."""
+    import torch
+    q32, k32, v32 = _t32(q), _t32(k), _t32(v)
+    Lq, D = q32.shape
+    Lk = k32.shape[0]
+    d = D // heads
+    nb = Lk // 128
+    out = torch.empty((Lq, D), dtype=torch.float64)
+    buf = torch.empty((min(chunk, Lq), Lk), dtype=torch.float32)
+    for hh in range(heads):
+        sl = slice(hh * d, (hh + 1) * d)
+        khT, vh = k32[:, sl].T.contiguous(), v32[:, sl].contiguous()
+        for r0 in range(0, Lq, chunk):
+            qc = q32[r0:r0 + chunk, sl]
+            s = buf[:qc.shape[0]]
+            torch.matmul(qc, khT, out=s)
+            s.sub_(s.amax(dim=-1, keepdim=True)).mul_(1.0 / math.sqrt(d)).exp_()
+            l = s[:, :nb * 128].reshape(s.shape[0], nb, 128).sum(dim=-1).to(torch.float64).sum(dim=-1, keepdim=True)
+            l += s[:, nb * 128:].sum(dim=-1, keepdim=True).to(torch.float64)
+            out[r0:r0 + chunk, sl] = (s @ vh).to(torch.float64) / l
+    return out
+
+
+def ffn_f32(h, w: Dict[str, np.ndarray], chunk: int = 4096):
+    """``ffn_branch`` with float32 products; the hidden layer (bias, GELU-tanh) in
+    float64, a block of rows at a time (rows are independent)."""
+    import torch
+    h = _t64(h)
+    out = torch.empty((h.shape[0], _f(w["w_2"]).shape[0]), dtype=torch.float64)
+    for r0 in range(0, h.shape[0], chunk):
+        u = linear_f32(h[r0:r0 + chunk], w["w_1"], w["b_1"])
+        u = 0.5 * u * (1.0 + torch.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+        out[r0:r0 + chunk] = linear_f32(u, w["w_2"], w["b_2"])
+    return out
+
+
+def dit_block_f32(x, e, w: Dict[str, np.ndarray], ctx, heads: int, eps: float = 1e-6, img_ctx=None,
+                  rows: Optional[Sequence[int]] = None):
+    """``dit_block`` with float32 products and float64 reductions (the section comment
+    above). ``x`` and the result are float64 torch tensors; ``rows`` as in ``dit_block``."""
+    import torch
+    x = _t64(x)
+    D = x.shape[-1]
+    shift_msa, scale_msa, gate_msa, shift_ffn, scale_ffn, gate_ffn = _t64(block_modulation(e, w["mod_bias"]))
+    h_all = layer_norm_f64(x, eps) * (1.0 + scale_msa) + shift_msa
+    if rows is None:
+        xr, hr = x, h_all
+    else:
+        idx = torch.from_numpy(np.asarray(rows, dtype=np.int64))
+        xr, hr = x[idx], h_all[idx]
+    wqkv, bqkv = w["w_qkv"], _f(w["b_qkv"])
+    q = linear_f32(hr, wqkv[:D], bqkv[:D])
+    kv = linear_f32(h_all, wqkv[D:], bqkv[D:])
+    o = attention_f32(q, kv[:, :D], kv[:, D:], heads)
+    x1 = xr + gate_msa * linear_f32(o, w["w_o"], w["b_o"])
+    hc = layer_norm_f64(x1, eps)
+    qc = linear_f32(hc, w["w_cq"], w["b_cq"])
+    kvc = linear_f32(ctx, w["w_ckv"], w["b_ckv"])
+    oc = attention_f32(qc, kvc[:, :D], kvc[:, D:], heads)
+    if img_ctx is not None:
+        kvi = linear_f32(img_ctx, w["w_ckv_img"], w["b_ckv_img"])
+        oc = oc + attention_f32(qc, kvi[:, :D], kvi[:, D:], heads)
+    x2 = x1 + linear_f32(oc, w["w_co"], w["b_co"])
+    hf = layer_norm_f64(x2, eps) * (1.0 + scale_ffn) + shift_ffn
+    return x2 + gate_ffn * ffn_f32(hf, w)
+
+
+def dit_stack_f32(latent, t: float, weights: Dict, blocks: Sequence[Dict], ctx, heads: int,
+                  eps: float = 1e-6, img_ctx=None, freq_dim: int = 256,
+                  rows: Optional[Sequence[int]] = None, progress=None) -> np.ndarray:
+    """``dit_stack`` with the blocks and the head in float32 products and float64
+    reductions (patchify and the time MLP are the float64 functions above). With
+    ``rows`` the last block and the head are evaluated for those tokens only (every
+    earlier block needs all tokens) and the result is the head output ``[len(rows),
+    out_ch*4]``; otherwise it is the unpatchified velocity ``[out_ch, F, H, W]``.
+    ``progress(i)`` is called after block ``i``."""
+    lat = _f(latent)
+    C, F, H, W = lat.shape
+    x = _t64(patchify(lat, weights["w_p"], weights["b_p"]))
+    e = time_mlp(t, weights["w_t1"], weights["b_t1"], weights["w_t2"], weights["b_t2"], freq_dim)
+    n = len(blocks)
+    for i, blk in enumerate(blocks):
+        x = dit_block_f32(x, e, blk, ctx, heads, eps, img_ctx=img_ctx,
+                          rows=rows if i == n - 1 else None)
+        if progress is not None:
+            progress(i)
+    if rows is not None and n == 0:
+        x = x[_t64(np.asarray(rows)).long()]
+    y = linear_f32(layer_norm_f64(x, eps), weights["w_head"], weights["b_head"]).numpy()
+    if rows is not None:
+        return y
+    return unpatchify(y, _f(weights["w_head"]).shape[0] // 4, F, H, W)

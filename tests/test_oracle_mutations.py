@@ -253,3 +253,39 @@ def test_attention_fp8_mutations_are_caught():
     _fails(P.check_attention_fp8, _attention_fp8_variant(v_axis=-1))            # a v scale per key row
     _fails(P.check_attention_fp8, _attention_fp8_variant(int_base=False))       # base at the row max itself
     P.check_attention_fp8(_attention_fp8_variant())                              # the unmutated restatement passes
+
+
+def test_f32_stack_mutations_are_caught():
+    import torch
+
+    def no_tail_sum(q, k, v, heads, chunk=2048):       # row sum misses the keys past the last 128-key block
+        q32, k32, v32 = (torch.as_tensor(np.float32(a)) for a in (q, k, v))
+        d = q32.shape[1] // heads
+        out = np.empty(q32.shape)
+        for h in range(heads):
+            sl = slice(h * d, (h + 1) * d)
+            s = q32[:, sl] @ k32[:, sl].T
+            p = torch.exp((s - s.amax(-1, keepdim=True)) / math.sqrt(d))
+            nb = s.shape[1] // 128
+            l = p[:, :nb * 128].sum(-1, keepdim=True).double()
+            out[:, sl] = ((p @ v32[:, sl]).double() / l).numpy()
+        return out
+
+    def scaled_after_exp(q, k, v, heads, chunk=2048):  # 1/sqrt(d) applied to the output, not the logits
+        return np.asarray(O.attention_f32(np.asarray(q) * math.sqrt(np.asarray(q).shape[1] // heads), k, v,
+                                          heads, chunk))
+    _fails(P.check_attention_f32, no_tail_sum)
+    _fails(P.check_attention_f32, scaled_after_exp)
+
+    def ungated_ffn(latent, t, weights, blocks, ctx, heads, eps=1e-6, img_ctx=None, rows=None):
+        mut = [dict(b) for b in blocks]
+        for b in mut:                                   # gate_ffn bias zeroed: the gate is e only
+            b["mod_bias"] = np.asarray(b["mod_bias"]).copy()
+            b["mod_bias"][5] = 0.0
+        return O.dit_stack_f32(latent, t, weights, mut, ctx, heads, eps, img_ctx=img_ctx, rows=rows)
+
+    def last_block_all_rows(latent, t, weights, blocks, ctx, heads, eps=1e-6, img_ctx=None, rows=None):
+        out = O.dit_stack_f32(latent, t, weights, blocks, ctx, heads, eps, img_ctx=img_ctx, rows=rows)
+        return out if rows is None else np.roll(out, 1, axis=0)   # rows returned out of order
+    _fails(P.check_stack_f32, ungated_ffn)
+    _fails(P.check_stack_f32, last_block_all_rows)

@@ -474,6 +474,58 @@ def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
     assert not np.allclose(v3, v2)
 
 
+# ----------------------------------------------------------------------------------------
+# The float32-product / float64-reduction stack used for the full-size 30-block stack
+# ----------------------------------------------------------------------------------------
+
+def check_attention_f32(attn_f32):
+    """Against the float64 ``attention``: scores spanning several 128-key partial sums
+    and a ragged tail, query blocks with a ragged last one, logit std 1 and 4."""
+    rng = RNG(40)
+    for scale in (1.0, 4.0):
+        q = rng.standard_normal((300, 256)) * scale / 64 ** 0.25 * 1.0
+        k = rng.standard_normal((300, 256)) / 64 ** 0.25
+        v = rng.standard_normal((300, 256))
+        got = np.asarray(attn_f32(q, k, v, 4, chunk=128))
+        ref = O.attention(np.float32(q), np.float32(k), np.float32(v), 4)
+        assert np.abs(got - ref).max() <= 2e-6 * np.abs(ref).max(), np.abs(got - ref).max()
+
+
+def check_stack_f32(stack_f32, block_f32=None):
+    """Against the float64 ``dit_stack``: a 3-block full-width stack at 144 tokens (one
+    whole 128-key block plus a ragged tail), T2V and I2V, the whole velocity and the
+    head outputs of sampled tokens, within 2e-6 of max|v| (float32 products)."""
+    import dataclasses
+    for name in ("wan13b_480p_stack30", "wan13b_480p_i2v_block"):
+        w = dataclasses.replace(WORKLOADS[name], frames=3, height=12, width=16, dim=256, heads=2, ffn=512,
+                                text_len=24, img_len=20 if name.endswith("i2v_block") else 0, img_feat=64,
+                                n_blocks=3)
+        inp = make_inputs(w, seed=3, block_input=False, zero_wx=False)
+        lat = inp["noise"][0]
+        img = None
+        if w.i2v:
+            img = round_bf16(RNG(41).standard_normal((w.img_len, w.dim)).astype(np.float32))
+            lat = np.concatenate([lat, inp["cond"][0], np.zeros((4, w.frames, w.height, w.width), np.float32)])
+        t = float(inp["u"][0] * 1000.0) if "u" in inp else float(inp["t"][0])
+        ref = O.dit_stack(lat, t, inp, inp["blocks"], inp["ctx"][0], w.heads, img_ctx=img)
+        got = stack_f32(lat, t, inp, inp["blocks"], inp["ctx"][0], w.heads, img_ctx=img)
+        den = np.abs(ref).max()
+        assert np.abs(got - ref).max() <= 2e-6 * den, (name, np.abs(got - ref).max() / den)
+        rows = np.array([0, 7, 100, 127, 128, 143])
+        y = np.asarray(ref).reshape(16, w.frames, w.height // 2, 2, w.width // 2, 2)
+        y = y.transpose(1, 2, 4, 0, 3, 5).reshape(w.tokens, 64)
+        got_rows = stack_f32(lat, t, inp, inp["blocks"], inp["ctx"][0], w.heads, img_ctx=img, rows=rows)
+        assert np.abs(got_rows - y[rows]).max() <= 2e-6 * den
+
+
+def test_attention_f32_matches_float64_attention():
+    check_attention_f32(O.attention_f32)
+
+
+def test_stack_f32_matches_float64_stack():
+    check_stack_f32(O.dit_stack_f32)
+
+
 def test_flow_matching_endpoints():
     rng = RNG(12)
     x1, x0 = rng.standard_normal((3, 4)), rng.standard_normal((3, 4))

@@ -20,13 +20,14 @@ here, once, so both the CUDA path and the oracle read identical numbers.
 from __future__ import annotations
 
 import dataclasses
+import hashlib
 from typing import Dict, List, Optional
 
 import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "make_inputs", "round_bf16", "bf16_bits",
-    "bits_to_f32", "sample_rows", "block_weight_names",
+    "bits_to_f32", "sample_rows", "block_weight_names", "input_digest",
 ]
 
 
@@ -227,3 +228,26 @@ def sample_rows(n_rows: int, tile: int = 128, count: int = 256, seed: int = 0) -
     while len(rows) < count:
         rows.add(int(rng.integers(0, n_rows)))
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def input_digest(inp: Dict[str, object]) -> str:
+    """SHA-256 over every array of a ``make_inputs`` result (keys in sorted order, block
+    dicts in block order, each array's dtype, shape and bytes). A stored expected value
+    records it, so a change of the input recipe shows up as a digest mismatch rather
+    than as a numerical failure."""
+    h = hashlib.sha256()
+
+    def add(name, a):
+        a = np.ascontiguousarray(a)
+        h.update(f"{name}:{a.dtype.str}:{a.shape};".encode())
+        h.update(a.view(np.uint8).reshape(-1).data)
+
+    for key in sorted(inp):
+        val = inp[key]
+        if isinstance(val, np.ndarray):
+            add(key, val)
+        elif key == "blocks":
+            for i, blk in enumerate(val):
+                for name in sorted(blk):
+                    add(f"blocks[{i}].{name}", blk[name])
+    return h.hexdigest()
