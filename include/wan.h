@@ -160,7 +160,9 @@ int wan_time_mlp(const wan_dit_config* cfg, const float* t, int B, const wan_tim
 int wan_adaln_modulate(const wan_dit_config* cfg, const float* x, int B, int L,
                        const float* e, const float* mod_bias, int chunk, void* h_out, void* stream);
 
-/* Self-attention branch with gated residual: x_inout[B, L, D] fp32 +=
+/* Self-attention branch with gated residual [Wan 2.1 page, "Diffusion Transformer":
+ * full spatio-temporal self-attention in every block, whose output is scaled by one of
+ * the six modulation vectors, the gate]: x_inout[B, L, D] fp32 +=
  * gate_msa * (Attn(h Wq, h Wk, h Wv) Wo^T + bo), gate_msa = e[b,2] + w->mod_bias[2].
  * h [B, L, D] act is the modulated LN output. Attention is full (non-causal) over the
  * L tokens of each sample, per head, scale 1/sqrt(head_dim). */
@@ -177,13 +179,18 @@ int wan_cross_attn_fwd(const wan_dit_config* cfg, const void* h, const void* ctx
                        const void* img_ctx, int Li, const wan_block_weights* w,
                        float* x_inout, int B, int L, void* workspace, size_t ws_bytes, void* stream);
 
-/* FFN branch with gated residual: x_inout += gate_ffn * (gelu_tanh(h W1^T + b1) W2^T + b2),
+/* FFN branch with gated residual [Wan 2.1 page, "Diffusion Transformer" and the config
+ * table (FFN dimension 8960 / 13824): the block's feed-forward network, its output scaled
+ * by the sixth modulation vector]: x_inout += gate_ffn * (gelu_tanh(h W1^T + b1) W2^T + b2),
  * gate_ffn = e[b,5] + w->mod_bias[5]. h [B, L, D] act. */
 int wan_ffn_fwd(const wan_dit_config* cfg, const void* h, const wan_block_weights* w,
                 const float* e, float* x_inout, int B, int L,
                 void* workspace, size_t ws_bytes, void* stream);
 
-/* One DiT block, in place on the residual stream x_inout [B, L, D] fp32:
+/* One DiT block [Wan 2.1 page, "Diffusion Transformer": self-attention, cross-attention
+ * to the text embedding, and an FFN; a shared MLP of the timestep gives six modulation
+ * vectors (shift, scale and gate of two branches) and each block learns its own bias on
+ * top of them], in place on the residual stream x_inout [B, L, D] fp32:
  * self-attention (modulated LN, gated), cross-attention (plain LN, ungated), FFN
  * (modulated LN, gated). e [B, 6, D] fp32 is the shared timestep-MLP output; the
  * block adds w->mod_bias. ctx [B, Lc, D] act; img_ctx [B, Li, D] act or NULL. */
@@ -228,7 +235,10 @@ int wan_head_fwd(const wan_dit_config* cfg, const float* x, int B, int F, int H,
  * before any launch. The call allocates nothing (no cudaMalloc, no cudaFree, no
  * allocating library routine).
  * The first call on a device looks up the array's device address (with that device
- * current) and caches it; make that first call before any stream capture. All calls
+ * current) and caches it; make that first call before any stream capture. The cached
+ * address belongs to the CUDA context it was looked up in: after a device reset, the
+ * next call on that device looks it up again, so make that call, too, before any
+ * capture. All calls
  * share the one array and each leaves its contents behind: calls whose work overlaps
  * on the GPU (other streams, other host threads) race on it, so the caller must order
  * them. No part of the array needs to start at zero. */

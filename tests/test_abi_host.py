@@ -251,3 +251,48 @@ def test_fp8_workspace_holds_the_bf16_workspace_codes_and_attention_operands(wan
     n = wan.fp8_workspace_bytes(cfg, B, L, Lc)
     assert base + extra <= n <= base + extra + 10 * 256
     assert wan.fp8_workspace_bytes(_cfg(wan, heads=7), B, 10, 10) == 0
+
+
+def test_both_patchify_calls_accept_and_reject_the_same_arguments(wan):
+    """wan_patchify and wan_patchify_noalloc run the same argument checks before any
+    launch: a config that one refuses, the other refuses with the same status."""
+    L = wan.lib
+    f = L.wan_patchify_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(wan.Config), ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    launches = wan.launch_count()
+    fake = 1 << 20
+    bad = []
+    c = _cfg(wan, heads=7)                      # dim != heads * head_dim
+    bad.append((c, -2))
+    c = _cfg(wan)
+    c.eps = 0.0                                 # eps must be positive
+    bad.append((c, -2))
+    c = _cfg(wan, out_ch=15)                    # odd output channels
+    bad.append((c, -2))
+    c = _cfg(wan, freq_dim=12)                  # frequency dim not a multiple of 8
+    bad.append((c, -2))
+    c = _cfg(wan, ffn=100)                      # FFN width not a multiple of 64
+    bad.append((c, -2))
+    c = _cfg(wan)
+    c.dtype = 5                                 # unknown dtype
+    bad.append((c, -3))
+    for cfg, code in bad:
+        a = L.wan_patchify(ctypes.byref(cfg), fake, 1, 2, 8, 8, fake, fake, fake, fake, 1 << 30, None)
+        b = f(ctypes.byref(cfg), fake, 1, 2, 8, 8, fake, fake, fake, None)
+        assert a == b == code, (a, b, code)
+    cfg = _cfg(wan)
+    # null and misaligned pointers, odd width: the same status from both
+    for args in [(0, fake, fake), (fake + 8, fake, fake), (fake, fake + 4, fake), (fake, fake, fake + 2)]:
+        lat, wp, out = args
+        a = L.wan_patchify(ctypes.byref(cfg), lat or None, 1, 2, 8, 8, wp, fake, out, fake, 1 << 30, None)
+        b = f(ctypes.byref(cfg), lat or None, 1, 2, 8, 8, wp, fake, out, None)
+        assert a == b and a < 0, (args, a, b)
+    assert L.wan_patchify(ctypes.byref(cfg), fake, 1, 2, 8, 7, fake, fake, fake, fake, 1 << 30, None) == \
+        f(ctypes.byref(cfg), fake, 1, 2, 8, 7, fake, fake, fake, None) == -2
+    # token counts whose product with the batch passes 2^31 are refused as a shape, not
+    # by a wrapped workspace size
+    assert L.wan_patchify(ctypes.byref(cfg), fake, 1 << 12, 1 << 10, 1 << 6, 1 << 6, fake, fake, fake, fake,
+                          1 << 62, None) == -2
+    assert wan.launch_count() == launches

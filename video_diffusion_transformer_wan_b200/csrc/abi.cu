@@ -18,21 +18,56 @@
 
 namespace wan {
 
+// ------------------------------------------------------------------ module symbols
+bool current_context_id(unsigned long long* id) {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+int SymbolCache::get(const void* symbol, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WAN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu_);
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  Entry& en = entry_[dev];
+  if (!have_ctx || !en.addr || en.ctx != ctx) {
+    void* p = nullptr;
+    // Looks the symbol up in this device's current context (creating the runtime's
+    // primary context if none exists yet), then records which context that was.
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return WAN_ERR_CUDA;
+    if (!current_context_id(&ctx)) return WAN_ERR_CUDA;
+    en.addr = p;
+    en.ctx = ctx;
+  }
+  *out = en.addr;
+  return WAN_OK;
+}
+
 // ------------------------------------------------------------------ device error flag
 __device__ int g_wan_error_flag;
 
 int* device_error_flag() {
-  static int* addr[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  dev &= 63;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_wan_error_flag) == cudaSuccess) addr[dev] = static_cast<int*>(p);
-  }
-  return addr[dev];
+  static SymbolCache cache;
+  void* p = nullptr;
+  return cache.get(&g_wan_error_flag, &p) == WAN_OK ? static_cast<int*>(p) : nullptr;
 }
 
 // ------------------------------------------------------------------ trace
@@ -127,8 +162,6 @@ static bool make_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* ba
 }
 
 // ------------------------------------------------------------------ validation helpers
-namespace {
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define WAN_REQUIRE(cond, code) \
@@ -147,15 +180,18 @@ int check_ptr(const void* p) {
   return WAN_OK;
 }
 int check_opt_ptr(const void* p) { return p ? check_ptr(p) : WAN_OK; }
+
+namespace {
+
 // Non-null and 4-byte aligned (fp32 scalars and scale vectors).
 int check_ptr_any(const void* p) {
   if (!p) return WAN_ERR_NULL;
   return (reinterpret_cast<uintptr_t>(p) & 3u) == 0 ? WAN_OK : WAN_ERR_ALIGN;
 }
 
-// `attention`: the call runs attention, which fixes head_dim (128 on the bf16 tensor-core
-// path, <= 128 on the fp32 path).
-int check_cfg(const wan_dit_config* c, bool attention = false) {
+}  // namespace
+
+int check_cfg(const wan_dit_config* c, bool attention) {
   WAN_REQUIRE(c, WAN_ERR_NULL);
   WAN_REQUIRE(c->dtype == WAN_F32 || c->dtype == WAN_BF16, WAN_ERR_DTYPE);
   WAN_REQUIRE(c->heads > 0 && c->head_dim > 0 && c->dim == c->heads * c->head_dim, WAN_ERR_SHAPE);
@@ -171,6 +207,8 @@ int check_cfg(const wan_dit_config* c, bool attention = false) {
   }
   return WAN_OK;
 }
+
+namespace {
 
 int check_block_w(const wan_dit_config* c, const wan_block_weights* w, bool need_img) {
   WAN_REQUIRE(w, WAN_ERR_NULL);
@@ -634,12 +672,14 @@ int wan_patchify(const wan_dit_config* cfg, const void* latent, int B, int F, in
   WAN_TRY(check_ptr(x_out));
   WAN_TRY(check_ptr(workspace));
   WAN_REQUIRE(B >= 0 && F >= 0 && H >= 0 && W >= 0 && H % 2 == 0 && W % 2 == 0, WAN_ERR_SHAPE);
-  const int L = F * (H / 2) * (W / 2);
+  const size_t rows = static_cast<size_t>(B) * F * (H / 2) * (W / 2);
+  WAN_REQUIRE(rows < (size_t(1) << 31), WAN_ERR_SHAPE);
   const int K = cfg->in_ch * 4;
-  WAN_REQUIRE(ws_bytes >= static_cast<size_t>(B) * L * K * dtype_size(cfg->dtype), WAN_ERR_WORKSPACE);
+  WAN_REQUIRE(ws_bytes >= rows * K * dtype_size(cfg->dtype), WAN_ERR_WORKSPACE);
   cudaStream_t s = as_stream(stream);
   WAN_TRY(launch_patch_gather(latent, B, cfg->in_ch, F, H, W, workspace, cfg->dtype, s));
-  return gemm(cfg, workspace, K, w_p, b_p, x_out, B * L, cfg->dim, K, 0, epi_store(cfg->dim, WAN_EPI_F32), s);
+  return gemm(cfg, workspace, K, w_p, b_p, x_out, static_cast<int>(rows), cfg->dim, K, 0,
+              epi_store(cfg->dim, WAN_EPI_F32), s);
 }
 
 int wan_time_mlp(const wan_dit_config* cfg, const float* t, int B, const wan_time_weights* w, float* e_out,

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "wan.h"
 
 namespace wan {
@@ -20,8 +22,39 @@ void count_launches(int n);
 void trace_launch_begin(int kind, cudaStream_t s, double work = 0.0);
 void trace_launch_end(int kind, cudaStream_t s);
 int* device_error_flag();   // device address of the error flag of the current device
+
+// Identity (cuCtxGetId) of the calling thread's current CUDA context; false if none.
+bool current_context_id(unsigned long long* id);
+// Device addresses of one __device__ symbol, one per device, each tagged with the
+// context it was looked up in. get() returns the cached address while the device's
+// current context is the one it came from, and looks it up again (cudaGetSymbolAddress,
+// with the device current) after that context has been replaced, e.g. by a device
+// reset that reloads the module at another address.
+class SymbolCache {
+ public:
+  int get(const void* symbol, void** out);
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  struct Entry {
+    void* addr = nullptr;
+    unsigned long long ctx = 0;
+  };
+  Entry entry_[kMaxDevices];
+  std::mutex mu_;
+};
 // One-thread kernel whose bounded wait runs out (about 1 s) and sets the error flag.
 int launch_wait_timeout_probe(cudaStream_t s);
+
+// ---------------------------------------------------------------- argument checks
+// The checks every entry point applies before any launch (defined in abi.cu).
+bool aligned16(const void* p);
+int check_ptr(const void* p);       // non-null and 16-byte aligned
+int check_opt_ptr(const void* p);   // null, or 16-byte aligned
+// Config consistency: dtype, dim == heads * head_dim, multiples of 64, even channel
+// counts, freq_dim, eps > 0. `attention`: the call runs attention, which fixes head_dim
+// (128 on the bf16 tensor-core path, <= 128 on the fp32 path).
+int check_cfg(const wan_dit_config* c, bool attention = false);
 
 // Returns WAN_ERR_CUDA if the last launch failed.
 inline int check_launch() {

@@ -13,13 +13,14 @@
 // use the array's name as a device address (on the host it is only a stand-in symbol),
 // so the first call on each device looks the address up with cudaGetSymbolAddress,
 // with that device current, and caches it; later calls reuse it. That first call should
-// therefore come before any stream capture. Every call shares the one array, so calls
-// whose work overlaps on the GPU (different streams, or different host threads on one
-// device) race on it and must be serialised by the caller. Nothing in the array has to
-// start at zero: each call writes every scratch byte it later reads.
+// therefore come before any stream capture. The cached address is tagged with the CUDA
+// context it came from: after a device reset (a new primary context, which reloads the
+// module, possibly at another address) the next call looks it up again, so that call
+// too should come before any capture. Every call shares the one array, so calls whose
+// work overlaps on the GPU (different streams, or different host threads on one device)
+// race on it and must be serialised by the caller. Nothing in the array has to start at
+// zero: each call writes every scratch byte it later reads.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "internal.h"
 
@@ -28,20 +29,10 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_patchify_scratch[WAN_PATCHIFY_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_patchify_scratch on the current device (looked up once per device).
+// Device address of g_patchify_scratch on the current device.
 int patchify_scratch(void** out) {
-  static void* addr[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return WAN_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_patchify_scratch) != cudaSuccess || !p) return WAN_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *out = addr[dev];
-  return WAN_OK;
+  static SymbolCache cache;
+  return cache.get(&g_patchify_scratch, out);
 }
 
 }  // namespace
@@ -51,23 +42,23 @@ using namespace wan;
 
 extern "C" int wan_patchify_noalloc(const wan_dit_config* cfg, const void* latent, int B, int F, int H, int W,
                                     const void* w_p, const void* b_p, float* x_out, void* stream) {
-  if (!cfg || !latent || !w_p || !x_out) return WAN_ERR_NULL;
-  if (cfg->dtype != WAN_F32 && cfg->dtype != WAN_BF16) return WAN_ERR_DTYPE;
-  const uintptr_t mis = reinterpret_cast<uintptr_t>(latent) | reinterpret_cast<uintptr_t>(w_p) |
-                        reinterpret_cast<uintptr_t>(b_p) | reinterpret_cast<uintptr_t>(x_out);
-  if (mis & 15u) return WAN_ERR_ALIGN;
-  if (cfg->dim <= 0 || cfg->dim % 64 != 0 || cfg->in_ch <= 0 || cfg->in_ch % 2 != 0) return WAN_ERR_SHAPE;
+  // The same argument checks, in the same order, as wan_patchify.
+  int st = check_cfg(cfg);
+  if (st == WAN_OK) st = check_ptr(latent);
+  if (st == WAN_OK) st = check_ptr(w_p);
+  if (st == WAN_OK) st = check_opt_ptr(b_p);
+  if (st == WAN_OK) st = check_ptr(x_out);
+  if (st != WAN_OK) return st;
   if (B < 0 || F < 0 || H < 0 || W < 0 || H % 2 != 0 || W % 2 != 0) return WAN_ERR_SHAPE;
-  const size_t L = static_cast<size_t>(F) * (H / 2) * (W / 2);
+  const size_t rows = static_cast<size_t>(B) * F * (H / 2) * (W / 2);
+  if (rows >= (size_t(1) << 31)) return WAN_ERR_SHAPE;
   const int K = cfg->in_ch * 4;
-  const size_t need = static_cast<size_t>(B) * L * K * dtype_size(cfg->dtype);
-  if (need > WAN_PATCHIFY_NOALLOC_SCRATCH_BYTES || static_cast<size_t>(B) * L >= (size_t(1) << 31))
-    return WAN_ERR_SHAPE;
+  if (rows * K * dtype_size(cfg->dtype) > WAN_PATCHIFY_NOALLOC_SCRATCH_BYTES) return WAN_ERR_SHAPE;
   void* scratch = nullptr;
-  int st = patchify_scratch(&scratch);
+  st = patchify_scratch(&scratch);
   if (st != WAN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int M = static_cast<int>(static_cast<size_t>(B) * L);
+  const int M = static_cast<int>(rows);
   st = launch_patch_gather(latent, B, cfg->in_ch, F, H, W, scratch, cfg->dtype, s);
   if (st != WAN_OK) return st;
   GemmEpi ep{};
