@@ -151,82 +151,163 @@ def replica_throughput(world: int, tokens_per_step: float, ms_per_step: float) -
     return world * tokens_per_step / (ms_per_step / 1e3)
 
 
-def _oracle_prefix(inp):
+def _oracle_inputs(w, inp):
+    """The oracle's view of one step's inputs: the latent (I2V: the 36-channel fusion),
+    the timestep, the text context and the image context (computed outside the timed
+    region, as the GPU step takes it precomputed)."""
     from oracle import wan_oracle as O
-    x = O.patchify(inp["noise"][0], inp["w_p"], inp["b_p"])
-    e = O.time_mlp(float(inp["t"][0]), inp["w_t1"], inp["b_t1"], inp["w_t2"], inp["b_t2"])
-    return x, e
+    lat = inp["noise"][0]
+    img = None
+    if w.i2v:
+        keep = [1] + [0] * (4 * (w.frames - 1))
+        lat = O.i2v_input(inp["noise"][0], inp["cond"][0], O.i2v_mask(keep, w.frames, w.height, w.width))
+        img = O.image_context_mlp(inp["img_feat"][0], *(inp[k] for k in ["w_i1", "b_i1", "w_i2", "b_i2",
+                                                                         "w_i3", "b_i3"]))
+    t = float(1000.0 * inp["u"][0]) if w.flow_matching else float(inp["t"][0])
+    return lat, t, inp["ctx"][0], img
 
 
-def _oracle_rows(w, inp, x, e, S, seed=1) -> float:
-    """Seconds the oracle takes for the block on S sampled query rows (keys and values
-    over all rows, since self-attention needs them)."""
+def oracle_step_seconds(w, inp) -> float:
+    """Seconds the fp64 oracle takes for exactly the work of one GPU step: ``dit_stack``
+    with the workload's blocks (patchify, timestep MLP, every block on all tokens, head,
+    unpatchify), one sample."""
     from oracle import wan_oracle as O
-    from wan_inputs import sample_rows
-    rows = sample_rows(w.tokens, count=S, seed=seed)
+    lat, t, ctx, img = _oracle_inputs(w, inp)
     t0 = time.perf_counter()
-    O.dit_block(x, e, inp["blocks"][0], inp["ctx"][0], w.heads, rows=rows)
+    O.dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads, img_ctx=img)
     return time.perf_counter() - t0
 
 
-def oracle_calibrate(w, inp, s_small=128, s_big=512):
-    """Time the CPU oracle on a bounded sample of one step: patchify and the timestep MLP
-    on all tokens, then the block for two query-row sample sizes. Returns
-    (t_prefix, fixed, per_row, seconds_spent): the full block is fixed + per_row * L."""
+def oracle_row_model(w, inp, s_small=64, s_big=256):
+    """Cross-check only (also the CPU warm-up): the block on two sampled query-row counts
+    (keys and values over all rows), fitted as fixed + per_row * rows and extended to all
+    L rows. Returns (model seconds per step, seconds spent)."""
+    from oracle import wan_oracle as O
+    from wan_inputs import sample_rows
+    lat, t, ctx, img = _oracle_inputs(w, inp)
     t0 = time.perf_counter()
-    x, e = _oracle_prefix(inp)
+    x = O.patchify(lat, inp["w_p"], inp["b_p"])
+    e = O.time_mlp(t, inp["w_t1"], inp["b_t1"], inp["w_t2"], inp["b_t2"])
     t_pre = time.perf_counter() - t0
-    ta = _oracle_rows(w, inp, x, e, s_small)
-    tb = _oracle_rows(w, inp, x, e, s_big)
-    per_row = max((tb - ta) / (s_big - s_small), 1e-9)
-    fixed = max(ta - per_row * s_small, 0.0)
-    return t_pre, fixed, per_row, time.perf_counter() - t0, (x, e)
+    ts = []
+    for S in (s_small, s_big):
+        rows = sample_rows(w.tokens, count=S, seed=1)
+        t1 = time.perf_counter()
+        for blk in inp["blocks"]:
+            O.dit_block(x, e, blk, ctx, w.heads, img_ctx=img, rows=rows)
+        ts.append(time.perf_counter() - t1)
+    per_row = max((ts[1] - ts[0]) / (s_big - s_small), 0.0)
+    fixed = max(ts[0] - per_row * s_small, 0.0)
+    return t_pre + fixed + per_row * w.tokens, time.perf_counter() - t0
 
 
-def oracle_sample(w, inp, s_small=128, s_big=512):
-    t_pre, fixed, per_row, spent, _ = oracle_calibrate(w, inp, s_small, s_big)
-    t_full = t_pre + fixed + per_row * w.tokens
-    desc = (f"fp64 numpy oracle: patchify + timestep MLP on all {w.tokens} tokens, then the block for "
-            f"{s_small} and {s_big} sampled query rows (K/V over all rows each time); the full-block time is "
-            f"extrapolated linearly in query rows: {t_full:.1f} s per step")
-    return w.tokens * w.batch / t_full, spent, desc
+def oracle_measure(w, inp):
+    """The CPU baseline: warm-up and per-row cross-check, then the oracle timed over one
+    whole step of the workload. Returns (tokens/s, step seconds, description, model seconds)."""
+    model_s, _ = oracle_row_model(w, inp)
+    step_s = oracle_step_seconds(w, inp)
+    desc = (f"fp64 numpy oracle timed over one whole step of {w.name} ({w.n_blocks} block(s) on all "
+            f"{w.tokens} tokens, patchify, timestep MLP and head): {step_s:.1f} s; warm-up: the block on 64 and "
+            f"256 sampled query rows, whose linear per-row model predicts {model_s:.1f} s (cross-check only)")
+    return w.tokens * w.batch / step_s, step_s, desc, model_s
 
 
 def run_reference(args, w):
-    """The oracle arm. Warm-up calibrates the per-row cost of the oracle; each timed step
-    evaluates the block on one bounded sample of query rows (keys and values over all
-    rows) and extrapolates its measured time to all L rows with that per-row cost."""
+    """The oracle arm. The fp64 oracle is the slow program on the host cores; one of its
+    steps at the 1.3B 480P shape takes on the order of 100 s, so the arm times ONE whole
+    step (the same work as one GPU step) after a bounded warm-up, and says so: its
+    ``steps`` is 1 whatever ``--steps`` asks for."""
     from wan_inputs import make_inputs
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    inp = make_inputs(w, seed=0, n_blocks=1, block_input=False)
-    t_pre, fixed, per_row, _, (x, e) = oracle_calibrate(w, inp, 64, 256)
-    for _ in range(max(args.warmup - 1, 0)):
-        _oracle_rows(w, inp, x, e, 64)
-    S = 64
-    vals = []
-    for i in range(args.steps):
-        t0 = time.perf_counter()
-        x, e = _oracle_prefix(inp)
-        ts = time.perf_counter() - t0 + _oracle_rows(w, inp, x, e, S, seed=100 + i)
-        vals.append(w.tokens * w.batch / (ts + per_row * (w.tokens - S)))
-    value = statistics.median(vals)
+    inp = make_inputs(w, seed=0, block_input=False)
+    value, step_s, desc, model_s = oracle_measure(w, inp)
     cores = blas_threads()
-    desc = (f"fp64 numpy oracle per step: patchify + timestep MLP on all tokens and the block for {S} sampled "
-            f"query rows (K/V over all rows); the remaining rows are added at the per-row cost calibrated in "
-            f"warm-up ({per_row * 1e3:.2f} ms/row)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.tokens * w.batch / value,
+        "steps": 1, "steps_requested": args.steps, "warmup": 1, "warmup_requested": args.warmup,
+        "ms_per_step": 1000.0 * step_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "tokens": w.tokens, "dim": w.dim, "heads": w.heads,
-                   "ffn": w.ffn, "text_tokens": w.text_len, "blocks": 1, "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+                   "ffn": w.ffn, "text_tokens": w.text_len, "image_tokens": w.img_len, "blocks": w.n_blocks,
+                   "parallelism": "replicas"},
+        "note": "one whole oracle step timed (about 100 s at this shape); the requested step count is not run",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                         "model_seconds": round(model_s, 1)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def choose_peak(peaks, peak_src, region_s):
+    """The bf16 denominator for kernels timed inside a region of ``region_s`` seconds:
+    the burst figure for a region under 1 s (the GPU does not reach its power-capped
+    steady state in that time), the sustained one otherwise."""
+    burst = region_s < 1.0
+    key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    return {"value": peaks[key], "hbm_gbs": peaks["hbm_gbs"],
+            "source": f"{peak_src} {key} ({'burst' if burst else 'sustained'}: timed region {region_s:.2f} s)"}
+
+
+def kernel_report(w, recs, steps, ms_step, clocks):
+    """Per-kernel durations and roofline fractions from the per-launch trace of ``steps``
+    steps. In each step the first GEMM is the patchify projection and the last the head
+    (both HBM-bound; algorithmic bytes = operands read once + output written once); the
+    attention launch with the most work is the self-attention, the others are
+    cross-attention; LayerNorm work is its algorithmic bytes."""
+    import video_diffusion_transformer_wan_b200 as wan
+    peaks, peak_src = load_peaks()
+    peak = choose_peak(peaks, peak_src, ms_step * steps / 1e3)
+    n = len(recs)
+    per = n // steps if steps and n % steps == 0 else None
+    if not per:
+        raise RuntimeError(f"trace holds {n} launches, not a multiple of {steps} steps")
+    B, L, D = w.batch, w.tokens, w.dim
+    K = w.in_ch * 4
+    patch_bytes = B * L * K * 2 + D * K * 2 + D * 2 + B * L * D * 4
+    head_bytes = B * L * D * 2 + w.out_ch * 4 * D * 2 + w.out_ch * 4 * 2 + B * L * w.out_ch * 4 * 4
+    acc = {k: [0.0, 0.0] for k in ["self_attention", "cross_attention", "gemm", "patchify_gemm", "head_gemm",
+                                   "layernorm", "small"]}
+    top = max(wk for k, _, wk in recs if k == wan.KIND_ATTN)
+    for i in range(steps):
+        chunk = recs[i * per:(i + 1) * per]
+        gi = [j for j, (k, _, _) in enumerate(chunk) if k == wan.KIND_GEMM]
+        for j, (k, ms, wk) in enumerate(chunk):
+            if k == wan.KIND_ATTN:
+                name = "self_attention" if wk == top else "cross_attention"
+            elif k == wan.KIND_GEMM:
+                name = "patchify_gemm" if j == gi[0] else "head_gemm" if j == gi[-1] else "gemm"
+                if name != "gemm":
+                    wk = patch_bytes if name == "patchify_gemm" else head_bytes
+            elif k == wan.KIND_NORM:
+                name = "layernorm"
+            else:
+                name = "small"
+            acc[name][0] += ms
+            acc[name][1] += wk
+    mhz = clocks.get("sm_mhz")
+    out = {}
+    for name, (ms, wk) in acc.items():
+        d = {"ms_per_step": ms / steps}
+        if name in ("self_attention", "cross_attention", "gemm") and ms > 0:
+            d.update({"tflops": wk / (ms / 1e3) / 1e12, "bound": "tensor"})
+            d["frac"] = d["tflops"] / peak["value"]
+        elif name in ("patchify_gemm", "head_gemm", "layernorm") and ms > 0:
+            d.update({"gbs": wk / (ms / 1e3) / 1e9, "bound": "hbm"})
+            d["frac"] = d["gbs"] / peak["hbm_gbs"]
+        d["sm_mhz"] = mhz
+        out[name] = d
+    out["peaks"] = {"bf16_tflops": peak["value"], "bf16_source": peak["source"], "hbm_gbs": peak["hbm_gbs"],
+                    "hbm_source": f"{peak_src} hbm_gbs"}
+    sa_ms = acc["self_attention"][0] / steps
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_tc_kernel (self-attention)",
+                "achieved": top / (sa_ms / 1e3) / 1e12, "peak": peak["value"], "unit": "TFLOP/s",
+                "frac": top / (sa_ms / 1e3) / 1e12 / peak["value"], "peak_source": peak["source"],
+                "sm_mhz": mhz, "work_per_launch": top, "ms_per_launch": sa_ms,
+                "traffic": attn_traffic_per_launch()}
+    return out, roofline, peak
 
 
 def main():
@@ -297,10 +378,8 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {wan.status_string(status)} after warm-up")
 
-    # ---------------- device-resident timed region (inputs already in HBM)
+    # ---------------- device-resident timed region (inputs already in HBM), untraced
     sampler = ClockSampler(local)
-    wan.trace_reset()
-    wan.trace_enable(True)
     launches0 = wan.launch_count()
     barrier()
     torch.cuda.synchronize()
@@ -316,26 +395,32 @@ def main():
     barrier()
     launches = wan.launch_count() - launches0
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
-    recs = wan.trace_launches()
-    wan.trace_enable(False)
     ms_step = ms_total / args.steps
     tokens_step = B * L
     value = replica_throughput(world, tokens_step, ms_step)
     flops = step_flops(w)
 
-    # dominant kernel: the self-attention launch (largest attention work per step)
-    attn = [(ms, work) for k, ms, work in recs if k == wan.KIND_ATTN]
-    top = max(wk for _, wk in attn)
-    self_attn = [(ms, wk) for ms, wk in attn if wk == top]
-    attn_ms = statistics.mean(ms for ms, _ in self_attn)
-    peaks, peak_src = load_peaks()
-    achieved = top / (attn_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    kind_ms = {}
-    for k, ms, _ in recs:
-        kind_ms[k] = kind_ms.get(k, 0.0) + ms
-    gemm_work = sum(wk for k, _, wk in recs if k == wan.KIND_GEMM)
-    norm = [(ms, wk) for k, ms, wk in recs if k == wan.KIND_NORM]
+    # ---------------- the same K steps again with the per-launch trace (CUDA events
+    # around every launch on the launch stream): per-kernel durations
+    sampler_t = ClockSampler(local)
+    wan.trace_reset()
+    wan.trace_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    sampler_t.start()
+    time.sleep(0.1)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record(stream)
+    for _ in range(args.steps):
+        step()
+    e5.record(stream)
+    torch.cuda.synchronize()
+    clocks_traced = sampler_t.stop()
+    barrier()
+    traced_ms_step = e4.elapsed_time(e5) / args.steps
+    recs = wan.trace_launches()
+    wan.trace_enable(False)
+    kernels, roofline, peak = kernel_report(w, recs, args.steps, traced_ms_step, clocks_traced)
 
     # ---------------- end to end through the C ABI with host buffers
     # Every step copies its inputs from pinned host memory and its velocity back. Two
@@ -396,9 +481,9 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_cpu, spent, desc = oracle_sample(w, inp)
+        v_cpu, step_s, desc, model_s = oracle_measure(w, inp)
         cpu = {"value": v_cpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc,
-               "seconds": round(spent, 1)}
+               "seconds": round(step_s, 1), "model_seconds": round(model_s, 1)}
 
     if rank == 0:
         line = {
@@ -413,24 +498,17 @@ def main():
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2 (per-step working set > 1 GB of activations)"},
             "tflops": flops / (ms_step / 1e3) / 1e12 * world,
-            "pct_bf16_peak": flops / (ms_step / 1e3) / 1e12 / peak,
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_tc_kernel (self-attention)",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained",
-                         "work_per_launch": top, "ms_per_launch": attn_ms,
-                         "traffic": attn_traffic_per_launch()},
-            "kernels_ms_per_step": {
-                "attention": kind_ms.get(wan.KIND_ATTN, 0.0) / args.steps,
-                "gemm": kind_ms.get(wan.KIND_GEMM, 0.0) / args.steps,
-                "layernorm": kind_ms.get(wan.KIND_NORM, 0.0) / args.steps,
-                "small": kind_ms.get(wan.KIND_SMALL, 0.0) / args.steps},
-            "gemm_tflops": gemm_work / (kind_ms.get(wan.KIND_GEMM, 1e-9) / 1e3) / 1e12,
-            "layernorm_gbs": (sum(wk for _, wk in norm) / (sum(ms for ms, _ in norm) / 1e3) / 1e9) if norm else None,
-            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "pct_bf16_peak": flops / (ms_step / 1e3) / 1e12 / peak["value"],
+            "pct_bf16_peak_basis": peak["source"],
+            "roofline": roofline,
+            "kernels": kernels,
+            "traced_ms_per_step": traced_ms_step,
+            "hbm_peak_gbs": peak["hbm_gbs"],
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": launches,
             "clocks": clocks,
+            "clocks_traced": clocks_traced,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

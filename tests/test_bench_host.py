@@ -60,3 +60,38 @@ def test_clock_sampler_parses_nvidia_smi_lines(bench):
 def test_peaks_source(bench):
     peaks, src = bench.load_peaks()
     assert peaks["bf16_tflops_sustained"] > 0 and src in ("measured", "fallback")
+
+
+def test_peak_rule_burst_for_short_regions(bench):
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    assert bench.choose_peak(peaks, "measured", 0.17)["value"] == 1600.0
+    assert bench.choose_peak(peaks, "measured", 2.5)["value"] == 1400.0
+    assert "burst" in bench.choose_peak(peaks, "measured", 0.5)["source"]
+
+
+def test_kernel_report_splits_a_step(bench):
+    """A synthetic trace of two steps in the launch order of wan_dit_stack_fwd with one
+    block: gather, patchify GEMM, time MLP, LN, QKV, self-attention, O, LN, cross q,
+    cross kv, cross-attention, cross o, LN, FFN1, FFN2, head LN, head GEMM."""
+    import video_diffusion_transformer_wan_b200 as wan
+    w = WORKLOADS["wan13b_480p_block"]
+    S, G, A, N = wan.KIND_SMALL, wan.KIND_GEMM, wan.KIND_ATTN, wan.KIND_NORM
+    sa, ca = 6.594e12, 0.103e12
+    step = [(S, 0.01, 1e6), (G, 0.05, 6.4e9), (S, 0.01, 1e6), (N, 0.05, 3e8), (G, 0.4, 4.6e11), (A, 5.5, sa),
+            (G, 0.15, 1.5e11), (N, 0.05, 3e8), (G, 0.13, 1.5e11), (G, 0.01, 4e9), (A, 0.2, ca), (G, 0.15, 1.5e11),
+            (N, 0.05, 3e8), (G, 0.7, 9e11), (G, 0.7, 9e11), (N, 0.05, 3e8), (G, 0.03, 6.4e9)]
+    recs = step * 2
+    k, roof, peak = bench.kernel_report(w, recs, 2, 8.5, {"sm_mhz": 1900})
+    assert k["self_attention"]["ms_per_step"] == pytest.approx(5.5)
+    assert roof["achieved"] == pytest.approx(sa / 5.5e-3 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / peak["value"])
+    assert k["cross_attention"]["tflops"] == pytest.approx(ca / 0.2e-3 / 1e12)
+    assert k["patchify_gemm"]["ms_per_step"] == pytest.approx(0.05)
+    assert k["head_gemm"]["ms_per_step"] == pytest.approx(0.03)
+    L, D = w.tokens, w.dim
+    assert k["patchify_gemm"]["gbs"] == pytest.approx((L * 64 * 2 + D * 64 * 2 + D * 2 + L * D * 4) / 0.05e-3 / 1e9)
+    assert k["head_gemm"]["gbs"] == pytest.approx((L * D * 2 + 64 * D * 2 + 64 * 2 + L * 64 * 4) / 0.03e-3 / 1e9)
+    assert k["gemm"]["ms_per_step"] == pytest.approx(0.4 + 0.15 + 0.13 + 0.01 + 0.15 + 0.7 + 0.7)
+    assert k["layernorm"]["gbs"] == pytest.approx(4 * 3e8 / 0.2e-3 / 1e9)
+    with pytest.raises(RuntimeError):
+        bench.kernel_report(w, recs[:-1], 2, 8.5, {"sm_mhz": 1900})
