@@ -2,16 +2,19 @@
 (``wan_dit_stack_fwd``): 256 sampled query rows (rows 0 and L-1 and the whole ragged
 last tile included) are compared with the oracle, which evaluates exactly those rows
 (keys and values over all rows). Everything but self-attention is row-local, so this
-is exact. The 30-block stack is checked at reduced token count with full-width
-blocks, and at full size through properties that hold at any size."""
+is exact. The 30-block stack is checked at full size against the oracle's velocity of
+256 sampled tokens (stored by a committed script that calls only the oracle), at
+reduced token count with full-width blocks, and at full size through properties that
+hold at any size."""
 import dataclasses
+import os
 
 import numpy as np
 import pytest
 
 from oracle import wan_oracle as O
-from wan_inputs import WORKLOADS, make_inputs, sample_rows
-from gpu_util import BF16_TOL, rel_err
+from wan_inputs import WORKLOADS, input_digest, make_inputs, sample_rows
+from gpu_util import BF16_TOL, rel_err, rms_err
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -149,13 +152,52 @@ def test_stack30_reduced_tokens_matches_oracle(wan):
     assert abs(float(loss[0]) - ref_loss) / ref_loss < 2e-2
 
 
-def test_stack30_full_size_properties(wan):
+GOLDEN_STACK30 = os.path.join(os.path.dirname(__file__), "golden", "wan13b_480p_stack30_seed0_velocity_rows.npz")
+
+
+@pytest.fixture(scope="module")
+def stack30_inputs():
+    return make_inputs(WORKLOADS["wan13b_480p_stack30"], seed=0, block_input=False)
+
+
+def test_stack30_full_size_matches_stored_oracle_velocity(wan, stack30_inputs):
+    """The 30-block 1.3B stack at 480P, 81 frames (32760 tokens) with one rectified-flow
+    velocity evaluation, through flow_matching_input and wan_dit_stack_fwd, against the
+    oracle's velocity of the 256 sampled tokens (rows 0 and L-1 and the ragged last tile
+    included), written by tests/golden/make_stack30_velocity.py (float32 products,
+    float64 reductions: ~1e-6 from the float64 definition)."""
+    g = np.load(GOLDEN_STACK30)
+    w = WORKLOADS["wan13b_480p_stack30"]
+    inp = stack30_inputs
+    assert str(g["digest"]) == input_digest(inp), "input recipe changed: regenerate the stored velocity"
+    rows = sample_rows(w.tokens)
+    assert np.array_equal(g["rows"], rows)
+    cfg, model, lat, ctx, img_ctx, keep, ws = _setup(wan, w, inp)
+    from video_diffusion_transformer_wan_b200.model import to_device
+    x1 = to_device(inp["x1"], model.act)
+    u = torch.from_numpy(inp["u"]).cuda()
+    xt = torch.empty_like(x1)
+    t = torch.empty(w.batch, dtype=torch.float32, device="cuda")
+    wan.flow_matching_input(cfg, x1, lat, u, xt, t)
+    v = torch.empty(w.batch, 16, w.frames, w.height, w.width, dtype=torch.float32, device="cuda")
+    wan.dit_stack_fwd(cfg, xt, t, model.stack_table, model.block_tables, ctx, None, v, ws)
+    torch.cuda.synchronize()
+    assert wan.device_status() == 0
+    got = _token_values(v[0].cpu().numpy(), rows, w)
+    del model, ws
+    torch.cuda.empty_cache()
+    err, rms = rel_err(got, g["values"]), rms_err(got, g["values"])
+    print(f"stack30 at {w.tokens} tokens, 30 blocks: max rel err {err:.3e}, rms {rms:.3e}")
+    assert err <= BF16_TOL
+
+
+def test_stack30_full_size_properties(wan, stack30_inputs):
     """Full-size 30-block stack: (1) with every block's weights zero, each block is the
     identity and the output is head(LN(patchify)) - row-local, so the oracle checks it
     on sampled tokens; (2) the stack with real weights equals 30 consecutive block calls
     between a patchify/timestep-MLP call and the head call, bitwise."""
     w = WORKLOADS["wan13b_480p_stack30"]
-    inp = make_inputs(w, seed=0, block_input=False)
+    inp = stack30_inputs
     cfg, model, lat, ctx, img_ctx, keep, ws = _setup(wan, w, inp)
     B, F, H, W, L, D = w.batch, w.frames, w.height, w.width, w.tokens, w.dim
     t = torch.from_numpy((1000.0 * inp["u"]).astype(np.float32)).cuda()
