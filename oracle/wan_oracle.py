@@ -549,7 +549,8 @@ def linear_fp8(x, weight, bias=None) -> np.ndarray:
     return y if bias is None else y + _f(bias)
 
 
-def attention_fp8(q, k, v, heads: int) -> np.ndarray:
+def attention_fp8(q, k, v, heads: int, running_base: bool = False, split_units=(), rows=None,
+                  prob=None) -> np.ndarray:
     """8-bit attention [Wan-P2, "Infra", inference optimisation: 8-bit FlashAttention,
     INT8 for q k^T and FP8 for the product with v]. reading: E4M3 for both products (the
     8-bit format of the tensor cores' f8 kind), with these scales, each an amax / 448
@@ -566,19 +567,99 @@ def attention_fp8(q, k, v, heads: int) -> np.ndarray:
       two base makes the rounding of p the same for any base a whole power of two
       away, which a one-pass kernel with a running base can reproduce.)
 
-    Per head: ``x = (q^ k^T) sq sk / (sqrt(d) ln 2)``, ``o = sv (E4M3(p) v^) / sum_j p``."""
+    Per head: ``x = (q^ k^T) sq sk / (sqrt(d) ln 2)``, ``o = sv (E4M3(p) v^) / sum_j p``.
+
+    ``running_base`` takes the base the way a one-pass kernel meets the keys instead of
+    from the row's final maximum (``_running_base_rows``); the two agree exactly unless
+    some p falls into E4M3's subnormal range under one base and not the other.
+    ``split_units``: (head, query block) pairs whose keys a kernel took in two halves
+    (query blocks of 256 rows). ``rows`` returns only those query rows (q still holds
+    every row: under the running base a row's result depends on its 32-row group).
+    ``prob`` (running base only): ``prob(S, c, base, first_key)`` evaluates a key tile's
+    probabilities ``2^(S c - base)``; by default exactly, in float64. A caller may pass a
+    model of some other arithmetic to study its effect."""
     q, k, v = (np.asarray(a, dtype=np.float32) for a in (q, k, v))
     Lq, D = q.shape
     d = D // heads
-    out = np.empty((Lq, D), dtype=F64)
+    sel = np.arange(Lq) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((len(sel), D), dtype=F64)
     for hh in range(heads):
         sl = slice(hh * d, (hh + 1) * d)
-        qq, sq = quantize_e4m3(q[:, sl], axis=-1)
         kq, sk = quantize_e4m3(k[:, sl])
         vq, sv = quantize_e4m3(v[:, sl])
+        if running_base:
+            qq, sq = quantize_e4m3(q[:, sl], axis=-1)
+            c = sq.astype(F64) * F64(sk) / (math.sqrt(d) * math.log(2.0))   # log2 units per unit of S
+            split = {qb for (h2, qb) in split_units if h2 == hh}
+            out[:, sl] = F64(sv) * _running_base_rows(qq, c, kq, vq, split, sel, prob=prob)
+            continue
+        qq, sq = quantize_e4m3(q[sel][:, sl], axis=-1)
         x = (qq @ kq.T) * sq.astype(F64) * F64(sk) / (math.sqrt(d) * math.log(2.0))
         p = np.exp2(x - np.ceil(x.max(axis=-1, keepdims=True)))
         out[:, sl] = F64(sv) * (round_e4m3(p) @ vq) / p.sum(axis=-1, keepdims=True)
+    return out
+
+
+def _running_base_rows(qq, c, kq, vq, split_blocks, rows, tile: int = 128, warp: int = 32, block: int = 256,
+                       threshold: float = 8.0, prob=None) -> np.ndarray:
+    """The rows ``rows`` of one head of ``attention_fp8`` with the base a one-pass kernel
+    keeps. ``qq`` [Lq, d] and ``kq``, ``vq`` [Lk, d] are E4M3 values, ``c`` [Lq, 1] the
+    log2 units of one unit of ``S = qq kq^T`` (exact). The keys come in tiles of ``tile``
+    in order; a row's running maximum m of S starts at its first tile's maximum and
+    moves to max(m, tile maximum) only when, for some row of its group of ``warp``
+    consecutive rows (groups from row 0), the tile maximum exceeds m by more than
+    ``threshold`` in log2 units -- then every row of the group moves; each tile's p is
+    taken against ``ceil(m c)``, and what was summed before a move is scaled by the exact
+    power of two between the old and the new base. Query blocks in ``split_blocks``
+    (rows [256 b, 256 b + 256)) take their keys in two halves of the key tiles (the
+    first floor(n/2) tiles, then the rest), each half with its own running base, merged
+    as ``(w0 O0 + w1 O1) / (w0 l0 + w1 l1)`` with ``w_i = 2^(b_i - max(b0, b1))``.
+    Returns the normalised ``E4M3(p) v^`` of those rows (without the v scale). ``prob``
+    as in ``attention_fp8``."""
+    Lq, Lk = qq.shape[0], kq.shape[0]
+    if prob is None:
+        def prob(St, cr, base, first_key):
+            return np.exp2(St * cr - base)
+    ntile = (Lk + tile - 1) // tile
+
+    def one_pass(S, cr, t0, t1):
+        # one group of rows over key tiles [t0, t1): (base, unnormalised output, sum)
+        m = None
+        o = np.zeros((S.shape[0], vq.shape[1]), dtype=F64)
+        l = np.zeros((S.shape[0], 1), dtype=F64)
+        for j in range(t0, t1):
+            St = S[:, j * tile:min((j + 1) * tile, Lk)]
+            mx = St.max(axis=-1, keepdims=True)
+            if m is None:
+                m = mx.copy()
+            elif ((mx - m) * cr > threshold).any():
+                m_new = np.maximum(m, mx)
+                alpha = np.exp2(np.ceil(m * cr) - np.ceil(m_new * cr))
+                o *= alpha
+                l *= alpha
+                m = m_new
+            p = prob(St, cr, np.ceil(m * cr), j * tile)
+            o += round_e4m3(p) @ vq[j * tile:j * tile + St.shape[1]]
+            l += p.sum(axis=-1, keepdims=True)
+        return np.ceil(m * cr), o, l
+
+    out = np.empty((len(rows), vq.shape[1]), dtype=F64)
+    where = {}
+    for i, r in enumerate(rows):
+        where.setdefault(int(r) // warp * warp, []).append(i)
+    for w0, idx in where.items():
+        w1 = min(w0 + warp, Lq)
+        S, cr = qq[w0:w1] @ kq.T, c[w0:w1]
+        if w0 // block in split_blocks:
+            b0, o0, l0 = one_pass(S, cr, 0, ntile // 2)
+            b1, o1, l1 = one_pass(S, cr, ntile // 2, ntile)
+            bm = np.maximum(b0, b1)
+            g0, g1 = np.exp2(b0 - bm), np.exp2(b1 - bm)
+            res = (g0 * o0 + g1 * o1) / (g0 * l0 + g1 * l1)
+        else:
+            _, o, l = one_pass(S, cr, 0, ntile)
+            res = o / l
+        out[idx] = res[np.asarray(rows)[idx] - w0]
     return out
 
 

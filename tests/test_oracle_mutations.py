@@ -289,3 +289,32 @@ def test_f32_stack_mutations_are_caught():
         return out if rows is None else np.roll(out, 1, axis=0)   # rows returned out of order
     _fails(P.check_stack_f32, ungated_ffn)
     _fails(P.check_stack_f32, last_block_all_rows)
+
+
+def _mutated(fn, old, new):
+    """A copy of oracle function ``fn`` with one source line changed."""
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(fn))
+    assert old in src, old
+    ns = dict(vars(O))
+    exec(src.replace(old, new, 1), ns)
+    return ns[fn.__name__]
+
+
+def test_attention_fp8_running_base_mutations_are_caught(monkeypatch):
+    import functools
+    base = O._running_base_rows
+    mutants = [
+        functools.partial(base, warp=1),                  # each row decides alone
+        functools.partial(base, threshold=6.0),           # moves too early
+        functools.partial(base, block=128),               # key split over 128-row blocks
+        _mutated(base, "o *= alpha", "pass"),                                    # output not rescaled
+        _mutated(base, "g0, g1 = np.exp2(b0 - bm), np.exp2(b1 - bm)", "g0, g1 = 1.0, 1.0"),  # halves summed
+        _mutated(base, "p = prob(St, cr, np.ceil(m * cr), j * tile)", "p = prob(St, cr, m * cr, j * tile)"),  # unrounded base
+    ]
+    for mut in mutants:
+        monkeypatch.setattr(O, "_running_base_rows", mut)
+        _fails(P.check_attention_fp8_running_base, O.attention_fp8)
+    monkeypatch.setattr(O, "_running_base_rows", base)
+    P.check_attention_fp8_running_base(O.attention_fp8)

@@ -830,3 +830,61 @@ def check_attention_fp8(attention_fp8):
 
 def test_attention_fp8_pins():
     check_attention_fp8(O.attention_fp8)
+
+
+def check_attention_fp8_running_base(attn):
+    """The running-base option of ``attention_fp8`` (the base a one-pass kernel keeps).
+
+    (1) Where every p stays in E4M3's normal range under both bases, the codes differ
+    only by exact powers of two, so the option equals the definition (whole and with
+    key-split query blocks) to rounding of float64 sums.
+    (2) A hand-built case whose base trajectory is known: one head (d = 128), keys in two
+    128-key tiles. Every query and key has one non-zero component, so logit (log2 units)
+    = alpha_r * k_j with k on the E4M3 grid (k scale 1/16). Tile 0: all k = 0 (p = 1 for
+    every row). Tile 1: a jump key k = 28, a key k = -20 whose value is e_0, and k = 0
+    elsewhere; key 0 (tile 0) has value e_1; the other values are zero.
+    Row 0 (alpha 0.5) jumps by 14 > 8 in tile 1, so its warp (rows 0-31) moves: row 1
+    (alpha 0.23, own jump 6.44 < 8) takes base ceil(6.44) = 7 and its p for the k = -20
+    key, 2^(-4.6 - 7), rounds to zero: out[1, 0] = 0. Row 32 (the same alpha, the next
+    warp, where nothing jumps; likewise row 160) keeps base 0, so that p is 2^-4.6 -> 11 * 2^-8:
+    out[32, 0] = 11 * 2^-8 / l with l = 254 + 2^6.44 + 2^-4.6. Row 0 moved to base 14, so
+    its tile-0 sum is scaled by 2^-14: out[0, 1] = 2^-14 / (1 + 254 * 2^-14 + 2^-24).
+    With the query block split in two key halves (tile 0 | tile 1), row 32's second
+    half starts at base 7: out[32, 0] = out[160, 0] = 0 and out[32, 1] = 2^-7 / (2^-7 * 128 + l1),
+    l1 = 2^(6.44 - 7) + 126 * 2^-7 + 2^(-4.6 - 7)."""
+    rng = RNG(52)
+    for std, Lq, Lk, H in [(0.3, 300, 900, 2), (0.25, 70, 2100, 1)]:
+        q = round_bf16(rng.standard_normal((Lq, H * 128)) * math.sqrt(std))
+        k = round_bf16(rng.standard_normal((Lk, H * 128)) * math.sqrt(std))
+        v = round_bf16(rng.standard_normal((Lk, H * 128)))
+        ref = O.attention_fp8(q, k, v, H)
+        for split in ((), [(0, 0)], [(h, b) for h in range(H) for b in range((Lq + 255) // 256)]):
+            got = attn(q, k, v, H, running_base=True, split_units=split)
+            assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max(), split
+    a = math.sqrt(128) * math.log(2.0)
+    q = np.zeros((192, 128))
+    q[0, 0], q[1, 0], q[32, 0], q[160, 0] = 0.5 * a, 0.23 * a, 0.23 * a, 0.23 * a
+    k = np.zeros((256, 128))
+    k[128, 0], k[129, 0] = 28.0, -20.0
+    v = np.zeros((256, 128))
+    v[129, 0], v[0, 1] = 1.0, 1.0
+    out = attn(q, k, v, 1, running_base=True)
+    l32 = 254 + 2 ** 6.44 + 2 ** -4.6
+    assert out[1, 0] == 0.0
+    np.testing.assert_allclose(out[32, 0], 11 * 2.0 ** -8 / l32, rtol=1e-6)
+    np.testing.assert_allclose(out[0, 1], 2.0 ** -14 / (1 + 254 * 2.0 ** -14 + 2.0 ** -24), rtol=1e-6)
+    out = attn(q, k, v, 1, running_base=True, split_units=[(0, 0)])
+    l1 = 2 ** (6.44 - 7) + 126 * 2.0 ** -7 + 2 ** (-4.6 - 7)
+    assert out[32, 0] == 0.0 and out[160, 0] == 0.0          # row 160 is in the same 256-row block
+    np.testing.assert_allclose(out[32, 1], 2.0 ** -7 / (2.0 ** -7 * 128 + l1), rtol=1e-6)
+    # the definition (final row maximum) gives zero for both rows' k = -20 key
+    ref = O.attention_fp8(q, k, v, 1)
+    assert ref[1, 0] == 0.0 and ref[32, 0] == 0.0
+    # a subset of rows is the same as those rows of the whole result
+    rows = np.array([0, 1, 33, 160, 191])
+    sub = attn(q, k, v, 1, running_base=True, split_units=[(0, 0)], rows=rows)
+    np.testing.assert_array_equal(sub, out[rows])
+
+
+def test_attention_fp8_running_base_pins():
+    check_attention_fp8_running_base(O.attention_fp8)
