@@ -1,0 +1,315 @@
+"""Derivation of the FP8 parity bars of the GPU tests (the FP8_* values in gpu_util).
+
+The Wan 2.1 page ("Wan: Open and Advanced Large-Scale Video Generative Models", section
+"Infra", inference optimisation) runs FP8 GEMMs and an 8-bit FlashAttention but states no
+accuracy; these bars come from the oracle alone. The GPU computes the inputs of its E4M3
+quantisers -- the attention outputs, the FFN hidden layer and, for the 8-bit attention,
+q, k and v -- as bf16 tensors whose values differ from the oracle's float64 ones by about
+one bf16 rounding step (2^-9 relative). E4M3 codes are 2^-3 apart, so such a difference
+moves a code with probability ~1/64, and then by a whole code. The study therefore moves
+exactly those tensors in the oracle by +-2^-9 (independent random signs) and measures how
+far the FP8 result moves, max-norm (max|d| / max|ref|) and RMS; the 8-bit attention also
+takes the one-pass kernel's running base (``attention_fp8(running_base=True)``), and in the
+sampling loop the DiT input is rounded to bf16 at every step, as the GPU's is. A bar is
+1.5x the worst case over the trials, rounded up to two significant digits.
+
+FP8_ATTN_TOL compares the oracle's running-base option with its definition (the base from
+the row's final maximum): they differ only where some p falls into E4M3's subnormal
+range under one base and not the other. FP8_ATTN_RB_TOL, the bar of the kernel against the
+running-base option, models the kernel's own arithmetic there (``kernel_prob_model``:
+float32 scores and exponent, the polynomial 2^x on one key in eight within its stated
+error bound, the bf16 output) on the tests' own inputs: a flipped E4M3 rounding of one of
+the few large probabilities of a peaked row moves that row.
+
+Calls only the oracle and the seeded input generator. ``python tests/fp8_tolerance_study.py``
+runs the reduced form (a minute or two); ``--full`` adds the 1.3B 480P block on 256
+sampled rows and 32760- and 75600-key attention (about an hour on 8 host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import math
+import os
+import sys
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(HERE))
+sys.path.insert(0, HERE)
+
+from oracle import wan_oracle as O  # noqa: E402
+from wan_inputs import WORKLOADS, make_inputs, round_bf16, sample_rows  # noqa: E402
+
+STEP = 2.0 ** -9
+
+
+def rel_max(got, ref) -> float:
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    return float(np.abs(got - ref).max() / np.abs(ref).max())
+
+
+def rel_rms(got, ref) -> float:
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    return float(np.sqrt(np.mean((got - ref) ** 2) / np.mean(ref ** 2)))
+
+
+def bar(worst: float) -> float:
+    """1.5x ``worst``, rounded up to two significant digits."""
+    v = 1.5 * worst
+    e = math.floor(math.log10(v)) - 1
+    return math.ceil(v / 10.0 ** e - 1e-9) * 10.0 ** e
+
+
+class QuantiserInputsMoved:
+    """Inside the context the oracle's ``attention`` and ``gelu_tanh`` outputs and the
+    8-bit attention's q, k, v and output are each moved by +-2^-9 (relative, random signs
+    from ``seed``), and the 8-bit attention takes the running base."""
+
+    def __init__(self, seed: int, bf16_dit_input: bool = False):
+        self.r = np.random.Generator(np.random.PCG64(seed))
+        self.bf16_dit_input = bf16_dit_input
+
+    def move(self, a):
+        a = np.asarray(a, np.float64)
+        return a * (1.0 + STEP * self.r.choice([-1.0, 1.0], size=a.shape))
+
+    def __enter__(self):
+        self.saved = O.attention, O.gelu_tanh, O.attention_fp8, O.dit_stack
+        attn, gelu, a8, stack = self.saved
+        O.attention = lambda q, k, v, h: self.move(attn(q, k, v, h))
+        O.gelu_tanh = lambda z: self.move(gelu(z))
+        O.attention_fp8 = lambda q, k, v, h: self.move(a8(self.move(q), self.move(k), self.move(v), h,
+                                                          running_base=True))
+        if self.bf16_dit_input:
+            # the sampling loop's DiT input is its float32 state rounded to bf16 each step
+            O.dit_stack = lambda latent, *a, **kw: stack(round_bf16(np.asarray(latent, np.float32)), *a, **kw)
+        return self
+
+    def __exit__(self, *exc):
+        O.attention, O.gelu_tanh, O.attention_fp8, O.dit_stack = self.saved
+        return False
+
+
+def _small(name: str, **kw):
+    extra = {"img_len": 7, "img_feat": 64} if "i2v" in name else {}
+    extra.update(kw)
+    return dataclasses.replace(WORKLOADS[name], dim=512, heads=4, ffn=1024, text_len=40, **extra)
+
+
+def _image_context(inp):
+    return O.image_context_mlp(inp["img_feat"][0], *(inp[k] for k in ["w_i1", "b_i1", "w_i2", "b_i2", "w_i3", "b_i3"]))
+
+
+def block_study(w, trials: int, seed0: int, fp8_attention: bool, rows=None):
+    """Worst (max, rms) movement of the FP8 block's branch delta ``x_out - x_in``."""
+    inp = make_inputs(w, seed=0, zero_wx=False)
+    x, e, blk, ctx = inp["x"][0], inp["e"][0], inp["blocks"][0], inp["ctx"][0]
+    img = _image_context(inp) if w.i2v else None
+    xr = x if rows is None else x[rows]
+
+    def delta():
+        return O.dit_block(x, e, blk, ctx, w.heads, img_ctx=img, rows=rows, fp8=True,
+                           fp8_attention=fp8_attention) - xr
+    ref = delta()
+    worst = [0.0, 0.0]
+    for s in range(trials):
+        with QuantiserInputsMoved(seed0 + s):
+            y = delta()
+        worst = [max(worst[0], rel_max(y, ref)), max(worst[1], rel_rms(y, ref))]
+    return worst
+
+
+def stack_study(trials: int, seed0: int, i2v: bool, fp8_attention: bool):
+    """Worst movement of a two-block FP8 stack's velocity, both samples of a batch of two."""
+    w = _small("wan13b_480p_i2v_block" if i2v else "wan13b_480p_block", frames=3, height=10, width=14,
+               n_blocks=2, batch=2)
+    inp = make_inputs(w, seed=0, zero_wx=False)
+    worst = [0.0, 0.0]
+    for b in range(w.batch):
+        lat = inp["noise"][b]
+        img = None
+        if i2v:
+            keep = [1] + [0] * (4 * (w.frames - 1))
+            lat = O.i2v_input(inp["noise"][b], inp["cond"][b], O.i2v_mask(keep, w.frames, w.height, w.width))
+            img = O.image_context_mlp(inp["img_feat"][b], *(inp[k] for k in ["w_i1", "b_i1", "w_i2", "b_i2",
+                                                                             "w_i3", "b_i3"]))
+
+        def vel():
+            return O.dit_stack(lat, float(inp["t"][b]), inp, inp["blocks"], inp["ctx"][b], w.heads, img_ctx=img,
+                               fp8=True, fp8_attention=fp8_attention)
+        ref = vel()
+        for s in range(trials):
+            with QuantiserInputsMoved(seed0 + 10 * b + s):
+                y = vel()
+            worst = [max(worst[0], rel_max(y, ref)), max(worst[1], rel_rms(y, ref))]
+    return worst
+
+
+def sampler_study(trials: int, seed0: int, fp8_attention: bool, cached: bool):
+    """Worst movement of the displacement ``x_n - x_0`` of guided FP8 sampling: three
+    plain Euler steps, or six with the diffusion cache (attention reused from step 1 every
+    second step, the unconditional pass skipped from step 3 with interval 3)."""
+    w = _small("wan13b_480p_block", frames=3, height=10, width=14, n_blocks=2, batch=2)
+    inp = make_inputs(w, seed=0, zero_wx=False, uncond=True)
+    x0, ctx, unc = inp["noise"][0], inp["ctx"][0], inp["ctx_uncond"][0]
+
+    def run():
+        if cached:
+            sched = O.diffusion_cache_schedule(6, 1, 2, 3, 3)
+            return O.sample_euler_cfg_cached(x0, 6, 5.0, inp, inp["blocks"], ctx, unc, w.heads, sched, fp8=True,
+                                             fp8_attention=fp8_attention) - x0
+        return O.sample_euler_cfg(x0, 3, 5.0, inp, inp["blocks"], ctx, unc, w.heads, fp8=True,
+                                  fp8_attention=fp8_attention) - x0
+    ref = run()
+    worst = [0.0, 0.0]
+    for s in range(trials):
+        with QuantiserInputsMoved(seed0 + s, bf16_dit_input=True):
+            y = run()
+        worst = [max(worst[0], rel_max(y, ref)), max(worst[1], rel_rms(y, ref))]
+    return worst
+
+
+def attention_study(cases, trials: int):
+    """Worst distance between the 8-bit attention under the running base (whole, and
+    with every query block split over two key halves) and under the definition's base.
+    ``cases``: (Lq, Lk, heads, logit std, rows or None)."""
+    worst = [0.0, 0.0]
+    for t in range(trials):
+        for Lq, Lk, H, std, rows in cases:
+            g = np.random.Generator(np.random.PCG64(100 * t + Lk + H))
+            s = math.sqrt(std)
+            q = round_bf16(g.standard_normal((Lq, H * 128)) * s)
+            k = round_bf16(g.standard_normal((Lk, H * 128)) * s)
+            v = round_bf16(g.standard_normal((Lk, H * 128)))
+            r = np.arange(Lq) if rows is None else rows
+            ref = O.attention_fp8(q[r], k, v, H)
+            blocks = [(h, b) for h in range(H) for b in range((Lq + 255) // 256)]
+            for split in ((), blocks):
+                got = O.attention_fp8(q, k, v, H, running_base=True, split_units=split, rows=r)
+                worst = [max(worst[0], rel_max(got, ref)), max(worst[1], rel_rms(got, ref))]
+    return worst
+
+
+POLY_REL_ERR = 7.5e-5   # stated relative error bound of the kernels' polynomial 2^x
+
+
+def kernel_prob_model(seed: int):
+    """A model of the 8-bit attention kernel's probabilities, from what the kernel states
+    about its arithmetic (no constant of its code): the score accumulated in float32
+    (rounded once here), the exponent ``S c - base`` as one float32 FMA and 2^x in
+    float32, except that the keys at tile positions 3 mod 8 take a polynomial 2^x whose
+    error is modelled as a seeded relative perturbation within its stated bound."""
+    r = np.random.Generator(np.random.PCG64(seed))
+
+    def prob(S, c, base, first_key):
+        S32 = np.asarray(S, np.float32).astype(np.float64)
+        c32 = np.asarray(c, np.float32).astype(np.float64)
+        x = (S32 * c32 - base).astype(np.float32).astype(np.float64)
+        p = np.exp2(x).astype(np.float32).astype(np.float64)
+        poly = (np.arange(S.shape[1]) % 8) == 3
+        if poly.any():
+            p[:, poly] *= 1.0 + POLY_REL_ERR * r.uniform(-1.0, 1.0, size=(S.shape[0], int(poly.sum())))
+        return p
+    return prob
+
+
+def _qkv(seed, B, Lq, Lk, H, logit_std):
+    """The 8-bit attention tests' inputs: q rows scaled by random powers of two (so that
+    the per-row q scales vary), k and v ~ N(0, 1) x sqrt(std), rounded to bf16."""
+    r = np.random.Generator(np.random.PCG64(seed))
+    s = np.sqrt(logit_std)
+    D = H * 128
+    q = round_bf16(r.standard_normal((B, Lq, D)) * s * np.exp2(r.integers(-3, 4, (B, Lq, 1))))
+    k = round_bf16(r.standard_normal((B, Lk, D)) * s)
+    v = round_bf16(r.standard_normal((B, Lk, D)))
+    return q, k, v
+
+
+def attention_kernel_model_study(cases, trials: int):
+    """Worst distance between the running-base oracle (exact exponentials) and the same
+    under ``kernel_prob_model`` with its output rounded to bf16, on the 8-bit attention
+    tests' own inputs: ``cases`` are (B, Lq, Lk, heads, logit std, input seed, rows or
+    None, split units: "all" or ()), each over ``trials`` perturbation seeds."""
+    worst = [0.0, 0.0]
+    for B, Lq, Lk, H, std, seed, rows, split in cases:
+        q, k, v = _qkv(seed, B, Lq, Lk, H, std)
+        units = [(h, b) for h in range(H) for b in range((Lq + 255) // 256)] if split == "all" else ()
+        r = np.arange(Lq) if rows is None else rows
+        for b in range(B):
+            ref = O.attention_fp8(q[b], k[b], v[b], H, running_base=True, split_units=units, rows=r)
+            for t in range(trials):
+                got = O.attention_fp8(q[b], k[b], v[b], H, running_base=True, split_units=units, rows=r,
+                                      prob=kernel_prob_model(1000 * t + b))
+                got = round_bf16(got.astype(np.float32))
+                worst = [max(worst[0], rel_max(got, ref)), max(worst[1], rel_rms(got, ref))]
+    return worst
+
+
+def warp_rows(n, count=8, seed=0):
+    from gpu_util import sample_warps
+    return sample_warps(n, count, seed)
+
+
+def study(full: bool = False, log=print):
+    """Runs every study; returns {bar name: (worst max, worst rms)}."""
+    out = {}
+    n = 6 if full else 2
+    blk = [block_study(_small(nm, frames=3, height=10, width=14), n, 100, False)
+           for nm in ("wan13b_480p_block", "wan13b_480p_i2v_block")]
+    if full:
+        w = WORKLOADS["wan13b_480p_block"]
+        blk.append(block_study(w, 3, 1000, False, rows=sample_rows(w.tokens)))
+    out["FP8_TOL"] = (max(b[0] for b in blk), max(b[1] for b in blk))
+    log("FP8_TOL", out["FP8_TOL"])
+    blk = [block_study(_small(nm, frames=5, height=24, width=32) if full else _small(nm, frames=3, height=10,
+                                                                                    width=14), n, 500, True)
+           for nm in ("wan13b_480p_block", "wan13b_480p_i2v_block")]
+    if full:
+        w = WORKLOADS["wan13b_480p_block"]
+        blk.append(block_study(w, 2, 1500, True, rows=sample_rows(w.tokens)))
+    out["FP8A_BLOCK_TOL"] = (max(b[0] for b in blk), max(b[1] for b in blk))
+    log("FP8A_BLOCK_TOL", out["FP8A_BLOCK_TOL"])
+    st = [stack_study(4 if full else 1, 300 + 37 * i, i2v, fa)
+          for i, (i2v, fa) in enumerate([(False, False), (True, False), (False, True), (True, True)])]
+    out["FP8_STACK_TOL"] = (max(s_[0] for s_ in st), max(s_[1] for s_ in st))
+    log("FP8_STACK_TOL", out["FP8_STACK_TOL"])
+    sa = [sampler_study(4 if full else 1, 700 + 13 * i, fa, cached)
+          for i, (fa, cached) in enumerate([(False, False), (True, False), (False, True), (True, True)])]
+    out["FP8_SAMPLE_TOL"] = (max(s_[0] for s_ in sa), max(s_[1] for s_ in sa))
+    log("FP8_SAMPLE_TOL", out["FP8_SAMPLE_TOL"])
+    cases = [(256, 700, 2, 0.6, None), (256, 700, 2, 1.0, None), (256, 2100, 2, 1.0, None),
+             (256, 700, 2, 4.0, None), (128, 3000, 1, 4.0, None)]
+    if full:
+        cases += [(32760, 32760, 1, 1.0, warp_rows(32760)), (75600, 75600, 1, 1.0, warp_rows(75600))]
+    out["FP8_ATTN_TOL"] = attention_study(cases, 6 if full else 1)
+    log("FP8_ATTN_TOL", out["FP8_ATTN_TOL"])
+    # the 8-bit attention tests' cases with their input seeds (Lq * 7 + Lk; the fused-layout
+    # test 11, the full-size ones 5, where every head but one is left out here)
+    kcases = [(1, 300, 700, 2, 1.0, 300 * 7 + 700, None, ()), (1, 300, 700, 2, 4.0, 300 * 7 + 700, None, ()),
+              (2, 257, 2100, 2, 1.0, 257 * 7 + 2100, None, "all"), (1, 130, 1, 1, 1.0, 130 * 7 + 1, None, ()),
+              (1, 1, 300, 2, 0.36, 1 * 7 + 300, None, ()), (2, 700, 700, 2, 1.0, 11, None, ())]
+    if full:
+        kcases += [(1, 32760, 32760, 1, 1.0, 5, warp_rows(32760), ()), (1, 75600, 75600, 1, 1.0, 5, warp_rows(75600), ())]
+    out["FP8_ATTN_RB_TOL"] = attention_kernel_model_study(kcases, 8 if full else 2)
+    log("FP8_ATTN_RB_TOL", out["FP8_ATTN_RB_TOL"])
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--full", action="store_true")
+    args = ap.parse_args()
+    import gpu_util as G
+    res = study(args.full)
+    print(f"{'bar':16s} {'worst max':>10s} {'worst rms':>10s} {'1.5x max':>9s} {'1.5x rms':>9s} "
+          f"{'used max':>9s} {'used rms':>9s}")
+    for name, (wm, wr) in res.items():
+        um, ur = getattr(G, name + "_MAX"), getattr(G, name + "_RMS")
+        print(f"{name:16s} {wm:10.4f} {wr:10.4f} {bar(wm):9.3g} {bar(wr):9.3g} {um:9.3g} {ur:9.3g}"
+              f"{'' if um >= 1.5 * wm and ur >= 1.5 * wr else '  BELOW 1.5x'}")
+
+
+if __name__ == "__main__":
+    main()

@@ -17,11 +17,15 @@ FP8_TOL_RMS = 3.2e-2
 # The same derivation for outputs further from the quantisers: the FP8 stack's velocity
 # (two blocks, LN, head) moves by at most 0.84 % (max) and 0.54 % (RMS) under those
 # perturbations (8 trials for each of the two samples, T2V and I2V, with and without
-# 8-bit self-attention), a 3-step guided FP8 sampling displacement by at most 1.31 %
-# and 1.0 % (4 trials); bars 1.5x, rounded up. The sampler bars separate FP8 from bf16
-# (4.5 % apart); at the stack the RMS bar does (1.5 % apart).
+# 8-bit self-attention); bars 1.5x, rounded up. Guided FP8 sampling (3 plain Euler
+# steps, or 6 with the diffusion cache, with and without 8-bit self-attention) also
+# rounds its DiT input to bf16 at every step, as the GPU does: its displacement moves by
+# at most 1.43 % (max) and 1.02 % (RMS); bars 1.5x, rounded up. The sampler bars
+# separate FP8 from bf16 (4.5 % apart); at the stack the RMS bar does (1.5 % apart).
+# Every number here is printed by tests/fp8_tolerance_study.py (``--full``), and
+# tests/test_fp8_tolerances.py re-runs its reduced form against these bars.
 FP8_STACK_TOL_MAX, FP8_STACK_TOL_RMS = 1.3e-2, 8.5e-3
-FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
+FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2.2e-2, 1.6e-2
 # 8-bit attention against the oracle's. The kernel takes each row's probabilities
 # against its running max (moved only when the max grows past 2^8), rounded up to a
 # whole power of two; the oracle against the row's final max. Whole powers of two leave
@@ -33,6 +37,17 @@ FP8_SAMPLE_TOL_MAX, FP8_SAMPLE_TOL_RMS = 2e-2, 1.5e-2
 # 2.0 % at 32760, 2.4 % at 75600); bars 1.5x: 8e-2 and 3.7e-2. (8-bit attention itself
 # is 4-18 % (max) and 4-12 % (RMS) away from exact attention there.)
 FP8_ATTN_TOL_MAX, FP8_ATTN_TOL_RMS = 8e-2, 3.7e-2
+# 8-bit attention against the oracle's running-base option (attention_fp8 with
+# running_base=True and the kernel's key-split units): the same codes and the same bases,
+# so what remains is the kernel's float32 scores and exponent, its approximate
+# exponentials (one in eight a degree-3 polynomial within 7.5e-5) and the bf16 rounding
+# of the output (2^-9 relative, about 1.6e-3 RMS). A float32 exponent that differs from
+# the exact one can flip the E4M3 rounding of a probability; in the few large
+# probabilities of a peaked row (logit std 4) that moves the row by a few percent.
+# Modelled on the tests' own inputs (fp8_tolerance_study.kernel_prob_model) the kernel
+# moves by at most 2.24 % (max) and 0.26 % (RMS) -- the GPU measured 2.24 % and 0.26 % on
+# the peaked case; bars 1.5x, rounded up.
+FP8_ATTN_RB_TOL_MAX, FP8_ATTN_RB_TOL_RMS = 3.4e-2, 4e-3
 # The FP8 block with 8-bit self-attention: the derivation of FP8_TOL_* with q, k and v
 # also moved by +-2^-9 and the running base emulated in the 8-bit attention moves the
 # block by at most 2.8 % (max) and 2.1 % (RMS) (960-token T2V and I2V blocks, 6 trials
@@ -65,3 +80,37 @@ def rms_err(got, ref) -> float:
     ref = np.asarray(ref, dtype=np.float64)
     den = np.sqrt(np.mean(ref ** 2))
     return float(np.sqrt(np.mean((got - ref) ** 2)) / (den if den > 0 else 1.0))
+
+
+def attention_split_units(B, H, Lq, Lk, nsm):
+    """(head, query block) pairs, per sample, whose keys the attention kernel takes in
+    two halves when the caller passes a workspace: units are (sample, head, 256-row
+    query block) in that order, one CTA each; when the last wave of ``units % nsm``
+    units would fill at most half of the ``nsm`` SMs and a unit has at least 16 key
+    tiles of 128, those last units are split over their key tiles (first half
+    floor(n/2) tiles) and merged after (the launch rule of the attention kernel)."""
+    pairs = (Lq + 255) // 256
+    units = B * H * pairs
+    rem = units % nsm
+    nkv = (Lk + 127) // 128
+    out = {b: [] for b in range(B)}
+    if rem > 0 and 2 * rem <= nsm and nkv >= 16:
+        for u in range(units - rem, units):
+            bh, pair = divmod(u, pairs)
+            b, h = divmod(bh, H)
+            out[b].append((h, pair))
+    return out
+
+
+def sample_warps(n_rows, count=8, seed=0, warp=32, tile=128):
+    """Query rows checked at long sequence lengths when a row's result depends on its
+    32-row group (the 8-bit attention's running base): ``count`` whole groups -- the
+    first, every group of the ragged last 128-row tile, then seeded ones; sorted."""
+    groups = {0}
+    tail0 = n_rows - (n_rows % tile or tile)
+    groups.update(range(tail0 // warp, (n_rows + warp - 1) // warp))
+    r = rng(seed)
+    while len(groups) < count:
+        groups.add(int(r.integers(0, (n_rows + warp - 1) // warp)))
+    rows = [i for g in sorted(groups) for i in range(g * warp, min((g + 1) * warp, n_rows))]
+    return np.array(rows, dtype=np.int64)
