@@ -4,6 +4,8 @@ command the committed ncu summaries were captured with.
   python -m video_diffusion_transformer_wan_b200.kernel_bench attention --L 32760 --heads 12
   python -m video_diffusion_transformer_wan_b200.kernel_bench gemm --M 32760 --N 4608 --K 1536 --epi store
   python -m video_diffusion_transformer_wan_b200.kernel_bench layernorm --L 32760 --dim 1536
+  python -m video_diffusion_transformer_wan_b200.kernel_bench patchify --frames 21 --height 60 --width 104
+  python -m video_diffusion_transformer_wan_b200.kernel_bench head --frames 21 --height 60 --width 104
   python -m video_diffusion_transformer_wan_b200.kernel_bench sample --blocks 30 --steps 2
 
 Inputs are random device tensors (the kernels' timing does not depend on values); the
@@ -99,9 +101,38 @@ def _block(a) -> dict:
                 tokens_per_s=B * L / (ms / 1e3), tflops=flops / ms / 1e9)
 
 
+def _patch_or_head(a, g) -> dict:
+    """wan_patchify (patch gather + the K = in_ch*4 projection, fp32 store) or wan_head_fwd
+    (plain LN + the N = 64 projection scattered into the latent) on one 480P-sized latent.
+    Both projections are HBM-bound; algorithmic bytes: inputs read once, outputs written
+    once (patchify: latent, gathered patches written and read, W, x; head: x, the LN
+    output written and read, W, v)."""
+    D, F, H, W = a.dim, a.frames, a.height, a.width
+    L = F * (H // 2) * (W // 2)
+    cfg = wan.make_config(D, D // 128, 4 * D, in_ch=a.in_ch)
+    if a.kernel == "patchify":
+        K = a.in_ch * 4
+        lat = torch.randn(1, a.in_ch, F, H, W, device="cuda", generator=g).to(torch.bfloat16)
+        wp = (torch.randn(D, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        bp = torch.zeros(D, dtype=torch.bfloat16, device="cuda")
+        x = torch.empty(1, L, D, dtype=torch.float32, device="cuda")
+        ws = torch.empty(L * K * 2, dtype=torch.uint8, device="cuda")
+        ms = _time(lambda: wan.patchify(cfg, lat, wp, bp, x, ws), a.iters, a.warmup)
+        byts = L * K * 2 * 3 + D * K * 2 + L * D * 4.0
+    else:
+        x = torch.randn(1, L, D, device="cuda", generator=g)
+        wh = (torch.randn(64, D, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        bh = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+        v = torch.empty(1, 16, F, H, W, dtype=torch.float32, device="cuda")
+        ws = torch.empty(L * D * 2, dtype=torch.uint8, device="cuda")
+        ms = _time(lambda: wan.head_fwd(cfg, x, F, H, W, wh, bh, v, ws), a.iters, a.warmup)
+        byts = L * D * 4 + L * D * 2 * 2 + 64 * D * 2 + L * 64 * 4.0
+    return dict(L=L, dim=D, ms=ms, gbs=byts / ms / 1e6, alg_bytes=byts)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block"])
+    ap.add_argument("kernel", choices=["attention", "gemm", "layernorm", "sample", "block", "patchify", "head"])
     ap.add_argument("--fp8", action="store_true", help="attention / gemm / block / sample: E4M3 operands (kind::f8f6f4)")
     ap.add_argument("--fp8-attention", action="store_true",
                     help="block / sample with --fp8: the self-attention on E4M3 operands as well")
@@ -120,6 +151,10 @@ def main(argv=None):
     ap.add_argument("--N", type=int, default=4608)
     ap.add_argument("--K", type=int, default=1536)
     ap.add_argument("--epi", choices=["store", "gelu", "residual", "f32"], default="store")
+    ap.add_argument("--frames", type=int, default=21, help="patchify / head: latent frames")
+    ap.add_argument("--height", type=int, default=60, help="patchify / head: latent height")
+    ap.add_argument("--width", type=int, default=104, help="patchify / head: latent width")
+    ap.add_argument("--in-ch", type=int, default=16, help="patchify: latent channels")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=2)
     a = ap.parse_args(argv)
@@ -173,6 +208,8 @@ def main(argv=None):
             ms = _time(lambda: wan.linear_fwd(cfg, A, W, bias, C, epi, rows_per_batch=a.M), a.iters, a.warmup)
         flops = 2.0 * a.M * a.N * a.K
         out.update(M=a.M, N=a.N, K=a.K, epi=a.epi, fp8=a.fp8, ms=ms, tflops=flops / ms / 1e9)
+    elif a.kernel in ("patchify", "head"):
+        out.update(_patch_or_head(a, g))
     elif a.kernel == "block":
         out.update(_block(a))
     elif a.kernel == "sample":
