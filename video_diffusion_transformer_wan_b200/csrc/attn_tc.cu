@@ -66,14 +66,21 @@ constexpr int kHalfBytes = kTile * 128;        // 128 rows of one 128-byte swizz
 // Operand shapes: bf16 tiles are two 64-column spans (32 KB), E4M3 tiles one span of
 // 128 codes (16 KB). K of one MMA is 16 (bf16) or 32 (E4M3), so a 128-deep product
 // takes 8 or 4 instructions. The 16 KB tiles leave room for a deeper K/V ring.
-template <bool kF8>
+// The persistent variant (kPersist, short key sequences) double-buffers Q so that the
+// next unit's Q lands while the current one computes; its K/V ring is 3 stages to fit.
+template <bool kF8, bool kPersist = false>
 struct AttnShape {
   static constexpr int kTileBytes = kTile * (kF8 ? 128 : 256);
   static constexpr int kSpans = kF8 ? 1 : 2;
-  static constexpr int kStages = kF8 ? 8 : 5;
+  static constexpr int kQBufs = kPersist ? 2 : 1;
+  static constexpr int kStages = kPersist ? 3 : (kF8 ? 8 : 5);
   static constexpr int kMmas = kF8 ? 4 : 8;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kTileBytes) * (kQTiles + kStages) + 256;
+  static constexpr size_t kSmem =
+      1024 + static_cast<size_t>(kTileBytes) * (kQBufs * kQTiles + kStages) + 256;
 };
+// Key sequences of at most this many 128-key tiles (the 512 text and 257 image tokens of
+// the cross-attention) run on the persistent variant.
+constexpr int kMaxPersistKeyTiles = 4;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kMinSplitKeyTiles = 16;          // see launch_attn_tc
 
@@ -91,6 +98,7 @@ struct AttnParams {
   // remaining units' key tiles in two halves (CTA n_full + 2u + half) and write
   // unnormalised partial outputs to part_o / part_ml, merged by attn_combine_kernel.
   int pairs, n_full;
+  int n_units;     // persistent variant: CTA c takes units c, c + gridDim.x, ...
   float* part_o;   // [split CTA][tile][128 rows][128] fp32
   float* part_ml;  // [split CTA][tile][128 rows][2] (row max, row sum) fp32
   // E4M3 operands only: q scale per (sample, query row, head) [B, Lq, H]; k and v scale
@@ -104,21 +112,24 @@ struct AttnParams {
 __device__ __forceinline__ int pos_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int pos_v(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 * j + 2; }
 
-template <bool kF8>
+template <bool kF8, bool kPersist>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const AttnParams p) {
-  constexpr int kTileBytes = AttnShape<kF8>::kTileBytes;
-  constexpr int kStages = AttnShape<kF8>::kStages;
-  constexpr int kSpans = AttnShape<kF8>::kSpans;
-  constexpr int kMmas = AttnShape<kF8>::kMmas;
+  using Shape = AttnShape<kF8, kPersist>;
+  constexpr int kTileBytes = Shape::kTileBytes;
+  constexpr int kStages = Shape::kStages;
+  constexpr int kSpans = Shape::kSpans;
+  constexpr int kMmas = Shape::kMmas;
+  constexpr int kQBufs = Shape::kQBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                  // [2][tile]
-  uint8_t* sKV = sQ + kQTiles * kTileBytes;            // [kStages][tile]
+  uint8_t* sQ = smem;                                  // [kQBufs][2][tile]
+  uint8_t* sKV = sQ + kQBufs * kQTiles * kTileBytes;   // [kStages][tile]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * kTileBytes);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_full = bars;                 // [kQBufs]
+  uint64_t* q_empty = q_full + kQBufs;     // [kQBufs] (persistent: Q buffer free again)
+  uint64_t* kv_full = q_empty + kQBufs;
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* s_full = kv_empty + kStages;   // [2]
   uint64_t* p_full = s_full + kQTiles;     // [2]
@@ -129,21 +140,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nkv_all = (p.Lk + kTile - 1) / kTile;
-  int unit = blockIdx.x, kv0 = 0, kv1 = nkv_all, split = -1;
-  if (unit >= p.n_full) {
-    split = unit - p.n_full;
-    unit = p.n_full + (split >> 1);
+  // Work of this CTA: one unit (possibly one key half of a split unit), or, persistent,
+  // units blockIdx.x, blockIdx.x + gridDim.x, ... over all key tiles. Every barrier
+  // phase below counts across the units a CTA takes: Q buffer fills per buffer, ring
+  // loads, key tiles (S ready / P ready) and units (O final).
+  int kv0 = 0, kv1 = nkv_all, split = -1;
+  int n_iter = 1;
+  if constexpr (kPersist) {
+    n_iter = blockIdx.x < p.n_units ? (p.n_units - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                    : 0;
+  } else if (static_cast<int>(blockIdx.x) >= p.n_full) {
+    split = blockIdx.x - p.n_full;
     kv0 = (split & 1) ? nkv_all / 2 : 0;
     kv1 = (split & 1) ? nkv_all : nkv_all / 2;
   }
-  const int nkv = kv1 - kv0;  // key tiles this CTA visits, from key tile kv0 on
-  const int bh = unit / p.pairs;
-  const int q0 = (unit - bh * p.pairs) * (kQTiles * kTile);
-  const int h = bh % p.H;
-  const int b = bh / p.H;
+  const int nkv = kv1 - kv0;  // key tiles this CTA visits per unit, from key tile kv0 on
+  auto unit_of = [&](int it) {
+    if constexpr (kPersist) return static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+    return split >= 0 ? p.n_full + (split >> 1) : static_cast<int>(blockIdx.x);
+  };
+  struct UnitPos {
+    int b, h, q0;
+  };
+  auto decode = [&](int unit) {
+    const int bh = unit / p.pairs;
+    return UnitPos{bh / p.H, bh % p.H, (unit - bh * p.pairs) * (kQTiles * kTile)};
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int q = 0; q < kQBufs; ++q) {
+      mbar_init(&q_full[q], 1);
+      mbar_init(&q_empty[q], 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -172,41 +200,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, kQTiles * kTileBytes);
-      const int qc = p.q_col0 + h * kHd;
-      for (int t = 0; t < kQTiles; ++t)
-        for (int c = 0; c < kSpans; ++c)
-          tma_load_3d(sQ + t * kTileBytes + c * kHalfBytes, &mapQ, q_full, qc + 64 * c, q0 + t * kTile, b);
       const int n_loads = 2 * nkv;
-      int issued = 0;
-      for (int ld = 0; ld < n_loads; ++ld) {
-        const int stage = ld % kStages;
-        const uint32_t phase = static_cast<uint32_t>((ld / kStages) & 1);
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1u, p.err)) break;
-        bool is_v;
-        int j;
-        if (ld == 0) {
-          is_v = false, j = 0;
-        } else if (ld == n_loads - 1) {
-          is_v = true, j = nkv - 1;
-        } else if (ld & 1) {
-          is_v = false, j = (ld + 1) >> 1;
-        } else {
-          is_v = true, j = (ld >> 1) - 1;
-        }
-        const CUtensorMap* map = is_v ? &mapV : &mapK;
-        const int col = (is_v ? p.v_col0 : p.k_col0) + h * kHd;
-        uint8_t* dst = sKV + stage * kTileBytes;
-        mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
-        if (kF8 && is_v) {  // V^T: 128 dims (rows) x 128 keys (x)
-          tma_load_3d(dst, map, &kv_full[stage], (kv0 + j) * kTile, p.v_col0 + h * kHd, b);
-        } else {
+      int issued = 0;  // ring loads issued so far (all units)
+      int q_loads = 0;
+      bool ok = true;
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const UnitPos u = decode(unit_of(it));
+        const int qb = it % kQBufs;
+        if (kPersist && it >= kQBufs &&
+            !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), p.err))
+          break;
+        uint8_t* sq = sQ + qb * kQTiles * kTileBytes;
+        mbar_arrive_expect_tx(&q_full[qb], kQTiles * kTileBytes);
+        const int qc = p.q_col0 + u.h * kHd;
+        for (int t = 0; t < kQTiles; ++t)
           for (int c = 0; c < kSpans; ++c)
-            tma_load_3d(dst + c * kHalfBytes, map, &kv_full[stage], col + 64 * c, (kv0 + j) * kTile, b);
+            tma_load_3d(sq + t * kTileBytes + c * kHalfBytes, &mapQ, &q_full[qb], qc + 64 * c, u.q0 + t * kTile, u.b);
+        ++q_loads;
+        for (int ld = 0; ld < n_loads; ++ld) {
+          const int stage = issued % kStages;
+          const uint32_t phase = static_cast<uint32_t>((issued / kStages) & 1);
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          bool is_v;
+          int j;
+          if (ld == 0) {
+            is_v = false, j = 0;
+          } else if (ld == n_loads - 1) {
+            is_v = true, j = nkv - 1;
+          } else if (ld & 1) {
+            is_v = false, j = (ld + 1) >> 1;
+          } else {
+            is_v = true, j = (ld >> 1) - 1;
+          }
+          const CUtensorMap* map = is_v ? &mapV : &mapK;
+          const int col = (is_v ? p.v_col0 : p.k_col0) + u.h * kHd;
+          uint8_t* dst = sKV + stage * kTileBytes;
+          mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
+          if (kF8 && is_v) {  // V^T: 128 dims (rows) x 128 keys (x)
+            tma_load_3d(dst, map, &kv_full[stage], (kv0 + j) * kTile, p.v_col0 + u.h * kHd, u.b);
+          } else {
+            for (int c = 0; c < kSpans; ++c)
+              tma_load_3d(dst + c * kHalfBytes, map, &kv_full[stage], col + 64 * c, (kv0 + j) * kTile, u.b);
+          }
+          ++issued;
         }
-        ++issued;
       }
-      mbar_wait(q_full, 0, p.err);
+      // Wait for every copy this thread started (the last fill of each buffer and stage).
+      for (int q = 0; q < kQBufs; ++q) {
+        const int n_q = q_loads / kQBufs + (q < q_loads % kQBufs ? 1 : 0);
+        if (n_q > 0) mbar_wait(&q_full[q], static_cast<uint32_t>((n_q - 1) & 1), p.err);
+      }
       for (int s = 0; s < kStages; ++s) {
         const int n_s = issued / kStages + (s < issued % kStages ? 1 : 0);
         if (n_s > 0) mbar_wait(&kv_full[s], static_cast<uint32_t>((n_s - 1) & 1), p.err);
@@ -242,8 +288,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, acc);
         }
       };
-      auto qk = [&](int t, int kstage) {
-        const uint64_t qd = q_desc + static_cast<uint32_t>((t * kTileBytes) >> 4);
+      auto qk = [&](int t, int qb, int kstage) {
+        const uint64_t qd = q_desc + static_cast<uint32_t>(((qb * kQTiles + t) * kTileBytes) >> 4);
         const uint64_t kd = k_desc + static_cast<uint32_t>((kstage * kTileBytes) >> 4);
         const uint32_t s_tmem = tmem_base + t * kTile;
 #pragma unroll
@@ -255,41 +301,60 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, p.err);
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int pk = pos_k(j);
-        if (!wait_pos(pk)) break;
-        int pvpos = -1;
-        if (j > 0) {
-          pvpos = pos_v(j - 1, nkv);
-          if (!wait_pos(pvpos)) break;
-        }
-        for (int t = 0; ok && t < kQTiles; ++t) {
+      bool ok = true;
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int qb = it % kQBufs;
+        const int base = it * 2 * nkv;   // ring position of this unit's first load
+        const int tiles = it * nkv;      // key tiles of earlier units (S / P phases)
+        if (!mbar_wait(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1), p.err)) break;
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int pk = base + pos_k(j);
+          if (!wait_pos(pk)) {
+            ok = false;
+            break;
+          }
+          int pvpos = -1;
           if (j > 0) {
-            if (!mbar_wait(&p_full[t], static_cast<uint32_t>((j - 1) & 1), p.err)) {
+            pvpos = base + pos_v(j - 1, nkv);
+            if (!wait_pos(pvpos)) {
               ok = false;
               break;
             }
-            tc_fence_after();
-            pv(t, j - 1, pvpos % kStages);
           }
-          qk(t, pk % kStages);
-          tc_commit(&s_full[t]);
+          for (int t = 0; ok && t < kQTiles; ++t) {
+            if (j > 0) {
+              if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + j - 1) & 1), p.err)) {
+                ok = false;
+                break;
+              }
+              // The first PV of a unit overwrites O_t. The softmax threads of tile t
+              // read the previous unit's O_t out (and waited for those reads) before
+              // they arrived on p_full for this unit's first key tile, so it is free.
+              tc_fence_after();
+              pv(t, j - 1, pvpos % kStages);
+            }
+            qk(t, qb, pk % kStages);
+            tc_commit(&s_full[t]);
+          }
+          if (!ok) break;
+          tc_commit(&kv_empty[pk % kStages]);
+          if (j > 0) tc_commit(&kv_empty[pvpos % kStages]);
         }
-        if (!ok) break;
-        tc_commit(&kv_empty[pk % kStages]);
-        if (j > 0) tc_commit(&kv_empty[pvpos % kStages]);
-      }
-      if (ok && nkv > 0) {
+        if (!ok || nkv == 0) break;
+        tc_commit(&q_empty[qb]);   // every QK of this unit issued: Q buffer free once they complete
         const int last = nkv - 1;
-        const int pvpos = pos_v(last, nkv);
+        const int pvpos = base + pos_v(last, nkv);
         ok = wait_pos(pvpos);
         for (int t = 0; ok && t < kQTiles; ++t) {
-          if (!mbar_wait(&p_full[t], static_cast<uint32_t>(last & 1), p.err)) break;
+          if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + last) & 1), p.err)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           pv(t, last, pvpos % kStages);
           tc_commit(&o_final[t]);
         }
+        if (!ok) break;
         tc_commit(&kv_empty[pvpos % kStages]);
       }
       tc_commit(drain);
@@ -303,172 +368,178 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t s_row = tmem_base + lane_off + t * kTile;
     const uint32_t o_row = tmem_base + lane_off + 256 + t * kTile;
-    float sl2 = p.scale_log2;
-    float v_scale = 1.0f;
-    if constexpr (kF8) {
-      // Logit = S q_scale k_scale / sqrt(d): the row's scales fold into its log2 scale;
-      // the v scale multiplies the output.
-      const float* kvs = p.kv_scale + 2 * (static_cast<int64_t>(b) * p.H + h);
-      const int grow0 = q0 + t * kTile + row;
-      sl2 *= kvs[0] * (grow0 < p.Lq ? p.q_scale[(static_cast<int64_t>(b) * p.Lq + grow0) * p.H + h] : 1.0f);
-      v_scale = kvs[1];
-    }
-    float m_run = -INFINITY;
-    float l_run = 0.f;
     bool ok = true;
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (!mbar_wait_warp(&s_full[t], static_cast<uint32_t>(j & 1), p.err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int valid = p.Lk - (kv0 + j) * kTile;  // keys of this tile that exist (mask the rest)
-      // The whole S row (128 fp32) is read with one wait; P is then packed in place into
-      // the first 64 registers (pair i of the row lands in register i <= 2i, so the pass
-      // never overwrites a value it still has to read) and stored over S in TMEM.
-      uint32_t r[kTile];
-      tmem_ld32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
-      tmem_ld32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-      tmem_ld32(s_row + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
-      tmem_ld32(s_row + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
-      tmem_ld_wait();
-      if (valid < kTile) {
-#pragma unroll
-        for (int i = 0; i < kTile; ++i)
-          if (i >= valid) r[i] = __float_as_uint(-INFINITY);
-      }
-      float mx8[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(r[a]);
-#pragma unroll
-      for (int i = 8; i < kTile; i += 2)
-        mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const bool grow = (mx - m_run) * sl2 > kRescaleLog2;
-      float alpha = 1.0f;
-      bool rescale = false;
-      if (j == 0) {
-        m_run = mx;
-      } else if (__any_sync(0xffffffffu, grow)) {
-        const float m_new = fmaxf(m_run, mx);
-        // E4M3 P: bases are whole powers of two (see below), so alpha is one as well.
-        alpha = kF8 ? pow2i(static_cast<int>(ceilf(m_run * sl2) - ceilf(m_new * sl2)))
-                    : ex2_approx((m_run - m_new) * sl2);
-        m_run = m_new;
-        rescale = true;
-      }
-      // E4M3 P is taken against the base rounded up to a whole power of two: p <= 2^8
-      // still, and its codes are those of the exact-max base times an exact power of two
-      // (outside the subnormal range), whatever this row's running max is.
-      const float nb = kF8 ? -ceilf(m_run * sl2) : -m_run * sl2;
-      const unsigned long long sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
-      unsigned long long rs4[4] = {0ull, 0ull, 0ull, 0ull};
+    for (int it = 0; ok && it < n_iter; ++it) {
+      const UnitPos u = decode(unit_of(it));
+      const int b = u.b, h = u.h, q0 = u.q0;
+      const int tiles = it * nkv;
+      float sl2 = p.scale_log2;
+      float v_scale = 1.0f;
       if constexpr (kF8) {
-        // E4M3 P: four codes per register (quad i of the row lands in register i <= 4i).
-#pragma unroll
-        for (int i = 0; i < kTile / 4; ++i) {
-          const unsigned long long s01 = f2_pack(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
-          const unsigned long long s23 = f2_pack(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-          const float2 x01 = f2_unpack(f2_fma(s01, sl2x2, nbx2));
-          const float2 x23 = f2_unpack(f2_fma(s23, sl2x2, nbx2));
-          const float e0 = ex2_approx(x01.x), e1 = ex2_approx(x01.y);
-          // one exponential in eight on the FMA pipes (MUFU is the busier unit here)
-          const float e2 = ex2_approx(x23.x);
-          const float e3 = (i & 1) == 0 ? exp2_poly(x23.y) : ex2_approx(x23.y);
-          rs4[(2 * i) & 3] = f2_add(rs4[(2 * i) & 3], f2_pack(e0, e1));
-          rs4[(2 * i + 1) & 3] = f2_add(rs4[(2 * i + 1) & 3], f2_pack(e2, e3));
-          r[i] = pack_e4m3x4(e0, e1, e2, e3);
-        }
-        tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
-      } else {
-#pragma unroll
-        for (int i = 0; i < kTile / 2; ++i) {
-          const unsigned long long s2 = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          const float2 x = f2_unpack(f2_fma(s2, sl2x2, nbx2));
-          const float e0 = ex2_approx(x.x);
-          const float e1 = ex2_approx(x.y);
-          rs4[i & 3] = f2_add(rs4[i & 3], f2_pack(e0, e1));
-          r[i] = pack_bf16x2(e0, e1);
-        }
-        tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
-        tmem_st32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        // Logit = S q_scale k_scale / sqrt(d): the row's scales fold into its log2 scale;
+        // the v scale multiplies the output.
+        const float* kvs = p.kv_scale + 2 * (static_cast<int64_t>(b) * p.H + h);
+        const int grow0 = q0 + t * kTile + row;
+        sl2 *= kvs[0] * (grow0 < p.Lq ? p.q_scale[(static_cast<int64_t>(b) * p.Lq + grow0) * p.H + h] : 1.0f);
+        v_scale = kvs[1];
       }
-      if (rescale) {
-        // S_t(j) ready implies PV_t(j-1) completed, and PV_t(j) waits for this thread's
-        // arrival below: O_t is current and idle while it is rescaled here.
+      float m_run = -INFINITY;
+      float l_run = 0.f;
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (!mbar_wait_warp(&s_full[t], static_cast<uint32_t>((tiles + j) & 1), p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int valid = p.Lk - (kv0 + j) * kTile;  // keys of this tile that exist (mask the rest)
+        // The whole S row (128 fp32) is read with one wait; P is then packed in place into
+        // the first 64 registers (pair i of the row lands in register i <= 2i, so the pass
+        // never overwrites a value it still has to read) and stored over S in TMEM.
+        uint32_t r[kTile];
+        tmem_ld32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_ld32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_ld32(s_row + 64, *reinterpret_cast<uint32_t(*)[32]>(r + 64));
+        tmem_ld32(s_row + 96, *reinterpret_cast<uint32_t(*)[32]>(r + 96));
+        tmem_ld_wait();
+        if (valid < kTile) {
+#pragma unroll
+          for (int i = 0; i < kTile; ++i)
+            if (i >= valid) r[i] = __float_as_uint(-INFINITY);
+        }
+        float mx8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(r[a]);
+#pragma unroll
+        for (int i = 8; i < kTile; i += 2)
+          mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], __uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const bool grow = (mx - m_run) * sl2 > kRescaleLog2;
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = mx;
+        } else if (__any_sync(0xffffffffu, grow)) {
+          const float m_new = fmaxf(m_run, mx);
+          // E4M3 P: bases are whole powers of two (see below), so alpha is one as well.
+          alpha = kF8 ? pow2i(static_cast<int>(ceilf(m_run * sl2) - ceilf(m_new * sl2)))
+                      : ex2_approx((m_run - m_new) * sl2);
+          m_run = m_new;
+          rescale = true;
+        }
+        // E4M3 P is taken against the base rounded up to a whole power of two: p <= 2^8
+        // still, and its codes are those of the exact-max base times an exact power of two
+        // (outside the subnormal range), whatever this row's running max is.
+        const float nb = kF8 ? -ceilf(m_run * sl2) : -m_run * sl2;
+        const unsigned long long sl2x2 = f2_pack(sl2, sl2), nbx2 = f2_pack(nb, nb);
+        unsigned long long rs4[4] = {0ull, 0ull, 0ull, 0ull};
+        if constexpr (kF8) {
+          // E4M3 P: four codes per register (quad i of the row lands in register i <= 4i).
+#pragma unroll
+          for (int i = 0; i < kTile / 4; ++i) {
+            const unsigned long long s01 = f2_pack(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]));
+            const unsigned long long s23 = f2_pack(__uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+            const float2 x01 = f2_unpack(f2_fma(s01, sl2x2, nbx2));
+            const float2 x23 = f2_unpack(f2_fma(s23, sl2x2, nbx2));
+            const float e0 = ex2_approx(x01.x), e1 = ex2_approx(x01.y);
+            // one exponential in eight on the FMA pipes (MUFU is the busier unit here)
+            const float e2 = ex2_approx(x23.x);
+            const float e3 = (i & 1) == 0 ? exp2_poly(x23.y) : ex2_approx(x23.y);
+            rs4[(2 * i) & 3] = f2_add(rs4[(2 * i) & 3], f2_pack(e0, e1));
+            rs4[(2 * i + 1) & 3] = f2_add(rs4[(2 * i + 1) & 3], f2_pack(e2, e3));
+            r[i] = pack_e4m3x4(e0, e1, e2, e3);
+          }
+          tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+        } else {
+#pragma unroll
+          for (int i = 0; i < kTile / 2; ++i) {
+            const unsigned long long s2 = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            const float2 x = f2_unpack(f2_fma(s2, sl2x2, nbx2));
+            const float e0 = ex2_approx(x.x);
+            const float e1 = ex2_approx(x.y);
+            rs4[i & 3] = f2_add(rs4[i & 3], f2_pack(e0, e1));
+            r[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st32(s_row, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_st32(s_row + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        }
+        if (rescale) {
+          // S_t(j) ready implies PV_t(j-1) completed, and PV_t(j) waits for this thread's
+          // arrival below: O_t is current and idle while it is rescaled here.
+#pragma unroll 1
+          for (int c = 0; c < kHd / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_row + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            tmem_st32(o_row + c * 32, o);
+          }
+          l_run *= alpha;
+        }
+        {
+          const float2 s01 = f2_unpack(f2_add(rs4[0], rs4[1])), s23 = f2_unpack(f2_add(rs4[2], rs4[3]));
+          l_run += (s01.x + s01.y) + (s23.x + s23.y);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      const bool done = ok && nkv > 0 && mbar_wait_warp(&o_final[t], static_cast<uint32_t>(it & 1), p.err);
+      if (!done) ok = false;
+      if (done && split >= 0) {
+        // Partial output of a key-split CTA: O unnormalised, with the row's base and sum.
+        tc_fence_after();
+        const int64_t slot = (static_cast<int64_t>(split) * kQTiles + t) * kTile + row;
+        float4* po = reinterpret_cast<float4*>(p.part_o + slot * kHd);
 #pragma unroll 1
         for (int c = 0; c < kHd / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_row + c * 32, o);
+          uint32_t r0[32];
+          tmem_ld32(o_row + c * 32, r0);
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(o_row + c * 32, o);
+          for (int g = 0; g < 8; ++g)
+            po[c * 8 + g] = make_float4(__uint_as_float(r0[4 * g]), __uint_as_float(r0[4 * g + 1]),
+                                        __uint_as_float(r0[4 * g + 2]), __uint_as_float(r0[4 * g + 3]));
         }
-        l_run *= alpha;
-      }
-      {
-        const float2 s01 = f2_unpack(f2_add(rs4[0], rs4[1])), s23 = f2_unpack(f2_add(rs4[2], rs4[3]));
-        l_run += (s01.x + s01.y) + (s23.x + s23.y);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
-    const bool done = ok && nkv > 0 && mbar_wait_warp(&o_final[t], 0, p.err);
-    if (done && split >= 0) {
-      // Partial output of a key-split CTA: O unnormalised, with the row's base and sum.
-      tc_fence_after();
-      const int64_t slot = (static_cast<int64_t>(split) * kQTiles + t) * kTile + row;
-      float4* po = reinterpret_cast<float4*>(p.part_o + slot * kHd);
-#pragma unroll 1
-      for (int c = 0; c < kHd / 32; ++c) {
-        uint32_t r0[32];
-        tmem_ld32(o_row + c * 32, r0);
-        tmem_ld_wait();
+        // E4M3: the whole-power-of-two base itself (the merge then uses scale 1).
+        const float m_common = kF8 ? ceilf(m_run * sl2) : m_run;
+        reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_common, l_run);
+      } else if (done) {
+        tc_fence_after();
+        const float inv = v_scale / l_run;
+        const int grow = q0 + t * kTile + row;
+        __nv_bfloat16* orow;
+        if (p.sc.ranks > 0) {
+          const int owner = min(grow / p.sc.rows_local, p.sc.ranks - 1);
+          const int64_t lrow = static_cast<int64_t>(b) * p.sc.rows_local + (grow - owner * p.sc.rows_local);
+          orow = static_cast<__nv_bfloat16*>(p.sc.dst[owner]) + lrow * p.o_row_stride + p.o_col0 + h * kHd;
+        } else {
+          orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride + static_cast<int64_t>(grow) * p.o_row_stride +
+                 p.o_col0 + h * kHd;
+        }
 #pragma unroll
-        for (int g = 0; g < 8; ++g)
-          po[c * 8 + g] = make_float4(__uint_as_float(r0[4 * g]), __uint_as_float(r0[4 * g + 1]),
-                                      __uint_as_float(r0[4 * g + 2]), __uint_as_float(r0[4 * g + 3]));
-      }
-      // E4M3: the whole-power-of-two base itself (the merge then uses scale 1).
-      const float m_common = kF8 ? ceilf(m_run * sl2) : m_run;
-      reinterpret_cast<float2*>(p.part_ml)[slot] = make_float2(m_common, l_run);
-    } else if (done) {
-      tc_fence_after();
-      const float inv = v_scale / l_run;
-      const int grow = q0 + t * kTile + row;
-      __nv_bfloat16* orow;
-      if (p.sc.ranks > 0) {
-        const int owner = min(grow / p.sc.rows_local, p.sc.ranks - 1);
-        const int64_t lrow = static_cast<int64_t>(b) * p.sc.rows_local + (grow - owner * p.sc.rows_local);
-        orow = static_cast<__nv_bfloat16*>(p.sc.dst[owner]) + lrow * p.o_row_stride + p.o_col0 + h * kHd;
-      } else {
-        orow = p.o + static_cast<int64_t>(b) * p.o_batch_stride + static_cast<int64_t>(grow) * p.o_row_stride +
-               p.o_col0 + h * kHd;
-      }
+        for (int c = 0; c < kHd / 64; ++c) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(o_row + c * 64, r0);
+          tmem_ld32(o_row + c * 64 + 32, r1);
+          tmem_ld_wait();
+          if (grow < p.Lq) {
 #pragma unroll
-      for (int c = 0; c < kHd / 64; ++c) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(o_row + c * 64, r0);
-        tmem_ld32(o_row + c * 64 + 32, r1);
-        tmem_ld_wait();
-        if (grow < p.Lq) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(r0[g * 8 + 0]) * inv, __uint_as_float(r0[g * 8 + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(r0[g * 8 + 2]) * inv, __uint_as_float(r0[g * 8 + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(r0[g * 8 + 4]) * inv, __uint_as_float(r0[g * 8 + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(r0[g * 8 + 6]) * inv, __uint_as_float(r0[g * 8 + 7]) * inv);
-            reinterpret_cast<uint4*>(orow + c * 64)[g] = u;
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r1[g * 8 + 0]) * inv, __uint_as_float(r1[g * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(r1[g * 8 + 2]) * inv, __uint_as_float(r1[g * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(r1[g * 8 + 4]) * inv, __uint_as_float(r1[g * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(r1[g * 8 + 6]) * inv, __uint_as_float(r1[g * 8 + 7]) * inv);
-            reinterpret_cast<uint4*>(orow + c * 64 + 32)[g] = w;
+            for (int g = 0; g < 4; ++g) {
+              uint4 u4;
+              u4.x = pack_bf16x2(__uint_as_float(r0[g * 8 + 0]) * inv, __uint_as_float(r0[g * 8 + 1]) * inv);
+              u4.y = pack_bf16x2(__uint_as_float(r0[g * 8 + 2]) * inv, __uint_as_float(r0[g * 8 + 3]) * inv);
+              u4.z = pack_bf16x2(__uint_as_float(r0[g * 8 + 4]) * inv, __uint_as_float(r0[g * 8 + 5]) * inv);
+              u4.w = pack_bf16x2(__uint_as_float(r0[g * 8 + 6]) * inv, __uint_as_float(r0[g * 8 + 7]) * inv);
+              reinterpret_cast<uint4*>(orow + c * 64)[g] = u4;
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(r1[g * 8 + 0]) * inv, __uint_as_float(r1[g * 8 + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(r1[g * 8 + 2]) * inv, __uint_as_float(r1[g * 8 + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(r1[g * 8 + 4]) * inv, __uint_as_float(r1[g * 8 + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(r1[g * 8 + 6]) * inv, __uint_as_float(r1[g * 8 + 7]) * inv);
+              reinterpret_cast<uint4*>(orow + c * 64 + 32)[g] = w;
+            }
           }
         }
       }
@@ -524,24 +595,26 @@ bool make_operand_map(CUtensorMap* map, const AttnOperand& op, int B, int L) {
   return make_tmap_bf16(map, op.ptr, 3, dims, strides, box);
 }
 
+template <bool kF8, bool kPersist>
+void set_attn_smem_once(int dev) {
+  static std::once_flag once[64];
+  std::call_once(once[dev & 63], [] {
+    cudaFuncSetAttribute(attn_fwd_tc_kernel<kF8, kPersist>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(AttnShape<kF8, kPersist>::kSmem));
+  });
+}
+
 // Grid, optional key split of a partial last wave, launch and merge (both operand kinds).
 template <bool kF8>
 int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, AttnParams& p, int B, int H,
                  int Lq, int Lk, cudaStream_t s, bool has_sc, void* scratch, size_t scratch_bytes) {
   p.err = device_error_flag();
-  constexpr size_t kSmem = AttnShape<kF8>::kSmem;
-  static std::once_flag once[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  std::call_once(once[dev & 63], [] {
-    cudaFuncSetAttribute(attn_fwd_tc_kernel<kF8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kSmem));
-  });
-  // One CTA per unit. When the last wave would leave more than half of the SMs idle,
-  // its units are split over the key tiles instead (two CTAs each) and merged after.
   p.pairs = (Lq + kQTiles * kTile - 1) / (kQTiles * kTile);
   const int64_t units = static_cast<int64_t>(B) * H * p.pairs;
   if (units >= (int64_t(1) << 31)) return WAN_ERR_SHAPE;
+  p.n_units = static_cast<int>(units);
   static int nsm_of[64] = {0};
   if (nsm_of[dev & 63] == 0) {
     int v = 0;
@@ -549,8 +622,28 @@ int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
     nsm_of[dev & 63] = v > 0 ? v : 148;
   }
   const int nsm = nsm_of[dev & 63];
-  const int64_t rem = units % nsm;
   const int nkv_all = (Lk + kTile - 1) / kTile;
+  const double work = 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd;
+  // Short key sequences (a unit is a few key tiles long, so loading Q, setting up and
+  // writing O would dominate a one-unit CTA): one persistent CTA per SM walks the
+  // units, loading the next unit's Q and starting its first products while the
+  // current unit's output is written.
+  if (!kF8 && nkv_all <= kMaxPersistKeyTiles) {
+    set_attn_smem_once<kF8, true>(dev);
+    p.n_full = p.n_units;
+    p.part_o = p.part_ml = nullptr;
+    const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
+    trace_launch_begin(WAN_KIND_ATTN, s, work);
+    attn_fwd_tc_kernel<kF8, true><<<grid, kAttnThreads, AttnShape<kF8, true>::kSmem, s>>>(mq, mk, mv, p);
+    const int st = check_launch();
+    trace_launch_end(WAN_KIND_ATTN, s);
+    return st;
+  }
+  set_attn_smem_once<kF8, false>(dev);
+  constexpr size_t kSmem = AttnShape<kF8>::kSmem;
+  // One CTA per unit. When the last wave would leave more than half of the SMs idle,
+  // its units are split over the key tiles instead (two CTAs each) and merged after.
+  const int64_t rem = units % nsm;
   const size_t part_o_bytes = static_cast<size_t>(2 * rem) * kQTiles * kTile * kHd * 4;
   const size_t part_bytes = part_o_bytes + static_cast<size_t>(2 * rem) * kQTiles * kTile * 8;
   // Only when a unit is long enough (16+ key tiles) for half of it to outweigh the
@@ -562,8 +655,8 @@ int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   p.part_o = split ? static_cast<float*>(scratch) : nullptr;
   p.part_ml = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + part_o_bytes) : nullptr;
   const unsigned grid = static_cast<unsigned>(split ? units + rem : units);
-  trace_launch_begin(WAN_KIND_ATTN, s, 4.0 * B * H * static_cast<double>(Lq) * Lk * kHd);
-  attn_fwd_tc_kernel<kF8><<<grid, kAttnThreads, kSmem, s>>>(mq, mk, mv, p);
+  trace_launch_begin(WAN_KIND_ATTN, s, work);
+  attn_fwd_tc_kernel<kF8, false><<<grid, kAttnThreads, kSmem, s>>>(mq, mk, mv, p);
   int st = check_launch();
   if (st == WAN_OK && split) {
     attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);

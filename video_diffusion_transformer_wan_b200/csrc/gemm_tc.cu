@@ -11,12 +11,14 @@
 //             overlaps the main loop of the next;
 //   warps 2-9: epilogue; warp w reads TMEM lanes 32*(w%4).. (rows of the tile) and one
 //             half of the tile's columns with tcgen05.ld, applies bias / activation /
-//             scale and writes global memory. The gated fp32 residual (its own
-//             instantiation) goes through a 32x32 shared-memory block per warp so that
-//             the read-modify-write of x moves whole 128-byte row segments; with the
-//             thread-per-row layout of the TMEM load it took 32 half-used sectors per
-//             instruction and the epilogue of the D x D projections did not hide under
-//             their short main loop.
+//             scale and writes global memory. The gated fp32 residual and the fp32
+//             store (their own instantiation) go through a 32x32 shared-memory block
+//             per warp so that the read-modify-write of x, or the store, moves whole
+//             128-byte row segments; with the thread-per-row layout of the TMEM load
+//             it took 32 half-used sectors per instruction, the epilogue of the D x D
+//             projections did not hide under their short main loop, and the patchify
+//             projection (K = 64, nearly all epilogue) stored at a quarter of the HBM
+//             bandwidth.
 //
 // Tile order: the row blocks are cut into groups of group_m; within a group the row
 // block varies fastest, so the 148 tiles in flight share a slab of at most
@@ -169,16 +171,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   }
 }
 
-// Gated residual epilogue through shared memory: for each 32-column chunk the warp
-// reads its 32 rows from TMEM (thread = row), scales and adds the bias, stages the
-// 32x32 block (16-byte units XOR-swizzled by row), then reads it back four rows per
-// instruction (8 threads x 16 bytes per row) so that every fp32 read-modify-write of x
-// moves whole 128-byte row segments.
+// Gated residual (and plain fp32 store) epilogue through shared memory: for each
+// 32-column chunk the warp reads its 32 rows from TMEM (thread = row), scales and adds
+// the bias, stages the 32x32 block (16-byte units XOR-swizzled by row), then reads it
+// back four rows per instruction (8 threads x 16 bytes per row) so that every fp32
+// read-modify-write of x (or store of the fp32 output) moves whole 128-byte row
+// segments.
 __device__ __forceinline__ void residual_staged(const GemmParams& p, float* stg, uint32_t t_row, int r0, int n0,
                                                 int lane, int chunks) {
   const int row = r0 + lane;
   const float sc = p.a_scale ? (row < p.M ? __ldg(p.a_scale + row) : 0.f) * __ldg(p.w_scale) : 1.0f;
   const int sub = lane >> 3, cq = lane & 7;
+  const bool residual = p.epi.kind == WAN_EPI_RESIDUAL;
 #pragma unroll 1
   for (int c = 0; c < chunks; ++c) {
     const int col0 = n0 + c * 32;
@@ -199,6 +203,18 @@ __device__ __forceinline__ void residual_staged(const GemmParams& p, float* stg,
     }
     __syncwarp();
     const int gcol = col0 + cq * 4;
+    if (!residual) {  // fp32 store
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = i * 4 + sub;
+        const int grow = r0 + rr;
+        if (grow < p.M && gcol < p.N)
+          *reinterpret_cast<float4*>(static_cast<float*>(p.out) + static_cast<int64_t>(grow) * p.epi.ldo + gcol) =
+              reinterpret_cast<const float4*>(stg + rr * 32)[cq ^ (rr & 7)];
+      }
+      __syncwarp();
+      continue;
+    }
     float4 gb = make_float4(0.f, 0.f, 0.f, 0.f);
     if (p.epi.gate_bias && gcol < p.N) gb = __ldg(reinterpret_cast<const float4*>(p.epi.gate_bias + gcol));
     float4 x[8];
@@ -470,8 +486,10 @@ int launch_bn(const void* A, int64_t lda, const void* W, const void* bias, void*
   p.err = device_error_flag();
   const int tiles = p.m_blocks * p.n_blocks;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  return epi.kind == WAN_EPI_RESIDUAL ? launch_inst<BN, kF8, true>(mapA, mapB, p, grid, s)
-                                      : launch_inst<BN, kF8, false>(mapA, mapB, p, grid, s);
+  // The gated residual and the fp32 store (the patchify projection, whose epilogue is
+  // nearly all of its time) take the staged epilogue.
+  const bool staged = epi.kind == WAN_EPI_RESIDUAL || epi.kind == WAN_EPI_F32;
+  return staged ? launch_inst<BN, kF8, true>(mapA, mapB, p, grid, s) : launch_inst<BN, kF8, false>(mapA, mapB, p, grid, s);
 }
 
 }  // namespace
