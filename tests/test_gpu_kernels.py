@@ -63,7 +63,10 @@ def test_layernorm_modulation(wan, dtype, D, B, L):
 
 # ------------------------------------------------------------------------------ K-c
 GEMM_SHAPES = [(300, 256, 1536), (129, 384, 192), (77, 64, 64), (50, 1536, 144), (1000, 4608, 128),
-               (513, 3072, 1536), (128, 8960 // 4, 256)]
+               (513, 3072, 1536), (128, 8960 // 4, 256),
+               # CTA-pair tiles (M >= 1024, N >= 256, K >= 256): a ragged last pair tile in
+               # rows (the odd CTA's half beyond M) and in columns
+               (1100, 768, 320), (2200, 1160, 512)]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

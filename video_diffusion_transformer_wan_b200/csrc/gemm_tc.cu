@@ -419,6 +419,195 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   gemm_body<BN, true, kRes>(mapA, mapB, p);
 }
 
+// ---------------------------------------------------------------- CTA-pair GEMM
+// bf16 GEMMs with N >= 256 on CTA pairs: a pair owns a 256 x 256 output tile; CTA r of
+// the pair loads rows [128 r, 128 r + 128) of the tile's A and of its W block (W rows =
+// output columns) into the same shared-memory offsets, and the even CTA's MMA thread
+// issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16), which reads both CTAs'
+// halves and leaves each CTA's 128 accumulator rows (all 256 columns) in its own TMEM.
+// Per SM and k-block of 64 this moves 32 KB into shared memory instead of 48 KB (the
+// 128 x 256 one-SM tile loads all of its 256 W rows), for the same FLOPs.
+// Barriers: each CTA's TMA loads complete on the even CTA's full[stage] (only the even
+// CTA's producer arms it, with both CTAs' bytes); the MMA commits release empty[stage]
+// and signal tfull[acc] in both CTAs; both CTAs' epilogue warps release tempty[acc] on
+// the even CTA. Barriers are initialised, and TMEM allocated, in both CTAs before a
+// cluster barrier; a second one precedes deallocation.
+constexpr int kPairStages = 6;
+constexpr int kPairStageBytes = 2 * kBM * 128;  // A half + W half: 128 rows x 128 bytes each
+template <bool kRes>
+struct PairCfg {
+  static constexpr size_t kEpiStageBytes = kRes ? static_cast<size_t>(kEpiWarps) * 32 * 32 * 4 : 0;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kPairStages) * kPairStageBytes + 256 + kEpiStageBytes;
+};
+
+template <bool kRes>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                          const GemmParams p) {
+  constexpr int kHalf = kBM * 128;  // bytes of one 128-row operand half per stage
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kHalf;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kHalf);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  float* epi_stage = reinterpret_cast<float*>(sB + kPairStages * kHalf + 256);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int num_tiles = p.m_blocks * p.n_blocks;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kPairStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 32 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  // The even CTA's barriers, as shared::cluster addresses.
+  const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+  const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
+        const int m0 = mb * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int n0 = nb * 2 * kBM + static_cast<int>(rank) * kBM;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+          const int kbw = p.wk_period_blocks > 0 ? kb % p.wk_period_blocks : kb;
+          const uint32_t bar = full0 + static_cast<uint32_t>(stage) * 8u;
+          tma_load_2d_pair(sA + stage * kHalf, &mapA, bar, kb * p.bk, m0);
+          tma_load_2d_pair(sB + stage * kHalf, &mapB, bar, kbw * p.bk, n0);
+          ++issued;
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: each slot's last load was consumed (the MMA's release reaches both CTAs),
+      // so no copy into this CTA's shared memory is in flight at exit.
+      for (int st = 0; st < kPairStages; ++st) {
+        const int64_t n_s = issued / kPairStages + (st < issued % kPairStages ? 1 : 0);
+        if (n_s > 0) mbar_wait(&empty[st], static_cast<uint32_t>((n_s - 1) & 1), p.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16_f32(2 * kBM, 2 * kBM, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; ok && tile < num_tiles; tile += npairs, ++it) {
+        const int acc = it & 1;
+        if (!mbar_wait(&tempty[acc], ((it >> 1) & 1) ^ 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * kHalf);
+          const uint32_t b_addr = smem_u32(sB + stage * kHalf);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {  // 32 bytes (16 bf16) of K per MMA
+            const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + k * 32, 16, 1024);
+            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit_pair(&tfull[acc], 0x3);
+      }
+      tc_commit_pair(drain, 0x1);
+      mbar_wait(drain, 0, p.err);
+    }
+  } else {
+    const int quarter = warp & 3;           // TMEM lanes 32*quarter .. (rows of this CTA's half)
+    const int colhalf = (warp - 2) >> 2;    // which 128 of the tile's 256 columns
+    constexpr int kMine = 4;                // 32-column chunks per warp
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+      const int acc = it & 1;
+      if (!mbar_wait_warp(&tfull[acc], (it >> 1) & 1, p.err)) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(p, tile, mb, nb);
+      const int m0 = mb * 2 * kBM + static_cast<int>(rank) * kBM;
+      const int n0 = nb * 2 * kBM + colhalf * kBM;
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * 256 + colhalf * kBM);
+      if constexpr (kRes) {
+        residual_staged(p, epi_stage + (warp - 2) * 1024, t_row, m0 + quarter * 32, n0, lane, kMine);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kMine; c += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_row + c * 32, r0);
+          tmem_ld32(t_row + (c + 1) * 32, r1);
+          tmem_ld_wait();
+          epilogue_chunk(p, row, n0 + c * 32, r0);
+          epilogue_chunk(p, row, n0 + (c + 1) * 32, r1);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(acc) * 8u);
+    }
+  }
+  // Both CTAs are done with TMEM (and no remote arrival is pending) before it is freed.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
 // Launch one instantiation (the shared-memory opt-in is set once per device for each).
 template <int BN, bool kF8, bool kRes>
 int launch_inst(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p, int grid, cudaStream_t s) {
@@ -445,6 +634,64 @@ int sm_count() {
     counts[dev] = n > 0 ? n : 148;
   }
   return counts[dev];
+}
+
+#ifndef WAN_GEMM_PAIR
+#define WAN_GEMM_PAIR 1  // bf16 GEMMs with N >= 256, K >= 256, M >= 1024 on CTA pairs
+#endif
+
+// bf16, N >= 256: the CTA-pair kernel (256 x 256 tiles).
+int launch_pair(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
+                int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+  CUtensorMap mapA, mapB;
+  const uint64_t dimsA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * 2};
+  const uint32_t box[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+  const int kw = w_k_period > 0 ? w_k_period : K;
+  const uint64_t dimsB[2] = {static_cast<uint64_t>(kw), static_cast<uint64_t>(N)};
+  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * 2};
+  if (!make_tmap_bf16(&mapA, A, 2, dimsA, strA, box) || !make_tmap_bf16(&mapB, W, 2, dimsB, strB, box))
+    return WAN_ERR_CUDA;
+  GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.bk = kBK;
+  p.k_blocks = (K + kBK - 1) / kBK;
+  p.wk_period_blocks = w_k_period > 0 ? w_k_period / kBK : 0;
+  p.m_blocks = (M + 2 * kBM - 1) / (2 * kBM);
+  p.n_blocks = (N + 2 * kBM - 1) / (2 * kBM);
+  {
+    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * 2 * 2 * kBM);
+    p.group_m = static_cast<int>(slab_rows < 1 ? 1 : (slab_rows > p.m_blocks ? p.m_blocks : slab_rows));
+  }
+  p.a_scale = nullptr;
+  p.w_scale = nullptr;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.out = out;
+  p.epi = epi;
+  p.err = device_error_flag();
+  const int tiles = p.m_blocks * p.n_blocks;
+  const int pairs = sm_count() / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  const bool staged = epi.kind == WAN_EPI_RESIDUAL || epi.kind == WAN_EPI_F32;
+  static std::once_flag once[2][64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (staged) {
+    std::call_once(once[1][dev & 63], [] {
+      cudaFuncSetAttribute(gemm_bf16_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(PairCfg<true>::kSmemBytes));
+    });
+    gemm_bf16_pair_kernel<true><<<grid, kGemmThreads, PairCfg<true>::kSmemBytes, s>>>(mapA, mapB, p);
+  } else {
+    std::call_once(once[0][dev & 63], [] {
+      cudaFuncSetAttribute(gemm_bf16_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(PairCfg<false>::kSmemBytes));
+    });
+    gemm_bf16_pair_kernel<false><<<grid, kGemmThreads, PairCfg<false>::kSmemBytes, s>>>(mapA, mapB, p);
+  }
+  return check_launch();
 }
 
 template <int BN, bool kF8>
@@ -505,6 +752,10 @@ int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, 
     st = launch_bn<64, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   else if (N <= 128)
     st = launch_bn<128, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+  else if (WAN_GEMM_PAIR && N >= 256 && K >= 256 && M >= 1024 && sm_count() >= 2)
+    // long enough main loops and enough row blocks for the pair tiles to pay (the patchify
+    // projection, K = 64, and the 512-row context projections stay on one SM)
+    st = launch_pair(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   else
     st = launch_bn<256, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   trace_launch_end(WAN_KIND_GEMM, s);
