@@ -440,10 +440,8 @@ struct PairCfg {
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kPairStages) * kPairStageBytes + 256 + kEpiStageBytes;
 };
 
-template <bool kRes>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                          const GemmParams p) {
+template <bool kF8, bool kRes>
+__device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
   constexpr int kHalf = kBM * 128;  // bytes of one 128-row operand half per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -529,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_bf16_f32(2 * kBM, 2 * kBM, 0, 0);
+      const uint32_t idesc = kF8 ? idesc_e4m3_f32(2 * kBM, 2 * kBM) : idesc_bf16_f32(2 * kBM, 2 * kBM, 0, 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -548,10 +546,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_addr = smem_u32(sA + stage * kHalf);
           const uint32_t b_addr = smem_u32(sB + stage * kHalf);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {  // 32 bytes (16 bf16) of K per MMA
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per MMA: 16 bf16 or 32 E4M3
             const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + k * 32, 16, 1024);
-            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (kF8)
+              tc_mma_e4m3_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
           if (++stage == kPairStages) {
@@ -608,6 +609,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+template <bool kRes>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                          const GemmParams p) {
+  gemm_pair_body<false, kRes>(mapA, mapB, p);
+}
+
+template <bool kRes>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_e4m3_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                          const GemmParams p) {
+  gemm_pair_body<true, kRes>(mapA, mapB, p);
+}
+
 // Launch one instantiation (the shared-memory opt-in is set once per device for each).
 template <int BN, bool kF8, bool kRes>
 int launch_inst(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p, int grid, cudaStream_t s) {
@@ -640,33 +655,39 @@ int sm_count() {
 #define WAN_GEMM_PAIR 1  // bf16 GEMMs with N >= 256, K >= 256, M >= 1024 on CTA pairs
 #endif
 
-// bf16, N >= 256: the CTA-pair kernel (256 x 256 tiles).
+// N >= 256: the CTA-pair kernels (256 x 256 tiles), bf16 or E4M3 operands.
+template <bool kF8>
 int launch_pair(const void* A, int64_t lda, const void* W, const void* bias, void* out, int M, int N, int K,
-                int w_k_period, const GemmEpi& epi, cudaStream_t s) {
+                int w_k_period, const GemmEpi& epi, cudaStream_t s, const float* a_scale = nullptr,
+                const float* w_scale = nullptr) {
+  constexpr int bk = kF8 ? 128 : 64;  // elements per 128-byte row
+  constexpr int es = kF8 ? 1 : 2;
   CUtensorMap mapA, mapB;
   const uint64_t dimsA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * 2};
-  const uint32_t box[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+  const uint64_t strA[1] = {static_cast<uint64_t>(lda) * es};
+  const uint32_t box[2] = {static_cast<uint32_t>(bk), static_cast<uint32_t>(kBM)};
   const int kw = w_k_period > 0 ? w_k_period : K;
   const uint64_t dimsB[2] = {static_cast<uint64_t>(kw), static_cast<uint64_t>(N)};
-  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * 2};
-  if (!make_tmap_bf16(&mapA, A, 2, dimsA, strA, box) || !make_tmap_bf16(&mapB, W, 2, dimsB, strB, box))
-    return WAN_ERR_CUDA;
+  const uint64_t strB[1] = {static_cast<uint64_t>(kw) * es};
+  const bool maps_ok = kF8 ? make_tmap_u8(&mapA, A, 2, dimsA, strA, box) && make_tmap_u8(&mapB, W, 2, dimsB, strB, box)
+                           : make_tmap_bf16(&mapA, A, 2, dimsA, strA, box) &&
+                                 make_tmap_bf16(&mapB, W, 2, dimsB, strB, box);
+  if (!maps_ok) return WAN_ERR_CUDA;
   GemmParams p;
   p.M = M;
   p.N = N;
   p.K = K;
-  p.bk = kBK;
-  p.k_blocks = (K + kBK - 1) / kBK;
-  p.wk_period_blocks = w_k_period > 0 ? w_k_period / kBK : 0;
+  p.bk = bk;
+  p.k_blocks = (K + bk - 1) / bk;
+  p.wk_period_blocks = w_k_period > 0 ? w_k_period / bk : 0;
   p.m_blocks = (M + 2 * kBM - 1) / (2 * kBM);
   p.n_blocks = (N + 2 * kBM - 1) / (2 * kBM);
   {
-    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * 2 * 2 * kBM);
+    const int64_t slab_rows = (static_cast<int64_t>(WAN_GEMM_SLAB_MB) << 20) / (static_cast<int64_t>(K) * es * 2 * kBM);
     p.group_m = static_cast<int>(slab_rows < 1 ? 1 : (slab_rows > p.m_blocks ? p.m_blocks : slab_rows));
   }
-  p.a_scale = nullptr;
-  p.w_scale = nullptr;
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
   p.bias = static_cast<const __nv_bfloat16*>(bias);
   p.out = out;
   p.epi = epi;
@@ -675,22 +696,16 @@ int launch_pair(const void* A, int64_t lda, const void* W, const void* bias, voi
   const int pairs = sm_count() / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
   const bool staged = epi.kind == WAN_EPI_RESIDUAL || epi.kind == WAN_EPI_F32;
+  auto kern = staged ? (kF8 ? gemm_e4m3_pair_kernel<true> : gemm_bf16_pair_kernel<true>)
+                     : (kF8 ? gemm_e4m3_pair_kernel<false> : gemm_bf16_pair_kernel<false>);
+  const size_t smem = staged ? PairCfg<true>::kSmemBytes : PairCfg<false>::kSmemBytes;
   static std::once_flag once[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (staged) {
-    std::call_once(once[1][dev & 63], [] {
-      cudaFuncSetAttribute(gemm_bf16_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(PairCfg<true>::kSmemBytes));
-    });
-    gemm_bf16_pair_kernel<true><<<grid, kGemmThreads, PairCfg<true>::kSmemBytes, s>>>(mapA, mapB, p);
-  } else {
-    std::call_once(once[0][dev & 63], [] {
-      cudaFuncSetAttribute(gemm_bf16_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(PairCfg<false>::kSmemBytes));
-    });
-    gemm_bf16_pair_kernel<false><<<grid, kGemmThreads, PairCfg<false>::kSmemBytes, s>>>(mapA, mapB, p);
-  }
+  std::call_once(once[staged ? 1 : 0][dev & 63],
+                 [kern, smem] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     static_cast<int>(smem)); });
+  kern<<<grid, kGemmThreads, smem, s>>>(mapA, mapB, p);
   return check_launch();
 }
 
@@ -755,7 +770,7 @@ int launch_gemm_tc(const void* A, int64_t lda, const void* W, const void* bias, 
   else if (WAN_GEMM_PAIR && N >= 256 && K >= 256 && M >= 1024 && sm_count() >= 2)
     // long enough main loops and enough row blocks for the pair tiles to pay (the patchify
     // projection, K = 64, and the 512-row context projections stay on one SM)
-    st = launch_pair(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
+    st = launch_pair<false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   else
     st = launch_bn<256, false>(A, lda, W, bias, out, M, N, K, w_k_period, epi, s);
   trace_launch_end(WAN_KIND_GEMM, s);
@@ -772,6 +787,8 @@ int launch_gemm_e4m3(const void* A, int64_t lda, const float* a_scale, const voi
     st = launch_bn<64, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
   else if (N <= 128)
     st = launch_bn<128, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
+  else if (WAN_GEMM_PAIR && N >= 256 && K >= 512 && M >= 1024 && sm_count() >= 2)
+    st = launch_pair<true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
   else
     st = launch_bn<256, true>(A, lda, W, bias, out, M, N, K, 0, epi, s, a_scale, w_scale);
   trace_launch_end(WAN_KIND_GEMM, s);
