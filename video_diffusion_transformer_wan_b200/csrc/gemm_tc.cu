@@ -432,16 +432,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // and signal tfull[acc] in both CTAs; both CTAs' epilogue warps release tempty[acc] on
 // the even CTA. Barriers are initialised, and TMEM allocated, in both CTAs before a
 // cluster barrier; a second one precedes deallocation.
-constexpr int kPairStages = 6;
+#ifndef WAN_PAIR_STAGES_PLAIN
+#define WAN_PAIR_STAGES_PLAIN 6  // ring depth of the pair kernel without the staged epilogue
+#endif
 constexpr int kPairStageBytes = 2 * kBM * 128;  // A half + W half: 128 rows x 128 bytes each
 template <bool kRes>
 struct PairCfg {
+  static constexpr int kStages = kRes ? 6 : WAN_PAIR_STAGES_PLAIN;
   static constexpr size_t kEpiStageBytes = kRes ? static_cast<size_t>(kEpiWarps) * 32 * 32 * 4 : 0;
-  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kPairStages) * kPairStageBytes + 256 + kEpiStageBytes;
+  static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kPairStageBytes + 256 + kEpiStageBytes;
 };
 
 template <bool kF8, bool kRes>
 __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
+  constexpr int kPairStages = PairCfg<kRes>::kStages;
   constexpr int kHalf = kBM * 128;  // bytes of one 128-row operand half per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
