@@ -67,20 +67,25 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def attn_traffic_per_launch():
+def attn_traffic_per_launch(w):
     """DRAM bytes (read + write) per self-attention launch from the committed ncu
-    summary, or None when the kernel source changed since the counters were taken."""
+    summary, or None when the kernel source changed since the counters were taken or
+    the summary's launch shape (batch, tokens, heads) is not this workload's."""
     p = os.path.join(PROFILES, "attn_fwd_tc_kernel__self_L32760_H12.md")
     src = os.path.join(ROOT, "video_diffusion_transformer_wan_b200", "csrc", "attn_tc.cu")
     if not os.path.exists(p):
         return None
-    sha = byts = None
+    sha = byts = shape = None
     for line in open(p):
         if line.startswith("- attn_tc.cu sha256:"):
             sha = line.split(":", 1)[1].strip()
         elif line.startswith("- dram bytes per launch (read+write):"):
             byts = float(line.split(":", 1)[1])
+        elif line.startswith("- launch shape (batch, tokens, heads):"):
+            shape = tuple(int(v) for v in line.split(":", 1)[1].split(","))
     if sha != hashlib.sha256(open(src, "rb").read()).hexdigest():
+        return None
+    if shape != (w.batch, w.tokens, w.heads):
         return None
     return byts
 
@@ -271,6 +276,8 @@ def kernel_report(w, recs, steps, ms_step, clocks):
     acc = {k: [0.0, 0.0] for k in ["self_attention", "cross_attention", "gemm", "patchify_gemm", "head_gemm",
                                    "layernorm", "small"]}
     top = max(wk for k, _, wk in recs if k == wan.KIND_ATTN)
+    # self-attention launches per step (one per block)
+    n_sa = sum(1 for k, _, wk in recs[:per] if k == wan.KIND_ATTN and wk == top)
     for i in range(steps):
         chunk = recs[i * per:(i + 1) * per]
         gi = [j for j, (k, _, _) in enumerate(chunk) if k == wan.KIND_GEMM]
@@ -301,12 +308,12 @@ def kernel_report(w, recs, steps, ms_step, clocks):
         out[name] = d
     out["peaks"] = {"bf16_tflops": peak["value"], "bf16_source": peak["source"], "hbm_gbs": peak["hbm_gbs"],
                     "hbm_source": f"{peak_src} hbm_gbs"}
-    sa_ms = acc["self_attention"][0] / steps
+    sa_ms = acc["self_attention"][0] / (steps * n_sa)
     roofline = {"bound": "tensor", "kernel": "attn_fwd_tc_kernel (self-attention)",
                 "achieved": top / (sa_ms / 1e3) / 1e12, "peak": peak["value"], "unit": "TFLOP/s",
                 "frac": top / (sa_ms / 1e3) / 1e12 / peak["value"], "peak_source": peak["source"],
                 "sm_mhz": mhz, "work_per_launch": top, "ms_per_launch": sa_ms,
-                "traffic": attn_traffic_per_launch()}
+                "traffic": attn_traffic_per_launch(w)}
     return out, roofline, peak
 
 

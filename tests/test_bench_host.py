@@ -95,3 +95,30 @@ def test_kernel_report_splits_a_step(bench):
     assert k["layernorm"]["gbs"] == pytest.approx(4 * 3e8 / 0.2e-3 / 1e9)
     with pytest.raises(RuntimeError):
         bench.kernel_report(w, recs[:-1], 2, 8.5, {"sm_mhz": 1900})
+
+
+def test_kernel_report_per_launch_roofline_with_several_blocks(bench):
+    """A stack step runs one self-attention per block: the roofline entry is per launch
+    (the step's self-attention time divided by the launches), the per-kind entry per step."""
+    import video_diffusion_transformer_wan_b200 as wan
+    w = WORKLOADS["wan13b_480p_stack30"]
+    G, A, N = wan.KIND_GEMM, wan.KIND_ATTN, wan.KIND_NORM
+    sa, ca = 6.594e12, 0.103e12
+    block = [(N, 0.05, 3e8), (G, 0.4, 4.6e11), (A, 5.5, sa), (G, 0.15, 1.5e11), (A, 0.2, ca), (G, 0.7, 9e11)]
+    step = [(G, 0.05, 6.4e9)] + block * 3 + [(G, 0.03, 6.4e9)]
+    k, roof, _ = bench.kernel_report(w, step * 2, 2, 20.0, {"sm_mhz": 1900})
+    assert k["self_attention"]["ms_per_step"] == pytest.approx(3 * 5.5)
+    assert k["self_attention"]["tflops"] == pytest.approx(sa / 5.5e-3 / 1e12)
+    assert roof["ms_per_launch"] == pytest.approx(5.5)
+    assert roof["achieved"] == pytest.approx(sa / 5.5e-3 / 1e12)
+
+
+def test_attention_traffic_only_for_the_profiled_launch_shape(bench):
+    """The committed ncu traffic is reported for workloads whose self-attention launch
+    has the captured shape (batch 1, 32760 tokens, 12 heads) and for no other."""
+    t = bench.attn_traffic_per_launch(WORKLOADS["wan13b_480p_block"])
+    assert bench.attn_traffic_per_launch(WORKLOADS["wan14b_720p_block"]) is None
+    if t is not None:   # None when attn_tc.cu changed since the capture
+        assert t > 0
+        assert bench.attn_traffic_per_launch(WORKLOADS["wan13b_480p_stack30"]) == t
+        assert bench.attn_traffic_per_launch(WORKLOADS["wan13b_480p_i2v_block"]) == t
