@@ -4,7 +4,8 @@
 // cross-attention over 512 umT5 tokens in every block). softmax(q k^T / sqrt(d)) v per
 // head, non-causal, bf16 inputs, fp32 accumulation and fp32 softmax, head_dim 128.
 //
-// One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 320 threads:
+// One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 384 threads in
+// three warpgroups:
 //   warp 0    : TMA producer - both Q tiles once, then K_0, K_1, V_0, K_2, V_1, ...
 //               (the order the MMA warp consumes them) through a 5-stage ring of 32 KB
 //               tiles (128 rows x 128 dims as two 64-dim halves, 128-byte swizzle);
@@ -13,7 +14,8 @@
 //               operand in shared memory), then S_t = Q_t K_j^T, then a commit that
 //               signals S_t ready. MMAs of one thread execute in issue order, so that
 //               signal also means P_t has been consumed and O_t holds every earlier PV;
-//   warps 2-5 : softmax of query tile 0, warps 6-9: of query tile 1; one thread per
+//   warps 2-3 : idle (they complete warpgroup 0, which hands registers to the softmax);
+//   warps 4-7 : softmax of query tile 0, warps 8-11: of query tile 1; one thread per
 //               query row (warp % 4 selects the TMEM lane quarter). The row's 128 S
 //               values are read from TMEM with a single wait (the wait covers every
 //               outstanding TMEM load, so reading in pieces would expose its latency
@@ -28,6 +30,12 @@
 //               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
 //               base and p <= 256 stays well inside fp32 and bf16 range.
 // While one tile's softmax runs, the tensor core works on the other tile's MMAs.
+// Registers: the CTA launches at 168 a thread (the most 384 threads may hold); then
+// warpgroup 0 gives up all but 88 (setmaxnreg.dec) and the two softmax warpgroups take
+// 208 (setmaxnreg.inc): 128 x 88 + 256 x 208 = 384 x 168, and on each SM sub-partition
+// (one warp of each warpgroup) 88 + 208 + 208 = 3 x 168, so every increase is covered
+// by the decrease. The softmax keeps a whole 128-value S row in registers; at 168 a
+// thread (320 threads, two warps per sub-partition spare) it spilled loop state.
 // Work units are (sample, head, pair of query tiles), one CTA each, in a 1D grid. When
 // the last wave would fill at most half of the SMs, its units are split over the key
 // tiles instead (two CTAs per unit, each over half of them); those CTAs write their
@@ -57,7 +65,11 @@
 namespace wan {
 namespace {
 
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;
+constexpr int kRegsLow = 88;    // warpgroup 0 (producer, MMA issuer, two idle warps)
+constexpr int kRegsHigh = 208;  // warpgroups 1-2 (softmax)
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kAttnThreads * 168, "register split above the launch");
+static_assert(kRegsLow + 2 * kRegsHigh <= 3 * 168, "register split above a sub-partition's share");
 constexpr int kTile = 128;                     // query rows per tile = key rows per tile
 constexpr int kHd = 128;                       // head dim
 constexpr int kQTiles = 2;                     // query tiles per CTA
@@ -198,171 +210,175 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      const int n_loads = 2 * nkv;
-      int issued = 0;  // ring loads issued so far (all units)
-      int q_loads = 0;
-      bool ok = true;
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const UnitPos u = decode(unit_of(it));
-        const int qb = it % kQBufs;
-        if (kPersist && it >= kQBufs &&
-            !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), p.err))
-          break;
-        uint8_t* sq = sQ + qb * kQTiles * kTileBytes;
-        mbar_arrive_expect_tx(&q_full[qb], kQTiles * kTileBytes);
-        const int qc = p.q_col0 + u.h * kHd;
-        for (int t = 0; t < kQTiles; ++t)
-          for (int c = 0; c < kSpans; ++c)
-            tma_load_3d(sq + t * kTileBytes + c * kHalfBytes, &mapQ, &q_full[qb], qc + 64 * c, u.q0 + t * kTile, u.b);
-        ++q_loads;
-        for (int ld = 0; ld < n_loads; ++ld) {
-          const int stage = issued % kStages;
-          const uint32_t phase = static_cast<uint32_t>((issued / kStages) & 1);
-          if (!mbar_wait(&kv_empty[stage], phase ^ 1u, p.err)) {
-            ok = false;
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsLow>();
+    if (warp == 0) {
+      if (lane == 0) {
+        const int n_loads = 2 * nkv;
+        int issued = 0;  // ring loads issued so far (all units)
+        int q_loads = 0;
+        bool ok = true;
+        for (int it = 0; ok && it < n_iter; ++it) {
+          const UnitPos u = decode(unit_of(it));
+          const int qb = it % kQBufs;
+          if (kPersist && it >= kQBufs &&
+              !mbar_wait(&q_empty[qb], static_cast<uint32_t>((it / kQBufs - 1) & 1), p.err))
             break;
-          }
-          bool is_v;
-          int j;
-          if (ld == 0) {
-            is_v = false, j = 0;
-          } else if (ld == n_loads - 1) {
-            is_v = true, j = nkv - 1;
-          } else if (ld & 1) {
-            is_v = false, j = (ld + 1) >> 1;
-          } else {
-            is_v = true, j = (ld >> 1) - 1;
-          }
-          const CUtensorMap* map = is_v ? &mapV : &mapK;
-          const int col = (is_v ? p.v_col0 : p.k_col0) + u.h * kHd;
-          uint8_t* dst = sKV + stage * kTileBytes;
-          mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
-          if (kF8 && is_v) {  // V^T: 128 dims (rows) x 128 keys (x)
-            tma_load_3d(dst, map, &kv_full[stage], (kv0 + j) * kTile, p.v_col0 + u.h * kHd, u.b);
-          } else {
+          uint8_t* sq = sQ + qb * kQTiles * kTileBytes;
+          mbar_arrive_expect_tx(&q_full[qb], kQTiles * kTileBytes);
+          const int qc = p.q_col0 + u.h * kHd;
+          for (int t = 0; t < kQTiles; ++t)
             for (int c = 0; c < kSpans; ++c)
-              tma_load_3d(dst + c * kHalfBytes, map, &kv_full[stage], col + 64 * c, (kv0 + j) * kTile, u.b);
-          }
-          ++issued;
-        }
-      }
-      // Wait for every copy this thread started (the last fill of each buffer and stage).
-      for (int q = 0; q < kQBufs; ++q) {
-        const int n_q = q_loads / kQBufs + (q < q_loads % kQBufs ? 1 : 0);
-        if (n_q > 0) mbar_wait(&q_full[q], static_cast<uint32_t>((n_q - 1) & 1), p.err);
-      }
-      for (int s = 0; s < kStages; ++s) {
-        const int n_s = issued / kStages + (s < issued % kStages ? 1 : 0);
-        if (n_s > 0) mbar_wait(&kv_full[s], static_cast<uint32_t>((n_s - 1) & 1), p.err);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(kTile, kTile) : idesc_bf16_f32(kTile, kTile, 0, 0);
-      // PV: bf16 V is an MN-major operand; E4M3 V arrives transposed, so K-major.
-      const uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(kTile, kHd) : idesc_bf16_f32(kTile, kHd, 0, 1);
-      // Shared-memory descriptors are built once: every operand below sits at a fixed
-      // byte offset from sQ or sKV, and an offset moves only the 14-bit address field
-      // (offset >> 4, no carry out of it since shared addresses stay below 256 KB). The
-      // single issuing thread then spends one add per operand on each MMA.
-      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t k_desc = sdesc_sw128(smem_u32(sKV), 16, 1024);
-      const uint64_t v_desc = sdesc_sw128(smem_u32(sKV), kF8 ? 16 : kHalfBytes, 1024);
-      auto wait_pos = [&](int pos) {
-        return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
-      };
-      auto pv = [&](int t, int i, int vstage) {
-        // A = P_t in TMEM, packed from the first column of S_t's region (bf16 pairs or
-        // E4M3 quads per column, so 8 columns per MMA either way).
-        const uint32_t p_tmem = tmem_base + t * kTile;
-        const uint64_t vd = v_desc + static_cast<uint32_t>((vstage * kTileBytes) >> 4);
-        const uint32_t o_tmem = tmem_base + 256 + t * kTile;
-#pragma unroll
-        for (int k = 0; k < kMmas; ++k) {
-          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          if constexpr (kF8)
-            tc_mma_e4m3_ts(o_tmem, p_tmem + k * 8, vd + ((k * 32) >> 4), idesc_pv, acc);
-          else
-            tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, acc);
-        }
-      };
-      auto qk = [&](int t, int qb, int kstage) {
-        const uint64_t qd = q_desc + static_cast<uint32_t>(((qb * kQTiles + t) * kTileBytes) >> 4);
-        const uint64_t kd = k_desc + static_cast<uint32_t>((kstage * kTileBytes) >> 4);
-        const uint32_t s_tmem = tmem_base + t * kTile;
-#pragma unroll
-        for (int k = 0; k < kMmas; ++k) {
-          const uint32_t off = ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4;  // 32 bytes of K per MMA
-          if constexpr (kF8)
-            tc_mma_e4m3(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
-          else
-            tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
-        }
-      };
-      bool ok = true;
-      for (int it = 0; ok && it < n_iter; ++it) {
-        const int qb = it % kQBufs;
-        const int base = it * 2 * nkv;   // ring position of this unit's first load
-        const int tiles = it * nkv;      // key tiles of earlier units (S / P phases)
-        if (!mbar_wait(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1), p.err)) break;
-        for (int j = 0; ok && j < nkv; ++j) {
-          const int pk = base + pos_k(j);
-          if (!wait_pos(pk)) {
-            ok = false;
-            break;
-          }
-          int pvpos = -1;
-          if (j > 0) {
-            pvpos = base + pos_v(j - 1, nkv);
-            if (!wait_pos(pvpos)) {
+              tma_load_3d(sq + t * kTileBytes + c * kHalfBytes, &mapQ, &q_full[qb], qc + 64 * c, u.q0 + t * kTile, u.b);
+          ++q_loads;
+          for (int ld = 0; ld < n_loads; ++ld) {
+            const int stage = issued % kStages;
+            const uint32_t phase = static_cast<uint32_t>((issued / kStages) & 1);
+            if (!mbar_wait(&kv_empty[stage], phase ^ 1u, p.err)) {
               ok = false;
               break;
             }
+            bool is_v;
+            int j;
+            if (ld == 0) {
+              is_v = false, j = 0;
+            } else if (ld == n_loads - 1) {
+              is_v = true, j = nkv - 1;
+            } else if (ld & 1) {
+              is_v = false, j = (ld + 1) >> 1;
+            } else {
+              is_v = true, j = (ld >> 1) - 1;
+            }
+            const CUtensorMap* map = is_v ? &mapV : &mapK;
+            const int col = (is_v ? p.v_col0 : p.k_col0) + u.h * kHd;
+            uint8_t* dst = sKV + stage * kTileBytes;
+            mbar_arrive_expect_tx(&kv_full[stage], kTileBytes);
+            if (kF8 && is_v) {  // V^T: 128 dims (rows) x 128 keys (x)
+              tma_load_3d(dst, map, &kv_full[stage], (kv0 + j) * kTile, p.v_col0 + u.h * kHd, u.b);
+            } else {
+              for (int c = 0; c < kSpans; ++c)
+                tma_load_3d(dst + c * kHalfBytes, map, &kv_full[stage], col + 64 * c, (kv0 + j) * kTile, u.b);
+            }
+            ++issued;
           }
-          for (int t = 0; ok && t < kQTiles; ++t) {
+        }
+        // Wait for every copy this thread started (the last fill of each buffer and stage).
+        for (int q = 0; q < kQBufs; ++q) {
+          const int n_q = q_loads / kQBufs + (q < q_loads % kQBufs ? 1 : 0);
+          if (n_q > 0) mbar_wait(&q_full[q], static_cast<uint32_t>((n_q - 1) & 1), p.err);
+        }
+        for (int s = 0; s < kStages; ++s) {
+          const int n_s = issued / kStages + (s < issued % kStages ? 1 : 0);
+          if (n_s > 0) mbar_wait(&kv_full[s], static_cast<uint32_t>((n_s - 1) & 1), p.err);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        const uint32_t idesc_qk = kF8 ? idesc_e4m3_f32(kTile, kTile) : idesc_bf16_f32(kTile, kTile, 0, 0);
+        // PV: bf16 V is an MN-major operand; E4M3 V arrives transposed, so K-major.
+        const uint32_t idesc_pv = kF8 ? idesc_e4m3_f32(kTile, kHd) : idesc_bf16_f32(kTile, kHd, 0, 1);
+        // Shared-memory descriptors are built once: every operand below sits at a fixed
+        // byte offset from sQ or sKV, and an offset moves only the 14-bit address field
+        // (offset >> 4, no carry out of it since shared addresses stay below 256 KB). The
+        // single issuing thread then spends one add per operand on each MMA.
+        const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t k_desc = sdesc_sw128(smem_u32(sKV), 16, 1024);
+        const uint64_t v_desc = sdesc_sw128(smem_u32(sKV), kF8 ? 16 : kHalfBytes, 1024);
+        auto wait_pos = [&](int pos) {
+          return mbar_wait(&kv_full[pos % kStages], static_cast<uint32_t>((pos / kStages) & 1), p.err);
+        };
+        auto pv = [&](int t, int i, int vstage) {
+          // A = P_t in TMEM, packed from the first column of S_t's region (bf16 pairs or
+          // E4M3 quads per column, so 8 columns per MMA either way).
+          const uint32_t p_tmem = tmem_base + t * kTile;
+          const uint64_t vd = v_desc + static_cast<uint32_t>((vstage * kTileBytes) >> 4);
+          const uint32_t o_tmem = tmem_base + 256 + t * kTile;
+#pragma unroll
+          for (int k = 0; k < kMmas; ++k) {
+            const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+            if constexpr (kF8)
+              tc_mma_e4m3_ts(o_tmem, p_tmem + k * 8, vd + ((k * 32) >> 4), idesc_pv, acc);
+            else
+              tc_mma_bf16_ts(o_tmem, p_tmem + k * 8, vd + ((k * 16 * 128) >> 4), idesc_pv, acc);
+          }
+        };
+        auto qk = [&](int t, int qb, int kstage) {
+          const uint64_t qd = q_desc + static_cast<uint32_t>(((qb * kQTiles + t) * kTileBytes) >> 4);
+          const uint64_t kd = k_desc + static_cast<uint32_t>((kstage * kTileBytes) >> 4);
+          const uint32_t s_tmem = tmem_base + t * kTile;
+#pragma unroll
+          for (int k = 0; k < kMmas; ++k) {
+            const uint32_t off = ((k >> 2) * kHalfBytes + (k & 3) * 32) >> 4;  // 32 bytes of K per MMA
+            if constexpr (kF8)
+              tc_mma_e4m3(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(s_tmem, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
+          }
+        };
+        bool ok = true;
+        for (int it = 0; ok && it < n_iter; ++it) {
+          const int qb = it % kQBufs;
+          const int base = it * 2 * nkv;   // ring position of this unit's first load
+          const int tiles = it * nkv;      // key tiles of earlier units (S / P phases)
+          if (!mbar_wait(&q_full[qb], static_cast<uint32_t>((it / kQBufs) & 1), p.err)) break;
+          for (int j = 0; ok && j < nkv; ++j) {
+            const int pk = base + pos_k(j);
+            if (!wait_pos(pk)) {
+              ok = false;
+              break;
+            }
+            int pvpos = -1;
             if (j > 0) {
-              if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + j - 1) & 1), p.err)) {
+              pvpos = base + pos_v(j - 1, nkv);
+              if (!wait_pos(pvpos)) {
                 ok = false;
                 break;
               }
-              // The first PV of a unit overwrites O_t. The softmax threads of tile t
-              // read the previous unit's O_t out (and waited for those reads) before
-              // they arrived on p_full for this unit's first key tile, so it is free.
-              tc_fence_after();
-              pv(t, j - 1, pvpos % kStages);
             }
-            qk(t, qb, pk % kStages);
-            tc_commit(&s_full[t]);
+            for (int t = 0; ok && t < kQTiles; ++t) {
+              if (j > 0) {
+                if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + j - 1) & 1), p.err)) {
+                  ok = false;
+                  break;
+                }
+                // The first PV of a unit overwrites O_t. The softmax threads of tile t
+                // read the previous unit's O_t out (and waited for those reads) before
+                // they arrived on p_full for this unit's first key tile, so it is free.
+                tc_fence_after();
+                pv(t, j - 1, pvpos % kStages);
+              }
+              qk(t, qb, pk % kStages);
+              tc_commit(&s_full[t]);
+            }
+            if (!ok) break;
+            tc_commit(&kv_empty[pk % kStages]);
+            if (j > 0) tc_commit(&kv_empty[pvpos % kStages]);
+          }
+          if (!ok || nkv == 0) break;
+          tc_commit(&q_empty[qb]);   // every QK of this unit issued: Q buffer free once they complete
+          const int last = nkv - 1;
+          const int pvpos = base + pos_v(last, nkv);
+          ok = wait_pos(pvpos);
+          for (int t = 0; ok && t < kQTiles; ++t) {
+            if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + last) & 1), p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            pv(t, last, pvpos % kStages);
+            tc_commit(&o_final[t]);
           }
           if (!ok) break;
-          tc_commit(&kv_empty[pk % kStages]);
-          if (j > 0) tc_commit(&kv_empty[pvpos % kStages]);
+          tc_commit(&kv_empty[pvpos % kStages]);
         }
-        if (!ok || nkv == 0) break;
-        tc_commit(&q_empty[qb]);   // every QK of this unit issued: Q buffer free once they complete
-        const int last = nkv - 1;
-        const int pvpos = base + pos_v(last, nkv);
-        ok = wait_pos(pvpos);
-        for (int t = 0; ok && t < kQTiles; ++t) {
-          if (!mbar_wait(&p_full[t], static_cast<uint32_t>((tiles + last) & 1), p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          pv(t, last, pvpos % kStages);
-          tc_commit(&o_final[t]);
-        }
-        if (!ok) break;
-        tc_commit(&kv_empty[pvpos % kStages]);
+        tc_commit(drain);
+        mbar_wait(drain, 0, p.err);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, p.err);
     }
   } else {
+    setmaxnreg_inc<kRegsHigh>();
     // Softmax: query tile t, TMEM lane quarter (warp % 4), row 32 * quarter + lane.
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
