@@ -5,7 +5,7 @@
 // head, non-causal, bf16 inputs, fp32 accumulation and fp32 softmax, head_dim 128.
 //
 // One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 384 threads in
-// three warpgroups:
+// three warpgroups (bf16; the E4M3 instantiation has 320, without warps 2-3):
 //   warp 0    : TMA producer - both Q tiles once, then K_0, K_1, V_0, K_2, V_1, ...
 //               (the order the MMA warp consumes them) through a 5-stage ring of 32 KB
 //               tiles (128 rows x 128 dims as two 64-dim halves, 128-byte swizzle);
@@ -30,12 +30,13 @@
 //               (O_t in TMEM and the sum are rescaled then): softmax is invariant to the
 //               base and p <= 256 stays well inside fp32 and bf16 range.
 // While one tile's softmax runs, the tensor core works on the other tile's MMAs.
-// Registers: the CTA launches at 168 a thread (the most 384 threads may hold); then
-// warpgroup 0 gives up all but 88 (setmaxnreg.dec) and the two softmax warpgroups take
-// 208 (setmaxnreg.inc): 128 x 88 + 256 x 208 = 384 x 168, and on each SM sub-partition
-// (one warp of each warpgroup) 88 + 208 + 208 = 3 x 168, so every increase is covered
-// by the decrease. The softmax keeps a whole 128-value S row in registers; at 168 a
-// thread (320 threads, two warps per sub-partition spare) it spilled loop state.
+// Registers (bf16): the CTA launches at 168 a thread (the most 384 threads may hold);
+// then warpgroup 0 gives up all but 88 (setmaxnreg.dec) and the two softmax warpgroups
+// take 208 (setmaxnreg.inc): 128 x 88 + 256 x 208 = 384 x 168, and on each SM
+// sub-partition (one warp of each warpgroup) 88 + 208 + 208 = 3 x 168, so every increase
+// is covered by the decrease. The softmax keeps a whole 128-value S row in registers; at
+// 168 a thread it spilled loop state. The E4M3 kernel did not spill at 168 and measured
+// about 1 % slower with the split, so it keeps 320 threads at 168.
 // Work units are (sample, head, pair of query tiles), one CTA each, in a 1D grid. When
 // the last wave would fill at most half of the SMs, its units are split over the key
 // tiles instead (two CTAs per unit, each over half of them); those CTAs write their
@@ -65,10 +66,9 @@
 namespace wan {
 namespace {
 
-constexpr int kAttnThreads = 384;
 constexpr int kRegsLow = 88;    // warpgroup 0 (producer, MMA issuer, two idle warps)
 constexpr int kRegsHigh = 208;  // warpgroups 1-2 (softmax)
-static_assert(128 * kRegsLow + 256 * kRegsHigh <= kAttnThreads * 168, "register split above the launch");
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split above the launch");
 static_assert(kRegsLow + 2 * kRegsHigh <= 3 * 168, "register split above a sub-partition's share");
 constexpr int kTile = 128;                     // query rows per tile = key rows per tile
 constexpr int kHd = 128;                       // head dim
@@ -87,6 +87,10 @@ struct AttnShape {
   static constexpr int kQBufs = kPersist ? 2 : 1;
   static constexpr int kStages = kPersist ? 3 : (kF8 ? 8 : 5);
   static constexpr int kMmas = kF8 ? 4 : 8;
+  // bf16: three warpgroups with the register split; E4M3: 320 threads, no split
+  static constexpr bool kRegSplit = !kF8;
+  static constexpr int kThreads = kRegSplit ? 384 : 320;
+  static constexpr int kSoftmaxWarp0 = kRegSplit ? 4 : 2;  // first softmax warp
   static constexpr size_t kSmem =
       1024 + static_cast<size_t>(kTileBytes) * (kQBufs * kQTiles + kStages) + 256;
 };
@@ -125,7 +129,7 @@ __device__ __forceinline__ int pos_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
 __device__ __forceinline__ int pos_v(int j, int n) { return j == n - 1 ? 2 * n - 1 : 2 * j + 2; }
 
 template <bool kF8, bool kPersist>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(AttnShape<kF8, kPersist>::kThreads, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const AttnParams p) {
   using Shape = AttnShape<kF8, kPersist>;
@@ -210,8 +214,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp < 4) {
-    setmaxnreg_dec<kRegsLow>();
+  if (warp < Shape::kSoftmaxWarp0) {
+    if constexpr (Shape::kRegSplit) setmaxnreg_dec<kRegsLow>();
     if (warp == 0) {
       if (lane == 0) {
         const int n_loads = 2 * nkv;
@@ -376,9 +380,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
   } else {
-    setmaxnreg_inc<kRegsHigh>();
+    if constexpr (Shape::kRegSplit) setmaxnreg_inc<kRegsHigh>();
     // Softmax: query tile t, TMEM lane quarter (warp % 4), row 32 * quarter + lane.
-    const int t = (warp - 4) >> 2;
+    const int t = (warp - Shape::kSoftmaxWarp0) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -650,7 +654,8 @@ int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
     p.part_o = p.part_ml = nullptr;
     const unsigned grid = static_cast<unsigned>(units < nsm ? units : nsm);
     trace_launch_begin(WAN_KIND_ATTN, s, work);
-    attn_fwd_tc_kernel<kF8, true><<<grid, kAttnThreads, AttnShape<kF8, true>::kSmem, s>>>(mq, mk, mv, p);
+    attn_fwd_tc_kernel<kF8, true>
+        <<<grid, AttnShape<kF8, true>::kThreads, AttnShape<kF8, true>::kSmem, s>>>(mq, mk, mv, p);
     const int st = check_launch();
     trace_launch_end(WAN_KIND_ATTN, s);
     return st;
@@ -672,7 +677,7 @@ int launch_units(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap
   p.part_ml = split ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + part_o_bytes) : nullptr;
   const unsigned grid = static_cast<unsigned>(split ? units + rem : units);
   trace_launch_begin(WAN_KIND_ATTN, s, work);
-  attn_fwd_tc_kernel<kF8, false><<<grid, kAttnThreads, kSmem, s>>>(mq, mk, mv, p);
+  attn_fwd_tc_kernel<kF8, false><<<grid, AttnShape<kF8, false>::kThreads, kSmem, s>>>(mq, mk, mv, p);
   int st = check_launch();
   if (st == WAN_OK && split) {
     attn_combine_kernel<<<dim3(static_cast<unsigned>(rem), kQTiles), 256, 0, s>>>(p);
