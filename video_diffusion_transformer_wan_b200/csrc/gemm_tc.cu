@@ -171,6 +171,65 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int row, int
   }
 }
 
+// bf16 store (plain or GELU) of one 32x32 block through shared memory: thread = row
+// applies scale, bias and GELU to its 32 columns, packs them to bf16 and stages the
+// 64-byte row (16-byte units XOR-swizzled by row); the warp then reads it back eight
+// rows per instruction (4 threads x 16 bytes per row), so each global store moves
+// whole 64-byte row segments instead of one 16-byte piece of 32 rows.
+__device__ __forceinline__ void store_staged_bf16(const GemmParams& p, uint32_t* stg, int r0, int n0, int lane,
+                                                  const uint32_t (&r)[32]) {
+  const int row = r0 + lane;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.a_scale) {
+    const float sc = row < p.M ? __ldg(p.a_scale + row) * __ldg(p.w_scale) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= sc;
+  }
+  if (p.bias) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (n0 + g * 8 < p.N) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.bias + n0) + g);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(h[j]);
+          v[g * 8 + 2 * j] += f.x;
+          v[g * 8 + 2 * j + 1] += f.y;
+        }
+      }
+    }
+  }
+  if (p.epi.kind == WAN_EPI_GELU) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_f(v[i]);
+  }
+  const int swz = (lane >> 1) & 3;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 u;
+    u.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+    u.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+    u.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+    u.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+    reinterpret_cast<uint4*>(stg + lane * 16)[g ^ swz] = u;
+  }
+  __syncwarp();
+  const int q = lane & 3;
+  const int gcol = n0 + q * 8;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = i * 8 + (lane >> 2);
+    const int grow = r0 + rr;
+    const uint4 u = reinterpret_cast<const uint4*>(stg + rr * 16)[q ^ ((rr >> 1) & 3)];
+    if (grow < p.M && gcol < p.N)
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(grow) * p.epi.ldo + gcol) = u;
+  }
+  __syncwarp();
+}
+
 // Gated residual (and plain fp32 store) epilogue through shared memory: for each
 // 32-column chunk the warp reads its 32 rows from TMEM (thread = row), scales and adds
 // the bias, stages the 32x32 block (16-byte units XOR-swizzled by row), then reads it
@@ -432,14 +491,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // and signal tfull[acc] in both CTAs; both CTAs' epilogue warps release tempty[acc] on
 // the even CTA. Barriers are initialised, and TMEM allocated, in both CTAs before a
 // cluster barrier; a second one precedes deallocation.
+// Epilogue: the gated residual stages fp32 blocks (residual_staged); the bf16 store and
+// GELU stage bf16 blocks (store_staged_bf16), so each store moves 64-byte row segments.
 #ifndef WAN_PAIR_STAGES_PLAIN
-#define WAN_PAIR_STAGES_PLAIN 6  // ring depth of the pair kernel without the staged epilogue
+#define WAN_PAIR_STAGES_PLAIN 6  // ring depth of the pair kernel without the gated residual
 #endif
 constexpr int kPairStageBytes = 2 * kBM * 128;  // A half + W half: 128 rows x 128 bytes each
 template <bool kRes>
 struct PairCfg {
   static constexpr int kStages = kRes ? 6 : WAN_PAIR_STAGES_PLAIN;
-  static constexpr size_t kEpiStageBytes = kRes ? static_cast<size_t>(kEpiWarps) * 32 * 32 * 4 : 0;
+  // fp32 32x32 block per epilogue warp (gated residual), or a bf16 one (staged store)
+  static constexpr size_t kEpiStageBytes = static_cast<size_t>(kEpiWarps) * 32 * 32 * (kRes ? 4 : 2);
   static constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * kPairStageBytes + 256 + kEpiStageBytes;
 };
 
@@ -587,6 +649,17 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CU
                              static_cast<uint32_t>(acc * 256 + colhalf * kBM);
       if constexpr (kRes) {
         residual_staged(p, epi_stage + (warp - 2) * 1024, t_row, m0 + quarter * 32, n0, lane, kMine);
+      } else if (p.epi.kind == WAN_EPI_STORE || p.epi.kind == WAN_EPI_GELU) {
+        uint32_t* stg = reinterpret_cast<uint32_t*>(epi_stage) + (warp - 2) * 512;
+#pragma unroll 1
+        for (int c = 0; c < kMine; c += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(t_row + c * 32, r0);
+          tmem_ld32(t_row + (c + 1) * 32, r1);
+          tmem_ld_wait();
+          store_staged_bf16(p, stg, m0 + quarter * 32, n0 + c * 32, lane, r0);
+          store_staged_bf16(p, stg, m0 + quarter * 32, n0 + (c + 1) * 32, lane, r1);
+        }
       } else {
 #pragma unroll 1
         for (int c = 0; c < kMine; c += 2) {
