@@ -307,6 +307,65 @@ __device__ __forceinline__ void residual_staged(const GemmParams& p, float* stg,
   }
 }
 
+// Gated residual (or fp32 store) by bulk tensor operations: for each 32-column chunk the
+// warp reads its 32 rows from TMEM (thread = row), forms g * (acc * scale + bias) (or
+// acc * scale + bias for the store), stages the 32 x 32 fp32 block in the 128-byte
+// swizzled layout of the x tensor map, and one lane issues a bulk reduce-add of the
+// block into x (x += block, element-wise in L2) or a bulk store. x is never read into
+// the SM. Each x element is updated by exactly one tile, so the result does not depend
+// on timing. The block is rewritten only after the previous bulk operation read it.
+__device__ __forceinline__ void residual_tma(const GemmParams& p, const CUtensorMap* map_x, float* stg,
+                                             uint32_t t_row, int r0, int n0, int lane, int chunks) {
+  const int row = r0 + lane;
+  const float sc = p.a_scale ? (row < p.M ? __ldg(p.a_scale + row) : 0.f) * __ldg(p.w_scale) : 1.0f;
+  const bool residual = p.epi.kind == WAN_EPI_RESIDUAL;
+  const float* gate_row = residual && p.epi.gate
+                              ? p.epi.gate + static_cast<int64_t>(min(row, p.M - 1) / p.epi.rows_per_batch) *
+                                                 p.epi.gate_bstride
+                              : nullptr;
+#pragma unroll 1
+  for (int c = 0; c < chunks; ++c) {
+    const int col0 = n0 + c * 32;
+    uint32_t r[32];
+    tmem_ld32(t_row + c * 32, r);
+    if (lane == 0) bulk_wait_read_all();
+    tmem_ld_wait();
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int col = col0 + 4 * k;
+      float4 v = make_float4(__uint_as_float(r[4 * k]) * sc, __uint_as_float(r[4 * k + 1]) * sc,
+                             __uint_as_float(r[4 * k + 2]) * sc, __uint_as_float(r[4 * k + 3]) * sc);
+      if (col < p.N) {
+        if (p.bias) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(p.bias + col));
+          const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+          const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+          v.x += b01.x; v.y += b01.y; v.z += b23.x; v.w += b23.y;
+        }
+        if (gate_row) {
+          float4 g = __ldg(reinterpret_cast<const float4*>(gate_row + col));
+          if (p.epi.gate_bias) {
+            const float4 gb = __ldg(reinterpret_cast<const float4*>(p.epi.gate_bias + col));
+            g.x += gb.x; g.y += gb.y; g.z += gb.z; g.w += gb.w;
+          }
+          v.x *= g.x; v.y *= g.y; v.z *= g.z; v.w *= g.w;
+        }
+      }
+      reinterpret_cast<float4*>(stg + lane * 32)[k ^ (lane & 7)] = v;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && r0 < p.M && col0 < p.N) {  // the tensor map clips the block at M and N
+      if (residual)
+        tma_reduce_add_2d(map_x, stg, col0, r0);
+      else
+        tma_store_2d(map_x, stg, col0, r0);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <int BN, bool kF8, bool kRes>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
   using C = GemmCfg<BN, kRes>;
@@ -491,8 +550,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // and signal tfull[acc] in both CTAs; both CTAs' epilogue warps release tempty[acc] on
 // the even CTA. Barriers are initialised, and TMEM allocated, in both CTAs before a
 // cluster barrier; a second one precedes deallocation.
-// Epilogue: the gated residual stages fp32 blocks (residual_staged); the bf16 store and
-// GELU stage bf16 blocks (store_staged_bf16), so each store moves 64-byte row segments.
+// Epilogue: the gated residual and the fp32 store stage fp32 blocks and hand them to
+// bulk tensor operations (residual_tma: a reduce-add into x, or a store), so x is never
+// read into the SM; the bf16 store and GELU stage bf16 blocks (store_staged_bf16), so
+// each store moves 64-byte row segments.
 #ifndef WAN_PAIR_STAGES_PLAIN
 #define WAN_PAIR_STAGES_PLAIN 6  // ring depth of the pair kernel without the gated residual
 #endif
@@ -506,20 +567,23 @@ struct PairCfg {
 };
 
 template <bool kF8, bool kRes>
-__device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const GemmParams& p) {
+__device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapX,
+                                               const GemmParams& p) {
   constexpr int kPairStages = PairCfg<kRes>::kStages;
   constexpr int kHalf = kBM * 128;  // bytes of one 128-row operand half per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kPairStages * kHalf;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kHalf);
+  // epilogue staging (1024-byte aligned, as the x tensor map's 128-byte swizzle needs),
+  // then the barriers
+  float* epi_stage = reinterpret_cast<float*>(sB + kPairStages * kHalf);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(epi_stage) + PairCfg<kRes>::kEpiStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  float* epi_stage = reinterpret_cast<float*>(sB + kPairStages * kHalf + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -543,6 +607,7 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CU
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapA);
     tma_prefetch_desc(&mapB);
+    if (kRes) tma_prefetch_desc(&mapX);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, 512);
@@ -648,7 +713,7 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CU
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * 256 + colhalf * kBM);
       if constexpr (kRes) {
-        residual_staged(p, epi_stage + (warp - 2) * 1024, t_row, m0 + quarter * 32, n0, lane, kMine);
+        residual_tma(p, &mapX, epi_stage + (warp - 2) * 1024, t_row, m0 + quarter * 32, n0, lane, kMine);
       } else if (p.epi.kind == WAN_EPI_STORE || p.epi.kind == WAN_EPI_GELU) {
         uint32_t* stg = reinterpret_cast<uint32_t*>(epi_stage) + (warp - 2) * 512;
 #pragma unroll 1
@@ -675,6 +740,8 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CU
       mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(acc) * 8u);
     }
   }
+  // The epilogue's bulk operations have completed before the CTA can exit.
+  if (kRes && warp >= 2 && lane == 0) bulk_wait_all();
   // Both CTAs are done with TMEM (and no remote arrival is pending) before it is freed.
   __syncwarp();
   tc_fence_before();
@@ -689,15 +756,15 @@ __device__ __forceinline__ void gemm_pair_body(const CUtensorMap& mapA, const CU
 template <bool kRes>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                          const GemmParams p) {
-  gemm_pair_body<false, kRes>(mapA, mapB, p);
+                          const __grid_constant__ CUtensorMap mapX, const GemmParams p) {
+  gemm_pair_body<false, kRes>(mapA, mapB, mapX, p);
 }
 
 template <bool kRes>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_e4m3_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                          const GemmParams p) {
-  gemm_pair_body<true, kRes>(mapA, mapB, p);
+                          const __grid_constant__ CUtensorMap mapX, const GemmParams p) {
+  gemm_pair_body<true, kRes>(mapA, mapB, mapX, p);
 }
 
 // Launch one instantiation (the shared-memory opt-in is set once per device for each).
@@ -773,6 +840,15 @@ int launch_pair(const void* A, int64_t lda, const void* W, const void* bias, voi
   const int pairs = sm_count() / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
   const bool staged = epi.kind == WAN_EPI_RESIDUAL || epi.kind == WAN_EPI_F32;
+  // x (fp32, [M, ldo]) for the bulk reduce-add / store of the staged epilogue: 32 x 32
+  // boxes; every box starts at a column that is a multiple of 32 (128 bytes).
+  CUtensorMap mapX = mapA;
+  if (staged) {
+    const uint64_t dimsX[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+    const uint64_t strX[1] = {static_cast<uint64_t>(epi.ldo) * 4};
+    const uint32_t boxX[2] = {32, 32};
+    if (!make_tmap_f32(&mapX, out, 2, dimsX, strX, boxX)) return WAN_ERR_CUDA;
+  }
   auto kern = staged ? (kF8 ? gemm_e4m3_pair_kernel<true> : gemm_bf16_pair_kernel<true>)
                      : (kF8 ? gemm_e4m3_pair_kernel<false> : gemm_bf16_pair_kernel<false>);
   const size_t smem = staged ? PairCfg<true>::kSmemBytes : PairCfg<false>::kSmemBytes;
@@ -782,7 +858,7 @@ int launch_pair(const void* A, int64_t lda, const void* W, const void* bias, voi
   std::call_once(once[staged ? 1 : 0][dev & 63],
                  [kern, smem] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                      static_cast<int>(smem)); });
-  kern<<<grid, kGemmThreads, smem, s>>>(mapA, mapB, p);
+  kern<<<grid, kGemmThreads, smem, s>>>(mapA, mapB, mapX, p);
   return check_launch();
 }
 

@@ -70,6 +70,8 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
 // The same for 8-bit elements (E4M3 codes).
 bool make_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                   const uint64_t* strides_bytes, const uint32_t* box);
+bool make_tmap_f32(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box);
 
 // ---------------------------------------------------------------- kernels
 // LayerNorm (+ modulation). rows = B*L; e/mod_bias may be NULL (chunk < 0: plain LN).
