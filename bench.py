@@ -67,9 +67,20 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def code_sha256(path):
+    """sha256 of a CUDA source with its // comments, surrounding whitespace and blank
+    lines removed: it changes with the code, not with the comments."""
+    lines = []
+    for line in open(path, encoding="utf-8"):
+        code = line.split("//", 1)[0].strip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def attn_traffic_per_launch(w):
     """DRAM bytes (read + write) per self-attention launch from the committed ncu
-    summary, or None when the kernel source changed since the counters were taken or
+    summary, or None when the kernel code changed since the counters were taken or
     the summary's launch shape (batch, tokens, heads) is not this workload's."""
     p = os.path.join(PROFILES, "attn_fwd_tc_kernel__self_L32760_H12.md")
     src = os.path.join(ROOT, "video_diffusion_transformer_wan_b200", "csrc", "attn_tc.cu")
@@ -77,13 +88,13 @@ def attn_traffic_per_launch(w):
         return None
     sha = byts = shape = None
     for line in open(p):
-        if line.startswith("- attn_tc.cu sha256:"):
+        if line.startswith("- attn_tc.cu code sha256:"):
             sha = line.split(":", 1)[1].strip()
         elif line.startswith("- dram bytes per launch (read+write):"):
             byts = float(line.split(":", 1)[1])
         elif line.startswith("- launch shape (batch, tokens, heads):"):
             shape = tuple(int(v) for v in line.split(":", 1)[1].split(","))
-    if sha != hashlib.sha256(open(src, "rb").read()).hexdigest():
+    if sha != code_sha256(src):
         return None
     if shape != (w.batch, w.tokens, w.heads):
         return None

@@ -122,3 +122,15 @@ def test_attention_traffic_only_for_the_profiled_launch_shape(bench):
         assert t > 0
         assert bench.attn_traffic_per_launch(WORKLOADS["wan13b_480p_stack30"]) == t
         assert bench.attn_traffic_per_launch(WORKLOADS["wan13b_480p_i2v_block"]) == t
+
+
+def test_code_hash_follows_code_not_comments(bench, tmp_path):
+    """The profile's traffic stays valid across comment edits and lapses on a code edit."""
+    a = tmp_path / "a.cu"
+    a.write_text("// header\nint f(int x) {  // trailing\n  return x + 1;\n}\n")
+    b = tmp_path / "b.cu"
+    b.write_text("// another header\n\nint f(int x) {\n  return x + 1;   // changed comment\n}\n")
+    c = tmp_path / "c.cu"
+    c.write_text("// header\nint f(int x) {\n  return x + 2;\n}\n")
+    assert bench.code_sha256(str(a)) == bench.code_sha256(str(b))
+    assert bench.code_sha256(str(a)) != bench.code_sha256(str(c))

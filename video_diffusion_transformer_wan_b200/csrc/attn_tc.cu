@@ -5,7 +5,8 @@
 // head, non-causal, bf16 inputs, fp32 accumulation and fp32 softmax, head_dim 128.
 //
 // One CTA = two 128-row query tiles (t = 0, 1) of one (sample, head); 384 threads in
-// three warpgroups (bf16; the E4M3 instantiation has 320, without warps 2-3):
+// three warpgroups (bf16; the E4M3 instantiation has 320 threads, no idle warps, and
+// its softmax warps are 2-5 and 6-9):
 //   warp 0    : TMA producer - both Q tiles once, then K_0, K_1, V_0, K_2, V_1, ...
 //               (the order the MMA warp consumes them) through a 5-stage ring of 32 KB
 //               tiles (128 rows x 128 dims as two 64-dim halves, 128-byte swizzle);
