@@ -318,3 +318,41 @@ def test_attention_fp8_running_base_mutations_are_caught(monkeypatch):
         _fails(P.check_attention_fp8_running_base, O.attention_fp8)
     monkeypatch.setattr(O, "_running_base_rows", base)
     P.check_attention_fp8_running_base(O.attention_fp8)
+
+
+def test_head_and_image_mlp_mutations_are_caught():
+    def no_norm(x, w, b, eps=1e-6):                     # LayerNorm dropped from the head
+        return O.linear(x, w, b)
+
+    def eps_outside_head(x, w, b, eps=1e-6):            # eps added to the deviation, not the variance
+        x = np.asarray(x, np.float64)
+        ln = (x - x.mean(-1, keepdims=True)) / (np.sqrt(x.var(-1, keepdims=True)) + eps)
+        return O.linear(ln, w, b)
+    _fails(P.check_head, no_norm)
+    _fails(P.check_head, eps_outside_head)
+
+    def relu_mlp(feat, w1, b1, w2, b2, w3, b3):         # ReLU for GELU-tanh
+        h = np.maximum(O.linear(feat, w1, b1), 0)
+        return O.linear(np.maximum(O.linear(h, w2, b2), 0), w3, b3)
+
+    def gelu_on_output(feat, w1, b1, w2, b2, w3, b3):   # activation after the last layer too
+        return O.gelu_tanh(O.image_context_mlp(feat, w1, b1, w2, b2, w3, b3))
+
+    def one_gelu(feat, w1, b1, w2, b2, w3, b3):         # the second activation dropped
+        return O.linear(O.linear(O.gelu_tanh(O.linear(feat, w1, b1)), w2, b2), w3, b3)
+    for mut in (relu_mlp, gelu_on_output, one_gelu):
+        _fails(P.check_image_context_mlp, mut)
+
+
+def test_flow_matching_mutations_are_caught():
+    def swapped_ends(x1, x0, u):                         # x_t = t x0 + (1 - t) x1
+        return O.flow_matching_input(x0, x1, u)
+
+    def flipped_target(x1, x0):                          # v = x0 - x1
+        return O.flow_matching_target(x0, x1)
+
+    def half_step(x1, x0, u):                            # t used as t / 2
+        return O.flow_matching_input(x1, x0, u / 2)
+    _fails(P.check_flow_matching, swapped_ends, O.flow_matching_target)
+    _fails(P.check_flow_matching, O.flow_matching_input, flipped_target)
+    _fails(P.check_flow_matching, half_step, O.flow_matching_target)

@@ -433,7 +433,8 @@ def test_i2v_zero_projection_equals_t2v():
     assert not np.allclose(O.patchify(x36, w36, b), O.patchify(noise, w16, b))
 
 
-def test_image_context_mlp_vs_torch():
+def check_image_context_mlp(mlp):
+    """Linear -> GELU-tanh -> Linear -> GELU-tanh -> Linear, re-expressed in torch."""
     rng = RNG(11)
     feat = rng.standard_normal((5, 24))
     ws = [rng.standard_normal(s) * 0.2 for s in [(16, 24), (16,), (16, 16), (16,), (16, 16), (16,)]]
@@ -442,7 +443,24 @@ def test_image_context_mlp_vs_torch():
         ref = tF.linear(ref, t64(ws[2 * i]), t64(ws[2 * i + 1]))
         if i < 2:
             ref = tF.gelu(ref, approximate="tanh")
-    np.testing.assert_allclose(O.image_context_mlp(feat, *ws), ref.numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(mlp(feat, *ws), ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_image_context_mlp_vs_torch():
+    check_image_context_mlp(O.image_context_mlp)
+
+
+def check_head(head):
+    """Plain LayerNorm (eps 1e-6, no affine) then Linear(D, out_ch * 4), in torch."""
+    rng = RNG(14)
+    x = rng.standard_normal((7, 32)) * 3 + 1.5
+    w, b = rng.standard_normal((64, 32)) * 0.1, rng.standard_normal(64)
+    ref = tF.linear(tF.layer_norm(t64(x), (32,), eps=1e-6), t64(w), t64(b))
+    np.testing.assert_allclose(head(x, w, b), ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_head_vs_torch():
+    check_head(O.head)
 
 
 def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
@@ -526,13 +544,19 @@ def test_stack_f32_matches_float64_stack():
     check_stack_f32(O.dit_stack_f32)
 
 
-def test_flow_matching_endpoints():
+def check_flow_matching(fm_input, fm_target):
+    """x_t runs from x0 at t = 0 to x1 at t = 1 on a straight line whose velocity is the
+    target: x_0.75 - x_0.25 = 0.5 v."""
     rng = RNG(12)
     x1, x0 = rng.standard_normal((3, 4)), rng.standard_normal((3, 4))
-    assert np.array_equal(O.flow_matching_input(x1, x0, 0.0), x0)
-    assert np.array_equal(O.flow_matching_input(x1, x0, 1.0), x1)
-    a, b = O.flow_matching_input(x1, x0, 0.25), O.flow_matching_input(x1, x0, 0.75)
-    np.testing.assert_allclose(b - a, 0.5 * O.flow_matching_target(x1, x0), rtol=1e-14, atol=1e-15)
+    assert np.array_equal(fm_input(x1, x0, 0.0), x0)
+    assert np.array_equal(fm_input(x1, x0, 1.0), x1)
+    a, b = fm_input(x1, x0, 0.25), fm_input(x1, x0, 0.75)
+    np.testing.assert_allclose(b - a, 0.5 * fm_target(x1, x0), rtol=1e-14, atol=1e-15)
+
+
+def test_flow_matching_endpoints():
+    check_flow_matching(O.flow_matching_input, O.flow_matching_target)
 
 
 # ----------------------------------------------------------------------------------------
