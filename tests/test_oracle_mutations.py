@@ -356,3 +356,14 @@ def test_flow_matching_mutations_are_caught():
     _fails(P.check_flow_matching, swapped_ends, O.flow_matching_target)
     _fails(P.check_flow_matching, O.flow_matching_input, flipped_target)
     _fails(P.check_flow_matching, half_step, O.flow_matching_target)
+
+
+def test_i2v_input_mutations_are_caught():
+    def cond_first(noise, cond, mask):                   # condition latent before the noise
+        return O.i2v_input(cond, noise, mask)
+
+    def mask_before_cond(noise, cond, mask):             # mask channels before the condition
+        return np.concatenate([np.asarray(noise, np.float64), np.asarray(mask, np.float64),
+                               np.asarray(cond, np.float64)], axis=0)
+    _fails(P.check_i2v_input, cond_first)
+    _fails(P.check_i2v_input, mask_before_cond)

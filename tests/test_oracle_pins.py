@@ -420,17 +420,27 @@ def test_i2v_mask_structure():
     check_i2v_mask(O.i2v_mask)
 
 
-def test_i2v_zero_projection_equals_t2v():
+def check_i2v_input(i2v_input):
+    """With the 20 extra input channels' weights at zero (their initialisation), the
+    36-channel patchify is the text-to-video one on the noise; the condition latent sits
+    in channels 16-31 and the mask in 32-35."""
     rng = RNG(10)
     D, F, H, W = 12, 2, 4, 6
     noise, cond = rng.standard_normal((16, F, H, W)), rng.standard_normal((16, F, H, W))
     keep = np.zeros(1 + 4 * (F - 1)); keep[0] = 1
-    x36 = O.i2v_input(noise, cond, O.i2v_mask(keep, F, H, W))
+    mask = O.i2v_mask(keep, F, H, W)
+    x36 = i2v_input(noise, cond, mask)
+    assert x36.shape == (36, F, H, W)
     w16 = rng.standard_normal((D, 16, 1, 2, 2)); b = rng.standard_normal(D)
     w36 = np.concatenate([w16, np.zeros((D, 20, 1, 2, 2))], axis=1)
     assert np.array_equal(O.patchify(x36, w36, b), O.patchify(noise, w16, b))
+    assert np.array_equal(x36[16:32], cond) and np.array_equal(x36[32:], mask)
     w36[:, 16:] = rng.standard_normal((D, 20, 1, 2, 2))
     assert not np.allclose(O.patchify(x36, w36, b), O.patchify(noise, w16, b))
+
+
+def test_i2v_zero_projection_equals_t2v():
+    check_i2v_input(O.i2v_input)
 
 
 def check_image_context_mlp(mlp):
