@@ -367,3 +367,16 @@ def test_i2v_input_mutations_are_caught():
                                np.asarray(cond, np.float64)], axis=0)
     _fails(P.check_i2v_input, cond_first)
     _fails(P.check_i2v_input, mask_before_cond)
+
+
+def test_stack_mutations_are_caught():
+    def reversed_blocks(latent, t, weights, blocks, ctx, heads, **kw):   # blocks applied last to first
+        return O.dit_stack(latent, t, weights, list(blocks)[::-1], ctx, heads, **kw)
+
+    def first_block_twice(latent, t, weights, blocks, ctx, heads, **kw):  # one block's weights for all
+        return O.dit_stack(latent, t, weights, [blocks[0]] * len(blocks), ctx, heads, **kw)
+
+    def time_in_thousandths(latent, t, weights, blocks, ctx, heads, **kw):  # t rescaled to [0, 1]
+        return O.dit_stack(latent, t / 1000.0, weights, blocks, ctx, heads, **kw)
+    for mut in (reversed_blocks, first_block_twice, time_in_thousandths):
+        _fails(P.check_stack, mut)

@@ -473,24 +473,31 @@ def test_head_vs_torch():
     check_head(O.head)
 
 
-def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
+def check_stack(dit_stack):
+    """All-zero blocks leave the stack as head(patchify) (in torch); two real blocks equal
+    the torch re-expression of the block applied in order with the shared MLP output."""
     w = WORKLOADS["tiny_f32_block"]
     inp = make_inputs(w, seed=1, n_blocks=2)
     lat, t, ctx = inp["noise"][0], float(inp["t"][0]), inp["ctx"][0]
     zero = [{k: np.zeros_like(v) for k, v in b.items()} for b in inp["blocks"]]
-    v = O.dit_stack(lat, t, inp, zero, ctx, w.heads)
+    v = dit_stack(lat, t, inp, zero, ctx, w.heads)
     x = O.patchify(lat, inp["w_p"], inp["b_p"])
     ref = O.unpatchify(tF.linear(tF.layer_norm(t64(x), (w.dim,), eps=1e-6), t64(inp["w_head"]),
                                  t64(inp["b_head"])).numpy(), 16, w.frames, w.height, w.width)
     np.testing.assert_allclose(v, ref, rtol=1e-12, atol=1e-12)
-    # two real blocks == the torch re-expression applied twice with the shared MLP output
-    v2 = O.dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads)
+    v2 = dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads)
     e = O.time_mlp(t, inp["w_t1"], inp["b_t1"], inp["w_t2"], inp["b_t2"])
     xx = x
     for b in inp["blocks"]:
         xx = torch_block(xx, e, b, ctx, w.heads)
     ref2 = O.unpatchify(O.head(xx, inp["w_head"], inp["b_head"]), 16, w.frames, w.height, w.width)
     np.testing.assert_allclose(v2, ref2, rtol=1e-10, atol=1e-11)
+    return inp, lat, t, ctx, x, e, v2
+
+
+def test_stack_with_zero_blocks_is_head_of_patchify_and_matches_blockwise():
+    w = WORKLOADS["tiny_f32_block"]
+    inp, lat, t, ctx, x, e, v2 = check_stack(O.dit_stack)
     # the FP8 stack == the torch re-expression of the FP8 block (torch's E4M3 conversion)
     # applied twice; patchify, the time MLP and the head unchanged
     v3 = O.dit_stack(lat, t, inp, inp["blocks"], ctx, w.heads, fp8=True)
